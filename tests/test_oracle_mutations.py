@@ -1,0 +1,53 @@
+"""The oracle's pins catch plausible mistakes planted in the oracle.
+
+Each case copies the oracle's C source, plants one mistake (a dropped term,
+a wrong sign, index or constant, a transposed operand, the wrong rounding
+rule), builds it with the oracle's own flags into a temporary library and
+runs the pin tests against it in a fresh process.  The pins must fail for
+every mutant.  Everything here runs on the CPU.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTANTS = {
+    "gamma_signed_mean": ("row += fabs((double)W[n * K + k]);", "row += (double)W[n * K + k];"),
+    "gamma_fp32_accumulate": ("double row = 0.0;", "float row = 0.0f;"),
+    "gamma_divides_by_rows": ("return (float)(total / (double)(N * K));", "return (float)(total / (double)(K));"),
+    "ternary_no_eps": ("float d = gamma + ORACLE_EPS;", "float d = gamma;"),
+    "ternary_round_half_away": ("float t = rintf(r);", "float t = roundf(r);"),
+    "ternary_no_clamp": ("if (t > 1.0f) t = 1.0f;", ";"),
+    "pack_swapped_fields": ("word |= code << (8 * b + 2 * j);", "word |= code << (8 * j + 2 * b);"),
+    "pack_signed_code": ("uint32_t code = (uint32_t)(t + 1);", "uint32_t code = (uint32_t)(t & 3);"),
+    "act_scale_128": ("float scale = 127.0f / fmaxf(amax, ORACLE_EPS);", "float scale = 128.0f / fmaxf(amax, ORACLE_EPS);"),
+    "act_round_half_away": ("float v = rintf(x[m * K + k] * scale);", "float v = roundf(x[m * K + k] * scale);"),
+    "act_signed_max": ("float a = fabsf(x[m * K + k]);", "float a = x[m * K + k];"),
+    "acc_transposed_weight": ("(int64_t)T[n * K + k];", "(int64_t)T[k * N + n];"),
+    "dequant_multiplies_scale": ("(double)gamma / (double)s[m];", "(double)gamma * (double)s[m];"),
+    "dequant_gamma_plus_eps": ("(double)gamma / (double)s[m];", "((double)gamma + 1e-5) / (double)s[m];"),
+    "bf16_via_fp32": ("double r = rint(ldexp(a, -qexp));", "double r = rint(ldexp((double)(float)a, -qexp));"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_mutant(name, tmp_path):
+    before, after = MUTANTS[name]
+    src = open(oracle._SRC).read()
+    assert src.count(before) == 1, "mutation site not found: " + name
+    mutated = tmp_path / "mutant.c"
+    mutated.write_text(src.replace(before, after))
+    so = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", *oracle.CFLAGS, str(mutated), "-o", str(so), "-lm"])
+    env = dict(os.environ, BITLINEAR_ORACLE_LIB=str(so))
+    res = subprocess.run(
+        [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600,
+    )
+    assert res.returncode != 0, "pins did not catch mutant %s:\n%s" % (name, res.stdout[-2000:])
