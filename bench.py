@@ -1,0 +1,556 @@
+#!/usr/bin/env python
+"""Benchmark of the BitLinear W1.58A8 forward on B200.
+
+Headline (``value``): decode GB/s of packed ternary weights streamed per
+second for the 2B-class decode step (one token through BitLinear K=2560 ->
+N=6912 and K=2560 -> N=2560, bf16 in/out), whole job over all ranks.  A step
+is one pass of the inference forward over one batch: per-token activation
+quantisation, ternary x int8 product with int32 accumulation and fused
+dequantisation, for every layer of the workload.  The weights are packed once
+at load time (absmean + ternarise + pack), as a deployed checkpoint is; that
+offline path is timed separately under ``pack``.
+
+Also reported in the same line: the 2B prefill GEMM (2048 tokens) in int8
+TOPS against the tensor-core roofline, and the 70B-class decode layer chain
+at 1 and 8 tokens in GB/s.  Inputs are seeded and synthetic with the pages'
+shapes and distributions; weights rotate over enough copies that every step
+reads them from HBM (more than 4x the L2 size).
+
+``--impl reference`` times the CPU oracle (plain scalar C, one core) on the
+same workload, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "BitLinear decode GB/s (% HBM peak) + prefill int8 TOPS (% peak), 1 B200"
+UNIT = "GB/s"
+DECODE_LAYERS = [(2560, 6912), (2560, 2560)]  # (K in, N out)
+PREFILL = dict(M=2048, K=2560, N=6912)
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_PER_BF16 = 2.0  # nominal dense ratio (4.5 POPS int8 / 2.25 PFLOPS bf16)
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100000, help="timed decode steps")
+    p.add_argument("--warmup", type=int, default=2000)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-extras", action="store_true", help="skip prefill / 70B chain / pack lines")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS, bf16_sustained=1400.0,
+                    source="fallback")
+
+
+# ----------------------------------------------------------------------------
+# clocks sampled while the GPU is busy
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.QUERY, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [s.strip() for s in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        busy = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (replicas: no data-path collective)
+# ----------------------------------------------------------------------------
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+# workloads
+# ----------------------------------------------------------------------------
+
+def l2_bytes():
+    import torch
+
+    return torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+
+
+def make_layer_sets(shapes, seed, min_bytes):
+    """Packed weights for each (K, N) layer, plus byte-identical copies at other
+    addresses until all sets together exceed ``min_bytes`` (cold L2 per step)."""
+    import torch
+
+    import synth
+    import ternary_weight_a8_b200 as tb
+
+    base = []
+    for i, (K, N) in enumerate(shapes):
+        W = torch.from_numpy(synth.latent_weights(N, K, seed=seed + i)).cuda()
+        packed, gamma = tb.pack_weights(W)
+        del W
+        base.append((packed, gamma))
+    set_bytes = sum(p.numel() for p, _ in base)
+    nsets = max(1, math.ceil(min_bytes / set_bytes))
+    sets = [base] + [[(p.clone(), g.clone()) for p, g in base] for _ in range(nsets - 1)]
+    torch.cuda.synchronize()
+    return sets, set_bytes
+
+
+def make_inputs(shapes, M, seed, shared=None):
+    import torch
+
+    import synth
+
+    xs = []
+    for i, (K, N) in enumerate(shapes):
+        if shared is not None and shared[i]:
+            xs.append(xs[-1])
+            continue
+        bits, _ = synth.activations_bf16(M, K, seed=seed + 100 + i)
+        xs.append(torch.from_numpy(bits.view("int16")).cuda().view(torch.bfloat16))
+    ys = [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for (K, N) in shapes]
+    return xs, ys
+
+
+def capture(fn, steps):
+    """A CUDA graph of `steps` calls fn(i)."""
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn(0)  # warm the launch paths outside the capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            for i in range(steps):
+                fn(i)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    return g
+
+
+def timed_graph_run(step_fn, steps, warmup, world, chunk=500, sampler=None):
+    """Times exactly `steps` calls of step_fn, replayed as CUDA graphs; returns seconds (max over ranks)."""
+    import torch
+
+    chunk = max(1, min(chunk, steps))
+    g_main = capture(lambda i: step_fn(i), chunk)
+    rem = steps % chunk
+    g_rem = capture(lambda i: step_fn(i), rem) if rem else None
+    w_chunk = max(1, min(chunk, warmup))
+    g_warm = capture(lambda i: step_fn(i), w_chunk)
+    for _ in range(max(1, warmup // w_chunk)):
+        g_warm.replay()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps // chunk):
+        g_main.replay()
+    if g_rem is not None:
+        g_rem.replay()
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    secs = start.elapsed_time(end) / 1e3
+    del g_main, g_rem, g_warm
+    return max_over_ranks(secs, world), clocks
+
+
+def kernel_event_times(launch_pre, launch_kernel, steps):
+    """Average device duration of one kernel, timed with events on its launching stream."""
+    import torch
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        launch_pre(i)
+        evs[i][0].record()
+        launch_kernel(i)
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    t = [a.elapsed_time(b) / 1e3 for a, b in evs]
+    return statistics.mean(t), statistics.median(t)
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import ternary_weight_a8_b200 as tb
+
+    torch.cuda.set_device(local)
+    peaks = load_peaks()
+    L2 = l2_bytes()
+    out = {}
+
+    # ---- decode 2B (headline) ----
+    sets, set_bytes = make_layer_sets(DECODE_LAYERS, seed=0, min_bytes=4 * L2)
+    nsets = len(sets)
+    xs, ys = make_inputs(DECODE_LAYERS, 1, seed=0)
+    ws = tb.new_workspace(max(tb.workspace_bytes(1, N, K) for K, N in DECODE_LAYERS))
+
+    def decode_step(i):
+        S = sets[i % nsets]
+        for (packed, gamma), x, y in zip(S, xs, ys):
+            tb.forward(packed, gamma, x, y=y, workspace=ws)
+
+    sampler = ClockSampler(torch.cuda.current_device())
+    secs, clocks = timed_graph_run(decode_step, args.steps, args.warmup, world, sampler=sampler)
+    units = args.steps * set_bytes * world
+    value = units / secs / 1e9
+    launches = args.steps * 2 * len(DECODE_LAYERS)
+    status = tb.device_status(ws)
+
+    # roofline of the dominant kernel: the GEMV of the N=6912 layer, timed per launch
+    K0, N0 = DECODE_LAYERS[0]
+    xq = torch.empty((1, K0), dtype=torch.int8, device="cuda")
+    sc = torch.empty(1, dtype=torch.float32, device="cuda")
+    rs = torch.empty(1, dtype=torch.int32, device="cuda")
+    nk = min(args.steps, 3000)
+    mean_s, med_s = kernel_event_times(
+        lambda i: tb.quant_act(xs[0], xq, sc, rs),
+        lambda i: tb.forward_quantized(sets[i % nsets][0][0], sets[i % nsets][0][1], xq, sc, rs, y=ys[0],
+                                       workspace=ws), nk)
+    gemv_bytes = N0 * K0 // 4 + K0 + N0 * 2 + 16
+    achieved = gemv_bytes / mean_s / 1e9
+    roofline = {"bound": "hbm", "kernel": "gemv_kernel (K=2560, N=6912, 1 token)", "achieved": round(achieved, 1),
+                "peak": peaks["hbm"], "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
+                "peak_source": peaks["source"], "traffic": None,
+                "algorithmic_bytes_per_launch": gemv_bytes, "launch_us_mean": round(mean_s * 1e6, 3),
+                "launch_us_median": round(med_s * 1e6, 3)}
+
+    # ---- e2e through the public API with host buffers ----
+    x_host = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in xs]
+    for h, x in zip(x_host, xs):
+        h.copy_(x.cpu())
+    y_host = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in ys]
+    ne = min(args.steps, 2000)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(ne):
+        S = sets[i % nsets]
+        for (packed, gamma), xh, x, y, yh in zip(S, x_host, xs, ys, y_host):
+            x.copy_(xh, non_blocking=True)
+            tb.forward(packed, gamma, x, y=y, workspace=ws)
+            yh.copy_(y, non_blocking=True)
+        torch.cuda.current_stream().synchronize()  # the step's result is on the host
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_secs = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+    e2e = {"value": round(ne * set_bytes * world / e2e_secs / 1e9, 2), "unit": UNIT,
+           "h2d_bytes_per_step": sum(x.numel() * 2 for x in xs),
+           "d2h_bytes_per_step": sum(y.numel() * 2 for y in ys), "steps": ne,
+           "ms_per_step": round(e2e_secs / ne * 1e3, 4)}
+    del sets
+
+    if not args.no_extras:
+        out["prefill"] = run_prefill(args, world, peaks, L2)
+        out["chain_70b"] = run_chain(args, world, peaks, L2)
+        out["pack"] = run_pack(world)
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic (seeded N(0,0.02) latent weights, N(0,1) bf16 activations with 1% x20 outlier channels)",
+        "config": {"workload": "decode_2b: BitLinear K=2560->N=6912 and K=2560->N=2560, 1 token, bf16 in/out, "
+                               "packed 2-bit ternary weights",
+                   "tokens": 1, "layers_k_n": DECODE_LAYERS, "weight_bytes_per_step": set_bytes,
+                   "l2": "rotating %d byte-identical weight sets (%.0f MB > 4x L2), cold L2 every step"
+                         % (nsets, nsets * set_bytes / 1e6),
+                   "graph": "steps replayed as CUDA graphs of 500 steps", "parallelism": "replicas x%d" % world},
+        "pct_hbm_measured": round(100 * value / world / peaks["hbm"], 2),
+        "pct_hbm_nominal_8tbs": round(100 * value / world / 8000.0, 2),
+        "roofline": roofline, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+        "device_status": status,
+    }
+    result.update(out)
+    return result
+
+
+def run_prefill(args, world, peaks, L2):
+    import torch
+
+    import ternary_weight_a8_b200 as tb
+
+    M, K, N = PREFILL["M"], PREFILL["K"], PREFILL["N"]
+    sets, set_bytes = make_layer_sets([(K, N)], seed=7, min_bytes=L2)
+    xs = []
+    import synth
+    for i in range(4):
+        bits, _ = synth.activations_bf16(M, K, seed=300 + i)
+        xs.append(torch.from_numpy(bits.view("int16")).cuda().view(torch.bfloat16))
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = tb.new_workspace(tb.workspace_bytes(M, N, K))
+
+    def step(i):
+        packed, gamma = sets[i % len(sets)][0]
+        tb.forward(packed, gamma, xs[i % len(xs)], y=y, workspace=ws)
+
+    steps = 400
+    secs, _ = timed_graph_run(step, steps, 20, world, chunk=100)
+    ops = 2.0 * M * N * K
+    tops = ops * steps * world / secs / 1e12
+    xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    sc = torch.empty(M, dtype=torch.float32, device="cuda")
+    rs = torch.empty(M, dtype=torch.int32, device="cuda")
+    mean_s, med_s = kernel_event_times(
+        lambda i: tb.quant_act(xs[i % len(xs)], xq, sc, rs),
+        lambda i: tb.forward_quantized(sets[i % len(sets)][0][0], sets[i % len(sets)][0][1], xq, sc, rs, y=y,
+                                       workspace=ws), 100)
+    peak_int8 = peaks["bf16"] * INT8_PER_BF16
+    k_tops = ops / mean_s / 1e12
+    status = tb.device_status(ws)
+    return {"metric": "prefill int8 TOPS", "value": round(tops, 1), "unit": "TOPS",
+            "workload": "prefill_2b: BitLinear K=2560->N=6912 over 2048 tokens (act quant + tcgen05 GEMM)",
+            "ms_per_step": round(secs / steps * 1e3, 5), "tokens_per_s": round(M * steps * world / secs, 0),
+            "roofline": {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 kind::i8)", "achieved": round(k_tops, 1),
+                         "peak": peak_int8, "unit": "TOPS", "frac": round(k_tops / peak_int8, 4),
+                         "peak_source": "%s bf16 burst x %.0f (nominal int8/bf16 ratio)" % (peaks["source"], INT8_PER_BF16),
+                         "launch_us_mean": round(mean_s * 1e6, 2), "launch_us_median": round(med_s * 1e6, 2),
+                         "traffic": None},
+            "pct_int8_nominal_4500": round(100 * tops / world / 4500.0, 2), "device_status": status}
+
+
+def run_chain(args, world, peaks, L2):
+    import torch
+
+    import synth
+    import ternary_weight_a8_b200 as tb
+
+    shapes = synth.CHAIN_70B
+    sets, set_bytes = make_layer_sets(shapes, seed=1000, min_bytes=3 * L2)
+    res = {"workload": "chain_70b: QKV 8192->10240, O 8192->8192, gate+up 8192->2x28672, down 28672->8192, "
+                       "bf16, gate/up share one quantised input", "weight_bytes_per_step": set_bytes}
+    for M in (1, 8):
+        xs, ys = make_inputs(shapes, M, seed=1000, shared=synth.CHAIN_70B_SHARED_INPUT)
+        layer_sets = [[tb.Layer(p, g, x, y) for (p, g), x, y in zip(S, xs, ys)] for S in sets]
+        ws = tb.new_workspace(tb.chain_workspace_bytes(layer_sets[0], M))
+
+        def step(i):
+            tb.layer_chain(layer_sets[i % len(layer_sets)], workspace=ws)
+
+        steps = 300
+        secs, _ = timed_graph_run(step, steps, 10, world, chunk=100)
+        gbs = set_bytes * steps * world / secs / 1e9
+        res["tokens_%d" % M] = {"GB/s": round(gbs, 1), "pct_hbm_measured": round(100 * gbs / world / peaks["hbm"], 2),
+                                "us_per_chain": round(secs / steps * 1e6, 2),
+                                "tokens_per_s": round(M * steps * world / secs, 1),
+                                "device_status": tb.device_status(ws)}
+    return res
+
+
+def run_pack(world):
+    import torch
+
+    import synth
+    import ternary_weight_a8_b200 as tb
+
+    K, N = 2560, 6912
+    W = torch.from_numpy(synth.latent_weights(N, K, seed=0)).cuda()
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device="cuda")
+    gamma = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = tb.new_workspace(tb.pack_workspace_bytes(N, K))
+    for _ in range(3):
+        tb.pack_weights(W, packed, gamma, ws)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    n = 20
+    for _ in range(n):
+        tb.pack_weights(W, packed, gamma, ws)
+    b.record()
+    torch.cuda.synchronize()
+    s = a.elapsed_time(b) / 1e3 / n
+    return {"workload": "pack K=2560, N=6912 fp32 latent -> 2-bit (gamma + ternarise + pack)",
+            "us_per_call": round(s * 1e6, 1), "GB/s_latent_read": round(N * K * 4 / s / 1e9, 1)}
+
+
+# ----------------------------------------------------------------------------
+# the oracle (CPU) on the same workload
+# ----------------------------------------------------------------------------
+
+def oracle_decode_setup():
+    import numpy as np
+
+    import oracle
+    import synth
+
+    layers = []
+    for i, (K, N) in enumerate(DECODE_LAYERS):
+        W = synth.latent_weights(N, K, seed=i)
+        packed, gamma, _ = oracle.pack_weights(W)
+        _, xf = synth.activations_bf16(1, K, seed=100 + i)
+        layers.append((packed, gamma, K, xf))
+    set_bytes = sum(p.size for p, *_ in layers)
+
+    def step():
+        for packed, gamma, K, xf in layers:
+            T, ok = oracle.unpack(packed, K)
+            acc, y, *_ = oracle.forward(T, gamma, xf)
+            oracle.round_bf16(y)
+
+    return step, set_bytes
+
+
+def cpu_baseline(target_s=10.0):
+    step, set_bytes = oracle_decode_setup()
+    t0 = time.perf_counter()
+    step()
+    one = time.perf_counter() - t0
+    reps = max(1, int(target_s / max(one, 1e-6)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        step()
+    secs = time.perf_counter() - t0
+    return {"value": round(reps * set_bytes / secs / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "%d full decode_2b steps (unpack + quantise + accumulate + dequantise + bf16 round, "
+                      "both layers) on one host core, %.1f s" % (reps, secs)}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    step, set_bytes = oracle_decode_setup()
+    steps = max(1, min(args.steps, 200))
+    warm = max(0, min(args.warmup, 3))
+    for _ in range(warm):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        step()
+    secs = time.perf_counter() - t0
+    value = steps * set_bytes / secs / 1e9
+    sample = "%d full decode_2b steps on one host core (steps capped at 200)" % steps
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+            "steps": steps, "warmup": warm, "ms_per_step": round(secs / steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": "decode_2b: BitLinear K=2560->N=6912 and K=2560->N=2560, 1 token, bf16 in/out"},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_init() if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    if args.impl == "reference":
+        res = run_reference(args, world, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    res = run_ours(args, world, rank, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

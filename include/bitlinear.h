@@ -1,0 +1,182 @@
+/*
+ * bitlinear.h — C ABI of the B200 (sm_100a) BitLinear W1.58A8 forward.
+ *
+ * The operation, from the BitNet b1.58 pages:
+ *  - "BitNet b1.58 and the 1-Bit AI Architecture Revolution", section "The
+ *    BitLinear Layer and AbsMean Quantization": gamma is the mean absolute
+ *    value of the whole latent weight matrix; every weight is divided by
+ *    (gamma + 1e-5), rounded to the nearest integer and clamped to [-1, 1];
+ *    gamma is kept beside the ternary matrix.
+ *  - "BitNet's Real Bet: Designing the Whole Inference Stack", section "A
+ *    low-bit model is a whole-stack design": weights in {-1, 0, +1},
+ *    activations on a separate per-token 8-bit path (W1.58A8); the GPU path
+ *    stores four ternary values in one int8, moves packed weights from HBM to
+ *    on-chip memory, unpacks them and computes with the 8-bit activations.
+ *  - same blog, section "The Energy Revolution": the product is integer
+ *    additions of 8-bit activations (int32 accumulation here).
+ *  - "A Two-Billion Ternary Bet": activations are quantised dynamically.
+ *
+ * Definitions this library implements (readings where the pages are silent):
+ *  gamma   = fp32( (sum_n sum_k |W[n][k]|) / (N*K) ), sums in double, k
+ *            ascending within a row, then rows ascending.
+ *  t[n][k] = clamp(rint(W[n][k] / (gamma + 1e-5f)), -1, 1), fp32 ops, ties to even.
+ *  s[m]    = 127 / max(max_k |x[m][k]|, 1e-5), fp32.
+ *  q[m][k] = clamp(rint(x[m][k] * s[m]), -128, 127), fp32 ops, ties to even.
+ *  acc     = sum_k q[m][k] * t[n][k]   (int32, exact)
+ *  y[m][n] = acc * gamma / s[m]          (fp32 arithmetic, then the output type)
+ *
+ * Packed weight layout ("four ternary values in one int8"): uint8 [N][K/4],
+ * row-major.  Code c = t + 1 in {0, 1, 2}.  The 32-bit little-endian word g of
+ * a row holds elements 16g .. 16g+15; element 16g + 4j + b sits in byte b at
+ * bits [2j, 2j+1].  So (word >> 2j) & 0x03030303 holds the four consecutive
+ * codes 16g+4j .. 16g+4j+3, one per byte.
+ *
+ * Conventions for every call:
+ *  - Pointers named "device" must be CUDA device (or managed, or mapped
+ *    pinned host) memory, 16-byte aligned; the workspace must be 256-byte
+ *    aligned.  Host-only pointers are rejected with BL_ERR_INVALID_ARG.
+ *  - The caller owns and allocates every buffer.  The library allocates no
+ *    device memory.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *    only enqueue work; they do not synchronise, except
+ *    bitlinear_device_status.
+ *  - Shapes: 1 <= N, 64 <= K, K % 64 == 0, 0 <= M.  M == 0 is a no-op.
+ *  - Return value: BL_OK or a negative BL_ERR_* code; the message of the most
+ *    recent failure on the calling thread is bitlinear_last_error().
+ *  - Device-side failures (a bounded wait that ran out) set a bit in the
+ *    workspace's status word; bitlinear_device_status reads and clears it.
+ *    The first 256 bytes of every workspace hold that status word and must
+ *    be zero before first use (zero the workspace once after allocating it).
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element types of activations and outputs. */
+typedef enum { BL_F32 = 0, BL_BF16 = 1 } bl_dtype;
+
+/* Status codes. */
+enum {
+  BL_OK = 0,
+  BL_ERR_INVALID_ARG = -1,         /* null / host-only pointer, bad dtype, negative size */
+  BL_ERR_UNSUPPORTED_SHAPE = -2,   /* K % 64 != 0, K < 64, N < 1, sizes past int32 indexing */
+  BL_ERR_MISALIGNED = -3,          /* device pointer not 16-byte (workspace: 256-byte) aligned */
+  BL_ERR_WORKSPACE_TOO_SMALL = -4, /* workspace_bytes below the *_workspace_bytes() figure */
+  BL_ERR_CUDA = -5,                /* a CUDA runtime call or kernel launch failed */
+  BL_ERR_DEVICE_TIMEOUT = -6       /* a device-side bounded wait ran out (device_status only) */
+};
+
+/*
+ * Workspace bytes bitlinear_pack_weights needs for an N x K matrix
+ * (status word + N per-row double sums).
+ */
+size_t bitlinear_pack_workspace_bytes(int N, int K);
+
+/*
+ * Offline weight path: absmean gamma, ternarisation and 2-bit packing
+ * ("The BitLinear Layer and AbsMean Quantization"; "A low-bit model is a
+ * whole-stack design").
+ *   W       device fp32 [N][K], row-major (nn.Linear: out x in) latent weights; read only.
+ *   packed  device uint8 [N][K/4] out, layout above.
+ *   gamma   device fp32 [1] out.
+ *   workspace / workspace_bytes: >= bitlinear_pack_workspace_bytes(N, K).
+ * The gamma sum order is fixed (see above), so results are bit-reproducible.
+ */
+int bitlinear_pack_weights(const float* W, int N, int K, uint8_t* packed, float* gamma,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Per-token 8-bit activation quantisation ("A low-bit model is a whole-stack
+ * design"; "A Two-Billion Ternary Bet"), one pass per token.
+ *   x       device [M][K] of x_dtype (BL_F32 or BL_BF16); read only.
+ *   xq      device int8 [M][K] out: q.
+ *   scale   device fp32 [M] out: s.
+ *   rowsum  device int32 [M] out, or NULL: sum_k q[m][k].
+ */
+int bitlinear_quant_act(const void* x, int x_dtype, int M, int K, int8_t* xq, float* scale,
+                        int32_t* rowsum, void* stream);
+
+/* Workspace bytes bitlinear_forward needs (status word + q, s, rowsum). */
+size_t bitlinear_workspace_bytes(int M, int N, int K);
+
+/*
+ * The BitLinear W1.58A8 forward: quantise x per token, ternary x int8
+ * product with int32 accumulation, fused dequantisation by gamma and s.
+ *   packed  device uint8 [N][K/4] (from bitlinear_pack_weights); gamma device fp32 [1].
+ *   x       device [M][K] of x_dtype.
+ *   y       device [M][N] of y_dtype out.
+ *   acc_out device int32 [M][N] out, or NULL: the exact accumulators
+ *           sum_k q*t (for parity checks).
+ * M <= 16 runs the decode GEMV kernel; larger M the tcgen05 tensor-core GEMM.
+ */
+int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, const void* x,
+                      int x_dtype, int M, void* y, int y_dtype, int32_t* acc_out, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/*
+ * The product and dequantisation on activations already quantised by
+ * bitlinear_quant_act (xq, scale, rowsum as it wrote them; rowsum required).
+ * workspace >= bitlinear_workspace_bytes(M, N, K) (only its status word is used).
+ */
+int bitlinear_forward_quantized(const uint8_t* packed, const float* gamma, int N, int K,
+                                const int8_t* xq, const float* scale, const int32_t* rowsum,
+                                int M, void* y, int y_dtype, int32_t* acc_out, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/* One BitLinear of a chain: weights, gamma, shape, input [M][K], output [M][N]. */
+typedef struct {
+  const uint8_t* packed;
+  const float* gamma;
+  int N;
+  int K;
+  const void* x;
+  void* y;
+} bl_layer;
+
+/* Workspace bytes bitlinear_layer_chain needs for these layers at M tokens. */
+size_t bitlinear_chain_workspace_bytes(const bl_layer* layers, int n_layers, int M);
+
+/*
+ * Runs n_layers BitLinear forwards back to back on one stream.  Consecutive
+ * layers that read the same x pointer with the same K (e.g. FFN gate and up)
+ * share one activation quantisation; each keeps its own gamma.  `layers` is a
+ * host array, read during the call only.
+ */
+int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dtype, int y_dtype,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, returns BL_OK or BL_ERR_DEVICE_TIMEOUT from the
+ * workspace's status word, and clears the word.
+ */
+int bitlinear_device_status(void* workspace, void* stream);
+
+/*
+ * Exercises the device-side bounded wait: launches one block that waits on a
+ * barrier nothing completes, with a limit of `limit_us` microseconds
+ * (1 .. 1000000); the wait gives up, sets the status word and returns.  A
+ * following bitlinear_device_status reports BL_ERR_DEVICE_TIMEOUT.
+ */
+int bitlinear_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int limit_us,
+                                    void* stream);
+
+/* Forces the product kernel: 0 = by M (default), 1 = GEMV (M <= 16 only), 2 = GEMM.  Per thread. */
+int bitlinear_set_path(int path);
+
+/* Message of the most recent failure on the calling thread ("" if none). */
+const char* bitlinear_last_error(void);
+
+/* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
+int bitlinear_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H */

@@ -1,0 +1,261 @@
+"""B200-native BitLinear W1.58A8 forward (BitNet b1.58), Python binding.
+
+A thin ctypes binding of ``libbitlinear.so``, whose C ABI is declared in
+``include/bitlinear.h``.  This module only marshals arguments: PyTorch
+provides device memory and the current stream; every step of the forward
+runs in the library's CUDA kernels.  There is no CPU fallback: if the
+library is missing or no GPU is present, the calls raise.
+
+Calls (same names as the C ABI, without the ``bitlinear_`` prefix):
+``pack_weights``, ``quant_act``, ``forward``, ``forward_quantized``,
+``layer_chain``, ``device_status``, plus workspace helpers.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbitlinear.so")
+
+BL_F32, BL_BF16 = 0, 1
+BL_OK = 0
+BL_ERR_INVALID_ARG = -1
+BL_ERR_UNSUPPORTED_SHAPE = -2
+BL_ERR_MISALIGNED = -3
+BL_ERR_WORKSPACE_TOO_SMALL = -4
+BL_ERR_CUDA = -5
+BL_ERR_DEVICE_TIMEOUT = -6
+
+PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__("bitlinear error %d: %s" % (code, message))
+        self.code = code
+
+
+class bl_layer(ctypes.Structure):
+    _fields_ = [
+        ("packed", ctypes.c_void_p),
+        ("gamma", ctypes.c_void_p),
+        ("N", ctypes.c_int),
+        ("K", ctypes.c_int),
+        ("x", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                "libbitlinear.so is not built; run `python -m ternary_weight_a8_b200._build` "
+                "(or __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        sigs = {
+            "bitlinear_pack_workspace_bytes": (sz, [i32, i32]),
+            "bitlinear_pack_weights": (i32, [vp, i32, i32, vp, vp, vp, sz, vp]),
+            "bitlinear_quant_act": (i32, [vp, i32, i32, i32, vp, vp, vp, vp]),
+            "bitlinear_workspace_bytes": (sz, [i32, i32, i32]),
+            "bitlinear_forward": (i32, [vp, vp, i32, i32, vp, i32, i32, vp, i32, vp, vp, sz, vp]),
+            "bitlinear_forward_quantized": (i32, [vp, vp, i32, i32, vp, vp, vp, i32, vp, i32, vp, vp, sz, vp]),
+            "bitlinear_chain_workspace_bytes": (sz, [ctypes.POINTER(bl_layer), i32, i32]),
+            "bitlinear_layer_chain": (i32, [ctypes.POINTER(bl_layer), i32, i32, i32, i32, vp, sz, vp]),
+            "bitlinear_device_status": (i32, [vp, vp]),
+            "bitlinear_selftest_wait_timeout": (i32, [vp, sz, i32, vp]),
+            "bitlinear_set_path": (i32, [i32]),
+            "bitlinear_last_error": (ctypes.c_char_p, []),
+            "bitlinear_version": (i32, []),
+        }
+        for name, (res, args) in sigs.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def last_error() -> str:
+    return lib().bitlinear_last_error().decode()
+
+
+def _check(rc: int) -> None:
+    if rc != BL_OK:
+        raise BitLinearError(rc, last_error())
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return BL_F32
+    if dt == torch.bfloat16:
+        return BL_BF16
+    raise ValueError("unsupported dtype %s (float32 or bfloat16)" % dt)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: torch.cuda.Stream | None = None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def set_path(path: int) -> None:
+    """Force the product kernel on this thread: PATH_AUTO, PATH_GEMV or PATH_GEMM."""
+    _check(lib().bitlinear_set_path(path))
+
+
+def version() -> int:
+    return lib().bitlinear_version()
+
+
+# ----------------------------------------------------------------------------
+# Workspaces
+# ----------------------------------------------------------------------------
+
+def pack_workspace_bytes(N: int, K: int) -> int:
+    return lib().bitlinear_pack_workspace_bytes(N, K)
+
+
+def workspace_bytes(M: int, N: int, K: int) -> int:
+    return lib().bitlinear_workspace_bytes(M, N, K)
+
+
+def new_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zeroed uint8 device buffer of at least ``nbytes`` (the status word starts at zero)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+# ----------------------------------------------------------------------------
+# Calls
+# ----------------------------------------------------------------------------
+
+def pack_weights(W: torch.Tensor, packed: torch.Tensor | None = None, gamma: torch.Tensor | None = None,
+                 workspace: torch.Tensor | None = None, stream=None):
+    """Latent fp32 weights ``[N][K]`` -> (packed uint8 ``[N][K/4]``, gamma fp32 ``[1]``)."""
+    N, K = W.shape
+    if packed is None:
+        packed = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    if workspace is None:
+        workspace = new_workspace(pack_workspace_bytes(N, K), W.device)
+    _check(lib().bitlinear_pack_weights(_ptr(W), N, K, _ptr(packed), _ptr(gamma), _ptr(workspace),
+                                        workspace.numel(), _stream(stream)))
+    return packed, gamma
+
+
+def quant_act(x: torch.Tensor, xq=None, scale=None, rowsum=None, stream=None):
+    """Activations ``[M][K]`` (fp32/bf16) -> (int8 q ``[M][K]``, fp32 s ``[M]``, int32 rowsum ``[M]``)."""
+    M, K = x.shape
+    dev = x.device
+    xq = torch.empty((M, K), dtype=torch.int8, device=dev) if xq is None else xq
+    scale = torch.empty(M, dtype=torch.float32, device=dev) if scale is None else scale
+    rowsum = torch.empty(M, dtype=torch.int32, device=dev) if rowsum is None else rowsum
+    _check(lib().bitlinear_quant_act(_ptr(x), _dtype_code(x.dtype), M, K, _ptr(xq), _ptr(scale),
+                                     _ptr(rowsum), _stream(stream)))
+    return xq, scale, rowsum
+
+
+def forward(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, out_dtype=torch.bfloat16,
+            y: torch.Tensor | None = None, acc_out: torch.Tensor | bool | None = None,
+            workspace: torch.Tensor | None = None, stream=None):
+    """y = BitLinear(x): returns y, or (y, acc) when ``acc_out`` is True or a tensor."""
+    N = packed.shape[0]
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    acc = None
+    if acc_out is True:
+        acc = torch.empty((M, N), dtype=torch.int32, device=x.device)
+    elif isinstance(acc_out, torch.Tensor):
+        acc = acc_out
+    if workspace is None:
+        workspace = new_workspace(workspace_bytes(M, N, K), x.device)
+    _check(lib().bitlinear_forward(_ptr(packed), _ptr(gamma), N, K, _ptr(x), _dtype_code(x.dtype), M,
+                                   _ptr(y), _dtype_code(y.dtype), _ptr(acc), _ptr(workspace),
+                                   workspace.numel(), _stream(stream)))
+    return (y, acc) if acc is not None else y
+
+
+def forward_quantized(packed: torch.Tensor, gamma: torch.Tensor, xq: torch.Tensor, scale: torch.Tensor,
+                      rowsum: torch.Tensor, out_dtype=torch.bfloat16, y: torch.Tensor | None = None,
+                      acc_out: torch.Tensor | bool | None = None, workspace: torch.Tensor | None = None,
+                      stream=None):
+    """The product + dequantisation on activations from ``quant_act``."""
+    N = packed.shape[0]
+    M, K = xq.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    acc = None
+    if acc_out is True:
+        acc = torch.empty((M, N), dtype=torch.int32, device=xq.device)
+    elif isinstance(acc_out, torch.Tensor):
+        acc = acc_out
+    if workspace is None:
+        workspace = new_workspace(256, xq.device)
+    _check(lib().bitlinear_forward_quantized(_ptr(packed), _ptr(gamma), N, K, _ptr(xq), _ptr(scale),
+                                             _ptr(rowsum), M, _ptr(y), _dtype_code(y.dtype), _ptr(acc),
+                                             _ptr(workspace), workspace.numel(), _stream(stream)))
+    return (y, acc) if acc is not None else y
+
+
+@dataclass
+class Layer:
+    packed: torch.Tensor
+    gamma: torch.Tensor
+    x: torch.Tensor
+    y: torch.Tensor
+
+
+def _layer_array(layers: Sequence[Layer]):
+    arr = (bl_layer * len(layers))()
+    for i, L in enumerate(layers):
+        arr[i] = bl_layer(_ptr(L.packed), _ptr(L.gamma), L.packed.shape[0], L.x.shape[1], _ptr(L.x), _ptr(L.y))
+    return arr
+
+
+def chain_workspace_bytes(layers: Sequence[Layer], M: int) -> int:
+    arr = _layer_array(layers)
+    return lib().bitlinear_chain_workspace_bytes(arr, len(layers), M)
+
+
+def layer_chain(layers: Sequence[Layer], workspace: torch.Tensor | None = None, stream=None) -> None:
+    """Runs the layers back to back; each writes its ``y``.  Same-x neighbours share one quantisation."""
+    if not layers:
+        return
+    M = layers[0].x.shape[0]
+    arr = _layer_array(layers)
+    if workspace is None:
+        workspace = new_workspace(lib().bitlinear_chain_workspace_bytes(arr, len(layers), M), layers[0].x.device)
+    _check(lib().bitlinear_layer_chain(arr, len(layers), M, _dtype_code(layers[0].x.dtype),
+                                       _dtype_code(layers[0].y.dtype), _ptr(workspace), workspace.numel(),
+                                       _stream(stream)))
+
+
+def device_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronises and returns BL_OK or BL_ERR_DEVICE_TIMEOUT (clearing the status word)."""
+    return lib().bitlinear_device_status(_ptr(workspace), _stream(stream))
+
+
+def selftest_wait_timeout(workspace: torch.Tensor, limit_us: int, stream=None) -> None:
+    _check(lib().bitlinear_selftest_wait_timeout(_ptr(workspace), workspace.numel(), limit_us, _stream(stream)))

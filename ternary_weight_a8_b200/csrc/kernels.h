@@ -1,0 +1,61 @@
+// Internal launchers of the BitLinear kernels (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace bl {
+
+enum OutType { kOutF32 = 0, kOutBF16 = 1 };
+
+// Launch helper: cudaLaunchKernelEx, optionally as a programmatic dependent
+// of the preceding kernel on the stream.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                   bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+int num_sms();
+
+// Offline weight path.
+cudaError_t launch_gamma(const float* W, int N, int K, double* row_sums, float* gamma,
+                         cudaStream_t stream);
+cudaError_t launch_ternary_pack(const float* W, int N, int K, const float* gamma, uint8_t* packed,
+                                cudaStream_t stream);
+
+// Per-token activation quantisation.
+cudaError_t launch_act_quant(const void* x, int x_bf16, int M, int K, int8_t* xq, float* scale,
+                             int32_t* rowsum, cudaStream_t stream, bool pdl);
+
+// Product + dequantisation on quantised activations.
+struct ProductArgs {
+  const uint8_t* packed;
+  const float* gamma;
+  int N, K, M;
+  const int8_t* xq;
+  const float* scale;
+  const int32_t* rowsum;
+  void* y;
+  int y_type;  // OutType
+  int32_t* acc_out;
+  uint32_t* status;
+};
+cudaError_t launch_gemv(const ProductArgs& a, cudaStream_t stream, bool pdl);
+cudaError_t launch_gemm(const ProductArgs& a, cudaStream_t stream, bool pdl);
+
+// Self-test of the bounded device wait.
+cudaError_t launch_wait_timeout_selftest(uint32_t* status, int limit_us, cudaStream_t stream);
+
+}  // namespace bl

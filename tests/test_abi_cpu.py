@@ -1,0 +1,99 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The library builds for sm_100a, loads, and exports every function that
+``include/bitlinear.h`` declares; argument checks that run before any CUDA
+call return the documented status codes; the workspace arithmetic matches
+the documented layout.  No call here launches work.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import ternary_weight_a8_b200 as tb
+from ternary_weight_a8_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return tb.lib()
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(bitlinear_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for required in ("bitlinear_pack_weights", "bitlinear_quant_act", "bitlinear_forward",
+                     "bitlinear_layer_chain"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    missing = [n for n in declared_functions() if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_host_side_validation(L):
+    vp = ctypes.c_void_p
+    assert L.bitlinear_set_path(5) == tb.BL_ERR_INVALID_ARG
+    assert "path" in tb.last_error()
+    assert L.bitlinear_set_path(0) == tb.BL_OK
+    # bad shapes are refused before any pointer is looked at
+    assert L.bitlinear_forward(None, None, 0, 256, None, 0, 1, None, 0, None, None, 0, None) == tb.BL_ERR_UNSUPPORTED_SHAPE
+    assert L.bitlinear_forward(None, None, 8, 100, None, 0, 1, None, 0, None, None, 0, None) == tb.BL_ERR_UNSUPPORTED_SHAPE
+    assert "K = 100" in tb.last_error()
+    assert L.bitlinear_forward(None, None, 8, 32, None, 0, 1, None, 0, None, None, 0, None) == tb.BL_ERR_UNSUPPORTED_SHAPE
+    assert L.bitlinear_forward(None, None, 8, 256, None, 7, 1, None, 0, None, None, 0, None) == tb.BL_ERR_INVALID_ARG
+    assert L.bitlinear_forward(None, None, 8, 256, None, 0, -1, None, 0, None, None, 0, None) == tb.BL_ERR_INVALID_ARG
+    assert L.bitlinear_quant_act(None, 3, 1, 256, None, None, None, None) == tb.BL_ERR_INVALID_ARG
+    assert L.bitlinear_pack_weights(None, 8, 48, None, None, None, 0, None) == tb.BL_ERR_UNSUPPORTED_SHAPE
+    assert L.bitlinear_layer_chain(None, 1, 1, 0, 0, None, 0, None) == tb.BL_ERR_INVALID_ARG
+    # empty inputs are a no-op that succeeds without touching memory
+    assert L.bitlinear_forward(vp(16), vp(16), 8, 256, vp(16), 0, 0, vp(16), 0, None, vp(256), 0, None) == tb.BL_OK
+    assert L.bitlinear_quant_act(vp(16), 0, 0, 256, vp(16), vp(16), None, None) == tb.BL_OK
+
+
+def test_workspace_layout(L):
+    # status word (256) + q (M*K, 256-rounded) + scale and rowsum (4*M each, 256-rounded)
+    assert tb.workspace_bytes(1, 6912, 2560) == 256 + 2560 + 256 + 256
+    assert tb.workspace_bytes(2048, 6912, 2560) == 256 + 2048 * 2560 + 8192 + 8192
+    assert tb.workspace_bytes(3, 10, 64) == 256 + 256 + 256 + 256
+    assert tb.pack_workspace_bytes(6912, 2560) == 256 + 6912 * 8
+    layers = (tb.bl_layer * 2)()
+    layers[0].N, layers[0].K = 10240, 8192
+    layers[1].N, layers[1].K = 8192, 28672
+    assert L.bitlinear_chain_workspace_bytes(layers, 2, 8) == tb.workspace_bytes(8, 8192, 28672)
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(tb, "_lib", None)
+    monkeypatch.setattr(tb, "LIB_PATH", "/nonexistent/libbitlinear.so")
+    with pytest.raises(RuntimeError, match="not built"):
+        tb.lib()
+
+
+def test_package_does_not_import_oracle():
+    import subprocess
+    import sys
+    code = "import sys, ternary_weight_a8_b200 as t; t.lib(); print('oracle' in sys.modules)"
+    out = subprocess.check_output([sys.executable, "-c", code], cwd=ROOT, text=True).strip()
+    assert out == "False"
+    src_dir = os.path.join(ROOT, "ternary_weight_a8_b200")
+    for dirpath, _, files in os.walk(src_dir):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert "import oracle" not in text and "from oracle" not in text, fn
+                assert "bitlinear_oracle" not in text, fn

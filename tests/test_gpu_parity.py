@@ -1,0 +1,310 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Every case draws seeded synthetic inputs once, hands the same arrays to both
+sides, and compares at the bars stated in ``parity.py``: packed weights,
+gamma, int8 activations, scales, row sums and int32 accumulators bit for bit;
+outputs within 1e-6 relative (fp32) or 1 ulp (bf16).  Sizes span several
+tiles with ragged tails; the full-size workloads of the pages (2B/3B decode,
+2B prefill, 70B layer chain) are checked on sampled output rows, which the
+oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import ternary_weight_a8_b200 as tb
+from conftest import read_golden
+from parity import activations, assert_y_matches, bf16_dev, dev, f32_bits, weights
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _auto_path():
+    tb.set_path(tb.PATH_AUTO)
+    yield
+    tb.set_path(tb.PATH_AUTO)
+
+
+# ----------------------------------------------------------------------------
+# offline weight path: gamma + ternarise + pack
+# ----------------------------------------------------------------------------
+
+PACK_SHAPES = [(1, 64), (17, 192), (33, 640), (256, 256), (6912, 2560), (2560, 2560), (8640, 3200),
+               (3200, 8640), (10240, 8192), (28672, 8192), (8192, 28672)]
+
+
+@pytest.mark.parametrize("N,K", PACK_SHAPES)
+def test_pack_parity(N, K):
+    W = weights(N, K, seed=N + K)
+    packed_ref, gamma_ref, _ = oracle.pack_weights(W)
+    packed, gamma = tb.pack_weights(dev(W))
+    assert f32_bits(gamma.cpu().numpy())[0] == f32_bits([gamma_ref])[0]
+    got = packed.cpu().numpy()
+    if not np.array_equal(got, packed_ref):
+        bad = np.argwhere(got != packed_ref)
+        raise AssertionError("%d packed bytes differ, first at %s" % (len(bad), bad[:5].tolist()))
+
+
+def _tie_matrix():
+    """W whose mean magnitude makes some weights exactly (gamma + 1e-5) / 2 (and 3/2 of it)."""
+    rng = np.random.default_rng(0)
+    N, K = 64, 64
+    signs = rng.choice([-1.0, 1.0], size=(N, K)).astype(np.float32)
+    kind = rng.integers(0, 4, size=(N, K))  # 0: tie h, 1: c, 2: 3h, 3: c/3
+    h = np.float32(0.2)
+    for _ in range(60):
+        mags = np.where(kind == 0, h, np.where(kind == 1, np.float32(0.5),
+                        np.where(kind == 2, np.float32(3) * h, np.float32(0.5) / np.float32(3))))
+        W = (signs * mags).astype(np.float32)
+        g, _ = oracle.absmean_gamma(W)
+        d = np.float32(g + np.float32(1e-5))
+        h_new = np.float32(d * np.float32(0.5))
+        if h_new == h:
+            break
+        h = h_new
+    return W, h, d
+
+
+def test_pack_exact_ties():
+    W, h, d = _tie_matrix()
+    assert float(h) * 2 == float(d)  # exact ties w / d = 0.5 by construction
+    packed_ref, gamma_ref, T_ref = oracle.pack_weights(W)
+    tie = np.abs(W) == h
+    assert tie.sum() > 500 and (T_ref[tie] == 0).all()  # half rounds to the even neighbour 0
+    packed, gamma = tb.pack_weights(dev(W))
+    assert f32_bits(gamma.cpu().numpy())[0] == f32_bits([gamma_ref])[0]
+    assert np.array_equal(packed.cpu().numpy(), packed_ref)
+
+
+def test_pack_special_matrices():
+    Z = np.zeros((8, 128), np.float32)
+    packed, gamma = tb.pack_weights(dev(Z))
+    assert gamma.item() == 0.0 and (packed.cpu().numpy() == 0x55).all()
+    C = np.full((8, 128), -0.03, np.float32)
+    packed, gamma = tb.pack_weights(dev(C))
+    assert (packed.cpu().numpy() == 0x00).all()
+    assert np.array_equal(packed.cpu().numpy(), oracle.pack_weights(C)[0])
+
+
+# ----------------------------------------------------------------------------
+# per-token activation quantisation
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,K,dtype", [(4, 256, "f32"), (3, 64, "f32"), (1, 2560, "bf16"), (16, 3200, "bf16"),
+                                       (2048, 2560, "bf16"), (8, 28672, "bf16"), (5, 8640, "f32")])
+def test_quant_parity(M, K, dtype):
+    x, xf = activations(M, K, seed=M * 7 + K, dtype=dtype)
+    q_ref, s_ref, r_ref = oracle.quant_act(xf)
+    q, s, r = tb.quant_act(x)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(f32_bits(s.cpu().numpy()), f32_bits(s_ref))
+    assert np.array_equal(r.cpu().numpy(), r_ref)
+
+
+def test_quant_golden_ties_and_degenerate_tokens():
+    rows = read_golden("act_quant.txt")
+    toks = [[float(v) for v in rows[i][1]] for i in range(0, len(rows), 4)]
+    K = 64
+    x = np.zeros((len(toks) + 2, K), np.float32)
+    for i, t in enumerate(toks):
+        x[i, :len(t)] = t
+    x[-1, 5] = 3e-6  # below the 1e-5 floor
+    q, s, r = tb.quant_act(dev(x))
+    q_ref, s_ref, r_ref = oracle.quant_act(x)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(f32_bits(s.cpu().numpy()), f32_bits(s_ref))
+    assert np.array_equal(r.cpu().numpy(), r_ref)
+    for i in range(0, len(rows), 4):
+        want = [int(v) for v in rows[i + 1][1]]
+        assert q.cpu().numpy()[i // 4, :len(want)].tolist() == want
+
+
+# ----------------------------------------------------------------------------
+# the forward: acc bit-exact, y within the bar
+# ----------------------------------------------------------------------------
+
+def _full_case(M, N, K, xdtype, ydtype, path, seed=0):
+    W = weights(N, K, seed=seed + 1)
+    packed_ref, gamma_ref, T = oracle.pack_weights(W)
+    x, xf = activations(M, K, seed=seed + 2, dtype=xdtype)
+    acc_ref, y_ref, *_ = oracle.forward(T, gamma_ref, xf)
+    tb.set_path(path)
+    y, acc = tb.forward(dev(packed_ref), dev(np.array([gamma_ref], np.float32)), x,
+                        out_dtype=ydtype, acc_out=True)
+    got = acc.cpu().numpy()
+    assert np.array_equal(got, acc_ref), "acc differs at %s" % np.argwhere(got != acc_ref)[:5].tolist()
+    assert_y_matches(y, y_ref, acc_ref)
+
+
+SMALL = [(1, 16, 64), (4, 256, 256), (3, 100, 192), (8, 300, 640), (9, 17, 128), (16, 1000, 320),
+         (17, 300, 192), (100, 513, 384), (130, 260, 256), (256, 512, 1024)]
+
+
+@pytest.mark.parametrize("M,N,K", [s for s in SMALL if s[0] <= 16])
+@pytest.mark.parametrize("ydtype", [torch.float32, torch.bfloat16])
+def test_forward_small_gemv(M, N, K, ydtype):
+    _full_case(M, N, K, "bf16", ydtype, tb.PATH_GEMV, seed=M * N + K)
+
+
+@pytest.mark.parametrize("M,N,K", SMALL)
+@pytest.mark.parametrize("ydtype", [torch.float32, torch.bfloat16])
+def test_forward_small_gemm(M, N, K, ydtype):
+    _full_case(M, N, K, "f32", ydtype, tb.PATH_GEMM, seed=M + N + K)
+
+
+def test_forward_single_256_both_paths():
+    """K = N = 256, 4 tokens, fp32 in and out (seed 0)."""
+    for path in (tb.PATH_GEMV, tb.PATH_GEMM, tb.PATH_AUTO):
+        _full_case(4, 256, 256, "f32", torch.float32, path, seed=0)
+
+
+@pytest.mark.parametrize("N", [6912, 2560])
+def test_forward_decode_2b(N):
+    _full_case(1, N, 2560, "bf16", torch.bfloat16, tb.PATH_AUTO, seed=N)
+
+
+@pytest.mark.parametrize("K,N", [(3200, 8640), (8640, 3200)])
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 16])
+def test_forward_decode_3b_sweep(K, N, M):
+    _full_case(M, N, K, "bf16", torch.bfloat16, tb.PATH_AUTO, seed=K + M)
+
+
+def _sampled_case(M, N, K, rows, seed, xdtype="bf16", ydtype=torch.bfloat16, path=tb.PATH_AUTO):
+    """Full-size run on the GPU; the oracle computes the sampled output rows only."""
+    W = weights(N, K, seed=seed)
+    gamma_ref, _ = oracle.absmean_gamma(W)
+    Wd = dev(W)
+    packed, gamma = tb.pack_weights(Wd)
+    del Wd
+    assert f32_bits(gamma.cpu().numpy())[0] == f32_bits([gamma_ref])[0]
+    x, xf = activations(M, K, seed=seed + 1, dtype=xdtype)
+    tb.set_path(path)
+    y, acc = tb.forward(packed, gamma, x, out_dtype=ydtype, acc_out=True)
+    T_rows = oracle.ternarize(W[rows], gamma_ref)
+    acc_ref, y_ref, *_ = oracle.forward(T_rows, gamma_ref, xf)
+    got = acc.cpu().numpy()[:, rows]
+    assert np.array_equal(got, acc_ref)
+    assert_y_matches(y[:, torch.as_tensor(rows, device=y.device)].contiguous(), y_ref, acc_ref)
+    # whole-output properties: finite, and zero exactly where acc is zero
+    yf = y.float()
+    assert torch.isfinite(yf).all()
+    assert ((acc == 0) == (yf == 0)).all()
+
+
+def test_forward_prefill_2b_sampled():
+    rng = np.random.default_rng(4)
+    rows = np.sort(np.concatenate([rng.choice(6912, 120, replace=False), [0, 255, 256, 6911]]))
+    _sampled_case(2048, 6912, 2560, np.unique(rows), seed=40)
+
+
+def test_forward_prefill_ragged_full():
+    """A prefill shape with ragged M, N and K tails, checked everywhere."""
+    _full_case(300, 1000, 576, "bf16", torch.bfloat16, tb.PATH_AUTO, seed=77)
+
+
+def test_forward_quantized_matches_forward():
+    W = weights(2560, 2560, seed=5)
+    packed, gamma = tb.pack_weights(dev(W))
+    for M in (1, 8, 16, 64):
+        x, _ = activations(M, 2560, seed=M, dtype="bf16")
+        y1, a1 = tb.forward(packed, gamma, x, acc_out=True)
+        xq, s, r = tb.quant_act(x)
+        y2, a2 = tb.forward_quantized(packed, gamma, xq, s, r, acc_out=True)
+        assert torch.equal(a1, a2) and torch.equal(y1, y2)
+
+
+def test_gemv_and_gemm_agree_on_decode_sizes():
+    W = weights(3200, 8640, seed=9)
+    packed, gamma = tb.pack_weights(dev(W))
+    for M in (1, 5, 16):
+        x, _ = activations(M, 8640, seed=M + 100, dtype="bf16")
+        tb.set_path(tb.PATH_GEMV)
+        y1, a1 = tb.forward(packed, gamma, x, acc_out=True, out_dtype=torch.float32)
+        tb.set_path(tb.PATH_GEMM)
+        y2, a2 = tb.forward(packed, gamma, x, acc_out=True, out_dtype=torch.float32)
+        assert torch.equal(a1, a2) and torch.equal(y1, y2)
+
+
+def test_forward_extreme_accumulators():
+    """|acc| = 127 * K at K = 28672 (all weights +1, every activation code 127) stays exact."""
+    K, N = 28672, 64
+    W = np.full((N, K), 0.02, np.float32)
+    W[1::2] *= -1
+    packed, gamma = tb.pack_weights(dev(W))
+    x = torch.full((3, K), 2.5, dtype=torch.bfloat16, device="cuda")
+    for path in (tb.PATH_GEMV, tb.PATH_GEMM):
+        tb.set_path(path)
+        y, acc = tb.forward(packed, gamma, x, acc_out=True, out_dtype=torch.float32)
+        a = acc.cpu().numpy()
+        assert (a[:, 0::2] == 127 * K).all() and (a[:, 1::2] == -127 * K).all()
+        want = 127 * K * float(np.float32(0.02)) / float(np.float32(127 / 2.5))
+        assert np.allclose(y.cpu().numpy()[:, 0], want, rtol=1e-6)
+
+
+def test_forward_zero_tokens_and_weights():
+    W = weights(300, 512, seed=3)
+    packed, gamma = tb.pack_weights(dev(W))
+    x = torch.zeros((20, 512), dtype=torch.bfloat16, device="cuda")
+    x[3, 7] = 1.0
+    for path in (tb.PATH_GEMM,):
+        tb.set_path(path)
+        y, acc = tb.forward(packed, gamma, x, acc_out=True)
+        assert (acc[torch.arange(20) != 3] == 0).all() and (y.float()[torch.arange(20) != 3] == 0).all()
+    packed0, gamma0 = tb.pack_weights(torch.zeros((300, 512), device="cuda"))
+    y, acc = tb.forward(packed0, gamma0, x[:4], acc_out=True)
+    assert (acc == 0).all() and (y.float() == 0).all()
+
+
+# ----------------------------------------------------------------------------
+# 70B-class layer chain at decode
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_layer_chain_70b_sampled(M):
+    layers_shape = synth.CHAIN_70B
+    shared = synth.CHAIN_70B_SHARED_INPUT
+    rng = np.random.default_rng(M)
+    layers, refs = [], []
+    x_prev = None
+    for li, (K, N) in enumerate(layers_shape):
+        W = weights(N, K, seed=1000 + li)  # re-randomised per layer from a seed
+        gamma_ref, _ = oracle.absmean_gamma(W)
+        Wd = dev(W)
+        packed, gamma = tb.pack_weights(Wd)
+        del Wd
+        assert f32_bits(gamma.cpu().numpy())[0] == f32_bits([gamma_ref])[0]
+        if shared[li]:
+            x, xf = x_prev
+        else:
+            x, xf = activations(M, K, seed=2000 + li, dtype="bf16")
+        x_prev = (x, xf)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        layers.append(tb.Layer(packed, gamma, x, y))
+        rows = np.unique(np.concatenate([rng.choice(N, 48, replace=False), [0, N - 1]]))
+        T_rows = oracle.ternarize(W[rows], gamma_ref)
+        acc_ref, y_ref, *_ = oracle.forward(T_rows, gamma_ref, xf)
+        refs.append((rows, acc_ref, y_ref))
+        del W
+    tb.layer_chain(layers)
+    torch.cuda.synchronize()
+    for L, (rows, acc_ref, y_ref) in zip(layers, refs):
+        assert_y_matches(L.y[:, torch.as_tensor(rows, device="cuda")].contiguous(), y_ref, acc_ref)
+        assert torch.isfinite(L.y.float()).all()
+
+
+def test_layer_chain_matches_separate_forwards():
+    K = 1024
+    x, _ = activations(4, K, seed=1, dtype="bf16")
+    specs = [(K, 700, x), (K, 900, x), (K, 300, None)]
+    layers, singles = [], []
+    for i, (k, n, xi) in enumerate(specs):
+        packed, gamma = tb.pack_weights(dev(weights(n, k, seed=50 + i)))
+        xi = xi if xi is not None else activations(4, k, seed=9, dtype="bf16")[0]
+        layers.append(tb.Layer(packed, gamma, xi, torch.empty((4, n), dtype=torch.bfloat16, device="cuda")))
+        singles.append(tb.forward(packed, gamma, xi))
+    tb.layer_chain(layers)
+    for L, y in zip(layers, singles):
+        assert torch.equal(L.y, y)
