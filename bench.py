@@ -254,17 +254,22 @@ def timed_graph_run(step_fn, steps, warmup, world, chunk=500, sampler=None):
     return max_over_ranks(secs, world), clocks
 
 
-def kernel_event_times(launch_pre, launch_kernel, steps):
-    """Average device duration of one kernel, timed with events on its launching stream."""
+def kernel_event_times(launch_pre, launch_kernel, steps, batch=100):
+    """Average device duration of one kernel, timed with events on its launching stream.
+
+    Each batch of launches is queued behind a spin of the stream, so the
+    events bracket the kernel's execution rather than the host's launch gaps."""
     import torch
 
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    for i in range(steps):
-        launch_pre(i)
-        evs[i][0].record()
-        launch_kernel(i)
-        evs[i][1].record()
-    torch.cuda.synchronize()
+    for b0 in range(0, steps, batch):
+        torch.cuda._sleep(int(20e6))  # ~10 ms: longer than enqueueing one batch
+        for i in range(b0, min(steps, b0 + batch)):
+            launch_pre(i)
+            evs[i][0].record()
+            launch_kernel(i)
+            evs[i][1].record()
+        torch.cuda.synchronize()
     t = [a.elapsed_time(b) / 1e3 for a, b in evs]
     return statistics.mean(t), statistics.median(t)
 

@@ -212,7 +212,7 @@ def forward_quantized(packed: torch.Tensor, gamma: torch.Tensor, xq: torch.Tenso
     elif isinstance(acc_out, torch.Tensor):
         acc = acc_out
     if workspace is None:
-        workspace = new_workspace(256, xq.device)
+        workspace = new_workspace(workspace_bytes(M, N, K), xq.device)
     _check(lib().bitlinear_forward_quantized(_ptr(packed), _ptr(gamma), N, K, _ptr(xq), _ptr(scale),
                                              _ptr(rowsum), M, _ptr(y), _dtype_code(y.dtype), _ptr(acc),
                                              _ptr(workspace), workspace.numel(), _stream(stream)))

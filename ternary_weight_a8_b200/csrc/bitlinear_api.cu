@@ -64,17 +64,32 @@ int check_dtype(int t, const char* name) {
 
 int check_nk(int N, int K) {
   if (N < 1) return fail(BL_ERR_UNSUPPORTED_SHAPE, "N = %d: need N >= 1", N);
+  if (N > bl::kGemvMaxCounters * bl::kGemvRowsPerBlock)
+    return fail(BL_ERR_UNSUPPORTED_SHAPE, "N = %d: need N <= %d", N, bl::kGemvMaxCounters * bl::kGemvRowsPerBlock);
   if (K < 64 || K % 64 != 0) return fail(BL_ERR_UNSUPPORTED_SHAPE, "K = %d: need K >= 64 and K %% 64 == 0", K);
   return BL_OK;
 }
 
+// Workspace layout (offsets from the 256-byte aligned base):
+//   [0, 256)            status word
+//   [256, 256 + 64 KB)  split-K counters, one per 128-row block (decode GEMV)
+//   partials            split-K partial-sum slots (decode GEMV, M <= 16)
+//   xq, scale, rowsum   the quantised activations of the call
+// The status word and the counters sit at fixed offsets whatever the shapes,
+// so a workspace shared by calls of different shapes stays consistent.
+constexpr size_t kCounterBytes = static_cast<size_t>(bl::kGemvMaxCounters) * 4;
+
 struct FwdLayout {
-  size_t xq, scale, rowsum, total;
+  size_t counters, partials, xq, scale, rowsum, total;
 };
 
-FwdLayout forward_layout(int M, int K) {
+FwdLayout forward_layout(int M, int N, int K) {
   FwdLayout l;
-  l.xq = kStatusBytes;
+  l.counters = kStatusBytes;
+  l.partials = kStatusBytes + kCounterBytes;
+  const size_t n_rb = (static_cast<size_t>(N) + bl::kGemvRowsPerBlock - 1) / bl::kGemvRowsPerBlock;
+  const size_t pbytes = (M <= 16) ? n_rb * bl::kGemvMaxSplits * static_cast<size_t>(M) * bl::kGemvRowsPerBlock * 4 : 0;
+  l.xq = l.partials + round_up(pbytes, 256);
   l.scale = l.xq + round_up(static_cast<size_t>(M) * K, 256);
   l.rowsum = l.scale + round_up(static_cast<size_t>(M) * 4, 256);
   l.total = l.rowsum + round_up(static_cast<size_t>(M) * 4, 256);
@@ -93,6 +108,12 @@ int run_product(const bl::ProductArgs& a, cudaStream_t stream) {
     if (a.M > 16) return fail(BL_ERR_UNSUPPORTED_SHAPE, "GEMV path forced with M = %d > 16", a.M);
     gemv = true;
   } else if (g_path == 2) {
+    gemv = false;
+  }
+  if (gemv && bl::plan_gemv(a.M, a.N, a.K).splits == 0) {
+    // The decode kernel stages the block's activations on chip; past that size use the GEMM.
+    if (g_path == 1) return fail(BL_ERR_UNSUPPORTED_SHAPE, "GEMV path forced but M*K = %lld is too large",
+                                 static_cast<long long>(a.M) * a.K);
     gemv = false;
   }
   cudaError_t e = gemv ? bl::launch_gemv(a, stream, true) : bl::launch_gemm(a, stream, true);
@@ -192,9 +213,8 @@ int bitlinear_quant_act(const void* x, int x_dtype, int M, int K, int8_t* xq, fl
 }
 
 size_t bitlinear_workspace_bytes(int M, int N, int K) {
-  (void)N;
-  if (M < 0 || K < 0) return 0;
-  return forward_layout(M, K).total;
+  if (M < 0 || N < 0 || K < 0) return 0;
+  return forward_layout(M, N, K).total;
 }
 
 int bitlinear_forward_quantized(const uint8_t* packed, const float* gamma, int N, int K,
@@ -213,10 +233,13 @@ int bitlinear_forward_quantized(const uint8_t* packed, const float* gamma, int N
   BL_TRY(check_ptr(y, "y", 16));
   BL_TRY(check_ptr(acc_out, "acc_out", 16, true));
   BL_TRY(check_ptr(workspace, "workspace", 256));
-  if (workspace_bytes < kStatusBytes)
-    return fail(BL_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, kStatusBytes);
+  const FwdLayout l = forward_layout(M, N, K);
+  if (workspace_bytes < l.total)
+    return fail(BL_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, l.total);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
   bl::ProductArgs a{packed, gamma, N, K, M, xq, scale, rowsum, y, y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32,
-                    acc_out, static_cast<uint32_t*>(workspace)};
+                    acc_out, reinterpret_cast<uint32_t*>(ws), reinterpret_cast<int32_t*>(ws + l.partials),
+                    reinterpret_cast<uint32_t*>(ws + l.counters)};
   return run_product(a, static_cast<cudaStream_t>(stream));
 }
 
@@ -234,7 +257,7 @@ int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, c
   BL_TRY(check_ptr(y, "y", 16));
   BL_TRY(check_ptr(acc_out, "acc_out", 16, true));
   BL_TRY(check_ptr(workspace, "workspace", 256));
-  const FwdLayout l = forward_layout(M, K);
+  const FwdLayout l = forward_layout(M, N, K);
   if (workspace_bytes < l.total)
     return fail(BL_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, l.total);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -245,18 +268,25 @@ int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, c
   cudaError_t e = bl::launch_act_quant(x, x_dtype == BL_BF16, M, K, xq, scale, rowsum, s, true);
   if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
   bl::ProductArgs a{packed, gamma, N, K, M, xq, scale, rowsum, y, y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32,
-                    acc_out, reinterpret_cast<uint32_t*>(ws)};
+                    acc_out, reinterpret_cast<uint32_t*>(ws), reinterpret_cast<int32_t*>(ws + l.partials),
+                    reinterpret_cast<uint32_t*>(ws + l.counters)};
   return run_product(a, s);
+}
+
+static void chain_extent(const bl_layer* layers, int n_layers, int* n_max, int* k_max) {
+  *n_max = 1;
+  *k_max = 64;
+  for (int i = 0; i < n_layers; ++i) {
+    if (layers[i].N > *n_max) *n_max = layers[i].N;
+    if (layers[i].K > *k_max) *k_max = layers[i].K;
+  }
 }
 
 size_t bitlinear_chain_workspace_bytes(const bl_layer* layers, int n_layers, int M) {
   if (!layers || n_layers <= 0 || M < 0) return 0;
-  size_t best = kStatusBytes;
-  for (int i = 0; i < n_layers; ++i) {
-    const size_t t = forward_layout(M, layers[i].K).total;
-    if (t > best) best = t;
-  }
-  return best;
+  int n_max, k_max;
+  chain_extent(layers, n_layers, &n_max, &k_max);
+  return forward_layout(M, n_max, k_max).total;
 }
 
 int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dtype, int y_dtype,
@@ -281,9 +311,11 @@ int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dty
     return fail(BL_ERR_WORKSPACE_TOO_SMALL, "chain workspace %zu < %zu bytes", workspace_bytes, need);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int n_max, k_max;
+  chain_extent(layers, n_layers, &n_max, &k_max);
+  const FwdLayout l = forward_layout(M, n_max, k_max);  // one layout for every layer
   for (int i = 0; i < n_layers; ++i) {
     const bl_layer& L = layers[i];
-    const FwdLayout l = forward_layout(M, L.K);
     int8_t* xq = reinterpret_cast<int8_t*>(ws + l.xq);
     float* scale = reinterpret_cast<float*>(ws + l.scale);
     int32_t* rowsum = reinterpret_cast<int32_t*>(ws + l.rowsum);
@@ -293,7 +325,8 @@ int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dty
       if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
     }
     bl::ProductArgs a{L.packed, L.gamma, L.N, L.K, M, xq, scale, rowsum, L.y,
-                      y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32, nullptr, reinterpret_cast<uint32_t*>(ws)};
+                      y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32, nullptr, reinterpret_cast<uint32_t*>(ws),
+                      reinterpret_cast<int32_t*>(ws + l.partials), reinterpret_cast<uint32_t*>(ws + l.counters)};
     BL_TRY(run_product(a, s));
   }
   return BL_OK;

@@ -51,7 +51,27 @@ struct ProductArgs {
   int y_type;  // OutType
   int32_t* acc_out;
   uint32_t* status;
+  int32_t* acc_ws;     // split-K partial-sum slots [row block][split][M][128] (GEMV only)
+  uint32_t* counters;  // one per 128-row block, zero between calls (GEMV only)
 };
+
+// Decode kernel launch plan: blocks of 128 rows, K split `splits` ways, one wave.
+struct GemvPlan {
+  int n_rb, n_st, splits, st_per_split, nring, x_pitch, smem;
+};
+GemvPlan plan_gemv(int M, int N, int K);
+constexpr int kGemvRowsPerBlock = 128;
+constexpr int kGemvMaxSplits = 8;
+constexpr int kGemvMaxCounters = 16384;  // row blocks: N <= 2^21
+
+// cuTensorMapEncodeTiled from the driver (no link-time dependency on libcuda).
+#ifdef CUDA_VERSION
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+#endif
+void* tensor_map_encoder();
 cudaError_t launch_gemv(const ProductArgs& a, cudaStream_t stream, bool pdl);
 cudaError_t launch_gemm(const ProductArgs& a, cudaStream_t stream, bool pdl);
 

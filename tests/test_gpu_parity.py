@@ -308,3 +308,17 @@ def test_layer_chain_matches_separate_forwards():
     tb.layer_chain(layers)
     for L, y in zip(layers, singles):
         assert torch.equal(L.y, y)
+
+
+def test_shared_workspace_across_shapes_stays_consistent():
+    """One workspace serves calls of different shapes in stream order (split counters reset)."""
+    shapes = [(1, 6912, 2560), (16, 300, 8640), (8, 3200, 8640), (3, 2560, 2560), (1, 6912, 2560)]
+    ws = tb.new_workspace(max(tb.workspace_bytes(M, N, K) for M, N, K in shapes))
+    for i, (M, N, K) in enumerate(shapes):
+        packed, gamma = tb.pack_weights(dev(weights(N, K, seed=70 + i)))
+        x, _ = activations(M, K, seed=80 + i, dtype="bf16")
+        y1, a1 = tb.forward(packed, gamma, x, acc_out=True, workspace=ws)
+        y2, a2 = tb.forward(packed, gamma, x, acc_out=True)  # fresh workspace
+        assert torch.equal(a1, a2) and torch.equal(y1, y2)
+    hdr = ws[:256 + 65536]
+    assert int(hdr.count_nonzero().item()) == 0

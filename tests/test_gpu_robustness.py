@@ -88,7 +88,7 @@ def test_no_writes_outside_outputs(M):
     acc = abuf[pad:pad + M * N * 4].view(torch.int32).view(M, N)
     ws_bytes = tb.workspace_bytes(M, N, K)
     wbuf = torch.full((ws_bytes + pad,), canary, dtype=torch.uint8, device="cuda")
-    wbuf[:256] = 0
+    wbuf[:256 + 65536] = 0  # status word and split counters start at zero
     ws = wbuf[:ws_bytes]
     tb.forward(packed, gamma, x, y=y, acc_out=acc, workspace=ws)
     torch.cuda.synchronize()
