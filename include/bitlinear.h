@@ -40,17 +40,14 @@
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
  *    only enqueue work; they do not synchronise, except
  *    bitlinear_device_status.
- *  - Shapes: 1 <= N <= 2^21, 64 <= K, K % 64 == 0, 0 <= M.  M == 0 is a no-op.
+ *  - Shapes: 1 <= N <= 2^24, 64 <= K, K % 64 == 0, 0 <= M.  M == 0 is a no-op.
  *  - Return value: BL_OK or a negative BL_ERR_* code; the message of the most
  *    recent failure on the calling thread is bitlinear_last_error().
  *  - Device-side failures (a bounded wait that ran out) set a bit in the
  *    workspace's status word; bitlinear_device_status reads and clears it.
- *  - A workspace starts with a status word (256 bytes) and the decode
- *    kernel's split counters (64 KB).  Zero the workspace once after
- *    allocating it; every call that completes leaves that header zero
- *    again, whatever the shapes, so one workspace can serve calls of
- *    different shapes in stream order.  After a device-side failure, zero it
- *    again.  Calls that overlap on the GPU must not share a workspace.
+ *  - A workspace starts with a 256-byte status word, which must be zero
+ *    before first use (zero the workspace once after allocating it).  Calls
+ *    that overlap on the GPU must not share a workspace.
  */
 #ifndef BITLINEAR_H
 #define BITLINEAR_H
@@ -106,8 +103,7 @@ int bitlinear_pack_weights(const float* W, int N, int K, uint8_t* packed, float*
 int bitlinear_quant_act(const void* x, int x_dtype, int M, int K, int8_t* xq, float* scale,
                         int32_t* rowsum, void* stream);
 
-/* Workspace bytes bitlinear_forward and bitlinear_forward_quantized need:
- * header, decode split-K slots (M <= 16), and q, s, rowsum. */
+/* Workspace bytes bitlinear_forward needs (status word + q, s, rowsum). */
 size_t bitlinear_workspace_bytes(int M, int N, int K);
 
 /*
@@ -118,7 +114,8 @@ size_t bitlinear_workspace_bytes(int M, int N, int K);
  *   y       device [M][N] of y_dtype out.
  *   acc_out device int32 [M][N] out, or NULL: the exact accumulators
  *           sum_k q*t (for parity checks).
- * M <= 16 runs the decode GEMV kernel; larger M the tcgen05 tensor-core GEMM.
+ * M <= 16 runs the decode GEMV kernel (which quantises small activations
+ * itself); larger M the quantisation kernel and the tcgen05 tensor-core GEMM.
  */
 int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, const void* x,
                       int x_dtype, int M, void* y, int y_dtype, int32_t* acc_out, void* workspace,
@@ -127,7 +124,7 @@ int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, c
 /*
  * The product and dequantisation on activations already quantised by
  * bitlinear_quant_act (xq, scale, rowsum as it wrote them; rowsum required).
- * workspace >= bitlinear_workspace_bytes(M, N, K).
+ * Only the workspace's status word is used (256 bytes suffice).
  */
 int bitlinear_forward_quantized(const uint8_t* packed, const float* gamma, int N, int K,
                                 const int8_t* xq, const float* scale, const int32_t* rowsum,

@@ -64,32 +64,20 @@ int check_dtype(int t, const char* name) {
 
 int check_nk(int N, int K) {
   if (N < 1) return fail(BL_ERR_UNSUPPORTED_SHAPE, "N = %d: need N >= 1", N);
-  if (N > bl::kGemvMaxCounters * bl::kGemvRowsPerBlock)
-    return fail(BL_ERR_UNSUPPORTED_SHAPE, "N = %d: need N <= %d", N, bl::kGemvMaxCounters * bl::kGemvRowsPerBlock);
+  if (N > (1 << 24)) return fail(BL_ERR_UNSUPPORTED_SHAPE, "N = %d: need N <= 2^24", N);
   if (K < 64 || K % 64 != 0) return fail(BL_ERR_UNSUPPORTED_SHAPE, "K = %d: need K >= 64 and K %% 64 == 0", K);
   return BL_OK;
 }
 
-// Workspace layout (offsets from the 256-byte aligned base):
-//   [0, 256)            status word
-//   [256, 256 + 64 KB)  split-K counters, one per 128-row block (decode GEMV)
-//   partials            split-K partial-sum slots (decode GEMV, M <= 16)
-//   xq, scale, rowsum   the quantised activations of the call
-// The status word and the counters sit at fixed offsets whatever the shapes,
-// so a workspace shared by calls of different shapes stays consistent.
-constexpr size_t kCounterBytes = static_cast<size_t>(bl::kGemvMaxCounters) * 4;
-
+// Workspace layout: [0, 256) status word, then the quantised activations of
+// the call (q [M][K], s [M], rowsum [M]), each region 256-byte aligned.
 struct FwdLayout {
-  size_t counters, partials, xq, scale, rowsum, total;
+  size_t xq, scale, rowsum, total;
 };
 
-FwdLayout forward_layout(int M, int N, int K) {
+FwdLayout forward_layout(int M, int K) {
   FwdLayout l;
-  l.counters = kStatusBytes;
-  l.partials = kStatusBytes + kCounterBytes;
-  const size_t n_rb = (static_cast<size_t>(N) + bl::kGemvRowsPerBlock - 1) / bl::kGemvRowsPerBlock;
-  const size_t pbytes = (M <= 16) ? n_rb * bl::kGemvMaxSplits * static_cast<size_t>(M) * bl::kGemvRowsPerBlock * 4 : 0;
-  l.xq = l.partials + round_up(pbytes, 256);
+  l.xq = kStatusBytes;
   l.scale = l.xq + round_up(static_cast<size_t>(M) * K, 256);
   l.rowsum = l.scale + round_up(static_cast<size_t>(M) * 4, 256);
   l.total = l.rowsum + round_up(static_cast<size_t>(M) * 4, 256);
@@ -102,23 +90,69 @@ FwdLayout forward_layout(int M, int N, int K) {
     if (_rc != BL_OK) return _rc; \
   } while (0)
 
-int run_product(const bl::ProductArgs& a, cudaStream_t stream) {
-  bool gemv = a.M <= 16;
+// The product kernel for this call: the decode GEMV for M <= 16 (unless its
+// activations do not fit on chip), else the tensor-core GEMM; bitlinear_set_path
+// overrides the choice on the calling thread.
+int choose_gemv(int M, int N, int K, bool* gemv) {
+  bool v = M <= 16;
   if (g_path == 1) {
-    if (a.M > 16) return fail(BL_ERR_UNSUPPORTED_SHAPE, "GEMV path forced with M = %d > 16", a.M);
-    gemv = true;
+    if (M > 16) return fail(BL_ERR_UNSUPPORTED_SHAPE, "GEMV path forced with M = %d > 16", M);
+    v = true;
   } else if (g_path == 2) {
-    gemv = false;
+    v = false;
   }
-  if (gemv && bl::plan_gemv(a.M, a.N, a.K).splits == 0) {
-    // The decode kernel stages the block's activations on chip; past that size use the GEMM.
-    if (g_path == 1) return fail(BL_ERR_UNSUPPORTED_SHAPE, "GEMV path forced but M*K = %lld is too large",
-                                 static_cast<long long>(a.M) * a.K);
-    gemv = false;
+  if (v && bl::plan_gemv(M, N, K).splits == 0) {
+    if (g_path == 1)
+      return fail(BL_ERR_UNSUPPORTED_SHAPE, "GEMV path forced but M*K = %lld does not fit on chip",
+                  static_cast<long long>(M) * K);
+    v = false;
   }
-  cudaError_t e = gemv ? bl::launch_gemv(a, stream, true) : bl::launch_gemm(a, stream, true);
+  *gemv = v;
+  return BL_OK;
+}
+
+int launch_product(bool gemv, const uint8_t* packed, const float* gamma, int N, int K, int M, const int8_t* xq,
+                   const float* scale, const int32_t* rowsum, void* y, int y_dtype, int32_t* acc_out,
+                   uint32_t* status, cudaStream_t s) {
+  const int yt = y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32;
+  cudaError_t e;
+  if (gemv) {
+    bl::GemvArgs a{packed, gamma, N, K, M, xq, bl::kInInt8, scale, y, yt, acc_out, status};
+    e = bl::launch_gemv(a, s, true);
+  } else {
+    bl::ProductArgs a{packed, gamma, N, K, M, xq, scale, rowsum, y, yt, acc_out, status};
+    e = bl::launch_gemm(a, s, true);
+  }
   if (e != cudaSuccess) return cuda_fail(e, gemv ? "GEMV launch" : "GEMM launch");
   return BL_OK;
+}
+
+// One forward on raw activations.  *xq_valid tells whether the workspace
+// already holds this x quantised (a chain's layers that share their input);
+// it is updated when this call quantises x into the workspace.
+int forward_one(const uint8_t* packed, const float* gamma, int N, int K, const void* x, int x_dtype, int M,
+                void* y, int y_dtype, int32_t* acc_out, uint8_t* ws, const FwdLayout& l, bool* xq_valid,
+                cudaStream_t s) {
+  bool gemv = false;
+  BL_TRY(choose_gemv(M, N, K, &gemv));
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  if (gemv && bl::gemv_fuses_quant(M, K)) {
+    // Small activations: the GEMV blocks quantise them on chip (one launch, no round trip).
+    bl::GemvArgs a{packed, gamma, N, K, M, x, x_dtype == BL_BF16 ? bl::kInBF16 : bl::kInF32, nullptr, y,
+                   y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32, acc_out, status};
+    cudaError_t e = bl::launch_gemv(a, s, true);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMV launch");
+    return BL_OK;
+  }
+  int8_t* xq = reinterpret_cast<int8_t*>(ws + l.xq);
+  float* scale = reinterpret_cast<float*>(ws + l.scale);
+  int32_t* rowsum = reinterpret_cast<int32_t*>(ws + l.rowsum);
+  if (!*xq_valid) {
+    cudaError_t e = bl::launch_act_quant(x, x_dtype == BL_BF16, M, K, xq, scale, rowsum, s, true);
+    if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+    *xq_valid = true;
+  }
+  return launch_product(gemv, packed, gamma, N, K, M, xq, scale, rowsum, y, y_dtype, acc_out, status, s);
 }
 
 }  // namespace
@@ -213,8 +247,9 @@ int bitlinear_quant_act(const void* x, int x_dtype, int M, int K, int8_t* xq, fl
 }
 
 size_t bitlinear_workspace_bytes(int M, int N, int K) {
-  if (M < 0 || N < 0 || K < 0) return 0;
-  return forward_layout(M, N, K).total;
+  (void)N;
+  if (M < 0 || K < 0) return 0;
+  return forward_layout(M, K).total;
 }
 
 int bitlinear_forward_quantized(const uint8_t* packed, const float* gamma, int N, int K,
@@ -233,14 +268,12 @@ int bitlinear_forward_quantized(const uint8_t* packed, const float* gamma, int N
   BL_TRY(check_ptr(y, "y", 16));
   BL_TRY(check_ptr(acc_out, "acc_out", 16, true));
   BL_TRY(check_ptr(workspace, "workspace", 256));
-  const FwdLayout l = forward_layout(M, N, K);
-  if (workspace_bytes < l.total)
-    return fail(BL_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, l.total);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  bl::ProductArgs a{packed, gamma, N, K, M, xq, scale, rowsum, y, y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32,
-                    acc_out, reinterpret_cast<uint32_t*>(ws), reinterpret_cast<int32_t*>(ws + l.partials),
-                    reinterpret_cast<uint32_t*>(ws + l.counters)};
-  return run_product(a, static_cast<cudaStream_t>(stream));
+  if (workspace_bytes < kStatusBytes)
+    return fail(BL_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, kStatusBytes);
+  bool gemv = false;
+  BL_TRY(choose_gemv(M, N, K, &gemv));
+  return launch_product(gemv, packed, gamma, N, K, M, xq, scale, rowsum, y, y_dtype, acc_out,
+                        static_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
 int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, const void* x,
@@ -257,36 +290,20 @@ int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, c
   BL_TRY(check_ptr(y, "y", 16));
   BL_TRY(check_ptr(acc_out, "acc_out", 16, true));
   BL_TRY(check_ptr(workspace, "workspace", 256));
-  const FwdLayout l = forward_layout(M, N, K);
+  const FwdLayout l = forward_layout(M, K);
   if (workspace_bytes < l.total)
     return fail(BL_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, l.total);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  int8_t* xq = reinterpret_cast<int8_t*>(ws + l.xq);
-  float* scale = reinterpret_cast<float*>(ws + l.scale);
-  int32_t* rowsum = reinterpret_cast<int32_t*>(ws + l.rowsum);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = bl::launch_act_quant(x, x_dtype == BL_BF16, M, K, xq, scale, rowsum, s, true);
-  if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
-  bl::ProductArgs a{packed, gamma, N, K, M, xq, scale, rowsum, y, y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32,
-                    acc_out, reinterpret_cast<uint32_t*>(ws), reinterpret_cast<int32_t*>(ws + l.partials),
-                    reinterpret_cast<uint32_t*>(ws + l.counters)};
-  return run_product(a, s);
-}
-
-static void chain_extent(const bl_layer* layers, int n_layers, int* n_max, int* k_max) {
-  *n_max = 1;
-  *k_max = 64;
-  for (int i = 0; i < n_layers; ++i) {
-    if (layers[i].N > *n_max) *n_max = layers[i].N;
-    if (layers[i].K > *k_max) *k_max = layers[i].K;
-  }
+  bool xq_valid = false;
+  return forward_one(packed, gamma, N, K, x, x_dtype, M, y, y_dtype, acc_out, static_cast<uint8_t*>(workspace),
+                     l, &xq_valid, static_cast<cudaStream_t>(stream));
 }
 
 size_t bitlinear_chain_workspace_bytes(const bl_layer* layers, int n_layers, int M) {
   if (!layers || n_layers <= 0 || M < 0) return 0;
-  int n_max, k_max;
-  chain_extent(layers, n_layers, &n_max, &k_max);
-  return forward_layout(M, n_max, k_max).total;
+  int k_max = 64;
+  for (int i = 0; i < n_layers; ++i)
+    if (layers[i].K > k_max) k_max = layers[i].K;
+  return forward_layout(M, k_max).total;
 }
 
 int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dtype, int y_dtype,
@@ -311,23 +328,13 @@ int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dty
     return fail(BL_ERR_WORKSPACE_TOO_SMALL, "chain workspace %zu < %zu bytes", workspace_bytes, need);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int n_max, k_max;
-  chain_extent(layers, n_layers, &n_max, &k_max);
-  const FwdLayout l = forward_layout(M, n_max, k_max);  // one layout for every layer
+  bool xq_valid = false;
   for (int i = 0; i < n_layers; ++i) {
     const bl_layer& L = layers[i];
-    int8_t* xq = reinterpret_cast<int8_t*>(ws + l.xq);
-    float* scale = reinterpret_cast<float*>(ws + l.scale);
-    int32_t* rowsum = reinterpret_cast<int32_t*>(ws + l.rowsum);
     const bool shared_input = i > 0 && layers[i - 1].x == L.x && layers[i - 1].K == L.K;
-    if (!shared_input) {
-      cudaError_t e = bl::launch_act_quant(L.x, x_dtype == BL_BF16, M, L.K, xq, scale, rowsum, s, true);
-      if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
-    }
-    bl::ProductArgs a{L.packed, L.gamma, L.N, L.K, M, xq, scale, rowsum, L.y,
-                      y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32, nullptr, reinterpret_cast<uint32_t*>(ws),
-                      reinterpret_cast<int32_t*>(ws + l.partials), reinterpret_cast<uint32_t*>(ws + l.counters)};
-    BL_TRY(run_product(a, s));
+    if (!shared_input) xq_valid = false;
+    BL_TRY(forward_one(L.packed, L.gamma, L.N, L.K, L.x, x_dtype, M, L.y, y_dtype, nullptr, ws,
+                       forward_layout(M, L.K), &xq_valid, s));
   }
   return BL_OK;
 }

@@ -3,37 +3,40 @@
 //
 // "BitNet's Real Bet: Designing the Whole Inference Stack", section "A
 // low-bit model is a whole-stack design": the GPU path moves packed weights
-// from HBM to shared memory, unpacks them and computes with the 8-bit
-// activations.  "BitNet b1.58 and the 1-Bit AI Architecture Revolution",
-// section "The Energy Revolution": the product is integer additions; here
-// they run on the tensor cores' int8 path (mma.sync m16n8k32, u8 x s8 -> s32).
+// from HBM to shared memory, unpacks them and computes with the per-token
+// 8-bit activations.  "BitNet b1.58 and the 1-Bit AI Architecture
+// Revolution", section "The Energy Revolution": the product is integer
+// additions; here they run on the tensor cores' int8 path (mma.sync
+// m16n8k32, u8 x s8 -> s32).
 //
 // Decode streams the weights once, so the kernel is built around the stream:
 //  * A block owns 128 output rows (8 consumer warps x 16 rows) and a range of
 //    K.  One producer thread streams the block's packed weights with TMA in
-//    stages of 128 rows x 128 bytes (512 inputs), written in the 128-byte
-//    swizzle so that each lane's 16-byte reads are free of bank conflicts,
-//    through a ring of mbarrier-tracked buffers.  Weight loads need nothing
-//    from the preceding kernel, so they start before the grid dependency
-//    wait (programmatic dependent launch) and overlap the activation
-//    quantisation.
-//  * The block's int8 activations are copied once into shared memory, with
-//    the 16-byte chunks of every 128-byte block rotated by twice the block
-//    index, which makes the activation fragment reads conflict-free too.
+//    stages of 128 rows x 128 bytes (512 inputs), in the 128-byte swizzle so
+//    that the lanes' 16-byte reads are free of bank conflicts, through a
+//    ring of mbarrier-tracked buffers.  The weights need nothing from the
+//    preceding kernel, so their loads start before the grid-dependency wait
+//    (programmatic dependent launch).
+//  * The block's activations are staged once in shared memory as int8, the
+//    16-byte chunks of every 128-byte block rotated by twice the block index
+//    so that fragment reads are conflict-free.  When the activations are
+//    small the block quantises them itself (per-token absmax over all of K,
+//    then its own K range), which saves a launch and a round trip through
+//    HBM; otherwise it copies codes written by the quantisation kernel.
 //  * Each lane takes 16-byte chunks 2t and 2t+1 of rows g and g+8 of its
 //    warp's 16 rows into registers and releases the stage at once.
 //    Unpacking is one AND per four weights: mask 0x03030303 << 2j keeps the
 //    codes of elements 4j..4j+3 of a word in place (scaled by 4^j); four
 //    accumulator sets, one per j, are shifted back and added at the end,
-//    which is exact because each set is a multiple of 4^j.  The k order
-//    inside an mma is free as long as both operands agree, so lane (g, t)
-//    feeds its own words to the A fragment and the matching activation bytes
-//    to the B fragment.
-//  * Stored codes are c = t + 1, so y = (sum c*q - rowsum(q)) * gamma / s.
-//    When K is split over blocks, each block stores its partial sums in its
-//    own workspace slot; the last block of a row block (an atomic counter
-//    tells) adds the slots in split order, applies the epilogue and resets
-//    the counter for the next call.
+//    exact because each set is a multiple of 4^j.  The k order inside an mma
+//    is free as long as both operands agree, so lane (g, t) feeds its own
+//    words to the A fragment and the matching activation bytes to B.
+//  * Stored codes are c = t + 1, so each block subtracts the sum of its own
+//    activation codes: sum_range (c - 1) q = sum_range t q.
+//  * When K is split over blocks, the blocks of one row block form a thread
+//    block cluster and add their partial sums through distributed shared
+//    memory; each block then finishes a slice of the rows:
+//    y = acc * (gamma / s).
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -49,6 +52,7 @@ constexpr int kGvStageBytes = kGvRows * 128;      // 16 KB of packed weights
 constexpr int kGvThreads = 32 * (kGvWarps + 1);   // + one producer warp
 constexpr int kGvConsumers = 32 * kGvWarps;
 constexpr int kGvXBudget = 64 * 1024;             // activation bytes staged per block
+constexpr int kGvFuseLimit = 16 * 1024;           // M*K up to which blocks quantise themselves
 
 __device__ __forceinline__ void mma_u8s8_16x8x32(int (&d)[4], uint32_t a0, uint32_t a1,
                                                  uint32_t a2, uint32_t a3, uint32_t b0,
@@ -68,6 +72,12 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t u4_get(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
@@ -76,33 +86,89 @@ __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kGvConsumers) : "memory");
 }
 
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+__device__ __forceinline__ int ld_cluster_s32(uint32_t local_addr, uint32_t rank) {
+  uint32_t remote;
+  int v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
+  return v;
+}
+
 // Byte offset of activation chunk (16 bytes) `c` of a staged token row.
 __device__ __forceinline__ int x_chunk_off(int c) {
   const int blk = c >> 3, ci = c & 7;
   return blk * 128 + (((ci + 2 * (blk & 3)) & 7) << 4);
 }
 
-template <int TG, typename TY>
+// Sum of the 16 signed bytes of a chunk.
+__device__ __forceinline__ int byte_sum16(const uint4& v) {
+  int s = __dp4a(static_cast<int>(v.x), 0x01010101, 0);
+  s = __dp4a(static_cast<int>(v.y), 0x01010101, s);
+  s = __dp4a(static_cast<int>(v.z), 0x01010101, s);
+  return __dp4a(static_cast<int>(v.w), 0x01010101, s);
+}
+
+// 8 activations as fp32 (bf16 -> fp32 is exact).
+__device__ __forceinline__ void load8f(const float* p, float (&f)[8]) {
+  const float4 a = __ldcg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldcg(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+__device__ __forceinline__ void load8f(const __nv_bfloat16* p, float (&f)[8]) {
+  const uint4 u = __ldcg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+template <int TT>
+__device__ __forceinline__ void warp_sum_tokens(int (&v)[TT]) {
+#pragma unroll
+  for (int m = 0; m < TT; ++m)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v[m] += __shfl_xor_sync(0xffffffffu, v[m], o);
+}
+
+template <int TG, typename TY, typename TX>
 __global__ void __launch_bounds__(kGvThreads) gemv_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const float* __restrict__ gamma_ptr, int N, int K,
-    int M, const int8_t* __restrict__ xq, const float* __restrict__ scale,
-    const int32_t* __restrict__ rowsum, TY* __restrict__ y, int32_t* __restrict__ acc_out,
-    int32_t* __restrict__ acc_ws, uint32_t* __restrict__ counters, int splits, int st_per_split,
-    int nring, int x_pitch, uint32_t* status) {
+    int M, const TX* __restrict__ x, const float* __restrict__ scale, TY* __restrict__ y,
+    int32_t* __restrict__ acc_out, int splits, int st_per_split, int nring, int x_pitch,
+    uint32_t* status) {
+  constexpr int TT = TG * 8;                // token slots
+  constexpr bool kFused = sizeof(TX) != 1;  // activations arrive unquantised
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   const uint32_t ring = sb;
-  const uint32_t xs = sb + nring * kGvStageBytes;
   const int x_bytes = ((M * x_pitch + 127) / 128) * 128;
+  const uint32_t xs = sb + nring * kGvStageBytes;
   uint8_t* misc = smem + nring * kGvStageBytes + x_bytes;
-  const uint32_t bar0 = smem_u32(misc);  // full[nring], empty[nring]
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 16 * nring);
+  int* red_buf = reinterpret_cast<int*>(misc);                       // [128 rows][TT] partial sums
+  float* s_tok = reinterpret_cast<float*>(misc + kGvRows * TT * 4);  // [TT] token scales
+  int* rs_tok = reinterpret_cast<int*>(s_tok + TT);                  // [TT] range code sums
+  int* wred = rs_tok + TT;                                           // [kGvWarps][TT] reductions
+  const uint32_t bar0 = smem_u32(wred + kGvWarps * TT);              // full[nring], empty[nring]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(wred + kGvWarps * TT + 4 * nring);
   volatile int* never = abort_flag + 1;
-  volatile int* last_flag = abort_flag + 2;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rb = blockIdx.x / splits, ks = blockIdx.x % splits;
+  const int rb = blockIdx.x / splits;
+  const int ks = (splits > 1) ? static_cast<int>(cluster_rank()) : 0;
   const int n_st = (K + kGvStageK - 1) / kGvStageK;
   const int st0 = ks * st_per_split;
   const int st1 = min(n_st, st0 + st_per_split);
@@ -121,6 +187,11 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(
   griddep_launch_dependents();
   const WaitCtl ctl{status, abort_flag, kWaitLimitNs};
 
+  int acc[TG][4];
+  const int g = lane >> 2, t = lane & 3;
+  const int r_lo = warp * 16 + g;  // rows of this lane within the block (and + 8)
+  bool ok = true;
+
   if (warp == kGvWarps) {
     // Producer: weights only, so no grid-dependency wait is needed.
     if (lane == 0) {
@@ -138,97 +209,176 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(
           mbar_wait(bar0 + 8 * (j % nring), (j / nring) & 1, drain);
       }
     }
-    return;
-  }
-
-  // ---- consumers ----
-  griddep_wait();  // activations, scales and row sums come from the preceding kernel
-  const int k0 = st0 * kGvStageK;
-  const int kr = min(K, st1 * kGvStageK) - k0;  // multiple of 64
-  {
-    const int chunks = kr >> 4;
-    for (int idx = threadIdx.x; idx < M * chunks; idx += kGvConsumers) {
-      const int m = idx / chunks, c = idx - m * chunks;
-      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(xq + static_cast<size_t>(m) * K + k0) + c);
-      asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(xs + m * x_pitch + x_chunk_off(c)),
-                   "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                   : "memory");
-    }
-  }
-  consumer_sync();
-
-  const int g = lane >> 2, t = lane & 3;
-  const int r_lo = warp * 16 + g;  // rows of this lane within the block (and + 8)
-  int d[TG][4][4];
-#pragma unroll
-  for (int tg = 0; tg < TG; ++tg)
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) d[tg][j][c] = 0;
-
-  bool ok = true;
-  for (int i = 0; i < nst; ++i) {
-    const int slot = i % nring;
-    const bool got = mbar_wait(bar0 + 8 * slot, (i / nring) & 1, ctl);
-    if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-    const uint32_t wt = ring + slot * kGvStageBytes;
-    // 128-byte swizzle: chunk c of row r sits at chunk position c ^ (r & 7); r & 7 == g here.
-    const uint4 wl0 = lds128(wt + r_lo * 128 + (((2 * t) ^ g) << 4));
-    const uint4 wl1 = lds128(wt + r_lo * 128 + (((2 * t + 1) ^ g) << 4));
-    const uint4 wh0 = lds128(wt + (r_lo + 8) * 128 + (((2 * t) ^ g) << 4));
-    const uint4 wh1 = lds128(wt + (r_lo + 8) * 128 + (((2 * t + 1) ^ g) << 4));
     __syncwarp();
-    if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // weights are in registers
-
-    const int qblk = i * 4 + t;  // this lane's 128-input block of the staged activations
+    if (splits == 1) return;
+  } else {
+    // ---- consumers: stage this block's activations ----
+    griddep_wait();  // the activations may be the preceding kernel's output
+    const int tid = threadIdx.x;
+    const int k0 = st0 * kGvStageK;
+    const int kr = min(K, st1 * kGvStageK) - k0;  // multiple of 64
+    const int chunks = kr >> 4;                   // 16-input chunks of this block's range
+    int rs[TT];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint4 wl = h ? wl1 : wl0, wh = h ? wh1 : wh0;
+    for (int m = 0; m < TT; ++m) rs[m] = 0;
+    if constexpr (kFused) {
+      // Per-token absmax over all of K, then s = 127 / max(amax, 1e-5).
+      float am[TT];
 #pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        const int c0 = 4 * h + 2 * p;  // activation chunks c0, c0+1 of block qblk
-        uint4 xa[TG], xb[TG];
+      for (int m = 0; m < TT; ++m) {
+        am[m] = 0.0f;
+        if (m < M) {
+          for (int v = tid; v < K / 8; v += kGvConsumers) {
+            float f[8];
+            load8f(x + static_cast<size_t>(m) * K + v * 8, f);
 #pragma unroll
-        for (int tg = 0; tg < TG; ++tg) {
-          const int m = tg * 8 + g;
-          if (m < M) {
-            const uint32_t row = xs + m * x_pitch + qblk * 128;
-            xa[tg] = lds128(row + (((c0 + 2 * t) & 7) << 4));
-            xb[tg] = lds128(row + (((c0 + 1 + 2 * t) & 7) << 4));
-          } else {
-            xa[tg] = make_uint4(0, 0, 0, 0);
-            xb[tg] = make_uint4(0, 0, 0, 0);
+            for (int e = 0; e < 8; ++e) am[m] = fmaxf(am[m], fabsf(f[e]));
           }
         }
-        const uint32_t lo0 = u4_get(wl, 2 * p), lo1 = u4_get(wl, 2 * p + 1);
-        const uint32_t hi0 = u4_get(wh, 2 * p), hi1 = u4_get(wh, 2 * p + 1);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t mask = 0x03030303u << (2 * j);
-          const uint32_t a0 = lo0 & mask, a1 = hi0 & mask, a2 = lo1 & mask, a3 = hi1 & mask;
+        for (int o = 16; o > 0; o >>= 1) am[m] = fmaxf(am[m], __shfl_xor_sync(0xffffffffu, am[m], o));
+      }
+      if (lane == 0) {
 #pragma unroll
-          for (int tg = 0; tg < TG; ++tg)
-            mma_u8s8_16x8x32(d[tg][j], a0, a1, a2, a3, u4_get(xa[tg], j), u4_get(xb[tg], j));
+        for (int m = 0; m < TT; ++m) reinterpret_cast<float*>(wred)[warp * TT + m] = am[m];
+      }
+      consumer_sync();
+      if (tid < TT) {
+        float a = 0.0f;
+        for (int w = 0; w < kGvWarps; ++w) a = fmaxf(a, reinterpret_cast<float*>(wred)[w * TT + tid]);
+        s_tok[tid] = __fdiv_rn(127.0f, fmaxf(a, 1e-5f));
+      }
+      consumer_sync();
+      // Quantise this block's range into shared memory: q = clamp(rint(x * s), -128, 127).
+#pragma unroll
+      for (int m = 0; m < TT; ++m) {
+        if (m < M) {
+          const float s = s_tok[m];
+          for (int c = tid; c < chunks; c += kGvConsumers) {
+            const TX* src = x + static_cast<size_t>(m) * K + k0 + c * 16;
+            uint32_t w[4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float f[8];
+              load8f(src + 8 * h, f);
+#pragma unroll
+              for (int e = 0; e < 8; e += 4) {
+                uint32_t word = 0;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                  int q = __float2int_rn(__fmul_rn(f[e + b], s));
+                  q = min(max(q, -128), 127);
+                  rs[m] += q;
+                  word |= (static_cast<uint32_t>(q) & 0xffu) << (8 * b);
+                }
+                w[2 * h + e / 4] = word;
+              }
+            }
+            sts128(xs + m * x_pitch + x_chunk_off(c), make_uint4(w[0], w[1], w[2], w[3]));
+          }
+        }
+      }
+    } else {
+      // Codes written by the quantisation kernel.
+#pragma unroll
+      for (int m = 0; m < TT; ++m) {
+        if (m < M) {
+          const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const int8_t*>(x) +
+                                                            static_cast<size_t>(m) * K + k0);
+          for (int c = tid; c < chunks; c += kGvConsumers) {
+            const uint4 v = __ldcg(src + c);
+            rs[m] += byte_sum16(v);
+            sts128(xs + m * x_pitch + x_chunk_off(c), v);
+          }
+        }
+      }
+      if (tid < TT && tid < M) s_tok[tid] = __ldcg(scale + tid);
+    }
+    warp_sum_tokens<TT>(rs);
+    if (lane == 0) {
+#pragma unroll
+      for (int m = 0; m < TT; ++m) wred[warp * TT + m] = rs[m];
+    }
+    consumer_sync();
+    if (tid < TT) {
+      int a = 0;
+      for (int w = 0; w < kGvWarps; ++w) a += wred[w * TT + tid];
+      rs_tok[tid] = a;
+    }
+    consumer_sync();
+
+    // ---- main loop over this block's stages ----
+    int d[TG][4][4];
+#pragma unroll
+    for (int tg = 0; tg < TG; ++tg)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) d[tg][j][c] = 0;
+
+    for (int i = 0; i < nst; ++i) {
+      const int slot = i % nring;
+      const bool got = mbar_wait(bar0 + 8 * slot, (i / nring) & 1, ctl);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      const uint32_t wt = ring + slot * kGvStageBytes;
+      // 128-byte swizzle: chunk c of row r sits at chunk position c ^ (r & 7); r & 7 == g here.
+      const uint4 wl0 = lds128(wt + r_lo * 128 + (((2 * t) ^ g) << 4));
+      const uint4 wl1 = lds128(wt + r_lo * 128 + (((2 * t + 1) ^ g) << 4));
+      const uint4 wh0 = lds128(wt + (r_lo + 8) * 128 + (((2 * t) ^ g) << 4));
+      const uint4 wh1 = lds128(wt + (r_lo + 8) * 128 + (((2 * t + 1) ^ g) << 4));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // the weights are in registers
+
+      const int qblk = i * 4 + t;  // this lane's 128-input block of the staged activations
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint4 wl = h ? wl1 : wl0, wh = h ? wh1 : wh0;
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+          const int c0 = 4 * h + 2 * p;  // activation chunks c0, c0+1 of block qblk
+          uint4 xa[TG], xb[TG];
+#pragma unroll
+          for (int tg = 0; tg < TG; ++tg) {
+            const int m = tg * 8 + g;
+            if (m < M) {
+              const uint32_t row = xs + m * x_pitch + qblk * 128;
+              xa[tg] = lds128(row + (((c0 + 2 * t) & 7) << 4));
+              xb[tg] = lds128(row + (((c0 + 1 + 2 * t) & 7) << 4));
+            } else {
+              xa[tg] = make_uint4(0, 0, 0, 0);
+              xb[tg] = make_uint4(0, 0, 0, 0);
+            }
+          }
+          const uint32_t lo0 = u4_get(wl, 2 * p), lo1 = u4_get(wl, 2 * p + 1);
+          const uint32_t hi0 = u4_get(wh, 2 * p), hi1 = u4_get(wh, 2 * p + 1);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t mask = 0x03030303u << (2 * j);
+            const uint32_t a0 = lo0 & mask, a1 = hi0 & mask, a2 = lo1 & mask, a3 = hi1 & mask;
+#pragma unroll
+            for (int tg = 0; tg < TG; ++tg)
+              mma_u8s8_16x8x32(d[tg][j], a0, a1, a2, a3, u4_get(xa[tg], j), u4_get(xb[tg], j));
+          }
         }
       }
     }
+#pragma unroll
+    for (int tg = 0; tg < TG; ++tg)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int m = tg * 8 + 2 * t + (c & 1);
+        acc[tg][c] = d[tg][0][c] + (d[tg][1][c] >> 2) + (d[tg][2][c] >> 4) + (d[tg][3][c] >> 6) -
+                     (m < M ? rs_tok[m] : 0);
+      }
   }
-  // Every consumer warp gets here (bounded waits); leave together if any wait ran out.
-  consumer_sync();
-  if (*abort_flag || !ok) return;  // the status word records it; no output is written
-
-  // ---- epilogue ----
-  int acc[TG][4];
-#pragma unroll
-  for (int tg = 0; tg < TG; ++tg)
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-      acc[tg][c] = d[tg][0][c] + (d[tg][1][c] >> 2) + (d[tg][2][c] >> 4) + (d[tg][3][c] >> 6);
 
   const float gamma = __ldg(gamma_ptr);
   const int n_base = rb * kGvRows;
+
   if (splits == 1) {
+    // Consumers only (the producer has left); all of K is in registers.
+    consumer_sync();
+    if (*abort_flag || !ok) return;  // the status word records it; no output is written
 #pragma unroll
     for (int tg = 0; tg < TG; ++tg)
 #pragma unroll
@@ -236,59 +386,60 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(
         const int n = n_base + r_lo + ((c & 2) ? 8 : 0);
         const int m = tg * 8 + 2 * t + (c & 1);
         if (n < N && m < M) {
-          const int a = acc[tg][c] - __ldg(rowsum + m);
-          const float v = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, __ldg(scale + m)));
+          const float v = __fmul_rn(static_cast<float>(acc[tg][c]), __fdiv_rn(gamma, s_tok[m]));
           const size_t o = static_cast<size_t>(m) * N + n;
           if constexpr (sizeof(TY) == 4) y[o] = v; else y[o] = __float2bfloat16_rn(v);
-          if (acc_out) acc_out[o] = a;
+          if (acc_out) acc_out[o] = acc[tg][c];
         }
       }
     return;
   }
 
-  // Split K: each block stores its partial sums in its own slot; the block that
-  // completes the row block adds the slots in split order (deterministic) and
-  // finishes the row block.  Only the per-row-block counter is shared, and the
-  // finishing block resets it.
-  int32_t* my_slot = acc_ws + (static_cast<size_t>(rb) * splits + ks) * M * kGvRows;
+  // ---- split K: the cluster's blocks add their partial sums through distributed shared memory ----
+  if (warp < kGvWarps) {
 #pragma unroll
-  for (int tg = 0; tg < TG; ++tg)
+    for (int tg = 0; tg < TG; ++tg)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int r = r_lo + ((c & 2) ? 8 : 0);
-      const int m = tg * 8 + 2 * t + (c & 1);
-      if (m < M) __stcg(my_slot + m * kGvRows + r, acc[tg][c]);
+      for (int c = 0; c < 4; ++c) {
+        const int r = r_lo + ((c & 2) ? 8 : 0);
+        const int m = tg * 8 + 2 * t + (c & 1);
+        red_buf[r * TT + m] = acc[tg][c];
+      }
+  }
+  cluster_sync_all();  // every thread of every block of the cluster arrives here
+  bool failed = false;  // did any block of the cluster give up a wait?
+  for (int p = 0; p < splits; ++p)
+    failed |= ld_cluster_s32(smem_u32(const_cast<int*>(abort_flag)), p) != 0;
+  if (warp < kGvWarps && !failed) {
+    // This block finishes rows [r0, r1) of the row block.
+    const int per = (kGvRows + splits - 1) / splits;
+    const int r0 = ks * per, r1 = min(kGvRows, r0 + per);
+    const int rows = min(r1, N - n_base) - r0;
+    const uint32_t red_addr = smem_u32(red_buf);
+    for (int idx = threadIdx.x; idx < rows * M; idx += kGvConsumers) {
+      const int m = idx / rows, r = r0 + (idx - m * rows);
+      int a = 0;
+      for (int p = 0; p < splits; ++p) a += ld_cluster_s32(red_addr + (r * TT + m) * 4, p);
+      const size_t o = static_cast<size_t>(m) * N + n_base + r;
+      const float v = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, s_tok[m]));
+      if constexpr (sizeof(TY) == 4) y[o] = v; else y[o] = __float2bfloat16_rn(v);
+      if (acc_out) acc_out[o] = a;
     }
-  __threadfence();
-  consumer_sync();
-  if (threadIdx.x == 0) {
-    const uint32_t prev = atomicAdd(counters + rb, 1u);
-    *last_flag = (prev + 1 == static_cast<uint32_t>(splits)) ? 1 : 0;
   }
-  consumer_sync();
-  if (!*last_flag) return;
-  __threadfence();
-  const int rows = min(kGvRows, N - n_base);
-  const int32_t* slots = acc_ws + static_cast<size_t>(rb) * splits * M * kGvRows;
-  for (int idx = threadIdx.x; idx < rows * M; idx += kGvConsumers) {
-    const int m = idx / rows, r = idx - m * rows;
-    int sum = 0;
-    for (int s = 0; s < splits; ++s) sum += __ldcg(slots + (static_cast<size_t>(s) * M + m) * kGvRows + r);
-    const int a = sum - __ldg(rowsum + m);
-    const size_t o = static_cast<size_t>(m) * N + n_base + r;
-    const float v = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, __ldg(scale + m)));
-    if constexpr (sizeof(TY) == 4) y[o] = v; else y[o] = __float2bfloat16_rn(v);
-    if (acc_out) acc_out[o] = a;
-  }
-  if (threadIdx.x == 0) counters[rb] = 0;
+  cluster_sync_all();  // no block leaves while another still reads its shared memory
 }
 
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
+static int gemv_smem_bytes(int M, int tt, int ring, int x_pitch) {
+  return ring * kGvStageBytes + ((M * x_pitch + 127) / 128) * 128 + kGvRows * tt * 4 + 2 * tt * 4 +
+         kGvWarps * tt * 4 + 16 * ring + 64 + 1024;
+}
 
 static GemvPlan plan_gemv_budget(int M, int N, int K, int x_budget) {
   const int sms = num_sms();
+  const int tt = M <= 8 ? 8 : 16;
   GemvPlan best{};
   double best_cost = 1e30;
   const int n_rb = (N + kGvRows - 1) / kGvRows;
@@ -302,7 +453,7 @@ static GemvPlan plan_gemv_budget(int M, int N, int K, int x_budget) {
     for (int ring : {2, 3, 4, 6}) {
       if (ring > spc && ring != 2) continue;
       const int r_eff = ring < spc ? ring : spc;
-      const int smem = r_eff * kGvStageBytes + ((M * x_pitch + 127) / 128) * 128 + 16 * r_eff + 64 + 1024;
+      const int smem = gemv_smem_bytes(M, tt, r_eff, x_pitch);
       if (smem > 227 * 1024) continue;
       int occ = (227 * 1024) / smem;
       if (occ > 2048 / kGvThreads) occ = 2048 / kGvThreads;
@@ -311,9 +462,9 @@ static GemvPlan plan_gemv_budget(int M, int N, int K, int x_budget) {
       const long long per_sm = (ctas + sms - 1) / sms;
       const long long waves = (ctas + slots - 1) / slots;
       const int in_flight = static_cast<int>(per_sm < occ ? per_sm : occ) * r_eff;
-      // Stages the busiest SM streams, a little extra per split for the partial sums,
+      // Stages the busiest SM streams, a little extra per split for the reduction,
       // a penalty for a short tail wave and for too few stages in flight per SM.
-      double cost = static_cast<double>(per_sm * spc) * (1.0 + 0.04 * (s - 1));
+      double cost = static_cast<double>(per_sm * spc) * (1.0 + 0.03 * (s - 1));
       if (waves > 1 && waves < 4) cost *= 1.1;
       if (in_flight < 3 && spc >= 3) cost *= 1.25;
       if (cost < best_cost - 1e-9) {
@@ -331,8 +482,10 @@ GemvPlan plan_gemv(int M, int N, int K) {
   return p;  // splits == 0: the activations do not fit; the caller uses the GEMM
 }
 
-template <int TG, typename TY>
-static cudaError_t launch_gemv_t(const ProductArgs& a, const GemvPlan& p, cudaStream_t stream, bool pdl) {
+bool gemv_fuses_quant(int M, int K) { return static_cast<long long>(M) * K <= kGvFuseLimit; }
+
+template <int TG, typename TY, typename TX>
+static cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, cudaStream_t stream, bool pdl) {
   EncodeTiledFn enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap tw;
@@ -345,28 +498,55 @@ static cudaError_t launch_gemv_t(const ProductArgs& a, const GemvPlan& p, cudaSt
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
     return cudaErrorInvalidValue;
   }
-  static int max_smem_set = 0;
-  if (p.smem > 48 * 1024 && p.smem > max_smem_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<TG, TY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         227 * 1024);
+  auto kernel = gemv_kernel<TG, TY, TX>;
+  static bool attr_set = false;  // per template instance
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     if (e != cudaSuccess) return e;
-    max_smem_set = 227 * 1024;
+    attr_set = true;
   }
-  return launch(gemv_kernel<TG, TY>, dim3(p.n_rb * p.splits), dim3(kGvThreads), static_cast<size_t>(p.smem),
-                stream, pdl, tw, a.gamma, a.N, a.K, a.M, a.xq, a.scale, a.rowsum, static_cast<TY*>(a.y),
-                a.acc_out, a.acc_ws, a.counters, p.splits, p.st_per_split, p.nring, p.x_pitch, a.status);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.n_rb * p.splits);
+  cfg.blockDim = dim3(kGvThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(p.smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeClusterDimension;
+  attr[n].val.clusterDim.x = p.splits;
+  attr[n].val.clusterDim.y = 1;
+  attr[n].val.clusterDim.z = 1;
+  ++n;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, tw, a.gamma, a.N, a.K, a.M, static_cast<const TX*>(a.x), a.scale,
+                            static_cast<TY*>(a.y), a.acc_out, p.splits, p.st_per_split, p.nring, p.x_pitch,
+                            a.status);
 }
 
-cudaError_t launch_gemv(const ProductArgs& a, cudaStream_t stream, bool pdl) {
+template <int TG, typename TY>
+static cudaError_t launch_gemv_x(const GemvArgs& a, const GemvPlan& p, cudaStream_t stream, bool pdl) {
+  switch (a.x_type) {
+    case kInBF16: return launch_gemv_t<TG, TY, __nv_bfloat16>(a, p, stream, pdl);
+    case kInF32: return launch_gemv_t<TG, TY, float>(a, p, stream, pdl);
+    default: return launch_gemv_t<TG, TY, int8_t>(a, p, stream, pdl);
+  }
+}
+
+cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t stream, bool pdl) {
   const GemvPlan p = plan_gemv(a.M, a.N, a.K);
   if (p.splits == 0) return cudaErrorInvalidConfiguration;
-  if (p.splits > 1 && (a.acc_ws == nullptr || a.counters == nullptr)) return cudaErrorInvalidValue;
   if (a.M <= 8) {
-    return a.y_type == kOutBF16 ? launch_gemv_t<1, __nv_bfloat16>(a, p, stream, pdl)
-                                : launch_gemv_t<1, float>(a, p, stream, pdl);
+    return a.y_type == kOutBF16 ? launch_gemv_x<1, __nv_bfloat16>(a, p, stream, pdl)
+                                : launch_gemv_x<1, float>(a, p, stream, pdl);
   }
-  return a.y_type == kOutBF16 ? launch_gemv_t<2, __nv_bfloat16>(a, p, stream, pdl)
-                              : launch_gemv_t<2, float>(a, p, stream, pdl);
+  return a.y_type == kOutBF16 ? launch_gemv_x<2, __nv_bfloat16>(a, p, stream, pdl)
+                              : launch_gemv_x<2, float>(a, p, stream, pdl);
 }
 
 }  // namespace bl

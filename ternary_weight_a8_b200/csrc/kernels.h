@@ -39,7 +39,9 @@ cudaError_t launch_ternary_pack(const float* W, int N, int K, const float* gamma
 cudaError_t launch_act_quant(const void* x, int x_bf16, int M, int K, int8_t* xq, float* scale,
                              int32_t* rowsum, cudaStream_t stream, bool pdl);
 
-// Product + dequantisation on quantised activations.
+enum InType { kInInt8 = 0, kInBF16 = 1, kInF32 = 2 };
+
+// Tensor-core GEMM on quantised activations (many tokens).
 struct ProductArgs {
   const uint8_t* packed;
   const float* gamma;
@@ -51,18 +53,30 @@ struct ProductArgs {
   int y_type;  // OutType
   int32_t* acc_out;
   uint32_t* status;
-  int32_t* acc_ws;     // split-K partial-sum slots [row block][split][M][128] (GEMV only)
-  uint32_t* counters;  // one per 128-row block, zero between calls (GEMV only)
 };
 
-// Decode kernel launch plan: blocks of 128 rows, K split `splits` ways, one wave.
+// Decode GEMV (M <= 16): activations as int8 codes with their scales, or raw
+// (fp32 / bf16) activations that the kernel quantises itself.
+struct GemvArgs {
+  const uint8_t* packed;
+  const float* gamma;
+  int N, K, M;
+  const void* x;
+  int x_type;           // InType
+  const float* scale;   // token scales when x_type == kInInt8
+  void* y;
+  int y_type;           // OutType
+  int32_t* acc_out;
+  uint32_t* status;
+};
+
+// Decode kernel launch plan: blocks of 128 rows; K split over a cluster of `splits` blocks.
 struct GemvPlan {
   int n_rb, n_st, splits, st_per_split, nring, x_pitch, smem;
 };
 GemvPlan plan_gemv(int M, int N, int K);
-constexpr int kGemvRowsPerBlock = 128;
+bool gemv_fuses_quant(int M, int K);
 constexpr int kGemvMaxSplits = 8;
-constexpr int kGemvMaxCounters = 16384;  // row blocks: N <= 2^21
 
 // cuTensorMapEncodeTiled from the driver (no link-time dependency on libcuda).
 #ifdef CUDA_VERSION
@@ -72,7 +86,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 #endif
 void* tensor_map_encoder();
-cudaError_t launch_gemv(const ProductArgs& a, cudaStream_t stream, bool pdl);
+cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t stream, bool pdl);
 cudaError_t launch_gemm(const ProductArgs& a, cudaStream_t stream, bool pdl);
 
 // Self-test of the bounded device wait.

@@ -66,21 +66,15 @@ def test_host_side_validation(L):
 
 
 def test_workspace_layout(L):
-    # header (status 256 + split counters 64 KB), decode split slots for M <= 16
-    # (128-row blocks x 8 splits x M x 128 x 4 bytes), then q (M*K), scale and rowsum
-    # (4*M each), every region rounded to 256 bytes.
-    head = 256 + 65536
-    def slots(M, N):
-        return ((N + 127) // 128) * 8 * M * 128 * 4 if M <= 16 else 0
-    assert tb.workspace_bytes(1, 6912, 2560) == head + slots(1, 6912) + 2560 + 256 + 256
-    assert tb.workspace_bytes(2048, 6912, 2560) == head + 2048 * 2560 + 8192 + 8192
-    assert tb.workspace_bytes(3, 10, 64) == head + slots(3, 10) + 256 + 256 + 256
+    # status word (256) + q (M*K, 256-rounded) + scale and rowsum (4*M each, 256-rounded)
+    assert tb.workspace_bytes(1, 6912, 2560) == 256 + 2560 + 256 + 256
+    assert tb.workspace_bytes(2048, 6912, 2560) == 256 + 2048 * 2560 + 8192 + 8192
+    assert tb.workspace_bytes(3, 10, 64) == 256 + 256 + 256 + 256
     assert tb.pack_workspace_bytes(6912, 2560) == 256 + 6912 * 8
     layers = (tb.bl_layer * 2)()
     layers[0].N, layers[0].K = 10240, 8192
     layers[1].N, layers[1].K = 8192, 28672
-    # one layout for the whole chain: the largest N and the largest K
-    assert L.bitlinear_chain_workspace_bytes(layers, 2, 8) == tb.workspace_bytes(8, 10240, 28672)
+    assert L.bitlinear_chain_workspace_bytes(layers, 2, 8) == tb.workspace_bytes(8, 8192, 28672)
 
 
 def test_binding_fails_loudly_without_library(monkeypatch):
