@@ -33,12 +33,19 @@
 //    words to the A fragment and the matching activation bytes to B.
 //  * Stored codes are c = t + 1, so each block subtracts the sum of its own
 //    activation codes: sum_range (c - 1) q = sum_range t q.
-//  * When K is split over blocks, the blocks of one row block form a thread
-//    block cluster and add their partial sums through distributed shared
-//    memory; each block then finishes a slice of the rows:
-//    y = acc * (gamma / s).
+//  * Two ways to cover the matrix, chosen by a host planner from a model of
+//    the bytes each SM keeps in flight: when there are enough row blocks,
+//    persistent blocks each take every gridDim-th row block over all of K,
+//    staging the activations once and streaming weights across row blocks
+//    without draining the ring; otherwise K is split, the blocks of one row
+//    block form a thread block cluster, add their partial sums through
+//    distributed shared memory and each finish a slice of the rows.
+//    Either way y = acc * (gamma / s).
+//  * The kernel is specialised on the number of token slots (1, 2, 4, 8 or
+//    16), so a one-token decode does no work for absent tokens.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -143,13 +150,13 @@ __device__ __forceinline__ void warp_sum_tokens(int (&v)[TT]) {
     for (int o = 16; o > 0; o >>= 1) v[m] += __shfl_xor_sync(0xffffffffu, v[m], o);
 }
 
-template <int TG, typename TY, typename TX>
-__global__ void __launch_bounds__(kGvThreads) gemv_kernel(
+template <int TT, typename TY, typename TX>
+__global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const float* __restrict__ gamma_ptr, int N, int K,
     int M, const TX* __restrict__ x, const float* __restrict__ scale, TY* __restrict__ y,
     int32_t* __restrict__ acc_out, int splits, int st_per_split, int nring, int x_pitch,
     uint32_t* status) {
-  constexpr int TT = TG * 8;                // token slots
+  constexpr int TG = (TT + 7) / 8;          // mma token groups of 8
   constexpr bool kFused = sizeof(TX) != 1;  // activations arrive unquantised
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -167,8 +174,13 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(
   volatile int* never = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rb = blockIdx.x / splits;
-  const int ks = (splits > 1) ? static_cast<int>(cluster_rank()) : 0;
+  const int n_rb = (N + kGvRows - 1) / kGvRows;
+  const bool clustered = splits > 1;
+  // Row blocks of this block: one per cluster when K is split, else every gridDim-th.
+  const int rb0 = clustered ? static_cast<int>(blockIdx.x) / splits : static_cast<int>(blockIdx.x);
+  const int rb_step = clustered ? n_rb : static_cast<int>(gridDim.x);
+  const int n_my_rb = rb0 < n_rb ? (n_rb - 1 - rb0) / rb_step + 1 : 0;
+  const int ks = clustered ? static_cast<int>(cluster_rank()) : 0;
   const int n_st = (K + kGvStageK - 1) / kGvStageK;
   const int st0 = ks * st_per_split;
   const int st1 = min(n_st, st0 + st_per_split);
@@ -196,21 +208,23 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(
     // Producer: weights only, so no grid-dependency wait is needed.
     if (lane == 0) {
       tma_prefetch_desc(&tmap_w);
+      const int total = n_my_rb * nst;  // (row block, stage) items, streamed without a break
       int i = 0;
-      for (; i < nst; ++i) {
+      for (; i < total; ++i) {
         const int slot = i % nring;
+        const int rb = rb0 + (i / nst) * rb_step, st = st0 + i % nst;
         if (!mbar_wait(bar0 + 8 * (nring + slot), ((i / nring) & 1) ^ 1, ctl)) break;
         mbar_arrive_expect_tx(bar0 + 8 * slot, kGvStageBytes);
-        tma_load_2d(ring + slot * kGvStageBytes, &tmap_w, (st0 + i) * 128, rb * kGvRows, bar0 + 8 * slot);
+        tma_load_2d(ring + slot * kGvStageBytes, &tmap_w, st * 128, rb * kGvRows, bar0 + 8 * slot);
       }
-      if (i < nst) {  // gave up: let copies in flight land before shared memory is released
+      if (i < total) {  // gave up: let copies in flight land before shared memory is released
         const WaitCtl drain{nullptr, never, 100000000ull};
         for (int j = (i > nring ? i - nring : 0); j < i; ++j)
           mbar_wait(bar0 + 8 * (j % nring), (j / nring) & 1, drain);
       }
     }
     __syncwarp();
-    if (splits == 1) return;
+    if (!clustered) return;
   } else {
     // ---- consumers: stage this block's activations ----
     griddep_wait();  // the activations may be the preceding kernel's output
@@ -307,93 +321,95 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(
     }
     consumer_sync();
 
-    // ---- main loop over this block's stages ----
-    int d[TG][4][4];
+    // ---- main loop: this block's row blocks, each over this block's stages ----
+    const float gamma = __ldg(gamma_ptr);
+    for (int r = 0; r < n_my_rb && ok; ++r) {
+      int d[TG][4][4];
 #pragma unroll
-    for (int tg = 0; tg < TG; ++tg)
+      for (int tg = 0; tg < TG; ++tg)
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) d[tg][j][c] = 0;
+          for (int c = 0; c < 4; ++c) d[tg][j][c] = 0;
 
-    for (int i = 0; i < nst; ++i) {
-      const int slot = i % nring;
-      const bool got = mbar_wait(bar0 + 8 * slot, (i / nring) & 1, ctl);
-      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-      const uint32_t wt = ring + slot * kGvStageBytes;
-      // 128-byte swizzle: chunk c of row r sits at chunk position c ^ (r & 7); r & 7 == g here.
-      const uint4 wl0 = lds128(wt + r_lo * 128 + (((2 * t) ^ g) << 4));
-      const uint4 wl1 = lds128(wt + r_lo * 128 + (((2 * t + 1) ^ g) << 4));
-      const uint4 wh0 = lds128(wt + (r_lo + 8) * 128 + (((2 * t) ^ g) << 4));
-      const uint4 wh1 = lds128(wt + (r_lo + 8) * 128 + (((2 * t + 1) ^ g) << 4));
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // the weights are in registers
+      for (int i = 0; i < nst; ++i) {
+        const int it = r * nst + i;
+        const int slot = it % nring;
+        const bool got = mbar_wait(bar0 + 8 * slot, (it / nring) & 1, ctl);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        const uint32_t wt = ring + slot * kGvStageBytes;
+        // 128-byte swizzle: chunk c of row r sits at chunk position c ^ (r & 7); r & 7 == g here.
+        const uint4 wl0 = lds128(wt + r_lo * 128 + (((2 * t) ^ g) << 4));
+        const uint4 wl1 = lds128(wt + r_lo * 128 + (((2 * t + 1) ^ g) << 4));
+        const uint4 wh0 = lds128(wt + (r_lo + 8) * 128 + (((2 * t) ^ g) << 4));
+        const uint4 wh1 = lds128(wt + (r_lo + 8) * 128 + (((2 * t + 1) ^ g) << 4));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // the weights are in registers
 
-      const int qblk = i * 4 + t;  // this lane's 128-input block of the staged activations
+        const int qblk = i * 4 + t;  // this lane's 128-input block of the staged activations
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint4 wl = h ? wl1 : wl0, wh = h ? wh1 : wh0;
+        for (int h = 0; h < 2; ++h) {
+          const uint4 wl = h ? wl1 : wl0, wh = h ? wh1 : wh0;
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-          const int c0 = 4 * h + 2 * p;  // activation chunks c0, c0+1 of block qblk
-          uint4 xa[TG], xb[TG];
+          for (int p = 0; p < 2; ++p) {
+            const int c0 = 4 * h + 2 * p;  // activation chunks c0, c0+1 of block qblk
+            uint4 xa[TG], xb[TG];
 #pragma unroll
-          for (int tg = 0; tg < TG; ++tg) {
-            const int m = tg * 8 + g;
-            if (m < M) {
-              const uint32_t row = xs + m * x_pitch + qblk * 128;
-              xa[tg] = lds128(row + (((c0 + 2 * t) & 7) << 4));
-              xb[tg] = lds128(row + (((c0 + 1 + 2 * t) & 7) << 4));
-            } else {
-              xa[tg] = make_uint4(0, 0, 0, 0);
-              xb[tg] = make_uint4(0, 0, 0, 0);
+            for (int tg = 0; tg < TG; ++tg) {
+              const int m = tg * 8 + g;
+              if (m < M) {
+                const uint32_t row = xs + m * x_pitch + qblk * 128;
+                xa[tg] = lds128(row + (((c0 + 2 * t) & 7) << 4));
+                xb[tg] = lds128(row + (((c0 + 1 + 2 * t) & 7) << 4));
+              } else {
+                xa[tg] = make_uint4(0, 0, 0, 0);
+                xb[tg] = make_uint4(0, 0, 0, 0);
+              }
+            }
+            const uint32_t lo0 = u4_get(wl, 2 * p), lo1 = u4_get(wl, 2 * p + 1);
+            const uint32_t hi0 = u4_get(wh, 2 * p), hi1 = u4_get(wh, 2 * p + 1);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t mask = 0x03030303u << (2 * j);
+              const uint32_t a0 = lo0 & mask, a1 = hi0 & mask, a2 = lo1 & mask, a3 = hi1 & mask;
+#pragma unroll
+              for (int tg = 0; tg < TG; ++tg)
+                mma_u8s8_16x8x32(d[tg][j], a0, a1, a2, a3, u4_get(xa[tg], j), u4_get(xb[tg], j));
             }
           }
-          const uint32_t lo0 = u4_get(wl, 2 * p), lo1 = u4_get(wl, 2 * p + 1);
-          const uint32_t hi0 = u4_get(wh, 2 * p), hi1 = u4_get(wh, 2 * p + 1);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t mask = 0x03030303u << (2 * j);
-            const uint32_t a0 = lo0 & mask, a1 = hi0 & mask, a2 = lo1 & mask, a3 = hi1 & mask;
-#pragma unroll
-            for (int tg = 0; tg < TG; ++tg)
-              mma_u8s8_16x8x32(d[tg][j], a0, a1, a2, a3, u4_get(xa[tg], j), u4_get(xb[tg], j));
-          }
         }
+      }
+#pragma unroll
+      for (int tg = 0; tg < TG; ++tg)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int m = tg * 8 + 2 * t + (c & 1);
+          acc[tg][c] = d[tg][0][c] + (d[tg][1][c] >> 2) + (d[tg][2][c] >> 4) + (d[tg][3][c] >> 6) -
+                       (m < M ? rs_tok[m] : 0);
+        }
+      if (!clustered && ok) {
+        // All of K is in registers: finish the row block.
+        const int n_base = (rb0 + r * rb_step) * kGvRows;
+#pragma unroll
+        for (int tg = 0; tg < TG; ++tg)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int n = n_base + r_lo + ((c & 2) ? 8 : 0);
+            const int m = tg * 8 + 2 * t + (c & 1);
+            if (n < N && m < M) {
+              const float v = __fmul_rn(static_cast<float>(acc[tg][c]), __fdiv_rn(gamma, s_tok[m]));
+              const size_t o = static_cast<size_t>(m) * N + n;
+              if constexpr (sizeof(TY) == 4) y[o] = v; else y[o] = __float2bfloat16_rn(v);
+              if (acc_out) acc_out[o] = acc[tg][c];
+            }
+          }
       }
     }
-#pragma unroll
-    for (int tg = 0; tg < TG; ++tg)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int m = tg * 8 + 2 * t + (c & 1);
-        acc[tg][c] = d[tg][0][c] + (d[tg][1][c] >> 2) + (d[tg][2][c] >> 4) + (d[tg][3][c] >> 6) -
-                     (m < M ? rs_tok[m] : 0);
-      }
   }
 
+  if (!clustered) return;  // (a wait that ran out is in the status word; outputs are then unspecified)
   const float gamma = __ldg(gamma_ptr);
-  const int n_base = rb * kGvRows;
-
-  if (splits == 1) {
-    // Consumers only (the producer has left); all of K is in registers.
-    consumer_sync();
-    if (*abort_flag || !ok) return;  // the status word records it; no output is written
-#pragma unroll
-    for (int tg = 0; tg < TG; ++tg)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int n = n_base + r_lo + ((c & 2) ? 8 : 0);
-        const int m = tg * 8 + 2 * t + (c & 1);
-        if (n < N && m < M) {
-          const float v = __fmul_rn(static_cast<float>(acc[tg][c]), __fdiv_rn(gamma, s_tok[m]));
-          const size_t o = static_cast<size_t>(m) * N + n;
-          if constexpr (sizeof(TY) == 4) y[o] = v; else y[o] = __float2bfloat16_rn(v);
-          if (acc_out) acc_out[o] = acc[tg][c];
-        }
-      }
-    return;
-  }
+  const int n_base = rb0 * kGvRows;
 
   // ---- split K: the cluster's blocks add their partial sums through distributed shared memory ----
   if (warp < kGvWarps) {
@@ -403,7 +419,7 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(
       for (int c = 0; c < 4; ++c) {
         const int r = r_lo + ((c & 2) ? 8 : 0);
         const int m = tg * 8 + 2 * t + (c & 1);
-        red_buf[r * TT + m] = acc[tg][c];
+        if (m < TT) red_buf[r * TT + m] = acc[tg][c];
       }
   }
   cluster_sync_all();  // every thread of every block of the cluster arrives here
@@ -432,44 +448,84 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
+static int token_slots(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
+
 static int gemv_smem_bytes(int M, int tt, int ring, int x_pitch) {
   return ring * kGvStageBytes + ((M * x_pitch + 127) / 128) * 128 + kGvRows * tt * 4 + 2 * tt * 4 +
          kGvWarps * tt * 4 + 16 * ring + 64 + 1024;
 }
 
+// Modelled time (us) of a plan: the busiest SM streams its bytes at the rate its
+// stages in flight allow (Little's law, ~1.5 us latency) or at its share of HBM,
+// plus a per-block start-up cost per wave and the cluster reduction.
+static double gemv_plan_cost(long long busiest_bytes, long long total_bytes, int in_flight_stages, int sms,
+                             long long waves, int splits) {
+  const double hbm = 6.5e6;     // bytes per us
+  const double latency = 1.5;   // us
+  const double per_sm_rate = in_flight_stages * static_cast<double>(kGvStageBytes) / latency;
+  double t = static_cast<double>(busiest_bytes) / per_sm_rate;
+  const double floor_t = static_cast<double>(total_bytes) / hbm;
+  if (t < floor_t) t = floor_t;
+  t += 2.0 * static_cast<double>(waves);
+  if (splits > 1) t += 1.0;
+  (void)sms;
+  return t;
+}
+
+static int env_int(const char* name) {
+  const char* v = getenv(name);
+  return v ? atoi(v) : 0;
+}
+
 static GemvPlan plan_gemv_budget(int M, int N, int K, int x_budget) {
   const int sms = num_sms();
-  const int tt = M <= 8 ? 8 : 16;
+  // Tuning knobs: pin the K split and / or the ring depth the model would choose.
+  const int force_s = env_int("BITLINEAR_GEMV_SPLITS");
+  const int force_ring = env_int("BITLINEAR_GEMV_RING");
+  const int tt = token_slots(M);
   GemvPlan best{};
   double best_cost = 1e30;
   const int n_rb = (N + kGvRows - 1) / kGvRows;
   const int n_st = (K + kGvStageK - 1) / kGvStageK;
+  const long long total = static_cast<long long>(n_rb) * n_st * kGvStageBytes;
   for (int s = 1; s <= n_st && s <= kGemvMaxSplits; ++s) {
     const int spc = (n_st + s - 1) / s;
     const int s_eff = (n_st + spc - 1) / spc;
     if (s_eff != s) continue;
+    if (force_s > 0 && s != force_s) continue;
     const int x_pitch = ((spc * kGvStageK + 127) / 128) * 128 + 16;
     if (M * x_pitch > x_budget) continue;
-    for (int ring : {2, 3, 4, 6}) {
+    for (int ring : {2, 3, 4, 6, 8}) {
       if (ring > spc && ring != 2) continue;
+      if (force_ring > 0 && ring != force_ring && !(ring == 2 && force_ring > spc)) continue;
       const int r_eff = ring < spc ? ring : spc;
       const int smem = gemv_smem_bytes(M, tt, r_eff, x_pitch);
       if (smem > 227 * 1024) continue;
       int occ = (227 * 1024) / smem;
       if (occ > 2048 / kGvThreads) occ = 2048 / kGvThreads;
-      const long long ctas = static_cast<long long>(n_rb) * s;
       const long long slots = static_cast<long long>(sms) * occ;
-      const long long per_sm = (ctas + sms - 1) / sms;
-      const long long waves = (ctas + slots - 1) / slots;
-      const int in_flight = static_cast<int>(per_sm < occ ? per_sm : occ) * r_eff;
-      // Stages the busiest SM streams, a little extra per split for the reduction,
-      // a penalty for a short tail wave and for too few stages in flight per SM.
-      double cost = static_cast<double>(per_sm * spc) * (1.0 + 0.03 * (s - 1));
-      if (waves > 1 && waves < 4) cost *= 1.1;
-      if (in_flight < 3 && spc >= 3) cost *= 1.25;
+      long long ctas, busiest;
+      int in_flight;
+      long long waves;
+      if (s == 1) {
+        // Persistent blocks over all of K: as many as fit at once, up to one per row block.
+        ctas = n_rb < slots ? n_rb : slots;
+        const long long per_sm = (ctas + sms - 1) / sms;
+        const long long rb_per_cta = (n_rb + ctas - 1) / ctas;
+        busiest = per_sm * rb_per_cta * n_st * kGvStageBytes;
+        in_flight = static_cast<int>(per_sm) * r_eff;
+        waves = 1;
+      } else {
+        ctas = static_cast<long long>(n_rb) * s;
+        const long long per_sm = (ctas + sms - 1) / sms;
+        busiest = per_sm * spc * kGvStageBytes;
+        waves = (ctas + slots - 1) / slots;
+        in_flight = static_cast<int>(per_sm < occ ? per_sm : occ) * r_eff;
+      }
+      const double cost = gemv_plan_cost(busiest, total, in_flight, sms, waves, s);
       if (cost < best_cost - 1e-9) {
         best_cost = cost;
-        best = GemvPlan{n_rb, n_st, s, spc, r_eff, x_pitch, smem};
+        best = GemvPlan{n_rb, n_st, s, spc, r_eff, x_pitch, smem, static_cast<int>(ctas)};
       }
     }
   }
@@ -484,7 +540,7 @@ GemvPlan plan_gemv(int M, int N, int K) {
 
 bool gemv_fuses_quant(int M, int K) { return static_cast<long long>(M) * K <= kGvFuseLimit; }
 
-template <int TG, typename TY, typename TX>
+template <int TT, typename TY, typename TX>
 static cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, cudaStream_t stream, bool pdl) {
   EncodeTiledFn enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
   if (!enc) return cudaErrorNotSupported;
@@ -494,11 +550,11 @@ static cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, cudaStrea
   const cuuint32_t box[2] = {128, kGvRows};
   const cuuint32_t estr[2] = {1, 1};
   if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.packed), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
     return cudaErrorInvalidValue;
   }
-  auto kernel = gemv_kernel<TG, TY, TX>;
+  auto kernel = gemv_kernel<TT, TY, TX>;
   static bool attr_set = false;  // per template instance
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
@@ -506,17 +562,19 @@ static cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, cudaStrea
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.n_rb * p.splits);
+  cfg.gridDim = dim3(p.grid);
   cfg.blockDim = dim3(kGvThreads);
   cfg.dynamicSmemBytes = static_cast<size_t>(p.smem);
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   int n = 0;
-  attr[n].id = cudaLaunchAttributeClusterDimension;
-  attr[n].val.clusterDim.x = p.splits;
-  attr[n].val.clusterDim.y = 1;
-  attr[n].val.clusterDim.z = 1;
-  ++n;
+  if (p.splits > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = p.splits;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
   if (pdl) {
     attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[n].val.programmaticStreamSerializationAllowed = 1;
@@ -529,24 +587,31 @@ static cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, cudaStrea
                             a.status);
 }
 
-template <int TG, typename TY>
+template <int TT, typename TY>
 static cudaError_t launch_gemv_x(const GemvArgs& a, const GemvPlan& p, cudaStream_t stream, bool pdl) {
   switch (a.x_type) {
-    case kInBF16: return launch_gemv_t<TG, TY, __nv_bfloat16>(a, p, stream, pdl);
-    case kInF32: return launch_gemv_t<TG, TY, float>(a, p, stream, pdl);
-    default: return launch_gemv_t<TG, TY, int8_t>(a, p, stream, pdl);
+    case kInBF16: return launch_gemv_t<TT, TY, __nv_bfloat16>(a, p, stream, pdl);
+    case kInF32: return launch_gemv_t<TT, TY, float>(a, p, stream, pdl);
+    default: return launch_gemv_t<TT, TY, int8_t>(a, p, stream, pdl);
+  }
+}
+
+template <typename TY>
+static cudaError_t launch_gemv_y(const GemvArgs& a, const GemvPlan& p, cudaStream_t stream, bool pdl) {
+  switch (token_slots(a.M)) {
+    case 1: return launch_gemv_x<1, TY>(a, p, stream, pdl);
+    case 2: return launch_gemv_x<2, TY>(a, p, stream, pdl);
+    case 4: return launch_gemv_x<4, TY>(a, p, stream, pdl);
+    case 8: return launch_gemv_x<8, TY>(a, p, stream, pdl);
+    default: return launch_gemv_x<16, TY>(a, p, stream, pdl);
   }
 }
 
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t stream, bool pdl) {
   const GemvPlan p = plan_gemv(a.M, a.N, a.K);
   if (p.splits == 0) return cudaErrorInvalidConfiguration;
-  if (a.M <= 8) {
-    return a.y_type == kOutBF16 ? launch_gemv_x<1, __nv_bfloat16>(a, p, stream, pdl)
-                                : launch_gemv_x<1, float>(a, p, stream, pdl);
-  }
-  return a.y_type == kOutBF16 ? launch_gemv_x<2, __nv_bfloat16>(a, p, stream, pdl)
-                              : launch_gemv_x<2, float>(a, p, stream, pdl);
+  return a.y_type == kOutBF16 ? launch_gemv_y<__nv_bfloat16>(a, p, stream, pdl)
+                              : launch_gemv_y<float>(a, p, stream, pdl);
 }
 
 }  // namespace bl

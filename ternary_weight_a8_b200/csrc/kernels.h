@@ -72,7 +72,7 @@ struct GemvArgs {
 
 // Decode kernel launch plan: blocks of 128 rows; K split over a cluster of `splits` blocks.
 struct GemvPlan {
-  int n_rb, n_st, splits, st_per_split, nring, x_pitch, smem;
+  int n_rb, n_st, splits, st_per_split, nring, x_pitch, smem, grid;
 };
 GemvPlan plan_gemv(int M, int N, int K);
 bool gemv_fuses_quant(int M, int K);
