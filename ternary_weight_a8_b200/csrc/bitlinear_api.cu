@@ -90,10 +90,13 @@ FwdLayout forward_layout(int M, int K) {
     if (_rc != BL_OK) return _rc; \
   } while (0)
 
-// The product kernel for this call: the decode GEMV for M <= 16 (unless its
-// activations do not fit on chip), else the tensor-core GEMM; bitlinear_set_path
+// Bytes [16, 24) of the status block: the decode kernel's ticket counters.
+uint32_t* tickets_of(void* ws) { return reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + 16); }
+
+// The product kernel for M tokens: the decode GEMV for M <= 16 (when its
+// activations fit on chip), else the tensor-core GEMM; bitlinear_set_path
 // overrides the choice on the calling thread.
-int choose_gemv(int M, int N, int K, bool* gemv) {
+int choose_gemv(int M, int K, bool* gemv) {
   bool v = M <= 16;
   if (g_path == 1) {
     if (M > 16) return fail(BL_ERR_UNSUPPORTED_SHAPE, "GEMV path forced with M = %d > 16", M);
@@ -101,7 +104,7 @@ int choose_gemv(int M, int N, int K, bool* gemv) {
   } else if (g_path == 2) {
     v = false;
   }
-  if (v && bl::plan_gemv(M, N, K).splits == 0) {
+  if (v && !bl::gemv_supported(M, K)) {
     if (g_path == 1)
       return fail(BL_ERR_UNSUPPORTED_SHAPE, "GEMV path forced but M*K = %lld does not fit on chip",
                   static_cast<long long>(M) * K);
@@ -111,48 +114,16 @@ int choose_gemv(int M, int N, int K, bool* gemv) {
   return BL_OK;
 }
 
-int launch_product(bool gemv, const uint8_t* packed, const float* gamma, int N, int K, int M, const int8_t* xq,
-                   const float* scale, const int32_t* rowsum, void* y, int y_dtype, int32_t* acc_out,
-                   uint32_t* status, cudaStream_t s) {
-  const int yt = y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32;
-  cudaError_t e;
-  if (gemv) {
-    bl::GemvArgs a{packed, gamma, N, K, M, xq, bl::kInInt8, scale, y, yt, acc_out, status};
-    e = bl::launch_gemv(a, s, true);
-  } else {
-    bl::ProductArgs a{packed, gamma, N, K, M, xq, scale, rowsum, y, yt, acc_out, status};
-    e = bl::launch_gemm(a, s, true);
-  }
-  if (e != cudaSuccess) return cuda_fail(e, gemv ? "GEMV launch" : "GEMM launch");
-  return BL_OK;
-}
+int gemv_fail(cudaError_t e) { return cuda_fail(e, "GEMV launch"); }
 
-// One forward on raw activations.  *xq_valid tells whether the workspace
-// already holds this x quantised (a chain's layers that share their input);
-// it is updated when this call quantises x into the workspace.
-int forward_one(const uint8_t* packed, const float* gamma, int N, int K, const void* x, int x_dtype, int M,
-                void* y, int y_dtype, int32_t* acc_out, uint8_t* ws, const FwdLayout& l, bool* xq_valid,
-                cudaStream_t s) {
-  bool gemv = false;
-  BL_TRY(choose_gemv(M, N, K, &gemv));
-  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
-  if (gemv && bl::gemv_fuses_quant(M, K)) {
-    // Small activations: the GEMV blocks quantise them on chip (one launch, no round trip).
-    bl::GemvArgs a{packed, gamma, N, K, M, x, x_dtype == BL_BF16 ? bl::kInBF16 : bl::kInF32, nullptr, y,
-                   y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32, acc_out, status};
-    cudaError_t e = bl::launch_gemv(a, s, true);
-    if (e != cudaSuccess) return cuda_fail(e, "GEMV launch");
-    return BL_OK;
-  }
-  int8_t* xq = reinterpret_cast<int8_t*>(ws + l.xq);
-  float* scale = reinterpret_cast<float*>(ws + l.scale);
-  int32_t* rowsum = reinterpret_cast<int32_t*>(ws + l.rowsum);
-  if (!*xq_valid) {
-    cudaError_t e = bl::launch_act_quant(x, x_dtype == BL_BF16, M, K, xq, scale, rowsum, s, true);
-    if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
-    *xq_valid = true;
-  }
-  return launch_product(gemv, packed, gamma, N, K, M, xq, scale, rowsum, y, y_dtype, acc_out, status, s);
+int launch_gemm_q(const uint8_t* packed, const float* gamma, int N, int K, int M, const int8_t* xq,
+                  const float* scale, const int32_t* rowsum, void* y, int y_dtype, int32_t* acc_out,
+                  uint32_t* status, cudaStream_t s) {
+  bl::ProductArgs a{packed, gamma, N, K, M, xq, scale, rowsum, y, y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32,
+                    acc_out, status};
+  cudaError_t e = bl::launch_gemm(a, s, true);
+  if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
+  return BL_OK;
 }
 
 }  // namespace
@@ -271,9 +242,16 @@ int bitlinear_forward_quantized(const uint8_t* packed, const float* gamma, int N
   if (workspace_bytes < kStatusBytes)
     return fail(BL_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, kStatusBytes);
   bool gemv = false;
-  BL_TRY(choose_gemv(M, N, K, &gemv));
-  return launch_product(gemv, packed, gamma, N, K, M, xq, scale, rowsum, y, y_dtype, acc_out,
-                        static_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream));
+  BL_TRY(choose_gemv(M, K, &gemv));
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (gemv) {
+    const bl::GemvLayerArgs L{packed, gamma, N, K, xq, scale, y, acc_out};
+    cudaError_t e = bl::launch_gemv_group(&L, 1, M, bl::kInInt8, y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32,
+                                          status, tickets_of(workspace), s, true);
+    return e == cudaSuccess ? BL_OK : gemv_fail(e);
+  }
+  return launch_gemm_q(packed, gamma, N, K, M, xq, scale, rowsum, y, y_dtype, acc_out, status, s);
 }
 
 int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, const void* x,
@@ -293,17 +271,46 @@ int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, c
   const FwdLayout l = forward_layout(M, K);
   if (workspace_bytes < l.total)
     return fail(BL_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, l.total);
-  bool xq_valid = false;
-  return forward_one(packed, gamma, N, K, x, x_dtype, M, y, y_dtype, acc_out, static_cast<uint8_t*>(workspace),
-                     l, &xq_valid, static_cast<cudaStream_t>(stream));
+  bool gemv = false;
+  BL_TRY(choose_gemv(M, K, &gemv));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int yt = y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32;
+  if (gemv && bl::gemv_fuses_quant(M, K, x_dtype == BL_BF16)) {
+    // Small activations: the decode kernel quantises them itself (one launch).
+    const bl::GemvLayerArgs L{packed, gamma, N, K, x, nullptr, y, acc_out};
+    cudaError_t e = bl::launch_gemv_group(&L, 1, M, x_dtype == BL_BF16 ? bl::kInBF16 : bl::kInF32, yt, status,
+                                          tickets_of(workspace), s, true);
+    return e == cudaSuccess ? BL_OK : gemv_fail(e);
+  }
+  int8_t* xq = reinterpret_cast<int8_t*>(ws + l.xq);
+  float* scale = reinterpret_cast<float*>(ws + l.scale);
+  int32_t* rowsum = reinterpret_cast<int32_t*>(ws + l.rowsum);
+  cudaError_t e = bl::launch_act_quant(x, x_dtype == BL_BF16, M, K, xq, scale, rowsum, s, true);
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+  if (gemv) {
+    const bl::GemvLayerArgs L{packed, gamma, N, K, xq, scale, y, acc_out};
+    e = bl::launch_gemv_group(&L, 1, M, bl::kInInt8, yt, status, tickets_of(workspace), s, true);
+    return e == cudaSuccess ? BL_OK : gemv_fail(e);
+  }
+  return launch_gemm_q(packed, gamma, N, K, M, xq, scale, rowsum, y, y_dtype, acc_out, status, s);
 }
+
+// Every layer of a chain has its own activation region (the layers of one
+// decode group are live together): status block, then per layer q, s, rowsum.
+static size_t chain_region_bytes(int M, int K) { return forward_layout(M, K).total - kStatusBytes; }
 
 size_t bitlinear_chain_workspace_bytes(const bl_layer* layers, int n_layers, int M) {
   if (!layers || n_layers <= 0 || M < 0) return 0;
-  int k_max = 64;
-  for (int i = 0; i < n_layers; ++i)
-    if (layers[i].K > k_max) k_max = layers[i].K;
-  return forward_layout(M, k_max).total;
+  size_t total = kStatusBytes;
+  for (int i = 0; i < n_layers; ++i) total += chain_region_bytes(M, layers[i].K);
+  return total;
+}
+
+static bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
 }
 
 int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dtype, int y_dtype,
@@ -327,14 +334,99 @@ int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dty
   if (workspace_bytes < need)
     return fail(BL_ERR_WORKSPACE_TOO_SMALL, "chain workspace %zu < %zu bytes", workspace_bytes, need);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  bool xq_valid = false;
-  for (int i = 0; i < n_layers; ++i) {
-    const bl_layer& L = layers[i];
-    const bool shared_input = i > 0 && layers[i - 1].x == L.x && layers[i - 1].K == L.K;
-    if (!shared_input) xq_valid = false;
-    BL_TRY(forward_one(L.packed, L.gamma, L.N, L.K, L.x, x_dtype, M, L.y, y_dtype, nullptr, ws,
-                       forward_layout(M, L.K), &xq_valid, s));
+  const bool x_bf16 = x_dtype == BL_BF16;
+  const size_t xsz = x_bf16 ? 2 : 4, ysz = y_dtype == BL_BF16 ? 2 : 4;
+  const int yt = y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32;
+
+  // Activation region of each layer.
+  size_t off[64];
+  if (n_layers > 64) return fail(BL_ERR_INVALID_ARG, "n_layers = %d > 64", n_layers);
+  {
+    size_t o = kStatusBytes;
+    for (int i = 0; i < n_layers; ++i) {
+      off[i] = o;
+      o += chain_region_bytes(M, layers[i].K);
+    }
+  }
+  auto region = [&](int i, int8_t** xq, float** sc, int32_t** rs) {
+    const FwdLayout l = forward_layout(M, layers[i].K);
+    *xq = reinterpret_cast<int8_t*>(ws + off[i] + (l.xq - kStatusBytes));
+    *sc = reinterpret_cast<float*>(ws + off[i] + (l.scale - kStatusBytes));
+    *rs = reinterpret_cast<int32_t*>(ws + off[i] + (l.rowsum - kStatusBytes));
+  };
+  // quant_src[i]: the layer whose region holds layer i's quantised input.
+  int quant_src[64];
+  for (int i = 0; i < n_layers; ++i) quant_src[i] = -1;
+  auto quantise = [&](int i) -> int {
+    for (int j = 0; j < i; ++j)
+      if (quant_src[j] == j && layers[j].x == layers[i].x && layers[j].K == layers[i].K) {
+        quant_src[i] = j;  // same input already quantised earlier in this call
+        return BL_OK;
+      }
+    int8_t* xq;
+    float* sc;
+    int32_t* rsum;
+    region(i, &xq, &sc, &rsum);
+    cudaError_t e = bl::launch_act_quant(layers[i].x, x_bf16, M, layers[i].K, xq, sc, rsum, s, true);
+    if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+    quant_src[i] = i;
+    return BL_OK;
+  };
+
+  int i = 0;
+  while (i < n_layers) {
+    bool gemv = false;
+    BL_TRY(choose_gemv(M, layers[i].K, &gemv));
+    if (!gemv) {
+      BL_TRY(quantise(i));
+      int8_t* xq;
+      float* sc;
+      int32_t* rsum;
+      region(quant_src[i], &xq, &sc, &rsum);
+      BL_TRY(launch_gemm_q(layers[i].packed, layers[i].gamma, layers[i].N, layers[i].K, M, xq, sc, rsum,
+                           layers[i].y, y_dtype, nullptr, status, s));
+      ++i;
+      continue;
+    }
+    // A decode group: following layers that also take the GEMV path the same way
+    // and neither read what the group writes nor write what it reads.
+    const bool fused = bl::gemv_fuses_quant(M, layers[i].K, x_bf16);
+    int j = i + 1;
+    while (j < n_layers && j - i < bl::kGvMaxLayers) {
+      bool gj = false;
+      if (choose_gemv(M, layers[j].K, &gj) != BL_OK || !gj) break;
+      if (bl::gemv_fuses_quant(M, layers[j].K, x_bf16) != fused) break;
+      bool independent = true;
+      const size_t xj = static_cast<size_t>(M) * layers[j].K * xsz, yj = static_cast<size_t>(M) * layers[j].N * ysz;
+      for (int k = i; k < j && independent; ++k) {
+        const size_t xk = static_cast<size_t>(M) * layers[k].K * xsz, yk = static_cast<size_t>(M) * layers[k].N * ysz;
+        if (ranges_overlap(layers[j].x, xj, layers[k].y, yk) || ranges_overlap(layers[j].y, yj, layers[k].x, xk) ||
+            ranges_overlap(layers[j].y, yj, layers[k].y, yk))
+          independent = false;
+      }
+      if (!independent) break;
+      ++j;
+    }
+    bl::GemvLayerArgs args[bl::kGvMaxLayers];
+    for (int k = i; k < j; ++k) {
+      const bl_layer& L = layers[k];
+      if (fused) {
+        args[k - i] = bl::GemvLayerArgs{L.packed, L.gamma, L.N, L.K, L.x, nullptr, L.y, nullptr};
+      } else {
+        BL_TRY(quantise(k));
+        int8_t* xq;
+        float* sc;
+        int32_t* rsum;
+        region(quant_src[k], &xq, &sc, &rsum);
+        args[k - i] = bl::GemvLayerArgs{L.packed, L.gamma, L.N, L.K, xq, sc, L.y, nullptr};
+      }
+    }
+    const int xt = fused ? (x_bf16 ? bl::kInBF16 : bl::kInF32) : bl::kInInt8;
+    cudaError_t e = bl::launch_gemv_group(args, j - i, M, xt, yt, status, tickets_of(workspace), s, true);
+    if (e != cudaSuccess) return gemv_fail(e);
+    i = j;
   }
   return BL_OK;
 }

@@ -55,28 +55,24 @@ struct ProductArgs {
   uint32_t* status;
 };
 
-// Decode GEMV (M <= 16): activations as int8 codes with their scales, or raw
-// (fp32 / bf16) activations that the kernel quantises itself.
-struct GemvArgs {
+// Decode GEMV (M <= 16) over a group of independent layers in one launch.
+// Each layer's activations are raw (fp32 / bf16, quantised in the kernel) or
+// int8 codes with their token scales; x_type is the same for the whole group.
+struct GemvLayerArgs {
   const uint8_t* packed;
   const float* gamma;
-  int N, K, M;
+  int N, K;
   const void* x;
-  int x_type;           // InType
-  const float* scale;   // token scales when x_type == kInInt8
+  const float* scale;  // token scales when the activations are int8 codes
   void* y;
-  int y_type;           // OutType
   int32_t* acc_out;
-  uint32_t* status;
 };
-
-// Decode kernel launch plan: blocks of 128 rows; K split over a cluster of `splits` blocks.
-struct GemvPlan {
-  int n_rb, n_st, splits, st_per_split, nring, x_pitch, smem, grid;
-};
-GemvPlan plan_gemv(int M, int N, int K);
-bool gemv_fuses_quant(int M, int K);
-constexpr int kGemvMaxSplits = 8;
+constexpr int kGvMaxLayers = 8;
+bool gemv_supported(int M, int K);
+bool gemv_fuses_quant(int M, int K, int x_bf16);
+// tickets: two zero-initialised uint32 in device memory (reset by the kernel after use).
+cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, int x_type, int y_type,
+                              uint32_t* status, uint32_t* tickets, cudaStream_t stream, bool pdl);
 
 // cuTensorMapEncodeTiled from the driver (no link-time dependency on libcuda).
 #ifdef CUDA_VERSION
@@ -86,7 +82,6 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 #endif
 void* tensor_map_encoder();
-cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t stream, bool pdl);
 cudaError_t launch_gemm(const ProductArgs& a, cudaStream_t stream, bool pdl);
 
 // Self-test of the bounded device wait.

@@ -74,7 +74,9 @@ def test_workspace_layout(L):
     layers = (tb.bl_layer * 2)()
     layers[0].N, layers[0].K = 10240, 8192
     layers[1].N, layers[1].K = 8192, 28672
-    assert L.bitlinear_chain_workspace_bytes(layers, 2, 8) == tb.workspace_bytes(8, 8192, 28672)
+    # a chain gives every layer its own q, s, rowsum region (a decode group's layers run together)
+    per_layer = lambda K: tb.workspace_bytes(8, 0, K) - 256
+    assert L.bitlinear_chain_workspace_bytes(layers, 2, 8) == 256 + per_layer(8192) + per_layer(28672)
 
 
 def test_binding_fails_loudly_without_library(monkeypatch):
