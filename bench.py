@@ -254,26 +254,6 @@ def timed_graph_run(step_fn, steps, warmup, world, chunk=500, sampler=None):
     return max_over_ranks(secs, world), clocks
 
 
-def kernel_event_times(launch_pre, launch_kernel, steps, batch=100):
-    """Average device duration of one kernel, timed with events on its launching stream.
-
-    Each batch of launches is queued behind a spin of the stream, so the
-    events bracket the kernel's execution rather than the host's launch gaps."""
-    import torch
-
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    for b0 in range(0, steps, batch):
-        torch.cuda._sleep(int(20e6))  # ~10 ms: longer than enqueueing one batch
-        for i in range(b0, min(steps, b0 + batch)):
-            launch_pre(i)
-            evs[i][0].record()
-            launch_kernel(i)
-            evs[i][1].record()
-        torch.cuda.synchronize()
-    t = [a.elapsed_time(b) / 1e3 for a, b in evs]
-    return statistics.mean(t), statistics.median(t)
-
-
 # ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
@@ -292,34 +272,32 @@ def run_ours(args, world, rank, local):
     sets, set_bytes = make_layer_sets(DECODE_LAYERS, seed=0, min_bytes=4 * L2)
     nsets = len(sets)
     xs, ys = make_inputs(DECODE_LAYERS, 1, seed=0)
-    ws = tb.new_workspace(max(tb.workspace_bytes(1, N, K) for K, N in DECODE_LAYERS))
+    layer_sets = [[tb.Layer(p, g, x, y) for (p, g), x, y in zip(S, xs, ys)] for S in sets]
+    ws = tb.new_workspace(tb.chain_workspace_bytes(layer_sets[0], 1))
 
     def decode_step(i):
-        S = sets[i % nsets]
-        for (packed, gamma), x, y in zip(S, xs, ys):
-            tb.forward(packed, gamma, x, y=y, workspace=ws)
+        # Both BitLinears of the step in one call; independent layers share one launch.
+        tb.layer_chain(layer_sets[i % nsets], workspace=ws)
 
     sampler = ClockSampler(torch.cuda.current_device())
     secs, clocks = timed_graph_run(decode_step, args.steps, args.warmup, world, sampler=sampler)
     units = args.steps * set_bytes * world
     value = units / secs / 1e9
-    launches = args.steps * len(DECODE_LAYERS)  # one fused GEMV launch per layer at one token
+    launches = args.steps  # one decode kernel per step
     status = tb.device_status(ws)
 
-    # roofline of the dominant kernel: the GEMV of the N=6912 layer (at one token it
-    # quantises its activations itself, so the forward is this one kernel), timed per launch
-    K0, N0 = DECODE_LAYERS[0]
-    nk = min(args.steps, 3000)
-    mean_s, med_s = kernel_event_times(
-        lambda i: None,
-        lambda i: tb.forward(sets[i % nsets][0][0], sets[i % nsets][0][1], xs[0], y=ys[0], workspace=ws), nk)
-    gemv_bytes = N0 * K0 // 4 + K0 + N0 * 2 + 16
-    achieved = gemv_bytes / mean_s / 1e9
-    roofline = {"bound": "hbm", "kernel": "gemv_kernel (K=2560, N=6912, 1 token)", "achieved": round(achieved, 1),
-                "peak": peaks["hbm"], "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
-                "peak_source": peaks["source"], "traffic": None,
-                "algorithmic_bytes_per_launch": gemv_bytes, "launch_us_mean": round(mean_s * 1e6, 3),
-                "launch_us_median": round(med_s * 1e6, 3)}
+    # Roofline of the dominant kernel: the decode kernel is the whole step, so its
+    # average launch duration is the timed region over the launches in it.
+    x_bytes = sum(K * 2 for K, N in DECODE_LAYERS)
+    y_bytes = sum(N * 2 for K, N in DECODE_LAYERS)
+    step_bytes = set_bytes + x_bytes + y_bytes + 8 * len(DECODE_LAYERS)
+    per_launch = secs / world / launches * world  # seconds per launch on one GPU
+    achieved = step_bytes / per_launch / 1e9
+    roofline = {"bound": "hbm", "kernel": "gemv_group_kernel (decode 2B step: K=2560 -> N=6912 and N=2560, 1 token)",
+                "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm"], 4), "peak_source": peaks["source"] + " HBM copy",
+                "traffic": None, "algorithmic_bytes_per_launch": step_bytes,
+                "launch_us_mean": round(per_launch * 1e6, 3)}
 
     # ---- e2e through the public API with host buffers ----
     x_host = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in xs]
@@ -332,10 +310,10 @@ def run_ours(args, world, rank, local):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for i in range(ne):
-        S = sets[i % nsets]
-        for (packed, gamma), xh, x, y, yh in zip(S, x_host, xs, ys, y_host):
+        for xh, x in zip(x_host, xs):
             x.copy_(xh, non_blocking=True)
-            tb.forward(packed, gamma, x, y=y, workspace=ws)
+        tb.layer_chain(layer_sets[i % nsets], workspace=ws)
+        for y, yh in zip(ys, y_host):
             yh.copy_(y, non_blocking=True)
         torch.cuda.current_stream().synchronize()  # the step's result is on the host
     e1.record()
@@ -345,7 +323,7 @@ def run_ours(args, world, rank, local):
            "h2d_bytes_per_step": sum(x.numel() * 2 for x in xs),
            "d2h_bytes_per_step": sum(y.numel() * 2 for y in ys), "steps": ne,
            "ms_per_step": round(e2e_secs / ne * 1e3, 4)}
-    del sets
+    del sets, layer_sets
 
     if not args.no_extras:
         out["prefill"] = run_prefill(args, world, peaks, L2)
@@ -395,13 +373,13 @@ def run_prefill(args, world, peaks, L2):
     secs, _ = timed_graph_run(step, steps, 20, world, chunk=100)
     ops = 2.0 * M * N * K
     tops = ops * steps * world / secs / 1e12
-    xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
-    sc = torch.empty(M, dtype=torch.float32, device="cuda")
-    rs = torch.empty(M, dtype=torch.int32, device="cuda")
-    mean_s, med_s = kernel_event_times(
-        lambda i: tb.quant_act(xs[i % len(xs)], xq, sc, rs),
+    # Roofline of the GEMM alone: a graph of back-to-back GEMM launches on quantised input.
+    xq, sc, rs = tb.quant_act(xs[0])
+    gsteps = 200
+    gsecs, _ = timed_graph_run(
         lambda i: tb.forward_quantized(sets[i % len(sets)][0][0], sets[i % len(sets)][0][1], xq, sc, rs, y=y,
-                                       workspace=ws), 100)
+                                       workspace=ws), gsteps, 10, world, chunk=100)
+    mean_s = gsecs / gsteps
     peak_int8 = peaks["bf16"] * INT8_PER_BF16
     k_tops = ops / mean_s / 1e12
     status = tb.device_status(ws)
@@ -411,7 +389,7 @@ def run_prefill(args, world, peaks, L2):
             "roofline": {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 kind::i8)", "achieved": round(k_tops, 1),
                          "peak": peak_int8, "unit": "TOPS", "frac": round(k_tops / peak_int8, 4),
                          "peak_source": "%s bf16 burst x %.0f (nominal int8/bf16 ratio)" % (peaks["source"], INT8_PER_BF16),
-                         "launch_us_mean": round(mean_s * 1e6, 2), "launch_us_median": round(med_s * 1e6, 2),
+                         "launch_us_mean": round(mean_s * 1e6, 2),
                          "traffic": None},
             "pct_int8_nominal_4500": round(100 * tops / world / 4500.0, 2), "device_status": status}
 
