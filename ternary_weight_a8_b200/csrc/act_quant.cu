@@ -1,4 +1,4 @@
-// Per-token 8-bit activation quantisation.
+// Per-token 8-bit activation quantisation, for one input or several at once.
 //
 // "BitNet's Real Bet: Designing the Whole Inference Stack", section "A
 // low-bit model is a whole-stack design": activations take a separate
@@ -6,11 +6,13 @@
 // quantised dynamically.  Reading (the pages print no formula): symmetric
 // absmax, s = 127 / max(amax, 1e-5), q = clamp(rint(x * s), -128, 127), in
 // fp32 with round-half-to-even.  The kernel also writes sum_k q[m][k], which
-// the product kernels use to turn sums over the stored codes c = t + 1 into
+// the tensor-core GEMM uses to turn sums over the stored codes c = t + 1 into
 // sums over t.
 //
-// One block per token; the token is read twice (absmax, then quantise), the
-// second time from L1/L2.
+// One block per (input, token).  A token of up to 32768 inputs is read once
+// into registers (16-input chunks, up to four per thread): block absmax,
+// then quantise from registers, pack four codes per word with byte permutes
+// and add the codes with dp4a.  Longer tokens are read a second time.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -18,95 +20,181 @@
 
 namespace bl {
 
-constexpr int kQuantThreads = 256;
+constexpr int kQuantMaxThreads = 512;
+constexpr int kQuantRegChunks = 4;
 
-struct Vec8 {
-  float v[8];
+struct QuantItem {
+  const void* x;
+  int8_t* xq;  // rows of ldq bytes; [K, ldq) is written as zeros
+  float* scale;
+  int32_t* rowsum;
+  int K, ldq;
 };
 
-__device__ __forceinline__ Vec8 load8(const float* p) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  return Vec8{{a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w}};
+struct QuantParams {
+  QuantItem item[kQuantMaxItems];
+  int n_items;
+};
+
+struct Chunk16 {
+  uint4 v[4];  // bf16: v[0..1]; fp32: v[0..3]
+};
+
+template <typename TX>
+__device__ __forceinline__ void load16(const TX* p, Chunk16& r) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+  r.v[0] = __ldcg(q);
+  r.v[1] = __ldcg(q + 1);
+  if constexpr (sizeof(TX) == 4) {
+    r.v[2] = __ldcg(q + 2);
+    r.v[3] = __ldcg(q + 3);
+  }
 }
 
-__device__ __forceinline__ Vec8 load8(const __nv_bfloat16* p) {
-  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-  Vec8 r;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    r.v[2 * i] = __uint_as_float(w[i] << 16);            // low half: element 2i
-    r.v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);  // high half: element 2i+1
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+template <typename TX>
+__device__ __forceinline__ float elem(const Chunk16& r, int e) {
+  if constexpr (sizeof(TX) == 4) {
+    return __uint_as_float(word_of(r.v[e >> 2], e & 3));
+  } else {
+    const uint32_t w = word_of(r.v[e >> 3], (e >> 1) & 3);  // bf16 -> fp32 is exact
+    return __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
   }
-  return r;
+}
+
+template <typename TX>
+__device__ __forceinline__ float chunk_absmax(const Chunk16& r) {
+  float a = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) a = fmaxf(a, fabsf(elem<TX>(r, e)));
+  return a;
+}
+
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+  const uint32_t lo = __byte_perm(static_cast<uint32_t>(a), static_cast<uint32_t>(b), 0x5140);
+  const uint32_t hi = __byte_perm(static_cast<uint32_t>(c), static_cast<uint32_t>(d), 0x5140);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
+// q for the 16 inputs of a chunk, written as one 16-byte store; returns sum q.
+template <typename TX>
+__device__ __forceinline__ int quant_chunk(const Chunk16& r, float s, int8_t* dst) {
+  uint32_t w[4];
+  int sum = 0;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    int q[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      q[e] = __float2int_rn(__fmul_rn(elem<TX>(r, 4 * b + e), s));
+      q[e] = min(max(q[e], -128), 127);
+    }
+    w[b] = pack4(q[0], q[1], q[2], q[3]);
+    sum = __dp4a(static_cast<int>(w[b]), 0x01010101, sum);
+  }
+  *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  return sum;
 }
 
 template <typename T, typename Op>
 __device__ __forceinline__ T block_reduce(T v, Op op, T* smem) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   if (lane == 0) smem[warp] = v;
   __syncthreads();
   T r = smem[0];
-  for (int i = 1; i < kQuantThreads / 32; ++i) r = op(r, smem[i]);
+  for (int i = 1; i < nw; ++i) r = op(r, smem[i]);
   __syncthreads();
   return r;
 }
 
 template <typename TX>
-__global__ void __launch_bounds__(kQuantThreads) act_quant_kernel(const TX* __restrict__ x, int K,
-                                                                  int8_t* __restrict__ xq,
-                                                                  float* __restrict__ scale,
-                                                                  int32_t* __restrict__ rowsum) {
-  __shared__ float red_f[kQuantThreads / 32];
-  __shared__ int red_i[kQuantThreads / 32];
+__global__ void __launch_bounds__(kQuantMaxThreads) act_quant_kernel(const __grid_constant__ QuantParams P) {
+  __shared__ float red_f[kQuantMaxThreads / 32];
+  __shared__ int red_i[kQuantMaxThreads / 32];
   griddep_launch_dependents();
-  griddep_wait();  // x may be the preceding kernel's output
+  griddep_wait();  // x may be the preceding kernel's output; q may still be read by it
 
-  const int m = blockIdx.x;
-  const TX* xr = x + static_cast<size_t>(m) * K;
-  int8_t* qr = xq + static_cast<size_t>(m) * K;
+  const QuantItem& it = P.item[blockIdx.y];
+  const int m = blockIdx.x, K = it.K, chunks = K >> 4, T = blockDim.x;
+  const TX* xr = static_cast<const TX*>(it.x) + static_cast<size_t>(m) * K;
+  int8_t* qr = it.xq + static_cast<size_t>(m) * it.ldq;
+  for (int c = K + 16 * threadIdx.x; c < it.ldq; c += 16 * T)  // row padding (K % 16 == 0)
+    *reinterpret_cast<uint4*>(qr + c) = make_uint4(0, 0, 0, 0);
+  const bool in_regs = chunks <= T * kQuantRegChunks;
 
+  Chunk16 reg[kQuantRegChunks];
   float amax = 0.0f;
-  for (int k = threadIdx.x * 8; k < K; k += kQuantThreads * 8) {
-    const Vec8 v = load8(xr + k);
+  if (in_regs) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v.v[i]));
+    for (int i = 0; i < kQuantRegChunks; ++i) {
+      const int c = threadIdx.x + i * T;
+      if (c < chunks) load16<TX>(xr + c * 16, reg[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < kQuantRegChunks; ++i) {
+      const int c = threadIdx.x + i * T;
+      if (c < chunks) amax = fmaxf(amax, chunk_absmax<TX>(reg[i]));
+    }
+  } else {
+    for (int c = threadIdx.x; c < chunks; c += T) {
+      Chunk16 r;
+      load16<TX>(xr + c * 16, r);
+      amax = fmaxf(amax, chunk_absmax<TX>(r));
+    }
   }
   amax = block_reduce(amax, [](float a, float b) { return fmaxf(a, b); }, red_f);
   const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
 
   int sum = 0;
-  for (int k = threadIdx.x * 8; k < K; k += kQuantThreads * 8) {
-    const Vec8 v = load8(xr + k);
-    uint32_t packed[2] = {0u, 0u};
+  if (in_regs) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      int q = __float2int_rn(__fmul_rn(v.v[i], s));
-      q = min(max(q, -128), 127);
-      sum += q;
-      packed[i >> 2] |= (static_cast<uint32_t>(q) & 0xffu) << (8 * (i & 3));
+    for (int i = 0; i < kQuantRegChunks; ++i) {
+      const int c = threadIdx.x + i * T;
+      if (c < chunks) sum += quant_chunk<TX>(reg[i], s, qr + c * 16);
     }
-    *reinterpret_cast<uint2*>(qr + k) = make_uint2(packed[0], packed[1]);
+  } else {
+    for (int c = threadIdx.x; c < chunks; c += T) {
+      Chunk16 r;
+      load16<TX>(xr + c * 16, r);
+      sum += quant_chunk<TX>(r, s, qr + c * 16);
+    }
   }
   sum = block_reduce(sum, [](int a, int b) { return a + b; }, red_i);
   if (threadIdx.x == 0) {
-    scale[m] = s;
-    if (rowsum) rowsum[m] = sum;
+    it.scale[m] = s;
+    if (it.rowsum) it.rowsum[m] = sum;
   }
 }
 
-cudaError_t launch_act_quant(const void* x, int x_bf16, int M, int K, int8_t* xq, float* scale,
-                             int32_t* rowsum, cudaStream_t stream, bool pdl) {
-  if (M <= 0) return cudaSuccess;
-  if (x_bf16) {
-    return launch(act_quant_kernel<__nv_bfloat16>, dim3(M), dim3(kQuantThreads), 0, stream, pdl,
-                  static_cast<const __nv_bfloat16*>(x), K, xq, scale, rowsum);
+cudaError_t launch_act_quant_group(const QuantArgs* items, int n_items, int M, int x_bf16, cudaStream_t stream,
+                                   bool pdl) {
+  if (M <= 0 || n_items <= 0) return cudaSuccess;
+  if (n_items > kQuantMaxItems) return cudaErrorInvalidValue;
+  QuantParams P = {};
+  int k_max = 0;
+  for (int i = 0; i < n_items; ++i) {
+    P.item[i] = QuantItem{items[i].x, items[i].xq, items[i].scale, items[i].rowsum, items[i].K, items[i].ldq};
+    if (items[i].K > k_max) k_max = items[i].K;
   }
-  return launch(act_quant_kernel<float>, dim3(M), dim3(kQuantThreads), 0, stream, pdl,
-                static_cast<const float*>(x), K, xq, scale, rowsum);
+  P.n_items = n_items;
+  // About two chunks per thread, in whole warps, 64 .. 512 threads.
+  int threads = ((k_max / 16 + 1) / 2 + 31) / 32 * 32;
+  if (threads < 64) threads = 64;
+  if (threads > kQuantMaxThreads) threads = kQuantMaxThreads;
+  const dim3 grid(M, n_items);
+  if (x_bf16) return launch(act_quant_kernel<__nv_bfloat16>, grid, dim3(threads), 0, stream, pdl, P);
+  return launch(act_quant_kernel<float>, grid, dim3(threads), 0, stream, pdl, P);
+}
+
+cudaError_t launch_act_quant(const void* x, int x_bf16, int M, int K, int ldq, int8_t* xq, float* scale,
+                             int32_t* rowsum, cudaStream_t stream, bool pdl) {
+  const QuantArgs a{x, xq, scale, rowsum, K, ldq};
+  return launch_act_quant_group(&a, 1, M, x_bf16, stream, pdl);
 }
 
 }  // namespace bl

@@ -69,8 +69,12 @@ int check_nk(int N, int K) {
   return BL_OK;
 }
 
-// Workspace layout: [0, 256) status word, then the quantised activations of
-// the call (q [M][K], s [M], rowsum [M]), each region 256-byte aligned.
+// Workspace layout: [0, 256) status block (status word, decode ticket
+// counters), then the quantised activations of the call: q [M][ldq] with
+// ldq = K rounded up to 128 (zero padding), s [M], rowsum [M]; every region
+// 256-byte aligned.
+int code_pitch(int K) { return (K + 127) / 128 * 128; }
+
 struct FwdLayout {
   size_t xq, scale, rowsum, total;
 };
@@ -78,7 +82,7 @@ struct FwdLayout {
 FwdLayout forward_layout(int M, int K) {
   FwdLayout l;
   l.xq = kStatusBytes;
-  l.scale = l.xq + round_up(static_cast<size_t>(M) * K, 256);
+  l.scale = l.xq + round_up(static_cast<size_t>(M) * code_pitch(K), 256);
   l.rowsum = l.scale + round_up(static_cast<size_t>(M) * 4, 256);
   l.total = l.rowsum + round_up(static_cast<size_t>(M) * 4, 256);
   return l;
@@ -104,23 +108,18 @@ int choose_gemv(int M, int K, bool* gemv) {
   } else if (g_path == 2) {
     v = false;
   }
-  if (v && !bl::gemv_supported(M, K)) {
-    if (g_path == 1)
-      return fail(BL_ERR_UNSUPPORTED_SHAPE, "GEMV path forced but M*K = %lld does not fit on chip",
-                  static_cast<long long>(M) * K);
-    v = false;
-  }
+  (void)K;
   *gemv = v;
   return BL_OK;
 }
 
 int gemv_fail(cudaError_t e) { return cuda_fail(e, "GEMV launch"); }
 
-int launch_gemm_q(const uint8_t* packed, const float* gamma, int N, int K, int M, const int8_t* xq,
+int launch_gemm_q(const uint8_t* packed, const float* gamma, int N, int K, int M, const int8_t* xq, int ldx,
                   const float* scale, const int32_t* rowsum, void* y, int y_dtype, int32_t* acc_out,
                   uint32_t* status, cudaStream_t s) {
-  bl::ProductArgs a{packed, gamma, N, K, M, xq, scale, rowsum, y, y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32,
-                    acc_out, status};
+  bl::ProductArgs a{packed, gamma, N, K, M, xq, ldx, scale, rowsum, y,
+                    y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32, acc_out, status};
   cudaError_t e = bl::launch_gemm(a, s, true);
   if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
   return BL_OK;
@@ -211,7 +210,7 @@ int bitlinear_quant_act(const void* x, int x_dtype, int M, int K, int8_t* xq, fl
   BL_TRY(check_ptr(xq, "xq", 16));
   BL_TRY(check_ptr(scale, "scale", 4));
   BL_TRY(check_ptr(rowsum, "rowsum", 4, true));
-  cudaError_t e = bl::launch_act_quant(x, x_dtype == BL_BF16, M, K, xq, scale, rowsum,
+  cudaError_t e = bl::launch_act_quant(x, x_dtype == BL_BF16, M, K, K, xq, scale, rowsum,
                                        static_cast<cudaStream_t>(stream), true);
   if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
   return BL_OK;
@@ -243,15 +242,20 @@ int bitlinear_forward_quantized(const uint8_t* packed, const float* gamma, int N
     return fail(BL_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, kStatusBytes);
   bool gemv = false;
   BL_TRY(choose_gemv(M, K, &gemv));
+  if (gemv && K % 128 != 0) {
+    // The decode kernel reads codes in 128-byte blocks; a [M][K] buffer with K % 128 != 0 has none.
+    if (g_path == 1) return fail(BL_ERR_UNSUPPORTED_SHAPE, "GEMV on caller codes needs K %% 128 == 0 (K = %d)", K);
+    gemv = false;
+  }
   uint32_t* status = static_cast<uint32_t*>(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (gemv) {
-    const bl::GemvLayerArgs L{packed, gamma, N, K, xq, scale, y, acc_out};
+    const bl::GemvLayerArgs L{packed, gamma, N, K, xq, scale, rowsum, K, y, acc_out};
     cudaError_t e = bl::launch_gemv_group(&L, 1, M, bl::kInInt8, y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32,
                                           status, tickets_of(workspace), s, true);
     return e == cudaSuccess ? BL_OK : gemv_fail(e);
   }
-  return launch_gemm_q(packed, gamma, N, K, M, xq, scale, rowsum, y, y_dtype, acc_out, status, s);
+  return launch_gemm_q(packed, gamma, N, K, M, xq, K, scale, rowsum, y, y_dtype, acc_out, status, s);
 }
 
 int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, const void* x,
@@ -279,7 +283,7 @@ int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, c
   const int yt = y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32;
   if (gemv && bl::gemv_fuses_quant(M, K, x_dtype == BL_BF16)) {
     // Small activations: the decode kernel quantises them itself (one launch).
-    const bl::GemvLayerArgs L{packed, gamma, N, K, x, nullptr, y, acc_out};
+    const bl::GemvLayerArgs L{packed, gamma, N, K, x, nullptr, nullptr, 0, y, acc_out};
     cudaError_t e = bl::launch_gemv_group(&L, 1, M, x_dtype == BL_BF16 ? bl::kInBF16 : bl::kInF32, yt, status,
                                           tickets_of(workspace), s, true);
     return e == cudaSuccess ? BL_OK : gemv_fail(e);
@@ -287,14 +291,15 @@ int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, c
   int8_t* xq = reinterpret_cast<int8_t*>(ws + l.xq);
   float* scale = reinterpret_cast<float*>(ws + l.scale);
   int32_t* rowsum = reinterpret_cast<int32_t*>(ws + l.rowsum);
-  cudaError_t e = bl::launch_act_quant(x, x_dtype == BL_BF16, M, K, xq, scale, rowsum, s, true);
+  const int ldq = code_pitch(K);
+  cudaError_t e = bl::launch_act_quant(x, x_dtype == BL_BF16, M, K, ldq, xq, scale, rowsum, s, true);
   if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
   if (gemv) {
-    const bl::GemvLayerArgs L{packed, gamma, N, K, xq, scale, y, acc_out};
+    const bl::GemvLayerArgs L{packed, gamma, N, K, xq, scale, rowsum, ldq, y, acc_out};
     e = bl::launch_gemv_group(&L, 1, M, bl::kInInt8, yt, status, tickets_of(workspace), s, true);
     return e == cudaSuccess ? BL_OK : gemv_fail(e);
   }
-  return launch_gemm_q(packed, gamma, N, K, M, xq, scale, rowsum, y, y_dtype, acc_out, status, s);
+  return launch_gemm_q(packed, gamma, N, K, M, xq, ldq, scale, rowsum, y, y_dtype, acc_out, status, s);
 }
 
 // Every layer of a chain has its own activation region (the layers of one
@@ -369,7 +374,8 @@ int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dty
     float* sc;
     int32_t* rsum;
     region(i, &xq, &sc, &rsum);
-    cudaError_t e = bl::launch_act_quant(layers[i].x, x_bf16, M, layers[i].K, xq, sc, rsum, s, true);
+    cudaError_t e = bl::launch_act_quant(layers[i].x, x_bf16, M, layers[i].K, code_pitch(layers[i].K), xq, sc, rsum,
+                                         s, true);
     if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
     quant_src[i] = i;
     return BL_OK;
@@ -385,8 +391,8 @@ int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dty
       float* sc;
       int32_t* rsum;
       region(quant_src[i], &xq, &sc, &rsum);
-      BL_TRY(launch_gemm_q(layers[i].packed, layers[i].gamma, layers[i].N, layers[i].K, M, xq, sc, rsum,
-                           layers[i].y, y_dtype, nullptr, status, s));
+      BL_TRY(launch_gemm_q(layers[i].packed, layers[i].gamma, layers[i].N, layers[i].K, M, xq,
+                           code_pitch(layers[i].K), sc, rsum, layers[i].y, y_dtype, nullptr, status, s));
       ++i;
       continue;
     }
@@ -410,17 +416,36 @@ int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dty
       ++j;
     }
     bl::GemvLayerArgs args[bl::kGvMaxLayers];
+    if (!fused) {
+      // Quantise the group's distinct inputs once, in one launch.
+      bl::QuantArgs qa[bl::kGvMaxLayers];
+      int nq = 0;
+      for (int k = i; k < j; ++k) {
+        int src = k;
+        for (int p = 0; p < k; ++p)
+          if (quant_src[p] == p && layers[p].x == layers[k].x && layers[p].K == layers[k].K) { src = p; break; }
+        quant_src[k] = src;
+        if (src == k) {
+          int8_t* xq;
+          float* sc;
+          int32_t* rsum;
+          region(k, &xq, &sc, &rsum);
+          qa[nq++] = bl::QuantArgs{layers[k].x, xq, sc, rsum, layers[k].K, code_pitch(layers[k].K)};
+        }
+      }
+      cudaError_t e = bl::launch_act_quant_group(qa, nq, M, x_bf16, s, true);
+      if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+    }
     for (int k = i; k < j; ++k) {
       const bl_layer& L = layers[k];
       if (fused) {
-        args[k - i] = bl::GemvLayerArgs{L.packed, L.gamma, L.N, L.K, L.x, nullptr, L.y, nullptr};
+        args[k - i] = bl::GemvLayerArgs{L.packed, L.gamma, L.N, L.K, L.x, nullptr, nullptr, 0, L.y, nullptr};
       } else {
-        BL_TRY(quantise(k));
         int8_t* xq;
         float* sc;
         int32_t* rsum;
         region(quant_src[k], &xq, &sc, &rsum);
-        args[k - i] = bl::GemvLayerArgs{L.packed, L.gamma, L.N, L.K, xq, sc, L.y, nullptr};
+        args[k - i] = bl::GemvLayerArgs{L.packed, L.gamma, L.N, L.K, xq, sc, rsum, code_pitch(L.K), L.y, nullptr};
       }
     }
     const int xt = fused ? (x_bf16 ? bl::kInBF16 : bl::kInF32) : bl::kInInt8;

@@ -303,11 +303,11 @@ void* tensor_map_encoder() {
 }
 
 static bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                        uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+                        uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz, uint64_t pitch = 0) {
   EncodeTiledFn fn = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {inner};  // bytes (uint8 elements)
+  const cuuint64_t strides[1] = {pitch ? pitch : inner};  // bytes (uint8 elements)
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
@@ -319,7 +319,7 @@ template <typename TY>
 static cudaError_t launch_gemm_t(const ProductArgs& a, cudaStream_t stream, bool pdl) {
   CUtensorMap ta, tb;
   if (!make_map_2d(&ta, a.xq, static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M), kBK, kBM,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+                   CU_TENSOR_MAP_SWIZZLE_128B, static_cast<uint64_t>(a.ldx)) ||
       !make_map_2d(&tb, a.packed, static_cast<uint64_t>(a.K / 4), static_cast<uint64_t>(a.N),
                    kBK / 4, kBN, CU_TENSOR_MAP_SWIZZLE_NONE)) {
     return cudaErrorInvalidValue;

@@ -12,23 +12,27 @@
 //
 // Decode streams every weight byte once, so the kernel is built around one
 // uninterrupted weight stream per SM:
-//  * Work unit: 128 output rows of one layer over all of its K.  Units are
+//  * Work unit: 64 output rows of one layer over all of its K (two blocks per SM).  Units are
 //    ordered largest-K layer first; each block takes its first unit by index
 //    and the rest from a ticket counter in the workspace, so the blocks end
 //    within a fraction of a unit of one another.  The block that finishes
 //    last resets the counter for the next launch.
-//  * One producer thread streams the block's units with TMA in stages of 128
+//  * One producer thread streams the block's units with TMA in stages of 64
 //    rows x 128 bytes (512 inputs), in the 128-byte swizzle so that the
 //    lanes' 16-byte reads are conflict-free, through a deep ring of
 //    mbarrier-tracked buffers that runs on from one unit to the next.  The
 //    first unit's loads start before the grid-dependency wait (programmatic
 //    dependent launch): weights never depend on the preceding kernel.
-//  * The activations of the current layer are staged in shared memory as
-//    int8, the 16-byte chunks of every 128-byte block rotated by twice the
-//    block index so that fragment reads are conflict-free.  Small
-//    activations are quantised by the block itself in one read (per-token
-//    absmax over all of K, s = 127 / max(amax, 1e-5), q = rint(x * s));
-//    larger ones arrive as codes from the quantisation kernel.
+//  * Activations quantised by the quantisation kernel stream with the
+//    weights: each stage also brings the stage's 512 inputs of every token,
+//    loaded through a 3-D tensor map (token, 128-input block, byte) in the
+//    128-byte swizzle, so shared-memory row 4m + q holds block q of token m
+//    and the fragment reads of the eight lanes of a phase hit eight
+//    different 16-byte bank groups.  Tiny activations (a one-token step of a
+//    small model) are instead quantised by the block itself in one read
+//    (per-token absmax over all of K, s = 127 / max(amax, 1e-5),
+//    q = rint(x * s)) and staged whole, the 16-byte chunks of every 128-byte
+//    block rotated by twice the block index; that saves a launch.
 //  * Each lane takes 16-byte chunks 2t and 2t+1 of rows g and g+8 of its
 //    warp's 16 rows into registers and releases the stage at once.
 //    Unpacking is one AND per four weights: mask 0x03030303 << 2j keeps the
@@ -50,25 +54,33 @@
 
 namespace bl {
 
-constexpr int kGvWarps = 8;
-constexpr int kGvRows = 16 * kGvWarps;           // 128 rows per unit
+constexpr int kGvWarps = 4;
+constexpr int kGvRows = 16 * kGvWarps;           // 64 rows per unit
 constexpr int kGvStageK = 512;                   // inputs per stage
-constexpr int kGvStageBytes = kGvRows * 128;     // 16 KB of packed weights
+constexpr int kGvStageBytes = kGvRows * 128;     // 8 KB of packed weights
 constexpr int kGvThreads = 32 * (kGvWarps + 1);  // + one producer warp
 constexpr int kGvConsumers = 32 * kGvWarps;
-constexpr int kGvMaxRing = 12;
+constexpr int kGvBlocksPerSM = 2;
+constexpr int kGvSmemPerBlock = 113 * 1024;
+constexpr int kGvMaxRing = 16;
 constexpr int kGvTagEnd = -1;
-constexpr int kGvFuseChunks = 8;  // 16-input chunks a consumer thread quantises itself (bf16)
+constexpr int kGvFuseChunks = 2;      // 16-input chunks a consumer thread quantises itself
+constexpr int kGvFuseElems = 4096;    // M*K up to which the blocks quantise activations themselves
 
 struct GvLayer {
-  CUtensorMap tmap;  // packed weights [N][K/4]: box 128 bytes x 128 rows, 128-byte swizzle
-  const void* x;
+  CUtensorMap tmap;  // packed weights [N][K/4]: box 128 bytes x 64 rows, 128-byte swizzle
+  CUtensorMap xmap;  // int8 codes as [M][K/128][128]: box 128 x 4 x token slots, 128-byte swizzle
+  const void* x;     // raw activations (quantised in the kernel) or int8 codes
   const float* scale;
+  const int32_t* rowsum;
   const float* gamma;
   void* y;
   int32_t* acc_out;
   int N, K, unit0;  // unit0: index of the layer's first unit
 };
+
+// Shared-memory bytes of one stage's activation tile: token slots x 4 blocks x 128.
+__host__ __device__ constexpr int x_tile_bytes(int tt) { return ((tt * 4 * 128 + 1023) / 1024) * 1024; }
 
 struct GvParams {
   GvLayer layer[kGvMaxLayers];
@@ -113,6 +125,13 @@ __device__ __forceinline__ void consumer_sync() {
 __device__ __forceinline__ int x_chunk_off(int c) {
   const int blk = c >> 3, ci = c & 7;
   return blk * 128 + (((ci + 2 * (blk & 3)) & 7) << 4);
+}
+
+// Low bytes of four ints, packed little-endian into one word.
+__device__ __forceinline__ uint32_t pack4_s8(int a, int b, int c, int d) {
+  const uint32_t lo = __byte_perm(static_cast<uint32_t>(a), static_cast<uint32_t>(b), 0x5140);
+  const uint32_t hi = __byte_perm(static_cast<uint32_t>(c), static_cast<uint32_t>(d), 0x5140);
+  return __byte_perm(lo, hi, 0x5410);
 }
 
 // Sum of the 16 signed bytes of a chunk.
@@ -205,22 +224,7 @@ __device__ __forceinline__ void stage_activations(const GvLayer& L, int M, uint3
   const int m = tid / G, j = tid % G;
   const int K = L.K;
   const int chunks = K >> 4;
-  if constexpr (sizeof(TX) == 1) {
-    int rs = 0;
-    if (m < M) {
-      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const int8_t*>(L.x) + static_cast<size_t>(m) * K);
-      for (int c = j; c < chunks; c += G) {
-        const uint4 v = __ldcg(src + c);
-        rs += byte_sum16(v);
-        sts128(xs + m * x_pitch + x_chunk_off(c), v);
-      }
-    }
-    rs = group_reduce_int<TT>(rs, reinterpret_cast<int*>(scratch));
-    if (j == 0 && m < TT) {
-      rs_tok[m] = rs;
-      s_tok[m] = (m < M) ? __ldcg(L.scale + m) : 1.0f;
-    }
-  } else {
+  {
     // At most kChunks chunks per thread (the host keeps M*K within that).
     constexpr int kChunks = sizeof(TX) == 4 ? kGvFuseChunks / 2 : kGvFuseChunks;
     RawChunk raw[kChunks];
@@ -246,13 +250,17 @@ __device__ __forceinline__ void stage_activations(const GvLayer& L, int M, uint3
     for (int i = 0; i < kChunks; ++i) {
       const int c = j + i * G;
       if (m < M && c < chunks) {
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        uint32_t w[4];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          int q = __float2int_rn(__fmul_rn(chunk_elem<TX>(raw[i], e), s));
-          q = min(max(q, -128), 127);
-          rs += q;
-          w[e >> 2] |= (static_cast<uint32_t>(q) & 0xffu) << (8 * (e & 3));
+        for (int b = 0; b < 4; ++b) {
+          int q[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            q[e] = __float2int_rn(__fmul_rn(chunk_elem<TX>(raw[i], 4 * b + e), s));
+            q[e] = min(max(q[e], -128), 127);
+          }
+          w[b] = pack4_s8(q[0], q[1], q[2], q[3]);
+          rs = __dp4a(static_cast<int>(w[b]), 0x01010101, rs);
         }
         sts128(xs + m * x_pitch + x_chunk_off(c), make_uint4(w[0], w[1], w[2], w[3]));
       }
@@ -267,15 +275,17 @@ __device__ __forceinline__ void stage_activations(const GvLayer& L, int M, uint3
 }
 
 template <int TT, typename TY, typename TX>
-__global__ void __launch_bounds__(kGvThreads, 1) gemv_group_kernel(const __grid_constant__ GvParams P) {
+__global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(const __grid_constant__ GvParams P) {
   constexpr int TG = (TT + 7) / 8;  // mma token groups of 8
+  constexpr bool kStream = sizeof(TX) == 1;  // int8 codes stream with the weights
+  constexpr int kSlot = kGvStageBytes + (kStream ? x_tile_bytes(TT) : 0);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nring = P.nring, M = P.M;
   const uint32_t sb = smem_u32(smem);
   const uint32_t ring = sb;
-  const uint32_t xs = sb + nring * kGvStageBytes;
-  uint8_t* misc = smem + nring * kGvStageBytes + ((M * P.x_pitch + 127) / 128) * 128;
+  const uint32_t xs = sb + nring * kSlot;  // whole-K activations (in-kernel quantisation only)
+  uint8_t* misc = smem + nring * kSlot + (kStream ? 0 : ((M * P.x_pitch + 127) / 128) * 128);
   float* s_tok = reinterpret_cast<float*>(misc);          // [16]
   int* rs_tok = reinterpret_cast<int*>(misc + 64);         // [16]
   float* scratch = reinterpret_cast<float*>(misc + 128);   // [kGvWarps]
@@ -315,8 +325,15 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_group_kernel(const __grid_
           const int slot = it % nring;
           if (!mbar_wait(bar0 + 8 * (nring + slot), ((it / nring) & 1) ^ 1, ctl)) { ok = false; break; }
           tags[slot] = unit;
-          mbar_arrive_expect_tx(bar0 + 8 * slot, kGvStageBytes);
-          tma_load_2d(ring + slot * kGvStageBytes, &L.tmap, st * 128, rb * kGvRows, bar0 + 8 * slot);
+          mbar_arrive_expect_tx(bar0 + 8 * slot, kStream ? kGvStageBytes + TT * 4 * 128 : kGvStageBytes);
+          tma_load_2d(ring + slot * kSlot, &L.tmap, st * 128, rb * kGvRows, bar0 + 8 * slot);
+          if constexpr (kStream) {
+            if (!waited) {
+              griddep_wait();  // the codes come from the preceding kernel
+              waited = true;
+            }
+            tma_load_3d(ring + slot * kSlot + kGvStageBytes, &L.xmap, 0, 4 * st, 0, bar0 + 8 * slot);
+          }
         }
         if (!waited) {
           griddep_wait();  // the ticket counter is reset by the preceding launch
@@ -355,10 +372,12 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_group_kernel(const __grid_
       while (l + 1 < P.n_layers && unit >= P.layer[l + 1].unit0) ++l;
       const GvLayer& L = P.layer[l];
       const int nst = (L.K + kGvStageK - 1) / kGvStageK;
-      if (l != staged) {
-        consumer_sync();  // every warp is done with the previous layer's activations
-        stage_activations<TT, TX>(L, M, xs, P.x_pitch, s_tok, rs_tok, scratch);
-        staged = l;
+      if constexpr (!kStream) {
+        if (l != staged) {
+          consumer_sync();  // every warp is done with the previous layer's activations
+          stage_activations<TT, TX>(L, M, xs, P.x_pitch, s_tok, rs_tok, scratch);
+          staged = l;
+        }
       }
 
       int d[TG][4][4];
@@ -375,7 +394,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_group_kernel(const __grid_
           const bool got = mbar_wait(bar0 + 8 * slot, (it / nring) & 1, ctl);
           if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         }
-        const uint32_t wt = ring + slot * kGvStageBytes;
+        const uint32_t wt = ring + slot * kSlot;
         // 128-byte swizzle: chunk c of row r sits at chunk position c ^ (r & 7); r & 7 == g here.
         const uint4 wl0 = lds128(wt + r_lo * 128 + (((2 * t) ^ g) << 4));
         const uint4 wl1 = lds128(wt + r_lo * 128 + (((2 * t + 1) ^ g) << 4));
@@ -396,9 +415,17 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_group_kernel(const __grid_
             for (int tg = 0; tg < TG; ++tg) {
               const int m = tg * 8 + g;
               if (m < M) {
-                const uint32_t row = xs + m * P.x_pitch + qblk * 128;
-                xa[tg] = lds128(row + (((c0 + 2 * t) & 7) << 4));
-                xb[tg] = lds128(row + (((c0 + 1 + 2 * t) & 7) << 4));
+                if constexpr (kStream) {
+                  // Row 4m + t of the stage's activation tile; chunk c sits at c ^ (row & 7).
+                  const uint32_t row = wt + kGvStageBytes + (4 * m + t) * 128;
+                  const int sw = (4 * m + t) & 7;
+                  xa[tg] = lds128(row + ((c0 ^ sw) << 4));
+                  xb[tg] = lds128(row + (((c0 + 1) ^ sw) << 4));
+                } else {
+                  const uint32_t row = xs + m * P.x_pitch + qblk * 128;
+                  xa[tg] = lds128(row + (((c0 + 2 * t) & 7) << 4));
+                  xb[tg] = lds128(row + (((c0 + 1 + 2 * t) & 7) << 4));
+                }
               } else {
                 xa[tg] = make_uint4(0, 0, 0, 0);
                 xb[tg] = make_uint4(0, 0, 0, 0);
@@ -430,8 +457,10 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_group_kernel(const __grid_
           const int n = n_base + r_lo + ((c & 2) ? 8 : 0);
           const int m = tg * 8 + 2 * t + (c & 1);
           if (n < L.N && m < M) {
-            const int a = d[tg][0][c] + (d[tg][1][c] >> 2) + (d[tg][2][c] >> 4) + (d[tg][3][c] >> 6) - rs_tok[m];
-            const float v = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, s_tok[m]));
+            const int rsum = kStream ? __ldcg(L.rowsum + m) : rs_tok[m];
+            const float sm = kStream ? __ldcg(L.scale + m) : s_tok[m];
+            const int a = d[tg][0][c] + (d[tg][1][c] >> 2) + (d[tg][2][c] >> 4) + (d[tg][3][c] >> 6) - rsum;
+            const float v = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, sm));
             const size_t o = static_cast<size_t>(m) * L.N + n;
             if constexpr (sizeof(TY) == 4) y[o] = v; else y[o] = __float2bfloat16_rn(v);
             if (L.acc_out) L.acc_out[o] = a;
@@ -458,20 +487,22 @@ static int token_slots(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M 
 
 int gemv_x_pitch(int K) { return ((K + 127) / 128) * 128 + 16; }
 
-int gemv_smem_bytes(int M, int K_max, int nring) {
-  return nring * kGvStageBytes + ((M * gemv_x_pitch(K_max) + 127) / 128) * 128 + 256 + 16 * nring + 1024;
-}
-
-bool gemv_supported(int M, int K) {
-  return M >= 1 && M <= 16 && gemv_smem_bytes(M, K, 3) <= 227 * 1024;
+// Shared memory of one block: the ring, then (in-kernel quantisation only) the
+// whole-K activations, then the small arrays and barriers.
+int gemv_smem_bytes(int M, int K_max, int nring, bool stream) {
+  const int slot = kGvStageBytes + (stream ? x_tile_bytes(token_slots(M)) : 0);
+  const int staged = stream ? 0 : ((M * gemv_x_pitch(K_max) + 127) / 128) * 128;
+  return nring * slot + staged + 256 + 16 * nring + 1024;
 }
 
 bool gemv_fuses_quant(int M, int K, int x_bf16) {
-  // Each consumer thread quantises at most kGvFuseChunks chunks of 16 inputs
-  // (half as many for fp32 inputs, which take twice the registers).
+  // Every block quantises the activations it uses, so only tiny ones are worth it;
+  // each consumer thread then holds at most kGvFuseChunks chunks of 16 inputs.
   const int G = kGvConsumers / token_slots(M);
   const int chunks_per_thread = (K / 16 + G - 1) / G;
-  return chunks_per_thread <= (x_bf16 ? kGvFuseChunks : kGvFuseChunks / 2);
+  const int max_chunks = x_bf16 ? kGvFuseChunks : (kGvFuseChunks + 1) / 2;
+  return M >= 1 && M <= 16 && static_cast<long long>(M) * K <= kGvFuseElems && chunks_per_thread <= max_chunks &&
+         gemv_smem_bytes(M, K, 4, false) <= kGvSmemPerBlock;
 }
 
 template <int TT, typename TY, typename TX>
@@ -479,7 +510,7 @@ static cudaError_t launch_group_t(const GvParams& P, int grid, int smem, cudaStr
   auto kernel = gemv_group_kernel<TT, TY, TX>;
   static bool attr_set = false;  // per template instance
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemPerBlock);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -511,6 +542,8 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   if (n_layers < 1 || n_layers > kGvMaxLayers || M < 1 || M > 16) return cudaErrorInvalidValue;
   EncodeTiledFn enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
   if (!enc) return cudaErrorNotSupported;
+  const bool stream_x = x_type == kInInt8;
+  const int tt = token_slots(M);
   // Largest K first: the longest units are handed out first.
   int order[kGvMaxLayers];
   for (int i = 0; i < n_layers; ++i) order[i] = i;
@@ -526,17 +559,33 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   for (int i = 0; i < n_layers; ++i) {
     const GemvLayerArgs& a = layers[order[i]];
     GvLayer& L = P.layer[i];
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K / 4), static_cast<cuuint64_t>(a.N)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K / 4)};
-    const cuuint32_t box[2] = {128, kGvRows};
-    const cuuint32_t estr[2] = {1, 1};
-    if (enc(&L.tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.packed), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
-      return cudaErrorInvalidValue;
+    {
+      const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K / 4), static_cast<cuuint64_t>(a.N)};
+      const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K / 4)};
+      const cuuint32_t box[2] = {128, kGvRows};
+      const cuuint32_t estr[2] = {1, 1};
+      if (enc(&L.tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.packed), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+        return cudaErrorInvalidValue;
+      }
+    }
+    if (stream_x) {
+      // Codes [M][ldx] viewed as [M][ldx/128][128]; blocks past K are zero in the buffer.
+      if (a.ldx % 128 != 0 || a.ldx < a.K) return cudaErrorInvalidValue;
+      const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(a.ldx / 128), static_cast<cuuint64_t>(M)};
+      const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(a.ldx)};
+      const cuuint32_t box[3] = {128, 4, static_cast<cuuint32_t>(tt)};
+      const cuuint32_t estr[3] = {1, 1, 1};
+      if (enc(&L.xmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(a.x), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+        return cudaErrorInvalidValue;
+      }
     }
     L.x = a.x;
     L.scale = a.scale;
+    L.rowsum = a.rowsum;
     L.gamma = a.gamma;
     L.y = a.y;
     L.acc_out = a.acc_out;
@@ -552,14 +601,16 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   P.x_pitch = gemv_x_pitch(k_max);
   P.status = status;
   P.tickets = tickets;
-  // One block per SM with the deepest ring that fits beside the activations.
-  const int x_bytes = gemv_smem_bytes(M, k_max, 0);
-  int nring = (227 * 1024 - x_bytes) / (kGvStageBytes + 16);
+  // Two blocks per SM, each with the deepest ring that fits beside its other data.
+  const int slot = kGvStageBytes + (stream_x ? x_tile_bytes(tt) : 0);
+  const int fixed = gemv_smem_bytes(M, k_max, 0, stream_x);
+  int nring = (kGvSmemPerBlock - fixed) / (slot + 16);
   if (nring > kGvMaxRing) nring = kGvMaxRing;
   if (nring < 2) return cudaErrorInvalidConfiguration;
   P.nring = nring;
-  const int smem = gemv_smem_bytes(M, k_max, nring);
-  const int grid = units < num_sms() ? units : num_sms();
+  const int smem = gemv_smem_bytes(M, k_max, nring, stream_x);
+  const int slots = kGvBlocksPerSM * num_sms();
+  const int grid = units < slots ? units : slots;
   return y_type == kOutBF16 ? launch_group_y<__nv_bfloat16>(x_type, P, grid, smem, stream, pdl)
                             : launch_group_y<float>(x_type, P, grid, smem, stream, pdl);
 }

@@ -35,9 +35,19 @@ cudaError_t launch_gamma(const float* W, int N, int K, double* row_sums, float* 
 cudaError_t launch_ternary_pack(const float* W, int N, int K, const float* gamma, uint8_t* packed,
                                 cudaStream_t stream);
 
-// Per-token activation quantisation.
-cudaError_t launch_act_quant(const void* x, int x_bf16, int M, int K, int8_t* xq, float* scale,
+// Per-token activation quantisation: one input, or several inputs in one launch.
+struct QuantArgs {
+  const void* x;
+  int8_t* xq;       // [M][ldq], zero past K
+  float* scale;
+  int32_t* rowsum;  // may be null
+  int K, ldq;
+};
+constexpr int kQuantMaxItems = 8;
+cudaError_t launch_act_quant(const void* x, int x_bf16, int M, int K, int ldq, int8_t* xq, float* scale,
                              int32_t* rowsum, cudaStream_t stream, bool pdl);
+cudaError_t launch_act_quant_group(const QuantArgs* items, int n_items, int M, int x_bf16, cudaStream_t stream,
+                                   bool pdl);
 
 enum InType { kInInt8 = 0, kInBF16 = 1, kInF32 = 2 };
 
@@ -47,6 +57,7 @@ struct ProductArgs {
   const float* gamma;
   int N, K, M;
   const int8_t* xq;
+  int ldx;  // row pitch of xq (>= K, multiple of 16)
   const float* scale;
   const int32_t* rowsum;
   void* y;
@@ -62,13 +73,14 @@ struct GemvLayerArgs {
   const uint8_t* packed;
   const float* gamma;
   int N, K;
-  const void* x;
-  const float* scale;  // token scales when the activations are int8 codes
+  const void* x;          // raw activations [M][K], or int8 codes [M][ldx]
+  const float* scale;     // token scales of the codes
+  const int32_t* rowsum;  // code sums of the codes
+  int ldx;                // row pitch of the codes: a multiple of 128 >= K, zero past K
   void* y;
   int32_t* acc_out;
 };
 constexpr int kGvMaxLayers = 8;
-bool gemv_supported(int M, int K);
 bool gemv_fuses_quant(int M, int K, int x_bf16);
 // tickets: two zero-initialised uint32 in device memory (reset by the kernel after use).
 cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, int x_type, int y_type,

@@ -66,10 +66,12 @@ def test_host_side_validation(L):
 
 
 def test_workspace_layout(L):
-    # status word (256) + q (M*K, 256-rounded) + scale and rowsum (4*M each, 256-rounded)
+    # status block (256) + q (M rows of K rounded up to 128, 256-rounded) + scale and
+    # rowsum (4*M each, 256-rounded)
     assert tb.workspace_bytes(1, 6912, 2560) == 256 + 2560 + 256 + 256
     assert tb.workspace_bytes(2048, 6912, 2560) == 256 + 2048 * 2560 + 8192 + 8192
-    assert tb.workspace_bytes(3, 10, 64) == 256 + 256 + 256 + 256
+    assert tb.workspace_bytes(3, 10, 64) == 256 + 512 + 256 + 256
+    assert tb.workspace_bytes(2, 10, 8640) == 256 + 2 * 8704 + 256 + 256
     assert tb.pack_workspace_bytes(6912, 2560) == 256 + 6912 * 8
     layers = (tb.bl_layer * 2)()
     layers[0].N, layers[0].K = 10240, 8192

@@ -205,11 +205,12 @@ def test_forward_prefill_ragged_full():
     _full_case(300, 1000, 576, "bf16", torch.bfloat16, tb.PATH_AUTO, seed=77)
 
 
-def test_forward_quantized_matches_forward():
-    W = weights(2560, 2560, seed=5)
+@pytest.mark.parametrize("K", [2560, 8640])
+def test_forward_quantized_matches_forward(K):
+    W = weights(640, K, seed=5)
     packed, gamma = tb.pack_weights(dev(W))
     for M in (1, 8, 16, 64):
-        x, _ = activations(M, 2560, seed=M, dtype="bf16")
+        x, _ = activations(M, K, seed=M, dtype="bf16")
         y1, a1 = tb.forward(packed, gamma, x, acc_out=True)
         xq, s, r = tb.quant_act(x)
         y2, a2 = tb.forward_quantized(packed, gamma, xq, s, r, acc_out=True)
