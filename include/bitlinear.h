@@ -168,6 +168,33 @@ int bitlinear_device_status(void* workspace, void* stream);
 int bitlinear_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int limit_us,
                                     void* stream);
 
+/*
+ * The forward of bitlinear_forward for callers that cannot allocate device
+ * memory.  (The pages have no counterpart: this is a deployment aid.)
+ *
+ * Who needs it: code where cudaMalloc is off limits because it can
+ * synchronise the device (latency-critical decode loops, real-time
+ * threads); plug-ins inside an engine that owns all device memory through
+ * its own pool and offers them no allocator; callers that hold a device-wide
+ * lock they must not block under.  Such callers pass only inputs and
+ * outputs (arguments as for bitlinear_forward, without the workspace).
+ *
+ * The scratch is a fixed 1 MiB array in device memory that the library
+ * declares once; every GPU that loads the library holds it until the
+ * process exits.  A call needs 256 bytes plus about M * K bytes of it
+ * (exactly bitlinear_workspace_bytes(M, N, K)); larger calls are refused
+ * with BL_ERR_WORKSPACE_TOO_SMALL.  All calls share the array and each call
+ * first clears its 256-byte control block, so calls in one stream are safe
+ * but calls that overlap on the GPU (other streams, other host threads)
+ * race on it.  The first call on a device looks up the array's device
+ * address (with that device current) and caches it; make that first call
+ * before any stream capture.  Device-side wait failures are recorded in the
+ * shared array and are not reported; use bitlinear_forward with a
+ * workspace and bitlinear_device_status to observe them.
+ */
+int bitlinear_forward_noalloc(const uint8_t* packed, const float* gamma, int N, int K, const void* x,
+                              int x_dtype, int M, void* y, int y_dtype, int32_t* acc_out, void* stream);
+
 /* Forces the product kernel: 0 = by M (default), 1 = GEMV (M <= 16 only), 2 = GEMM.  Per thread. */
 int bitlinear_set_path(int path);
 

@@ -5,6 +5,7 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <mutex>
 #include <string>
 
 #include "bitlinear.h"
@@ -484,3 +485,103 @@ int bitlinear_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// bitlinear_forward_noalloc: the forward for callers that cannot allocate.
+//
+// Some callers have no way to hand the library a workspace: code that runs
+// where cudaMalloc is off limits (it can synchronise the whole device, so a
+// latency-critical decode loop or a real-time thread avoids it), plug-ins
+// hosted by an engine that owns every device allocation through its own
+// pool and exposes no allocator to them, and callers holding a device-wide
+// lock they must not block under.  This entry point gives them the same
+// forward as bitlinear_forward, with the scratch in a fixed array that this
+// file declares in device memory, so nothing is allocated per call.
+//
+// The array costs every GPU that loads the library kNoAllocScratchBytes of
+// memory until the process exits.  Every call uses the same array, so calls
+// whose work overlaps on the GPU (two streams, or two host threads issuing
+// at once) race on it; calls in one stream are fine.  Each call clears the
+// array's 256-byte control block first, so nothing left by an earlier call
+// carries over.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB
+
+// The scratch.  On the host this name is only a shadow of the device symbol,
+// never an address to give a kernel; noalloc_scratch() looks the address up.
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[64] = {nullptr};
+
+// Device address of the scratch on the current device: looked up once per
+// device, with that device current, then cached.
+int noalloc_scratch(uint8_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(BL_ERR_CUDA, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    if (p == nullptr) return fail(BL_ERR_CUDA, "cudaGetSymbolAddress(scratch) returned NULL");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = static_cast<uint8_t*>(g_noalloc_ptr[dev]);
+  return BL_OK;
+}
+
+}  // namespace
+
+extern "C" int bitlinear_forward_noalloc(const uint8_t* packed, const float* gamma, int N, int K, const void* x,
+                                         int x_dtype, int M, void* y, int y_dtype, int32_t* acc_out,
+                                         void* stream) {
+  BL_TRY(check_nk(N, K));
+  BL_TRY(check_dtype(x_dtype, "x_dtype"));
+  BL_TRY(check_dtype(y_dtype, "y_dtype"));
+  if (M < 0) return fail(BL_ERR_INVALID_ARG, "M = %d < 0", M);
+  if (M == 0) return BL_OK;
+  BL_TRY(check_ptr(packed, "packed", 16));
+  BL_TRY(check_ptr(gamma, "gamma", 4));
+  BL_TRY(check_ptr(x, "x", 16));
+  BL_TRY(check_ptr(y, "y", 16));
+  BL_TRY(check_ptr(acc_out, "acc_out", 16, true));
+  // Same layout as a bitlinear_forward workspace: control block, then q, s, rowsum.
+  const FwdLayout l = forward_layout(M, K);
+  if (l.total > kNoAllocScratchBytes)
+    return fail(BL_ERR_WORKSPACE_TOO_SMALL,
+                "M = %d, K = %d needs %zu bytes of scratch but the fixed scratch holds %zu; "
+                "use bitlinear_forward with a workspace",
+                M, K, l.total, kNoAllocScratchBytes);
+  uint8_t* scratch = nullptr;
+  BL_TRY(noalloc_scratch(&scratch));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(scratch, 0, kStatusBytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the scratch control block");
+  bool gemv = false;
+  BL_TRY(choose_gemv(M, K, &gemv));
+  uint32_t* status = reinterpret_cast<uint32_t*>(scratch);
+  const int yt = y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32;
+  if (gemv && bl::gemv_fuses_quant(M, K, x_dtype == BL_BF16)) {
+    const bl::GemvLayerArgs L{packed, gamma, N, K, x, nullptr, nullptr, 0, y, acc_out};
+    e = bl::launch_gemv_group(&L, 1, M, x_dtype == BL_BF16 ? bl::kInBF16 : bl::kInF32, yt, status,
+                              tickets_of(scratch), s, true);
+    return e == cudaSuccess ? BL_OK : gemv_fail(e);
+  }
+  int8_t* xq = reinterpret_cast<int8_t*>(scratch + l.xq);
+  float* scale = reinterpret_cast<float*>(scratch + l.scale);
+  int32_t* rowsum = reinterpret_cast<int32_t*>(scratch + l.rowsum);
+  const int ldq = code_pitch(K);
+  e = bl::launch_act_quant(x, x_dtype == BL_BF16, M, K, ldq, xq, scale, rowsum, s, true);
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+  if (gemv) {
+    const bl::GemvLayerArgs L{packed, gamma, N, K, xq, scale, rowsum, ldq, y, acc_out};
+    e = bl::launch_gemv_group(&L, 1, M, bl::kInInt8, yt, status, tickets_of(scratch), s, true);
+    return e == cudaSuccess ? BL_OK : gemv_fail(e);
+  }
+  return launch_gemm_q(packed, gamma, N, K, M, xq, ldq, scale, rowsum, y, y_dtype, acc_out, status, s);
+}

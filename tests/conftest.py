@@ -32,3 +32,11 @@ def read_golden(name: str):
 @pytest.fixture
 def golden():
     return read_golden
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _library_built():
+    """Compile the CUDA library (sm_100a) if it is missing or older than its sources."""
+    from ternary_weight_a8_b200 import _build
+
+    _build.build()
