@@ -12,19 +12,19 @@
 //
 // Decode streams every weight byte once, so the kernel is built around one
 // uninterrupted weight stream per SM:
-//  * Work unit: 64 output rows of one layer over all of its K (two blocks per SM).  Units are
+//  * Work unit: 64 output rows of one layer over all of its K (three blocks per SM).  Units are
 //    ordered largest-K layer first; each block takes its first unit by index
 //    and the rest from a ticket counter in the workspace, so the blocks end
 //    within a fraction of a unit of one another.  The block that finishes
 //    last resets the counter for the next launch.
 //  * One producer thread streams the block's units with TMA in stages of 64
-//    rows x 128 bytes (512 inputs), in the 128-byte swizzle so that the
-//    lanes' 16-byte reads are conflict-free, through a deep ring of
+//    rows x 256 bytes (1024 inputs, two 128-byte halves), in the 128-byte
+//    swizzle so that the lanes' 16-byte reads are conflict-free, through a deep ring of
 //    mbarrier-tracked buffers that runs on from one unit to the next.  The
 //    first unit's loads start before the grid-dependency wait (programmatic
 //    dependent launch): weights never depend on the preceding kernel.
 //  * Activations quantised by the quantisation kernel stream with the
-//    weights: each stage also brings the stage's 512 inputs of every token,
+//    weights: each stage also brings the stage's 1024 inputs of every token,
 //    loaded through a 3-D tensor map (token, 128-input block, byte) in the
 //    128-byte swizzle, so shared-memory row 4m + q holds block q of token m
 //    and the fragment reads of the eight lanes of a phase hit eight
@@ -56,12 +56,12 @@ namespace bl {
 
 constexpr int kGvWarps = 4;
 constexpr int kGvRows = 16 * kGvWarps;           // 64 rows per unit
-constexpr int kGvStageK = 512;                   // inputs per stage
-constexpr int kGvStageBytes = kGvRows * 128;     // 8 KB of packed weights
+constexpr int kGvStageK = 1024;                  // inputs per stage
+constexpr int kGvStageBytes = kGvRows * 256;     // 16 KB of packed weights (two 128-byte halves)
 constexpr int kGvThreads = 32 * (kGvWarps + 1);  // + one producer warp
 constexpr int kGvConsumers = 32 * kGvWarps;
-constexpr int kGvBlocksPerSM = 2;
-constexpr int kGvSmemPerBlock = 113 * 1024;
+constexpr int kGvBlocksPerSM = 3;
+constexpr int kGvSmemPerBlock = 75 * 1024;
 constexpr int kGvMaxRing = 16;
 constexpr int kGvTagEnd = -1;
 constexpr int kGvFuseChunks = 2;      // 16-input chunks a consumer thread quantises itself
@@ -79,8 +79,9 @@ struct GvLayer {
   int N, K, unit0;  // unit0: index of the layer's first unit
 };
 
-// Shared-memory bytes of one stage's activation tile: token slots x 4 blocks x 128.
-__host__ __device__ constexpr int x_tile_bytes(int tt) { return ((tt * 4 * 128 + 1023) / 1024) * 1024; }
+// Shared-memory bytes of half a stage's activation tile: token slots x 4 blocks x 128,
+// rounded to the 1024-byte period of the 128-byte swizzle.
+__host__ __device__ constexpr int x_half_bytes(int tt) { return ((tt * 4 * 128 + 1023) / 1024) * 1024; }
 
 struct GvParams {
   GvLayer layer[kGvMaxLayers];
@@ -276,9 +277,10 @@ __device__ __forceinline__ void stage_activations(const GvLayer& L, int M, uint3
 
 template <int TT, typename TY, typename TX>
 __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(const __grid_constant__ GvParams P) {
-  constexpr int TG = (TT + 7) / 8;  // mma token groups of 8
+  constexpr int TG = (TT + 7) / 8;           // mma token groups of 8
   constexpr bool kStream = sizeof(TX) == 1;  // int8 codes stream with the weights
-  constexpr int kSlot = kGvStageBytes + (kStream ? x_tile_bytes(TT) : 0);
+  constexpr int kXHalf = x_half_bytes(TT);   // one half-stage activation tile
+  constexpr int kSlot = kGvStageBytes + (kStream ? 2 * kXHalf : 0);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nring = P.nring, M = P.M;
@@ -311,7 +313,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
   if (warp == kGvWarps) {
     // ---- producer: one thread streams the block's units ----
     if (lane == 0) {
-      int it = 0;           // stages issued
+      int slot = 0, phase = 0, issued = 0;
       bool waited = false;  // grid dependency
       bool ok = true;
       int unit = blockIdx.x;
@@ -321,19 +323,23 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         const GvLayer& L = P.layer[l];
         const int rb = unit - L.unit0;
         const int nst = (L.K + kGvStageK - 1) / kGvStageK;
-        for (int st = 0; st < nst; ++st, ++it) {
-          const int slot = it % nring;
-          if (!mbar_wait(bar0 + 8 * (nring + slot), ((it / nring) & 1) ^ 1, ctl)) { ok = false; break; }
+        for (int st = 0; st < nst; ++st) {
+          if (!mbar_wait(bar0 + 8 * (nring + slot), phase ^ 1, ctl)) { ok = false; break; }
           tags[slot] = unit;
-          mbar_arrive_expect_tx(bar0 + 8 * slot, kStream ? kGvStageBytes + TT * 4 * 128 : kGvStageBytes);
-          tma_load_2d(ring + slot * kSlot, &L.tmap, st * 128, rb * kGvRows, bar0 + 8 * slot);
+          const uint32_t full = bar0 + 8 * slot, dst = ring + slot * kSlot;
+          mbar_arrive_expect_tx(full, kStream ? kGvStageBytes + 2 * TT * 4 * 128 : kGvStageBytes);
+          tma_load_2d(dst, &L.tmap, st * 256, rb * kGvRows, full);
+          tma_load_2d(dst + kGvStageBytes / 2, &L.tmap, st * 256 + 128, rb * kGvRows, full);
           if constexpr (kStream) {
             if (!waited) {
               griddep_wait();  // the codes come from the preceding kernel
               waited = true;
             }
-            tma_load_3d(ring + slot * kSlot + kGvStageBytes, &L.xmap, 0, 4 * st, 0, bar0 + 8 * slot);
+            tma_load_3d(dst + kGvStageBytes, &L.xmap, 0, 8 * st, 0, full);
+            tma_load_3d(dst + kGvStageBytes + kXHalf, &L.xmap, 0, 8 * st + 4, 0, full);
           }
+          ++issued;
+          if (++slot == nring) { slot = 0; phase ^= 1; }
         }
         if (!waited) {
           griddep_wait();  // the ticket counter is reset by the preceding launch
@@ -343,15 +349,14 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       }
       if (ok) {
         // End marker: one more phase on the next slot, with no data.
-        const int slot = it % nring;
-        if (mbar_wait(bar0 + 8 * (nring + slot), ((it / nring) & 1) ^ 1, ctl)) {
+        if (mbar_wait(bar0 + 8 * (nring + slot), phase ^ 1, ctl)) {
           tags[slot] = kGvTagEnd;
           mbar_arrive(bar0 + 8 * slot);
         }
       } else {
         // Gave up: let copies in flight land before shared memory is released.
         const WaitCtl drain{nullptr, never, 100000000ull};
-        for (int j = (it > nring ? it - nring : 0); j < it; ++j)
+        for (int j = (issued > nring ? issued - nring : 0); j < issued; ++j)
           mbar_wait(bar0 + 8 * (j % nring), (j / nring) & 1, drain);
       }
     }
@@ -360,13 +365,25 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
     griddep_wait();  // activations may be the preceding kernel's output
     const int g = lane >> 2, t = lane & 3;
     const int r_lo = warp * 16 + g;  // rows of this lane within the unit (and + 8)
-    int staged = -1;                 // layer whose activations are in shared memory
-    int it = 0;
+    // Byte offsets of this lane's weight chunks 2t, 2t+1 of rows r_lo, r_lo+8 within a
+    // 128-byte-swizzled half-stage: chunk c of row r sits at chunk position c ^ (r & 7).
+    const uint32_t w_lo0 = r_lo * 128 + (((2 * t) ^ g) << 4), w_lo1 = r_lo * 128 + (((2 * t + 1) ^ g) << 4);
+    const uint32_t w_hi0 = w_lo0 + 8 * 128, w_hi1 = w_lo1 + 8 * 128;
+    // Streamed activations: row 4m + t of a half tile holds block t of token m.
+    uint32_t x_row[TG];
+    int x_sw[TG];
+#pragma unroll
+    for (int tg = 0; tg < TG; ++tg) {
+      const int m = tg * 8 + g;
+      x_row[tg] = (4 * m + t) * 128;
+      x_sw[tg] = (4 * m + t) & 7;
+    }
+    int staged = -1;  // layer whose activations are in shared memory
+    int slot = 0, phase = 0;
     while (true) {
-      const int slot0 = it % nring;
-      const bool got0 = mbar_wait(bar0 + 8 * slot0, (it / nring) & 1, ctl);
+      const bool got0 = mbar_wait(bar0 + 8 * slot, phase, ctl);
       if (!__all_sync(0xffffffffu, got0)) break;
-      const int unit = tags[slot0];
+      const int unit = tags[slot];
       if (unit == kGvTagEnd) break;
       int l = 0;
       while (l + 1 < P.n_layers && unit >= P.layer[l + 1].unit0) ++l;
@@ -388,61 +405,67 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
 #pragma unroll
           for (int c = 0; c < 4; ++c) d[tg][j][c] = 0;
       bool ok = true;
-      for (int i = 0; i < nst; ++i, ++it) {
-        const int slot = it % nring;
+      for (int i = 0; i < nst; ++i) {
         if (i > 0) {
-          const bool got = mbar_wait(bar0 + 8 * slot, (it / nring) & 1, ctl);
+          const bool got = mbar_wait(bar0 + 8 * slot, phase, ctl);
           if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         }
         const uint32_t wt = ring + slot * kSlot;
-        // 128-byte swizzle: chunk c of row r sits at chunk position c ^ (r & 7); r & 7 == g here.
-        const uint4 wl0 = lds128(wt + r_lo * 128 + (((2 * t) ^ g) << 4));
-        const uint4 wl1 = lds128(wt + r_lo * 128 + (((2 * t + 1) ^ g) << 4));
-        const uint4 wh0 = lds128(wt + (r_lo + 8) * 128 + (((2 * t) ^ g) << 4));
-        const uint4 wh1 = lds128(wt + (r_lo + 8) * 128 + (((2 * t + 1) ^ g) << 4));
+        uint4 w[2][4];  // [half][lo0, lo1, hi0, hi1]
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const uint32_t base = wt + hf * (kGvStageBytes / 2);
+          w[hf][0] = lds128(base + w_lo0);
+          w[hf][1] = lds128(base + w_lo1);
+          w[hf][2] = lds128(base + w_hi0);
+          w[hf][3] = lds128(base + w_hi1);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // the weights are in registers
+        const uint32_t xt = wt + kGvStageBytes;
 
-        const int qblk = i * 4 + t;  // this lane's 128-input block of the staged activations
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint4 wl = h ? wl1 : wl0, wh = h ? wh1 : wh0;
+        for (int hf = 0; hf < 2; ++hf) {
+          const int qblk = i * 8 + hf * 4 + t;  // this lane's 128-input block (whole-K staging)
 #pragma unroll
-          for (int p = 0; p < 2; ++p) {
-            const int c0 = 4 * h + 2 * p;  // activation chunks c0, c0+1 of block qblk
-            uint4 xa[TG], xb[TG];
+          for (int h = 0; h < 2; ++h) {
+            const uint4 wl = w[hf][h], wh = w[hf][2 + h];
 #pragma unroll
-            for (int tg = 0; tg < TG; ++tg) {
-              const int m = tg * 8 + g;
-              if (m < M) {
-                if constexpr (kStream) {
-                  // Row 4m + t of the stage's activation tile; chunk c sits at c ^ (row & 7).
-                  const uint32_t row = wt + kGvStageBytes + (4 * m + t) * 128;
-                  const int sw = (4 * m + t) & 7;
-                  xa[tg] = lds128(row + ((c0 ^ sw) << 4));
-                  xb[tg] = lds128(row + (((c0 + 1) ^ sw) << 4));
+            for (int p = 0; p < 2; ++p) {
+              const int c0 = 4 * h + 2 * p;  // activation chunks c0, c0+1 of the lane's block
+              uint4 xa[TG], xb[TG];
+#pragma unroll
+              for (int tg = 0; tg < TG; ++tg) {
+                const int m = tg * 8 + g;
+                if (m < M) {
+                  if constexpr (kStream) {
+                    const uint32_t row = xt + hf * kXHalf + x_row[tg];
+                    xa[tg] = lds128(row + ((c0 ^ x_sw[tg]) << 4));
+                    xb[tg] = lds128(row + (((c0 + 1) ^ x_sw[tg]) << 4));
+                  } else {
+                    const uint32_t row = xs + m * P.x_pitch + qblk * 128;
+                    xa[tg] = lds128(row + (((c0 + 2 * t) & 7) << 4));
+                    xb[tg] = lds128(row + (((c0 + 1 + 2 * t) & 7) << 4));
+                  }
                 } else {
-                  const uint32_t row = xs + m * P.x_pitch + qblk * 128;
-                  xa[tg] = lds128(row + (((c0 + 2 * t) & 7) << 4));
-                  xb[tg] = lds128(row + (((c0 + 1 + 2 * t) & 7) << 4));
+                  xa[tg] = make_uint4(0, 0, 0, 0);
+                  xb[tg] = make_uint4(0, 0, 0, 0);
                 }
-              } else {
-                xa[tg] = make_uint4(0, 0, 0, 0);
-                xb[tg] = make_uint4(0, 0, 0, 0);
               }
-            }
-            const uint32_t lo0 = u4_get(wl, 2 * p), lo1 = u4_get(wl, 2 * p + 1);
-            const uint32_t hi0 = u4_get(wh, 2 * p), hi1 = u4_get(wh, 2 * p + 1);
+              const uint32_t lo0 = u4_get(wl, 2 * p), lo1 = u4_get(wl, 2 * p + 1);
+              const uint32_t hi0 = u4_get(wh, 2 * p), hi1 = u4_get(wh, 2 * p + 1);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t mask = 0x03030303u << (2 * j);
-              const uint32_t a0 = lo0 & mask, a1 = hi0 & mask, a2 = lo1 & mask, a3 = hi1 & mask;
+              for (int j = 0; j < 4; ++j) {
+                const uint32_t mask = 0x03030303u << (2 * j);
+                const uint32_t a0 = lo0 & mask, a1 = hi0 & mask, a2 = lo1 & mask, a3 = hi1 & mask;
 #pragma unroll
-              for (int tg = 0; tg < TG; ++tg)
-                mma_u8s8_16x8x32(d[tg][j], a0, a1, a2, a3, u4_get(xa[tg], j), u4_get(xb[tg], j));
+                for (int tg = 0; tg < TG; ++tg)
+                  mma_u8s8_16x8x32(d[tg][j], a0, a1, a2, a3, u4_get(xa[tg], j), u4_get(xb[tg], j));
+              }
             }
           }
         }
+        if (++slot == nring) { slot = 0; phase ^= 1; }
       }
       if (!ok) break;
 
@@ -490,7 +513,7 @@ int gemv_x_pitch(int K) { return ((K + 127) / 128) * 128 + 16; }
 // Shared memory of one block: the ring, then (in-kernel quantisation only) the
 // whole-K activations, then the small arrays and barriers.
 int gemv_smem_bytes(int M, int K_max, int nring, bool stream) {
-  const int slot = kGvStageBytes + (stream ? x_tile_bytes(token_slots(M)) : 0);
+  const int slot = kGvStageBytes + (stream ? 2 * x_half_bytes(token_slots(M)) : 0);
   const int staged = stream ? 0 : ((M * gemv_x_pitch(K_max) + 127) / 128) * 128;
   return nring * slot + staged + 256 + 16 * nring + 1024;
 }
@@ -602,7 +625,7 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   P.status = status;
   P.tickets = tickets;
   // Two blocks per SM, each with the deepest ring that fits beside its other data.
-  const int slot = kGvStageBytes + (stream_x ? x_tile_bytes(tt) : 0);
+  const int slot = kGvStageBytes + (stream_x ? 2 * x_half_bytes(tt) : 0);
   const int fixed = gemv_smem_bytes(M, k_max, 0, stream_x);
   int nring = (kGvSmemPerBlock - fixed) / (slot + 16);
   if (nring > kGvMaxRing) nring = kGvMaxRing;
