@@ -34,7 +34,9 @@
 //    q = rint(x * s)) and staged whole, the 16-byte chunks of every 128-byte
 //    block rotated by twice the block index; that saves a launch.
 //  * Each lane takes 16-byte chunks 2t and 2t+1 of rows g and g+8 of its
-//    warp's 16 rows into registers and releases the stage at once.
+//    warp's 16 rows into registers; a warp releases a stage once it has
+//    read everything it needs from it (at once when the activations are
+//    staged whole, after the stage's products when they stream with it).
 //    Unpacking is one AND per four weights: mask 0x03030303 << 2j keeps the
 //    codes of elements 4j..4j+3 of a word in place (scaled by 4^j); four
 //    accumulator sets, one per j, are shifted back and added at the end,
@@ -420,8 +422,10 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           w[hf][2] = lds128(base + w_hi0);
           w[hf][3] = lds128(base + w_hi1);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // the weights are in registers
+        if constexpr (!kStream) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // the slot held only weights, now in registers
+        }
         const uint32_t xt = wt + kGvStageBytes;
 
 #pragma unroll
@@ -464,6 +468,10 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
               }
             }
           }
+        }
+        if constexpr (kStream) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // done with the slot's activations too
         }
         if (++slot == nring) { slot = 0; phase ^= 1; }
       }
