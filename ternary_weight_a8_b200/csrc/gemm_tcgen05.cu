@@ -8,15 +8,18 @@
 // "A Two-Billion Ternary Bet": the pack-store-load-unpack-compute sequence.
 //
 // Tile: 128 tokens x 256 output rows x 128 inputs per k-block.  Warp roles
-// in a persistent block of 12 warps (one block per SM):
-//   warp 0      TMA producer: the activation tile (128-byte swizzle) and the
-//               packed weight tile (256 rows x 32 bytes) per k-block;
+// in a persistent block of 16 warps (one block per SM):
+//   warp 0      TMA producer of the activation tiles (128-byte swizzle);
+//   warp 2      TMA producer of the packed weight tiles (256 rows x 32 bytes),
+//               on a ring of its own that the unpack warps release as soon
+//               as they hold the words in registers, so weight tiles are
+//               requested well ahead of the tensor cores;
 //   warp 1      tensor-memory owner and the single thread that issues the
 //               4 tcgen05.mma (K = 32 each) per k-block;
-//   warps 4-7   unpack: packed words -> one 16-byte chunk of codes
+//   warps 4-11  unpack: packed words -> one 16-byte chunk of codes
 //               ((w >> 2j) & 0x03030303, j = 0..3) written at its 128-byte
 //               swizzle position, then a proxy fence and an mbarrier arrive;
-//   warps 8-11  epilogue: tcgen05.ld of the int32 accumulators, then
+//   warps 12-15 epilogue: tcgen05.ld of the int32 accumulators, then
 //               y = (acc - rowsum[m]) * (gamma / s[m]) stored as fp32 / bf16.
 // Two accumulators (2 x 256 tensor-memory columns) let the epilogue of one
 // tile overlap the main loop of the next.  Every mbarrier wait is bounded in
@@ -31,18 +34,20 @@
 namespace bl {
 
 constexpr int kBM = 128, kBN = 256, kBK = 128;
-constexpr int kStages = 4, kUStages = 2;
+constexpr int kAStages = 5, kPStages = 6, kUStages = 3;
 constexpr int kABytes = kBM * kBK;       // 16 KB activation tile
 constexpr int kBPBytes = kBN * kBK / 4;  // 8 KB packed weight tile
 constexpr int kBUBytes = kBN * kBK;      // 32 KB unpacked code tile
-constexpr int kGemmThreads = 384;
+constexpr int kGemmThreads = 512;
+constexpr int kUnpackThreads = 256;  // warps 4-11
 constexpr int kOffA = 0;
-constexpr int kOffBU = kOffA + kStages * kABytes;
+constexpr int kOffBU = kOffA + kAStages * kABytes;
 constexpr int kOffBP = kOffBU + kUStages * kBUBytes;
-constexpr int kOffBar = kOffBP + kStages * kBPBytes;
-constexpr int kNumBars = 17;
+constexpr int kOffBar = kOffBP + kPStages * kBPBytes;
+constexpr int kNumBars = 2 * (kAStages + kPStages + kUStages) + 5;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory per block");
 constexpr uint32_t kTmemCols = 512;
 
 // Instruction descriptor: D s32, A s8, B s8, both K-major, N = 256, M = 128.
@@ -110,12 +115,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
-  auto full_bar = [&](int i) { return sb + kOffBar + 8 * i; };
-  auto empty_bar = [&](int i) { return sb + kOffBar + 8 * (kStages + i); };
-  auto ufull_bar = [&](int i) { return sb + kOffBar + 8 * (2 * kStages + i); };
-  auto uempty_bar = [&](int i) { return sb + kOffBar + 8 * (2 * kStages + kUStages + i); };
-  auto tfull_bar = [&](int i) { return sb + kOffBar + 8 * (2 * kStages + 2 * kUStages + i); };
-  auto tempty_bar = [&](int i) { return sb + kOffBar + 8 * (2 * kStages + 2 * kUStages + 2 + i); };
+  constexpr int kBarP = 2 * kAStages, kBarU = kBarP + 2 * kPStages, kBarT = kBarU + 2 * kUStages;
+  auto afull_bar = [&](int i) { return sb + kOffBar + 8 * i; };
+  auto aempty_bar = [&](int i) { return sb + kOffBar + 8 * (kAStages + i); };
+  auto pfull_bar = [&](int i) { return sb + kOffBar + 8 * (kBarP + i); };
+  auto pempty_bar = [&](int i) { return sb + kOffBar + 8 * (kBarP + kPStages + i); };
+  auto ufull_bar = [&](int i) { return sb + kOffBar + 8 * (kBarU + i); };
+  auto uempty_bar = [&](int i) { return sb + kOffBar + 8 * (kBarU + kUStages + i); };
+  auto tfull_bar = [&](int i) { return sb + kOffBar + 8 * (kBarT + i); };
+  auto tempty_bar = [&](int i) { return sb + kOffBar + 8 * (kBarT + 2 + i); };
   const uint32_t done_bar = sb + kOffBar + 8 * (kNumBars - 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 16);
@@ -123,12 +131,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(full_bar(i), 1);
-      mbar_init(empty_bar(i), 1);
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(afull_bar(i), 1);
+      mbar_init(aempty_bar(i), 1);
+    }
+    for (int i = 0; i < kPStages; ++i) {
+      mbar_init(pfull_bar(i), 1);
+      mbar_init(pempty_bar(i), kUnpackThreads);
     }
     for (int i = 0; i < kUStages; ++i) {
-      mbar_init(ufull_bar(i), 128);
+      mbar_init(ufull_bar(i), kUnpackThreads);
       mbar_init(uempty_bar(i), 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -140,10 +152,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
     *never = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmap_a);
-    tma_prefetch_desc(&tmap_b);
-  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmap_a);
+  if (warp == 2 && lane == 0) tma_prefetch_desc(&tmap_b);
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -162,26 +172,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
   const int tiles = m_tiles * n_tiles;
   const int kblocks = (K + kBK - 1) / kBK;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 2) {
     if (lane == 0) {
-      int it = 0;
+      // warp 0: activation tiles; warp 2: packed weight tiles.
+      const bool is_a = (warp == 0);
+      const int nst = is_a ? kAStages : kPStages;
+      int it = 0, s = 0;
+      uint32_t ph = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
         const int mt = tile % m_tiles, nt = tile / m_tiles;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          if (!mbar_wait(empty_bar(s), ph ^ 1, ctl)) { ok = false; break; }
-          mbar_arrive_expect_tx(full_bar(s), kABytes + kBPBytes);
-          tma_load_2d(sb + kOffA + s * kABytes, &tmap_a, kb * kBK, mt * kBM, full_bar(s));
-          tma_load_2d(sb + kOffBP + s * kBPBytes, &tmap_b, kb * (kBK / 4), nt * kBN, full_bar(s));
+          const uint32_t full = is_a ? afull_bar(s) : pfull_bar(s);
+          if (!mbar_wait(is_a ? aempty_bar(s) : pempty_bar(s), ph ^ 1, ctl)) { ok = false; break; }
+          if (is_a) {
+            mbar_arrive_expect_tx(full, kABytes);
+            tma_load_2d(sb + kOffA + s * kABytes, &tmap_a, kb * kBK, mt * kBM, full);
+          } else {
+            mbar_arrive_expect_tx(full, kBPBytes);
+            tma_load_2d(sb + kOffBP + s * kBPBytes, &tmap_b, kb * (kBK / 4), nt * kBN, full);
+          }
+          if (++s == nst) { s = 0; ph ^= 1; }
         }
       }
       if (!ok) {
         // Let copies already in flight land before the block's shared memory goes away.
         const WaitCtl drain{nullptr, never, 100000000ull};
-        for (int i = (it > kStages ? it - kStages : 0); i < it; ++i)
-          mbar_wait(full_bar(i % kStages), (i / kStages) & 1, drain);
+        for (int i = (it > nst ? it - nst : 0); i < it; ++i)
+          mbar_wait(is_a ? afull_bar(i % nst) : pfull_bar(i % nst), (i / nst) & 1, drain);
       }
     }
   } else if (warp == 1) {
@@ -194,8 +212,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + a * kBN;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          const int s = it % kStages, u = it % kUStages;
-          if (!mbar_wait(full_bar(s), (it / kStages) & 1, ctl)) { ok = false; break; }
+          const int s = it % kAStages, u = it % kUStages;
+          if (!mbar_wait(afull_bar(s), (it / kAStages) & 1, ctl)) { ok = false; break; }
           if (!mbar_wait(ufull_bar(u), (it / kUStages) & 1, ctl)) { ok = false; break; }
           tc_fence_after();
           const uint64_t adesc = sw128_kmajor_desc(sb + kOffA + s * kABytes);
@@ -205,7 +223,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
             tc_mma_i8(d_tmem, adesc + 2 * k, bdesc + 2 * k, kIdesc, (kb | k) != 0);
           }
           issued = true;
-          tc_commit(empty_bar(s));
+          tc_commit(aempty_bar(s));
           tc_commit(uempty_bar(u));
         }
         if (ok) tc_commit(tfull_bar(a));
@@ -217,37 +235,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
         mbar_wait(done_bar, 0, drain);
       }
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4 && warp < 12) {
     const int ut = threadIdx.x - 128;
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
       for (int kb = 0; kb < kblocks; ++kb, ++it) {
-        const int s = it % kStages, u = it % kUStages;
-        if (!mbar_wait(full_bar(s), (it / kStages) & 1, ctl)) { ok = false; break; }
-        if (!mbar_wait(uempty_bar(u), ((it / kUStages) & 1) ^ 1, ctl)) { ok = false; break; }
+        const int s = it % kPStages, u = it % kUStages;
+        if (!mbar_wait(pfull_bar(s), (it / kPStages) & 1, ctl)) { ok = false; break; }
+        constexpr int kPer = kBPBytes / 16 / kUnpackThreads;  // packed uint4 per thread
         const uint4* bp = reinterpret_cast<const uint4*>(smem + kOffBP + s * kBPBytes);
-        uint8_t* bu = smem + kOffBU + u * kBUBytes;
+        uint4 codes[kPer][4];
 #pragma unroll
-        for (int q = ut; q < kBPBytes / 16; q += 128) {
-          const uint4 v = bp[q];
-          const int r = q >> 1;              // weight row in the tile (32 packed bytes per row)
-          const int c0 = (q & 1) * 4;        // first 16-byte chunk (= packed word) of this uint4
+        for (int j = 0; j < kPer; ++j) {
+          const uint4 v = bp[ut + j * kUnpackThreads];
           const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-          uint8_t* rowp = bu + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const uint32_t w = w4[i];
-            const uint4 codes = make_uint4(w & 0x03030303u, (w >> 2) & 0x03030303u,
-                                           (w >> 4) & 0x03030303u, (w >> 6) & 0x03030303u);
-            *reinterpret_cast<uint4*>(rowp + (((c0 + i) ^ (r & 7)) << 4)) = codes;
+            codes[j][i] = make_uint4(w & 0x03030303u, (w >> 2) & 0x03030303u, (w >> 4) & 0x03030303u,
+                                     (w >> 6) & 0x03030303u);
           }
         }
+        if (!mbar_wait(uempty_bar(u), ((it / kUStages) & 1) ^ 1, ctl)) { ok = false; break; }
+        uint8_t* bu = smem + kOffBU + u * kBUBytes;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+          const int q = ut + j * kUnpackThreads;
+          const int r = q >> 1;              // weight row in the tile (32 packed bytes per row)
+          const int c0 = (q & 1) * 4;        // first 16-byte chunk (= packed word) of this uint4
+          uint8_t* rowp = bu + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<uint4*>(rowp + (((c0 + i) ^ (r & 7)) << 4)) = codes[j][i];
+        }
+        // The stores above consumed every packed word, so no read of the packed
+        // slot can still be in flight: hand it back to its producer.
+        mbar_arrive(pempty_bar(s));
         fence_proxy_async_smem();
         mbar_arrive(ufull_bar(u));
       }
     }
-  } else if (warp >= 8) {
+  } else if (warp >= 12) {
     const int q = warp & 3;  // tensor-memory lane quarter this warp may read
     const float gamma = __ldg(gamma_ptr);
     int tc = 0;
