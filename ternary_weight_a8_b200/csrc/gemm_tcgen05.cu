@@ -7,24 +7,32 @@
 // shared memory, are unpacked there and meet the 8-bit activations.
 // "A Two-Billion Ternary Bet": the pack-store-load-unpack-compute sequence.
 //
-// Tile: 128 tokens x 256 output rows x 128 inputs per k-block.  Warp roles
-// in a persistent block of 16 warps (one block per SM):
+// Tiles: 128 tokens per CTA x 256 output rows x 128 inputs per k-block.
+// Two forms of one kernel:
+//   CG = 1  one CTA per tile (used for up to 128 tokens);
+//   CG = 2  a cluster of two CTAs on two SMs shares a 256-token x 256-row
+//           tile through tcgen05.mma.cta_group::2: each CTA loads its own 128
+//           tokens and unpacks only its half (128 rows) of the weight tile, so
+//           per SM the unpack stores and the tensor cores' shared-memory reads
+//           of codes are halved.  The MMA thread of the even CTA issues for
+//           both; commits are multicast to both CTAs.
+// Warp roles in a persistent block of 16 warps (one block per SM):
 //   warp 0      TMA producer of the activation tiles (128-byte swizzle);
-//   warp 2      TMA producer of the packed weight tiles (256 rows x 32 bytes),
-//               on a ring of its own that the unpack warps release as soon
-//               as they hold the words in registers, so weight tiles are
-//               requested well ahead of the tensor cores;
-//   warp 1      tensor-memory owner and the single thread that issues the
-//               4 tcgen05.mma (K = 32 each) per k-block;
+//   warp 2      TMA producer of the packed weight tiles, on a ring of its own
+//               that the unpack warps release once their stores have consumed
+//               the words, so weight tiles are requested well ahead;
+//   warp 1      tensor-memory owner; in the even CTA, the single thread that
+//               issues the 4 tcgen05.mma (K = 32 each) per k-block;
 //   warps 4-11  unpack: packed words -> one 16-byte chunk of codes
 //               ((w >> 2j) & 0x03030303, j = 0..3) written at its 128-byte
-//               swizzle position, then a proxy fence and an mbarrier arrive;
+//               swizzle position, a proxy fence, then one arrive per warp;
 //   warps 12-15 epilogue: tcgen05.ld of the int32 accumulators, then
 //               y = (acc - rowsum[m]) * (gamma / s[m]) stored as fp32 / bf16.
 // Two accumulators (2 x 256 tensor-memory columns) let the epilogue of one
 // tile overlap the main loop of the next.  Every mbarrier wait is bounded in
 // time; a wait that runs out records the timeout in the workspace status
-// word and the block winds down without touching global memory further.
+// word, raises the abort flag of both CTAs of the pair, and the block winds
+// down without touching global memory further.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -34,25 +42,34 @@
 namespace bl {
 
 constexpr int kBM = 128, kBN = 256, kBK = 128;
-constexpr int kAStages = 5, kPStages = 6, kUStages = 3;
-constexpr int kABytes = kBM * kBK;       // 16 KB activation tile
-constexpr int kBPBytes = kBN * kBK / 4;  // 8 KB packed weight tile
-constexpr int kBUBytes = kBN * kBK;      // 32 KB unpacked code tile
+constexpr int kABytes = kBM * kBK;  // 16 KB activation tile per CTA
 constexpr int kGemmThreads = 512;
-constexpr int kUnpackThreads = 256;  // warps 4-11
-constexpr int kOffA = 0;
-constexpr int kOffBU = kOffA + kAStages * kABytes;
-constexpr int kOffBP = kOffBU + kUStages * kBUBytes;
-constexpr int kOffBar = kOffBP + kPStages * kBPBytes;
-constexpr int kNumBars = 2 * (kAStages + kPStages + kUStages) + 5;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
-static_assert(kSmemBytes <= 232448, "shared memory per block");
+constexpr int kUnpackWarps = 8;     // warps 4-11
+constexpr int kUnpackThreads = 32 * kUnpackWarps;
+constexpr int kEpiWarps = 4;        // warps 12-15
 constexpr uint32_t kTmemCols = 512;
 
-// Instruction descriptor: D s32, A s8, B s8, both K-major, N = 256, M = 128.
-constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) |
-                            ((kBM >> 4) << 24);
+template <int CG>
+struct GemmCfg {
+  static constexpr int kRowsB = kBN / CG;            // weight rows unpacked by one CTA
+  static constexpr int kBPBytes = kRowsB * kBK / 4;  // packed weight tile per CTA
+  static constexpr int kBUBytes = kRowsB * kBK;      // unpacked code tile per CTA
+  static constexpr int kAStages = CG == 1 ? 5 : 6;
+  static constexpr int kPStages = CG == 1 ? 6 : 8;
+  static constexpr int kUStages = CG == 1 ? 3 : 4;
+  static constexpr int kOffA = 0;
+  static constexpr int kOffBU = kOffA + kAStages * kABytes;
+  static constexpr int kOffBP = kOffBU + kUStages * kBUBytes;
+  static constexpr int kOffBar = kOffBP + kPStages * kBPBytes;
+  static constexpr int kNumBars = 2 * (kAStages + kPStages + kUStages) + 5;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
+  // Instruction descriptor: D s32, A s8, B s8, both K-major, N = 256, M = 128 * CG.
+  static constexpr uint32_t kIdesc =
+      (2u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | (((kBM * CG) >> 4) << 24);
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+  static_assert(kBPBytes / 16 % kUnpackThreads == 0, "packed words per unpack thread");
+};
 
 template <typename TY>
 __device__ __forceinline__ void store_row32(TY* __restrict__ y, int32_t* __restrict__ acc_out,
@@ -106,46 +123,87 @@ __device__ __forceinline__ void store_row32(TY* __restrict__ y, int32_t* __restr
   }
 }
 
-template <typename TY>
+// Bounded wait for the GEMM: as mbar_wait, and in the pair form a wait that
+// gives up raises the abort flag of the peer CTA too.
+template <int CG>
+__device__ __forceinline__ bool gemm_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl,
+                                          uint32_t peer_abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    if (*ctl.abort) return false;
+    if (global_ns() - t0 > ctl.limit_ns) {
+      *ctl.abort = 1;
+      if (CG == 2) st_shared_cluster_u32(peer_abort, 1u);
+      if (ctl.status) atomicOr(ctl.status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+// Arrive on a barrier of the even CTA of the pair (this CTA's own when CG = 1).
+template <int CG>
+__device__ __forceinline__ void arrive_leader(uint32_t bar) {
+  if constexpr (CG == 1) {
+    mbar_arrive(bar);
+  } else {
+    mbar_arrive_cluster(mapa_shared(bar, 0));
+  }
+}
+
+template <int CG>
+__device__ __forceinline__ void commit_to(uint32_t bar) {
+  if constexpr (CG == 1) {
+    tc_commit(bar);
+  } else {
+    tc_commit_pair_mc(bar, static_cast<uint16_t>(0x3));
+  }
+}
+
+template <typename TY, int CG>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
     const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
     const float* __restrict__ gamma_ptr, int N, int K, int M, const float* __restrict__ scale,
     const int32_t* __restrict__ rowsum, TY* __restrict__ y, int32_t* __restrict__ acc_out,
     uint32_t* status) {
+  using C = GemmCfg<CG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
-  constexpr int kBarP = 2 * kAStages, kBarU = kBarP + 2 * kPStages, kBarT = kBarU + 2 * kUStages;
-  auto afull_bar = [&](int i) { return sb + kOffBar + 8 * i; };
-  auto aempty_bar = [&](int i) { return sb + kOffBar + 8 * (kAStages + i); };
-  auto pfull_bar = [&](int i) { return sb + kOffBar + 8 * (kBarP + i); };
-  auto pempty_bar = [&](int i) { return sb + kOffBar + 8 * (kBarP + kPStages + i); };
-  auto ufull_bar = [&](int i) { return sb + kOffBar + 8 * (kBarU + i); };
-  auto uempty_bar = [&](int i) { return sb + kOffBar + 8 * (kBarU + kUStages + i); };
-  auto tfull_bar = [&](int i) { return sb + kOffBar + 8 * (kBarT + i); };
-  auto tempty_bar = [&](int i) { return sb + kOffBar + 8 * (kBarT + 2 + i); };
-  const uint32_t done_bar = sb + kOffBar + 8 * (kNumBars - 1);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 16);
-  volatile int* never = reinterpret_cast<volatile int*>(smem + kOffMisc + 32);
+  constexpr int kBarP = 2 * C::kAStages, kBarU = kBarP + 2 * C::kPStages, kBarT = kBarU + 2 * C::kUStages;
+  auto afull_bar = [&](int i) { return sb + C::kOffBar + 8 * i; };
+  auto aempty_bar = [&](int i) { return sb + C::kOffBar + 8 * (C::kAStages + i); };
+  auto pfull_bar = [&](int i) { return sb + C::kOffBar + 8 * (kBarP + i); };
+  auto pempty_bar = [&](int i) { return sb + C::kOffBar + 8 * (kBarP + C::kPStages + i); };
+  auto ufull_bar = [&](int i) { return sb + C::kOffBar + 8 * (kBarU + i); };
+  auto uempty_bar = [&](int i) { return sb + C::kOffBar + 8 * (kBarU + C::kUStages + i); };
+  auto tfull_bar = [&](int i) { return sb + C::kOffBar + 8 * (kBarT + i); };
+  auto tempty_bar = [&](int i) { return sb + C::kOffBar + 8 * (kBarT + 2 + i); };
+  const uint32_t done_bar = sb + C::kOffBar + 8 * (C::kNumBars - 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 16);
+  volatile int* never = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 32);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+  const uint32_t peer_abort = CG == 2 ? mapa_shared(sb + C::kOffMisc + 16, rank ^ 1u) : 0u;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kAStages; ++i) {
-      mbar_init(afull_bar(i), 1);
-      mbar_init(aempty_bar(i), 1);
+    for (int i = 0; i < C::kAStages; ++i) {
+      mbar_init(afull_bar(i), 1);   // the even CTA's expect-tx arrive (bytes of both CTAs)
+      mbar_init(aempty_bar(i), 1);  // MMA commit
     }
-    for (int i = 0; i < kPStages; ++i) {
+    for (int i = 0; i < C::kPStages; ++i) {
       mbar_init(pfull_bar(i), 1);
-      mbar_init(pempty_bar(i), kUnpackThreads);
+      mbar_init(pempty_bar(i), kUnpackWarps);
     }
-    for (int i = 0; i < kUStages; ++i) {
-      mbar_init(ufull_bar(i), kUnpackThreads);
+    for (int i = 0; i < C::kUStages; ++i) {
+      mbar_init(ufull_bar(i), kUnpackWarps * CG);  // unpack warps of both CTAs
       mbar_init(uempty_bar(i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(tfull_bar(i), 1);
-      mbar_init(tempty_bar(i), 128);
+      mbar_init(tempty_bar(i), kEpiWarps * CG);  // epilogue warps of both CTAs
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
@@ -155,42 +213,66 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
   if (warp == 0 && lane == 0) tma_prefetch_desc(&tmap_a);
   if (warp == 2 && lane == 0) tma_prefetch_desc(&tmap_b);
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    tmem_relinquish();
+    if constexpr (CG == 1) {
+      tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+      tmem_relinquish();
+    } else {
+      tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+      tmem_relinquish_pair();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 1) {
+    __syncthreads();
+  } else {
+    cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive
+  }
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Only the roles that touch the activations, scales, row sums or outputs
+  // wait for the preceding kernel; the weight tiles (never written by a
+  // kernel that lets its dependents start early) are fetched and unpacked
+  // meanwhile.
   griddep_launch_dependents();
-  griddep_wait();  // activations, scales and row sums come from the preceding kernel
 
   const WaitCtl ctl{status, abort_flag, kWaitLimitNs};
-  const int m_tiles = (M + kBM - 1) / kBM;
+  const int m_tiles = (M + kBM * CG - 1) / (kBM * CG);
   const int n_tiles = (N + kBN - 1) / kBN;
   const int tiles = m_tiles * n_tiles;
   const int kblocks = (K + kBK - 1) / kBK;
+  const int cluster_id = blockIdx.x / CG, n_clusters = gridDim.x / CG;
 
   if (warp == 0 || warp == 2) {
     if (lane == 0) {
       // warp 0: activation tiles; warp 2: packed weight tiles.
       const bool is_a = (warp == 0);
-      const int nst = is_a ? kAStages : kPStages;
+      if (is_a) griddep_wait();  // the activation codes come from the preceding kernel
+      const int nst = is_a ? C::kAStages : C::kPStages;
       int it = 0, s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+      for (int tile = cluster_id; ok && tile < tiles; tile += n_clusters) {
         const int mt = tile % m_tiles, nt = tile / m_tiles;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          const uint32_t full = is_a ? afull_bar(s) : pfull_bar(s);
-          if (!mbar_wait(is_a ? aempty_bar(s) : pempty_bar(s), ph ^ 1, ctl)) { ok = false; break; }
+          if (!gemm_wait<CG>(is_a ? aempty_bar(s) : pempty_bar(s), ph ^ 1, ctl, peer_abort)) {
+            ok = false;
+            break;
+          }
           if (is_a) {
-            mbar_arrive_expect_tx(full, kABytes);
-            tma_load_2d(sb + kOffA + s * kABytes, &tmap_a, kb * kBK, mt * kBM, full);
+            const uint32_t dst = sb + C::kOffA + s * kABytes;
+            const int row = mt * kBM * CG + static_cast<int>(rank) * kBM;
+            if constexpr (CG == 1) {
+              mbar_arrive_expect_tx(afull_bar(s), kABytes);
+              tma_load_2d(dst, &tmap_a, kb * kBK, row, afull_bar(s));
+            } else {
+              if (rank == 0) mbar_arrive_expect_tx(afull_bar(s), CG * kABytes);
+              tma_load_2d_pair(dst, &tmap_a, kb * kBK, row, mapa_shared(afull_bar(s), 0));
+            }
           } else {
-            mbar_arrive_expect_tx(full, kBPBytes);
-            tma_load_2d(sb + kOffBP + s * kBPBytes, &tmap_b, kb * (kBK / 4), nt * kBN, full);
+            mbar_arrive_expect_tx(pfull_bar(s), C::kBPBytes);
+            tma_load_2d(sb + C::kOffBP + s * C::kBPBytes, &tmap_b, kb * (kBK / 4),
+                        nt * kBN + static_cast<int>(rank) * C::kRowsB, pfull_bar(s));
           }
           if (++s == nst) { s = 0; ph ^= 1; }
         }
@@ -198,53 +280,71 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
       if (!ok) {
         // Let copies already in flight land before the block's shared memory goes away.
         const WaitCtl drain{nullptr, never, 100000000ull};
-        for (int i = (it > nst ? it - nst : 0); i < it; ++i)
-          mbar_wait(is_a ? afull_bar(i % nst) : pfull_bar(i % nst), (i / nst) & 1, drain);
+        if (!is_a || CG == 1) {
+          for (int i = (it > nst ? it - nst : 0); i < it; ++i)
+            gemm_wait<1>(is_a ? afull_bar(i % nst) : pfull_bar(i % nst), (i / nst) & 1, drain, 0u);
+        } else {
+          // Completion of the pair's activation copies is counted in the even
+          // CTA; give copies in flight a fixed millisecond instead.
+          const uint64_t t0 = global_ns();
+          while (global_ns() - t0 < 1000000ull) __nanosleep(10000);
+        }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       int it = 0, tc = 0;
       bool ok = true, issued = false;
-      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x, ++tc) {
+      for (int tile = cluster_id; ok && tile < tiles; tile += n_clusters, ++tc) {
         const int a = tc & 1;
-        if (!mbar_wait(tempty_bar(a), ((tc >> 1) & 1) ^ 1, ctl)) { ok = false; break; }
+        if (!gemm_wait<CG>(tempty_bar(a), ((tc >> 1) & 1) ^ 1, ctl, peer_abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + a * kBN;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          const int s = it % kAStages, u = it % kUStages;
-          if (!mbar_wait(afull_bar(s), (it / kAStages) & 1, ctl)) { ok = false; break; }
-          if (!mbar_wait(ufull_bar(u), (it / kUStages) & 1, ctl)) { ok = false; break; }
+          const int s = it % C::kAStages, u = it % C::kUStages;
+          if (!gemm_wait<CG>(afull_bar(s), (it / C::kAStages) & 1, ctl, peer_abort)) { ok = false; break; }
+          if (!gemm_wait<CG>(ufull_bar(u), (it / C::kUStages) & 1, ctl, peer_abort)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t adesc = sw128_kmajor_desc(sb + kOffA + s * kABytes);
-          const uint64_t bdesc = sw128_kmajor_desc(sb + kOffBU + u * kBUBytes);
+          const uint64_t adesc = sw128_kmajor_desc(sb + C::kOffA + s * kABytes);
+          const uint64_t bdesc = sw128_kmajor_desc(sb + C::kOffBU + u * C::kBUBytes);
 #pragma unroll
           for (int k = 0; k < kBK / 32; ++k) {
-            tc_mma_i8(d_tmem, adesc + 2 * k, bdesc + 2 * k, kIdesc, (kb | k) != 0);
+            if constexpr (CG == 1) {
+              tc_mma_i8(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::kIdesc, (kb | k) != 0);
+            } else {
+              tc_mma_i8_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::kIdesc, (kb | k) != 0);
+            }
           }
           issued = true;
-          tc_commit(aempty_bar(s));
-          tc_commit(uempty_bar(u));
+          commit_to<CG>(aempty_bar(s));
+          commit_to<CG>(uempty_bar(u));
         }
-        if (ok) tc_commit(tfull_bar(a));
+        if (ok) commit_to<CG>(tfull_bar(a));
       }
       if (issued) {
-        // Every MMA must be finished before tensor memory is released.
-        tc_commit(done_bar);
+        // Every MMA must be finished before tensor memory is released (the odd
+        // CTA learns of it through the closing cluster barrier).
+        if constexpr (CG == 1) {
+          tc_commit(done_bar);
+        } else {
+          tc_commit_pair(done_bar);
+        }
         const WaitCtl drain{nullptr, never, 100000000ull};
-        mbar_wait(done_bar, 0, drain);
+        gemm_wait<1>(done_bar, 0, drain, 0u);
       }
     }
-  } else if (warp >= 4 && warp < 12) {
+  } else if (warp >= 4 && warp < 4 + kUnpackWarps) {
     const int ut = threadIdx.x - 128;
     int it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+    for (int tile = cluster_id; ok && tile < tiles; tile += n_clusters) {
       for (int kb = 0; kb < kblocks; ++kb, ++it) {
-        const int s = it % kPStages, u = it % kUStages;
-        if (!mbar_wait(pfull_bar(s), (it / kPStages) & 1, ctl)) { ok = false; break; }
-        constexpr int kPer = kBPBytes / 16 / kUnpackThreads;  // packed uint4 per thread
-        const uint4* bp = reinterpret_cast<const uint4*>(smem + kOffBP + s * kBPBytes);
+        const int s = it % C::kPStages, u = it % C::kUStages;
+        // Wait outcomes are made warp-uniform: the warp then syncs and arrives as one.
+        ok = __all_sync(0xffffffffu, gemm_wait<1>(pfull_bar(s), (it / C::kPStages) & 1, ctl, peer_abort));
+        if (!ok) break;
+        constexpr int kPer = C::kBPBytes / 16 / kUnpackThreads;  // packed uint4 per thread
+        const uint4* bp = reinterpret_cast<const uint4*>(smem + C::kOffBP + s * C::kBPBytes);
         uint4 codes[kPer][4];
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
@@ -257,37 +357,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
                                      (w >> 6) & 0x03030303u);
           }
         }
-        if (!mbar_wait(uempty_bar(u), ((it / kUStages) & 1) ^ 1, ctl)) { ok = false; break; }
-        uint8_t* bu = smem + kOffBU + u * kBUBytes;
+        ok = __all_sync(0xffffffffu,
+                        gemm_wait<CG>(uempty_bar(u), ((it / C::kUStages) & 1) ^ 1, ctl, peer_abort));
+        if (!ok) break;
+        uint8_t* bu = smem + C::kOffBU + u * C::kBUBytes;
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
           const int q = ut + j * kUnpackThreads;
-          const int r = q >> 1;              // weight row in the tile (32 packed bytes per row)
-          const int c0 = (q & 1) * 4;        // first 16-byte chunk (= packed word) of this uint4
+          const int r = q >> 1;        // weight row in the CTA's tile (32 packed bytes per row)
+          const int c0 = (q & 1) * 4;  // first 16-byte chunk (= packed word) of this uint4
           uint8_t* rowp = bu + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             *reinterpret_cast<uint4*>(rowp + (((c0 + i) ^ (r & 7)) << 4)) = codes[j][i];
         }
-        // The stores above consumed every packed word, so no read of the packed
-        // slot can still be in flight: hand it back to its producer.
-        mbar_arrive(pempty_bar(s));
         fence_proxy_async_smem();
-        mbar_arrive(ufull_bar(u));
+        __syncwarp();
+        if (lane == 0) {
+          // The warp's stores consumed its packed words: release the packed
+          // slot, and report the codes to the MMA issuer.
+          mbar_arrive(pempty_bar(s));
+          arrive_leader<CG>(ufull_bar(u));
+        }
       }
     }
   } else if (warp >= 12) {
     const int q = warp & 3;  // tensor-memory lane quarter this warp may read
+    griddep_wait();          // scales and row sums come from the preceding kernel; y may be read by it
     const float gamma = __ldg(gamma_ptr);
     int tc = 0;
-    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
+    for (int tile = cluster_id; tile < tiles; tile += n_clusters, ++tc) {
       const int mt = tile % m_tiles, nt = tile / m_tiles;
       const int a = tc & 1;
       // tcgen05.ld below is warp-collective: take the wait's outcome warp-wide.
-      const bool got = mbar_wait(tfull_bar(a), (tc >> 1) & 1, ctl);
+      const bool got = gemm_wait<CG>(tfull_bar(a), (tc >> 1) & 1, ctl, peer_abort);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      const int m = mt * kBM + q * 32 + lane;
+      const int m = mt * kBM * CG + static_cast<int>(rank) * kBM + q * 32 + lane;
       const bool mvalid = m < M;
       float gs = 0.0f;
       int rs = 0;
@@ -304,14 +410,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
         if (mvalid && n0 < N) store_row32<TY>(y, acc_out, static_cast<size_t>(m) * N, n0, N, r, rs, gs);
       }
       tc_fence_before();
-      mbar_arrive(tempty_bar(a));
+      __syncwarp();
+      if (lane == 0) arrive_leader<CG>(tempty_bar(a));
     }
   }
 
-  __syncthreads();
+  tc_fence_before();
+  if constexpr (CG == 1) {
+    __syncthreads();
+  } else {
+    cluster_sync_all();  // no CTA leaves while its peer may still signal it
+  }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (CG == 1) {
+      tmem_dealloc(tmem_base, kTmemCols);
+    } else {
+      tmem_dealloc_pair(tmem_base, kTmemCols);
+    }
   }
 }
 
@@ -344,33 +460,76 @@ static bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename TY>
+template <typename TY, int CG>
 static cudaError_t launch_gemm_t(const ProductArgs& a, cudaStream_t stream, bool pdl) {
+  using C = GemmCfg<CG>;
   CUtensorMap ta, tb;
   if (!make_map_2d(&ta, a.xq, static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M), kBK, kBM,
                    CU_TENSOR_MAP_SWIZZLE_128B, static_cast<uint64_t>(a.ldx)) ||
-      !make_map_2d(&tb, a.packed, static_cast<uint64_t>(a.K / 4), static_cast<uint64_t>(a.N),
-                   kBK / 4, kBN, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+      !make_map_2d(&tb, a.packed, static_cast<uint64_t>(a.K / 4), static_cast<uint64_t>(a.N), kBK / 4,
+                   C::kRowsB, CU_TENSOR_MAP_SWIZZLE_NONE)) {
     return cudaErrorInvalidValue;
   }
-  static bool attr_set = false;  // per template instance; the attribute is per function
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<TY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
+  static int max_clusters = 0;  // per template instance; attributes are per function
+  if (max_clusters == 0) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<TY, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    int n = num_sms() / CG;
+    if (CG > 1) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(CG * n);
+      q.blockDim = dim3(kGemmThreads);
+      q.dynamicSmemBytes = C::kSmemBytes;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = CG;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      q.attrs = at;
+      q.numAttrs = 1;
+      int c = 0;
+      e = cudaOccupancyMaxActiveClusters(&c, gemm_kernel<TY, CG>, &q);
+      if (e != cudaSuccess) return e;
+      if (c > 0 && c < n) n = c;
+    }
+    max_clusters = n > 0 ? n : 1;
   }
-  const int tiles = ((a.M + kBM - 1) / kBM) * ((a.N + kBN - 1) / kBN);
-  const int grid = tiles < num_sms() ? tiles : num_sms();
-  return launch(gemm_kernel<TY>, dim3(grid), dim3(kGemmThreads), kSmemBytes, stream, pdl, ta, tb,
-                a.gamma, a.N, a.K, a.M, a.scale, a.rowsum, static_cast<TY*>(a.y), a.acc_out,
-                a.status);
+  const int tiles = ((a.M + kBM * CG - 1) / (kBM * CG)) * ((a.N + kBN - 1) / kBN);
+  const int clusters = tiles < max_clusters ? tiles : max_clusters;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CG * clusters);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (CG > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = CG;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<TY, CG>, ta, tb, a.gamma, a.N, a.K, a.M, a.scale, a.rowsum,
+                            static_cast<TY*>(a.y), a.acc_out, a.status);
 }
 
+// Up to 128 tokens one CTA per tile; beyond, CTA pairs on 256-token tiles.
 cudaError_t launch_gemm(const ProductArgs& a, cudaStream_t stream, bool pdl) {
   if (a.M <= 0) return cudaSuccess;
-  return a.y_type == kOutBF16 ? launch_gemm_t<__nv_bfloat16>(a, stream, pdl)
-                              : launch_gemm_t<float>(a, stream, pdl);
+  const bool pair = a.M > kBM;
+  if (a.y_type == kOutBF16)
+    return pair ? launch_gemm_t<__nv_bfloat16, 2>(a, stream, pdl) : launch_gemm_t<__nv_bfloat16, 1>(a, stream, pdl);
+  return pair ? launch_gemm_t<float, 2>(a, stream, pdl) : launch_gemm_t<float, 1>(a, stream, pdl);
 }
 
 }  // namespace bl
