@@ -55,12 +55,16 @@ struct GemmCfg {
   static constexpr int kBPBytes = kRowsB * kBK / 4;  // packed weight tile per CTA
   static constexpr int kBUBytes = kRowsB * kBK;      // unpacked code tile per CTA
   static constexpr int kAStages = CG == 1 ? 5 : 6;
-  static constexpr int kPStages = CG == 1 ? 6 : 8;
+  static constexpr int kPStages = CG == 1 ? 6 : 6;
   static constexpr int kUStages = CG == 1 ? 3 : 4;
+  // Output staging of the pair form: per epilogue warp two 32 x 32 boxes of
+  // up to 4-byte elements, written out by TMA bulk-tensor stores.
+  static constexpr int kOutWarpBytes = CG == 2 ? 2 * 4096 : 0;
   static constexpr int kOffA = 0;
   static constexpr int kOffBU = kOffA + kAStages * kABytes;
   static constexpr int kOffBP = kOffBU + kUStages * kBUBytes;
-  static constexpr int kOffBar = kOffBP + kPStages * kBPBytes;
+  static constexpr int kOffOut = kOffBP + kPStages * kBPBytes;
+  static constexpr int kOffBar = kOffOut + kEpiWarps * kOutWarpBytes;
   static constexpr int kNumBars = 2 * (kAStages + kPStages + kUStages) + 5;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
@@ -69,6 +73,7 @@ struct GemmCfg {
       (2u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | (((kBM * CG) >> 4) << 24);
   static_assert(kSmemBytes <= 232448, "shared memory per block");
   static_assert(kBPBytes / 16 % kUnpackThreads == 0, "packed words per unpack thread");
+  static_assert(kOffOut % 1024 == 0, "swizzled staging alignment");
 };
 
 template <typename TY>
@@ -123,6 +128,47 @@ __device__ __forceinline__ void store_row32(TY* __restrict__ y, int32_t* __restr
   }
 }
 
+// One 32-token x 32-output box of the epilogue through shared memory: lane i
+// holds token row i.  The box is written in the swizzle of its tensor map
+// (64-byte rows for bf16, 128-byte rows for 4-byte elements) so that the
+// lanes' 16-byte stores are free of bank conflicts, then one lane issues the
+// TMA store, which skips elements outside the output.
+__device__ __forceinline__ void stage_box_b16(uint8_t* buf, int lane, const uint32_t (&p)[16]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+        make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
+}
+__device__ __forceinline__ void stage_box_b32(uint8_t* buf, int lane, const uint32_t (&w)[32]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+        make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+}
+
+template <typename TY>
+__device__ __forceinline__ void stage_y(uint8_t* buf, int lane, const uint32_t (&r)[32], int rs, float gs) {
+  if constexpr (sizeof(TY) == 2) {
+    uint32_t p[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const __nv_bfloat16 lo =
+          __float2bfloat16_rn(__fmul_rn(static_cast<float>(static_cast<int>(r[2 * i]) - rs), gs));
+      const __nv_bfloat16 hi =
+          __float2bfloat16_rn(__fmul_rn(static_cast<float>(static_cast<int>(r[2 * i + 1]) - rs), gs));
+      p[i] = static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
+             (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+    }
+    stage_box_b16(buf, lane, p);
+  } else {
+    uint32_t w[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      w[i] = __float_as_uint(__fmul_rn(static_cast<float>(static_cast<int>(r[i]) - rs), gs));
+    stage_box_b32(buf, lane, w);
+  }
+}
+
 // Bounded wait for the GEMM: as mbar_wait, and in the pair form a wait that
 // gives up raises the abort flag of the peer CTA too.
 template <int CG>
@@ -164,6 +210,7 @@ __device__ __forceinline__ void commit_to(uint32_t bar) {
 template <typename TY, int CG>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
     const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+    const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_acc, int tma_out,
     const float* __restrict__ gamma_ptr, int N, int K, int M, const float* __restrict__ scale,
     const int32_t* __restrict__ rowsum, TY* __restrict__ y, int32_t* __restrict__ acc_out,
     uint32_t* status) {
@@ -385,6 +432,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
     const int q = warp & 3;  // tensor-memory lane quarter this warp may read
     griddep_wait();          // scales and row sums come from the preceding kernel; y may be read by it
     const float gamma = __ldg(gamma_ptr);
+    const bool staged = C::kOutWarpBytes > 0 && tma_out;
+    uint8_t* obuf = smem + C::kOffOut + (warp - 12) * C::kOutWarpBytes;
+    int ob = 0;  // staging buffer of the next box
+    if (staged && lane == 0) {
+      tma_prefetch_desc(&tmap_y);
+      if (acc_out) tma_prefetch_desc(&tmap_acc);
+    }
     int tc = 0;
     for (int tile = cluster_id; tile < tiles; tile += n_clusters, ++tc) {
       const int mt = tile % m_tiles, nt = tile / m_tiles;
@@ -393,7 +447,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
       const bool got = gemm_wait<CG>(tfull_bar(a), (tc >> 1) & 1, ctl, peer_abort);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      const int m = mt * kBM * CG + static_cast<int>(rank) * kBM + q * 32 + lane;
+      const int m0 = mt * kBM * CG + static_cast<int>(rank) * kBM + q * 32;  // first row of this warp
+      const int m = m0 + lane;
       const bool mvalid = m < M;
       float gs = 0.0f;
       int rs = 0;
@@ -407,12 +462,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kBN + c * 32, r);
         tmem_ld_wait();
         const int n0 = nt * kBN + c * 32;
-        if (mvalid && n0 < N) store_row32<TY>(y, acc_out, static_cast<size_t>(m) * N, n0, N, r, rs, gs);
+        if (staged) {
+          if (n0 < N && m0 < M) {  // warp-uniform
+            if (acc_out) {
+              // y and the accumulators: one box each, both buffers, every step.
+              if (lane == 0) bulk_wait_group_read<0>();
+              __syncwarp();
+              stage_y<TY>(obuf, lane, r, rs, gs);
+              uint32_t w[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) w[i] = static_cast<uint32_t>(static_cast<int>(r[i]) - rs);
+              stage_box_b32(obuf + 4096, lane, w);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmap_y, smem_u32(obuf), n0, m0);
+                tma_store_2d(&tmap_acc, smem_u32(obuf + 4096), n0, m0);
+                bulk_commit_group();
+              }
+            } else {
+              // The buffer's previous box (two groups ago) must have been read.
+              if (lane == 0) bulk_wait_group_read<1>();
+              __syncwarp();
+              uint8_t* b = obuf + ob * 4096;
+              stage_y<TY>(b, lane, r, rs, gs);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmap_y, smem_u32(b), n0, m0);
+                bulk_commit_group();
+              }
+              ob ^= 1;
+            }
+          }
+        } else if (mvalid && n0 < N) {
+          store_row32<TY>(y, acc_out, static_cast<size_t>(m) * N, n0, N, r, rs, gs);
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) arrive_leader<CG>(tempty_bar(a));
     }
+    if (staged && lane == 0) bulk_wait_group_all();  // stores done before the block's shared memory goes away
   }
 
   tc_fence_before();
@@ -447,17 +538,19 @@ void* tensor_map_encoder() {
   return fn;
 }
 
+// 2-D map over a row-major matrix of `outer` rows of `inner` elements, rows
+// `pitch` bytes apart (default: dense).
 static bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                        uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz, uint64_t pitch = 0) {
+                        uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz, uint64_t pitch = 0,
+                        CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_UINT8, uint32_t esize = 1) {
   EncodeTiledFn fn = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {pitch ? pitch : inner};  // bytes (uint8 elements)
+  const cuuint64_t strides[1] = {pitch ? pitch : inner * esize};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <typename TY, int CG>
@@ -469,6 +562,23 @@ static cudaError_t launch_gemm_t(const ProductArgs& a, cudaStream_t stream, bool
       !make_map_2d(&tb, a.packed, static_cast<uint64_t>(a.K / 4), static_cast<uint64_t>(a.N), kBK / 4,
                    C::kRowsB, CU_TENSOR_MAP_SWIZZLE_NONE)) {
     return cudaErrorInvalidValue;
+  }
+  // The pair form writes its outputs by TMA when the rows are 16-byte
+  // multiples and the buffers 16-byte aligned; otherwise by plain stores.
+  CUtensorMap ty = {}, tacc = {};
+  const uint64_t esz = sizeof(TY);
+  int tma_out = CG == 2 && (static_cast<uint64_t>(a.N) * esz) % 16 == 0 &&
+                (static_cast<uint64_t>(a.N) * 4) % 16 == 0 && reinterpret_cast<uintptr_t>(a.y) % 16 == 0 &&
+                reinterpret_cast<uintptr_t>(a.acc_out) % 16 == 0;
+  if (tma_out) {
+    const bool ok_y = make_map_2d(&ty, a.y, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.M), 32, 32,
+                                  esz == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, 0,
+                                  esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                                  static_cast<uint32_t>(esz));
+    const bool ok_acc = !a.acc_out || make_map_2d(&tacc, a.acc_out, static_cast<uint64_t>(a.N),
+                                                  static_cast<uint64_t>(a.M), 32, 32, CU_TENSOR_MAP_SWIZZLE_128B,
+                                                  0, CU_TENSOR_MAP_DATA_TYPE_INT32, 4);
+    if (!ok_y || !ok_acc) return cudaErrorInvalidValue;
   }
   static int max_clusters = 0;  // per template instance; attributes are per function
   if (max_clusters == 0) {
@@ -519,8 +629,8 @@ static cudaError_t launch_gemm_t(const ProductArgs& a, cudaStream_t stream, bool
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, gemm_kernel<TY, CG>, ta, tb, a.gamma, a.N, a.K, a.M, a.scale, a.rowsum,
-                            static_cast<TY*>(a.y), a.acc_out, a.status);
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<TY, CG>, ta, tb, ty, tacc, tma_out, a.gamma, a.N, a.K, a.M,
+                            a.scale, a.rowsum, static_cast<TY*>(a.y), a.acc_out, a.status);
 }
 
 // Up to 128 tokens one CTA per tile; beyond, CTA pairs on 256-token tiles.

@@ -205,6 +205,20 @@ def test_forward_prefill_ragged_full():
     _full_case(300, 1000, 576, "bf16", torch.bfloat16, tb.PATH_AUTO, seed=77)
 
 
+@pytest.mark.parametrize("M,N,K,ydtype", [(300, 1000, 576, torch.bfloat16), (300, 1000, 576, torch.float32),
+                                          (513, 772, 320, torch.float32), (2048, 512, 256, torch.bfloat16)])
+def test_forward_y_only_many_tokens(M, N, K, ydtype):
+    """Without the accumulator output (the serving call), checked everywhere."""
+    seed = M + N
+    W = weights(N, K, seed=seed)
+    packed_ref, gamma_ref, T = oracle.pack_weights(W)
+    x, xf = activations(M, K, seed=seed + 1, dtype="bf16")
+    acc_ref, y_ref, *_ = oracle.forward(T, gamma_ref, xf)
+    tb.set_path(tb.PATH_AUTO)
+    y = tb.forward(dev(packed_ref), dev(np.array([gamma_ref], np.float32)), x, out_dtype=ydtype)
+    assert_y_matches(y, y_ref, acc_ref)
+
+
 @pytest.mark.parametrize("K", [2560, 8640])
 def test_forward_quantized_matches_forward(K):
     W = weights(640, K, seed=5)
