@@ -16,17 +16,17 @@
 //           per SM the unpack stores and the tensor cores' shared-memory reads
 //           of codes are halved.  The MMA thread of the even CTA issues for
 //           both; commits are multicast to both CTAs.
-// Warp roles in a persistent block of 16 warps (one block per SM):
+// Warp roles in a persistent block (one per SM) of 16 warps (12 in the pair form):
 //   warp 0      TMA producer of the activation tiles (128-byte swizzle);
 //   warp 2      TMA producer of the packed weight tiles, on a ring of its own
 //               that the unpack warps release once their stores have consumed
 //               the words, so weight tiles are requested well ahead;
 //   warp 1      tensor-memory owner; in the even CTA, the single thread that
 //               issues the 4 tcgen05.mma (K = 32 each) per k-block;
-//   warps 4-11  unpack: packed words -> one 16-byte chunk of codes
+//   warps 4-11  unpack (4-7 in the pair form): packed words -> 16-byte chunks of codes
 //               ((w >> 2j) & 0x03030303, j = 0..3) written at its 128-byte
 //               swizzle position, a proxy fence, then one arrive per warp;
-//   warps 12-15 epilogue: tcgen05.ld of the int32 accumulators, then
+//   next 4      epilogue: tcgen05.ld of the int32 accumulators, then
 //               y = (acc - rowsum[m]) * (gamma / s[m]) stored as fp32 / bf16.
 // Two accumulators (2 x 256 tensor-memory columns) let the epilogue of one
 // tile overlap the main loop of the next.  Every mbarrier wait is bounded in
@@ -43,14 +43,18 @@ namespace bl {
 
 constexpr int kBM = 128, kBN = 256, kBK = 128;
 constexpr int kABytes = kBM * kBK;  // 16 KB activation tile per CTA
-constexpr int kGemmThreads = 512;
-constexpr int kUnpackWarps = 8;     // warps 4-11
-constexpr int kUnpackThreads = 32 * kUnpackWarps;
-constexpr int kEpiWarps = 4;        // warps 12-15
+constexpr int kEpiWarps = 4;        // the last four warps of the block
 constexpr uint32_t kTmemCols = 512;
 
 template <int CG>
 struct GemmCfg {
+  // Warps 4 .. 4 + kUnpackWarps - 1 unpack, the next four run the epilogue.
+  // The pair form unpacks half a weight tile per CTA and needs half the
+  // unpack warps (measured: as fast, and the smaller block is slightly faster).
+  static constexpr int kUnpackWarps = CG == 1 ? 8 : 4;
+  static constexpr int kUnpackThreads = 32 * kUnpackWarps;
+  static constexpr int kEpiWarp0 = 4 + kUnpackWarps;
+  static constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
   static constexpr int kRowsB = kBN / CG;            // weight rows unpacked by one CTA
   static constexpr int kBPBytes = kRowsB * kBK / 4;  // packed weight tile per CTA
   static constexpr int kBUBytes = kRowsB * kBK;      // unpacked code tile per CTA
@@ -73,6 +77,7 @@ struct GemmCfg {
       (2u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | (((kBM * CG) >> 4) << 24);
   static_assert(kSmemBytes <= 232448, "shared memory per block");
   static_assert(kBPBytes / 16 % kUnpackThreads == 0, "packed words per unpack thread");
+  static_assert(kEpiWarp0 % 4 == 0, "epilogue warp w reads tensor-memory lanes 32 * (w % 4) ..");
   static_assert(kOffOut % 1024 == 0, "swizzled staging alignment");
 };
 
@@ -208,7 +213,7 @@ __device__ __forceinline__ void commit_to(uint32_t bar) {
 }
 
 template <typename TY, int CG>
-__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
+__global__ void __maxnreg__(128) gemm_kernel(
     const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
     const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_acc, int tma_out,
     const float* __restrict__ gamma_ptr, int N, int K, int M, const float* __restrict__ scale,
@@ -242,10 +247,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
     }
     for (int i = 0; i < C::kPStages; ++i) {
       mbar_init(pfull_bar(i), 1);
-      mbar_init(pempty_bar(i), kUnpackWarps);
+      mbar_init(pempty_bar(i), C::kUnpackWarps);
     }
     for (int i = 0; i < C::kUStages; ++i) {
-      mbar_init(ufull_bar(i), kUnpackWarps * CG);  // unpack warps of both CTAs
+      mbar_init(ufull_bar(i), C::kUnpackWarps * CG);  // unpack warps of both CTAs
       mbar_init(uempty_bar(i), 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -380,7 +385,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
         gemm_wait<1>(done_bar, 0, drain, 0u);
       }
     }
-  } else if (warp >= 4 && warp < 4 + kUnpackWarps) {
+  } else if (warp >= 4 && warp < C::kEpiWarp0) {
     const int ut = threadIdx.x - 128;
     int it = 0;
     bool ok = true;
@@ -390,12 +395,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
         // Wait outcomes are made warp-uniform: the warp then syncs and arrives as one.
         ok = __all_sync(0xffffffffu, gemm_wait<1>(pfull_bar(s), (it / C::kPStages) & 1, ctl, peer_abort));
         if (!ok) break;
-        constexpr int kPer = C::kBPBytes / 16 / kUnpackThreads;  // packed uint4 per thread
+        constexpr int kPer = C::kBPBytes / 16 / C::kUnpackThreads;  // packed uint4 per thread
         const uint4* bp = reinterpret_cast<const uint4*>(smem + C::kOffBP + s * C::kBPBytes);
         uint4 codes[kPer][4];
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
-          const uint4 v = bp[ut + j * kUnpackThreads];
+          const uint4 v = bp[ut + j * C::kUnpackThreads];
           const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -410,7 +415,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
         uint8_t* bu = smem + C::kOffBU + u * C::kBUBytes;
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
-          const int q = ut + j * kUnpackThreads;
+          const int q = ut + j * C::kUnpackThreads;
           const int r = q >> 1;        // weight row in the CTA's tile (32 packed bytes per row)
           const int c0 = (q & 1) * 4;  // first 16-byte chunk (= packed word) of this uint4
           uint8_t* rowp = bu + (r >> 3) * 1024 + (r & 7) * 128;
@@ -428,12 +433,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(
         }
       }
     }
-  } else if (warp >= 12) {
+  } else if (warp >= C::kEpiWarp0) {
     const int q = warp & 3;  // tensor-memory lane quarter this warp may read
     griddep_wait();          // scales and row sums come from the preceding kernel; y may be read by it
     const float gamma = __ldg(gamma_ptr);
     const bool staged = C::kOutWarpBytes > 0 && tma_out;
-    uint8_t* obuf = smem + C::kOffOut + (warp - 12) * C::kOutWarpBytes;
+    uint8_t* obuf = smem + C::kOffOut + (warp - C::kEpiWarp0) * C::kOutWarpBytes;
     int ob = 0;  // staging buffer of the next box
     if (staged && lane == 0) {
       tma_prefetch_desc(&tmap_y);
@@ -589,7 +594,7 @@ static cudaError_t launch_gemm_t(const ProductArgs& a, cudaStream_t stream, bool
     if (CG > 1) {
       cudaLaunchConfig_t q = {};
       q.gridDim = dim3(CG * n);
-      q.blockDim = dim3(kGemmThreads);
+      q.blockDim = dim3(C::kThreads);
       q.dynamicSmemBytes = C::kSmemBytes;
       cudaLaunchAttribute at[1];
       at[0].id = cudaLaunchAttributeClusterDimension;
@@ -610,7 +615,7 @@ static cudaError_t launch_gemm_t(const ProductArgs& a, cudaStream_t stream, bool
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(CG * clusters);
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];

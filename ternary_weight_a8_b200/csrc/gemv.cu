@@ -20,9 +20,10 @@
 //  * One producer thread streams the block's units with TMA in stages of 64
 //    rows x 256 bytes (1024 inputs, two 128-byte halves), in the 128-byte
 //    swizzle so that the lanes' 16-byte reads are conflict-free, through a deep ring of
-//    mbarrier-tracked buffers that runs on from one unit to the next.  The
-//    first unit's loads start before the grid-dependency wait (programmatic
-//    dependent launch): weights never depend on the preceding kernel.
+//    mbarrier-tracked buffers that runs on from one unit to the next.  A whole
+//    ring of the first unit's weight loads is issued before the
+//    grid-dependency wait (programmatic dependent launch): weights never
+//    depend on the preceding kernel, so they stream while it still runs.
 //  * Activations quantised by the quantisation kernel stream with the
 //    weights: each stage also brings the stage's 1024 inputs of every token,
 //    loaded through a 3-D tensor map (token, 128-input block, byte) in the
@@ -319,13 +320,45 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       bool waited = false;  // grid dependency
       bool ok = true;
       int unit = blockIdx.x;
+      int st0 = 0;  // first stage of the current unit still to issue
+      if constexpr (kStream) {
+        // Before the grid dependency: the weights of the first unit's first
+        // stages (a whole ring of them); their activation tiles, written by
+        // the preceding kernel, follow once it has finished.
+        if (unit < P.total_units) {
+          int l = 0;
+          while (l + 1 < P.n_layers && unit >= P.layer[l + 1].unit0) ++l;
+          const GvLayer& L = P.layer[l];
+          const int rb = unit - L.unit0;
+          const int nst = (L.K + kGvStageK - 1) / kGvStageK;
+          const int pre = nst < nring ? nst : nring;
+          for (int st = 0; st < pre; ++st) {  // fresh slots 0 .. pre-1
+            tags[st] = unit;
+            const uint32_t full = bar0 + 8 * st, dst = ring + st * kSlot;
+            mbar_arrive_expect_tx(full, kGvStageBytes + 2 * TT * 4 * 128);
+            tma_load_2d(dst, &L.tmap, st * 256, rb * kGvRows, full);
+            tma_load_2d(dst + kGvStageBytes / 2, &L.tmap, st * 256 + 128, rb * kGvRows, full);
+          }
+          griddep_wait();  // the codes come from the preceding kernel
+          waited = true;
+          for (int st = 0; st < pre; ++st) {
+            const uint32_t full = bar0 + 8 * st, dst = ring + st * kSlot;
+            tma_load_3d(dst + kGvStageBytes, &L.xmap, 0, 8 * st, 0, full);
+            tma_load_3d(dst + kGvStageBytes + kXHalf, &L.xmap, 0, 8 * st + 4, 0, full);
+          }
+          issued = pre;
+          slot = pre % nring;
+          phase = pre == nring ? 1 : 0;
+          st0 = pre;
+        }
+      }
       while (ok && unit < P.total_units) {
         int l = 0;
         while (l + 1 < P.n_layers && unit >= P.layer[l + 1].unit0) ++l;
         const GvLayer& L = P.layer[l];
         const int rb = unit - L.unit0;
         const int nst = (L.K + kGvStageK - 1) / kGvStageK;
-        for (int st = 0; st < nst; ++st) {
+        for (int st = st0; st < nst; ++st) {
           if (!mbar_wait(bar0 + 8 * (nring + slot), phase ^ 1, ctl)) { ok = false; break; }
           tags[slot] = unit;
           const uint32_t full = bar0 + 8 * slot, dst = ring + slot * kSlot;
@@ -347,6 +380,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           griddep_wait();  // the ticket counter is reset by the preceding launch
           waited = true;
         }
+        st0 = 0;
         unit = static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(P.tickets, 1u));
       }
       if (ok) {

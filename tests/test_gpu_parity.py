@@ -94,7 +94,10 @@ def test_pack_special_matrices():
 # ----------------------------------------------------------------------------
 
 @pytest.mark.parametrize("M,K,dtype", [(4, 256, "f32"), (3, 64, "f32"), (1, 2560, "bf16"), (16, 3200, "bf16"),
-                                       (2048, 2560, "bf16"), (8, 28672, "bf16"), (5, 8640, "f32")])
+                                       (2048, 2560, "bf16"), (8, 28672, "bf16"), (5, 8640, "f32"),
+                                       # many tokens, short and long rows
+                                       (700, 2048, "f32"), (600, 576, "bf16"), (640, 4096, "bf16"),
+                                       (600, 4160, "bf16"), (1200, 64, "f32")])
 def test_quant_parity(M, K, dtype):
     x, xf = activations(M, K, seed=M * 7 + K, dtype=dtype)
     q_ref, s_ref, r_ref = oracle.quant_act(xf)
@@ -206,7 +209,8 @@ def test_forward_prefill_ragged_full():
 
 
 @pytest.mark.parametrize("M,N,K,ydtype", [(300, 1000, 576, torch.bfloat16), (300, 1000, 576, torch.float32),
-                                          (513, 772, 320, torch.float32), (2048, 512, 256, torch.bfloat16)])
+                                          (513, 772, 320, torch.float32), (2048, 512, 256, torch.bfloat16),
+                                          (700, 520, 192, torch.bfloat16)])
 def test_forward_y_only_many_tokens(M, N, K, ydtype):
     """Without the accumulator output (the serving call), checked everywhere."""
     seed = M + N
