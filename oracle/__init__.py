@@ -63,6 +63,8 @@ def _lib():
         lib.oracle_round_f32.restype = None
         lib.oracle_round_bf16.argtypes = [vp, i64, vp]
         lib.oracle_round_bf16.restype = None
+        lib.oracle_rmsnorm.argtypes = [vp, i64, i64, vp, ctypes.c_float, ctypes.c_int, vp]
+        lib.oracle_rmsnorm.restype = None
         _handle = lib
     return _handle
 
@@ -172,3 +174,21 @@ def forward(T: np.ndarray, gamma, x: np.ndarray):
     q, s, r = quant_act(x)
     acc = accumulate(q, T)
     return acc, dequant(acc, gamma, s), q, s, r
+
+
+def rmsnorm(x: np.ndarray, gain: np.ndarray | None, eps: float, out_bf16: bool) -> np.ndarray:
+    """Per-token RMSNorm ``[M][K]`` -> fp32 values, rounded to bf16 when ``out_bf16``."""
+    x = _c(x, np.float32)
+    M, K = x.shape
+    g = None if gain is None else _c(gain, np.float32)
+    out = np.empty((M, K), dtype=np.float32)
+    _lib().oracle_rmsnorm(x.ctypes.data, M, K, None if g is None else g.ctypes.data, float(np.float32(eps)),
+                          1 if out_bf16 else 0, out.ctypes.data)
+    return out
+
+
+def rmsnorm_quant(x: np.ndarray, gain: np.ndarray | None, eps: float, out_bf16: bool):
+    """The fused pre-norm: RMSNorm then per-token quantisation; returns (v, q, s, rowsum)."""
+    v = rmsnorm(x, gain, eps, out_bf16)
+    q, s, r = quant_act(v)
+    return v, q, s, r

@@ -24,6 +24,11 @@
  *            (W1.58A8); the GPU path stores four ternary values in one int8.
  *  [Energy]  same blog as [AbsMean], section "The Energy Revolution": the
  *            product reduces to integer additions of 8-bit activations.
+ *  [Norm]    "BitNet's Real Bet: Designing the Whole Inference Stack" (native
+ *            training section: the 2024 model uses RMSNorm, the 2B4T model
+ *            sub-layer normalisation) and "A Two-Billion Ternary Bet"
+ *            (sub-layer normalisation stabilises training): the normalisation
+ *            that precedes a BitLinear's activation quantisation.
  *
  * Readings where the pages are silent (each one is listed in the design notes):
  *  - gamma is summed in double precision in a fixed order: each row's |w|
@@ -38,6 +43,12 @@
  *  - Storage: code c = t + 1 in {0, 1, 2}, two bits each, four to a byte;
  *    32-bit little-endian word g of a row holds elements 16g .. 16g+15, and
  *    element 16g + 4j + b sits in byte b at bits [2j, 2j+1].
+ *  - RMSNorm (the pages name it without a formula): v = x * r * g with
+ *    r = 1 / sqrt(mean(x^2) + eps), g an optional per-channel gain; the
+ *    squares are summed in double over k ascending, r is formed in double
+ *    and rounded once to fp32, the products x * r then * g are fp32, and v
+ *    is rounded to the activation type (bf16 round-to-nearest-even for bf16
+ *    inputs), as an unfused norm that writes its output would store it.
  */
 #include <math.h>
 #include <stdint.h>
@@ -196,4 +207,28 @@ static uint16_t oracle_bf16_of(double y) {
 
 void oracle_round_bf16(const double* y, int64_t n, uint16_t* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_of(y[i]);
+}
+
+/* [Norm]: per-token RMSNorm, output rounded to the activation type (values as fp32). */
+void oracle_rmsnorm(const float* x, int64_t M, int64_t K, const float* g, float eps, int out_bf16,
+                    float* out) {
+  for (int64_t m = 0; m < M; ++m) {
+    double ss = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+      double v = (double)x[m * K + k];
+      ss += v * v;
+    }
+    double ms = ss / (double)K;
+    float r = (float)(1.0 / sqrt(ms + (double)eps));
+    for (int64_t k = 0; k < K; ++k) {
+      float v = x[m * K + k] * r;
+      if (g) v = v * g[k];
+      if (out_bf16) {
+        uint16_t h = oracle_bf16_of((double)v);
+        uint32_t u = (uint32_t)h << 16;
+        memcpy(&v, &u, 4);
+      }
+      out[m * K + k] = v;
+    }
+  }
 }

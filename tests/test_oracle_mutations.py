@@ -32,6 +32,12 @@ MUTANTS = {
     "dequant_multiplies_scale": ("(double)gamma / (double)s[m];", "(double)gamma * (double)s[m];"),
     "dequant_gamma_plus_eps": ("(double)gamma / (double)s[m];", "((double)gamma + 1e-5) / (double)s[m];"),
     "bf16_via_fp32": ("double r = rint(ldexp(a, -qexp));", "double r = rint(ldexp((double)(float)a, -qexp));"),
+    "rms_divides_by_k_minus_1": ("double ms = ss / (double)K;", "double ms = ss / (double)(K - 1);"),
+    "rms_eps_outside_sqrt": ("float r = (float)(1.0 / sqrt(ms + (double)eps));",
+                             "float r = (float)(1.0 / (sqrt(ms) + (double)eps));"),
+    "rms_gain_ignored": ("if (g) v = v * g[k];", ";"),
+    "rms_sum_of_abs": ("ss += v * v;", "ss += fabs(v);"),
+    "rms_no_bf16_rounding": ("if (out_bf16) {", "if (0) {"),
 }
 
 

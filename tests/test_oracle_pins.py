@@ -14,6 +14,10 @@ Passages (web pages on BitNet b1.58):
             section "A low-bit model is a whole-stack design".
   [Energy]  "BitNet b1.58 and the 1-Bit AI Architecture Revolution",
             section "The Energy Revolution".
+  [Norm]    "BitNet's Real Bet: Designing the Whole Inference Stack" (native
+            training: RMSNorm, sub-layer normalisation) and "BitNet b1.58 and
+            the 1-Bit AI Architecture Revolution", section "Empirical
+            Performance and The New Scaling Law" (RMSNorm).
 """
 import math
 from fractions import Fraction
@@ -340,3 +344,69 @@ def test_forward_approximates_full_precision_layer():
     full = x.astype(np.float64) @ W.astype(np.float64).T
     corr = np.corrcoef(y.ravel(), full.ravel())[0, 1]
     assert corr > 0.85
+
+
+# ----------------------------------------------------------------------------
+# RMSNorm before the activation quantisation  [Norm]
+# ----------------------------------------------------------------------------
+
+def _golden_rmsnorm_cases():
+    rows = read_golden("rmsnorm.txt")
+    for i in range(0, len(rows), 5):
+        (kx, x), (kg, g), (ke, e), (kv, v), (ku, u) = rows[i:i + 5]
+        assert (kx, kg, ke, kv, ku) == ("x", "g", "eps", "v", "ulps")
+        yield ([float(t) for t in x], None if g == ["-"] else [float(t) for t in g], float(e[0]),
+               [float(t) for t in v], int(u[0]))
+
+
+def test_rmsnorm_golden_cases():
+    n = 0
+    for x, g, eps, v, ulps in _golden_rmsnorm_cases():
+        got = oracle.rmsnorm(np.array([x], np.float32), None if g is None else np.array(g, np.float32), eps, False)[0]
+        for a, b in zip(got, v):
+            assert abs(float(a) - b) <= ulps * max(ulp32(b), 1e-45), (x, g, eps, got, v)
+        n += 1
+    assert n == 6
+
+
+@pytest.mark.parametrize("K,seed", [(2560, 0), (64, 1), (8640, 2)])
+def test_rmsnorm_output_has_unit_rms(K, seed):
+    """With eps = 0 and no gain the output's mean square is 1 (fp32 rounding only)."""
+    _, x = synth.activations_bf16(4, K, seed=seed)
+    v = oracle.rmsnorm(x, None, 0.0, False)
+    for row in v.astype(np.float64):
+        ms = math.fsum(float(t) * float(t) for t in row) / K
+        assert abs(ms - 1.0) < 4e-7
+
+
+def test_rmsnorm_power_of_two_scaling_and_gain():
+    """Scaling x by 2^j leaves the output unchanged; a gain of 2^j scales it exactly."""
+    _, x = synth.activations_bf16(3, 512, seed=5)
+    base = oracle.rmsnorm(x, None, 0.0, False)
+    for j in (-3, 1, 7):
+        assert np.array_equal(oracle.rmsnorm(x * np.float32(2.0 ** j), None, 0.0, False), base)
+        g = np.full(512, 2.0 ** j, np.float32)
+        assert np.array_equal(oracle.rmsnorm(x, g, 0.0, False), base * np.float32(2.0 ** j))
+
+
+def _bf16_rne_bits(f: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 round-to-nearest-even, on the bit patterns (finite inputs)."""
+    u = f.astype(np.float32).view(np.uint32).astype(np.uint64)
+    lower = u & 0xFFFF
+    upper = u >> 16
+    round_up = (lower > 0x8000) | ((lower == 0x8000) & ((upper & 1) == 1))
+    return (upper + round_up.astype(np.uint64)).astype(np.uint16)
+
+
+def test_rmsnorm_bf16_output_is_the_rounded_fp32_output():
+    _, x = synth.activations_bf16(5, 2560, seed=6)
+    g = synth.activations_bf16(1, 2560, seed=7)[1][0]
+    f32 = oracle.rmsnorm(x, g, 1e-6, False)
+    b16 = oracle.rmsnorm(x, g, 1e-6, True)
+    want = (_bf16_rne_bits(f32).astype(np.uint32) << 16).view(np.float32)
+    assert np.array_equal(b16, want)
+
+
+def test_rmsnorm_quant_of_a_zero_token():
+    v, q, s, r = oracle.rmsnorm_quant(np.zeros((1, 64), np.float32), None, 1e-6, True)
+    assert not v.any() and not q.any() and r[0] == 0 and s[0] == np.float32(127.0) / EPS32
