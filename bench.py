@@ -52,7 +52,7 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-extras", action="store_true", help="skip prefill / 70B chain / pack lines")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--only", choices=["prefill", "chain70b"], default=None,
+    p.add_argument("--only", choices=["prefill", "chain70b", "next"], default=None,
                    help="run one secondary workload alone and print its own line (a small case for profiling)")
     return p.parse_args()
 
@@ -363,6 +363,7 @@ def run_ours(args, world, rank, local):
         out["prefill"] = run_prefill(args, world, peaks, L2)
         out["chain_70b"] = run_chain(args, world, peaks, L2)
         out["pack"] = run_pack(world)
+        out["next"] = run_next(args, world, peaks, L2)
 
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -455,6 +456,43 @@ def run_chain(args, world, peaks, L2):
                                 "tokens_per_s": round(M * steps * world / secs, 1),
                                 "device_status": tb.device_status(ws)}
     return res
+
+
+def run_next(args, world, peaks, L2):
+    """The rows beyond the forward: fused RMSNorm + quantisation (prefill and decode sizes)."""
+    import torch
+
+    import synth
+    import ternary_weight_a8_b200 as tb
+
+    out = {}
+    for M, K in ((2048, 2560), (1, 8192)):
+        n_in = max(4, int(4 * L2 // (M * K * 2)) + 1)  # inputs larger than L2 in total
+        xs = []
+        for i in range(min(n_in, 64)):
+            bits, _ = synth.activations_bf16(M, K, seed=500 + i)
+            xs.append(torch.from_numpy(bits.view("int16")).cuda().view(torch.bfloat16))
+        g = torch.ones(K, dtype=torch.float32, device="cuda")
+        xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+        sc = torch.empty(M, dtype=torch.float32, device="cuda")
+        rs = torch.empty(M, dtype=torch.int32, device="cuda")
+        steps = 400
+        secs, _ = timed_graph_run(lambda i: tb.rmsnorm_quant(xs[i % len(xs)], g, 1e-6, None, xq, sc, rs),
+                                  steps, 20, world, chunk=100)
+        nb = M * K * 3 + M * 8 + K * 4
+        gbs = nb / (secs / steps) / 1e9
+        res = {"us": round(secs / steps * 1e6, 3), "GB/s": round(gbs, 1),
+               "pct_hbm_measured": round(100 * gbs / peaks["hbm"], 2), "bytes_per_call": nb}
+        # Unfused comparison: the norm as separate torch ops writing bf16, then the quantisation kernel.
+        def unfused(i):
+            x = xs[i % len(xs)]
+            xf = x.float()
+            v = (xf * torch.rsqrt(xf.pow(2).mean(-1, keepdim=True) + 1e-6) * g).to(torch.bfloat16)
+            tb.quant_act(v, xq, sc, rs)
+        usecs, _ = timed_graph_run(unfused, steps, 20, world, chunk=100)
+        res["unfused_torch_norm_then_quant_us"] = round(usecs / steps * 1e6, 3)
+        out["rmsnorm_quant_%dx%d" % (M, K)] = res
+    return out
 
 
 def run_pack(world):
@@ -560,7 +598,7 @@ def main():
         import torch
 
         torch.cuda.set_device(local)
-        fn = run_prefill if args.only == "prefill" else run_chain
+        fn = {"prefill": run_prefill, "chain70b": run_chain, "next": run_next}[args.only]
         res = fn(args, world, load_peaks(), l2_bytes())
         if rank == 0:
             print(json.dumps(res), flush=True)

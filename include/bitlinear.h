@@ -103,6 +103,29 @@ int bitlinear_pack_weights(const float* W, int N, int K, uint8_t* packed, float*
 int bitlinear_quant_act(const void* x, int x_dtype, int M, int K, int8_t* xq, float* scale,
                         int32_t* rowsum, void* stream);
 
+/*
+ * The normalisation before a BitLinear fused with its activation
+ * quantisation: RMSNorm (the 2024 model) / sub-layer normalisation (the 2B4T
+ * model), "BitNet's Real Bet: Designing the Whole Inference Stack", native
+ * training section; "BitNet b1.58 and the 1-Bit AI Architecture Revolution",
+ * section "Empirical Performance and The New Scaling Law".  The pages give no
+ * formula; the reading is v = x * r * g, r = 1 / sqrt(mean_k x^2 + eps),
+ * with the squares summed in double, r rounded once to fp32, fp32 products
+ * (x * r, then * g), and v rounded to x_dtype as an unfused norm would store
+ * it; v is then quantised exactly as bitlinear_quant_act does.  One pass
+ * over x per token.
+ *   x       device [M][K] of x_dtype (BL_F32 or BL_BF16); read only; 16-byte aligned.
+ *   gain    device fp32 [K] (the norm's per-channel weight), or NULL for 1.
+ *   eps     the norm's epsilon (>= 0, finite).
+ *   x_norm  device [M][K] of x_dtype out, or NULL: v itself (the residual
+ *           branch may need it).
+ *   xq, scale, rowsum: as bitlinear_quant_act (rowsum may be NULL).
+ * Errors: as bitlinear_quant_act; BL_ERR_INVALID_ARG for a negative or
+ * non-finite eps.
+ */
+int bitlinear_rmsnorm_quant(const void* x, int x_dtype, int M, int K, const float* gain, float eps, void* x_norm,
+                            int8_t* xq, float* scale, int32_t* rowsum, void* stream);
+
 /* Workspace bytes bitlinear_forward needs (status word + q, s, rowsum). */
 size_t bitlinear_workspace_bytes(int M, int N, int K);
 

@@ -68,6 +68,7 @@ def lib() -> ctypes.CDLL:
             "bitlinear_pack_workspace_bytes": (sz, [i32, i32]),
             "bitlinear_pack_weights": (i32, [vp, i32, i32, vp, vp, vp, sz, vp]),
             "bitlinear_quant_act": (i32, [vp, i32, i32, i32, vp, vp, vp, vp]),
+            "bitlinear_rmsnorm_quant": (i32, [vp, i32, i32, i32, vp, ctypes.c_float, vp, vp, vp, vp, vp]),
             "bitlinear_workspace_bytes": (sz, [i32, i32, i32]),
             "bitlinear_forward": (i32, [vp, vp, i32, i32, vp, i32, i32, vp, i32, vp, vp, sz, vp]),
             "bitlinear_forward_quantized": (i32, [vp, vp, i32, i32, vp, vp, vp, i32, vp, i32, vp, vp, sz, vp]),
@@ -174,6 +175,21 @@ def quant_act(x: torch.Tensor, xq=None, scale=None, rowsum=None, stream=None):
     _check(lib().bitlinear_quant_act(_ptr(x), _dtype_code(x.dtype), M, K, _ptr(xq), _ptr(scale),
                                      _ptr(rowsum), _stream(stream)))
     return xq, scale, rowsum
+
+
+def rmsnorm_quant(x: torch.Tensor, gain: torch.Tensor | None = None, eps: float = 1e-6, x_norm=None, xq=None,
+                  scale=None, rowsum=None, stream=None):
+    """RMSNorm fused with the per-token quantisation: returns (xq, scale, rowsum), and also
+    the normalised activations first when ``x_norm`` is True or a tensor."""
+    M, K = x.shape
+    dev = x.device
+    xq = torch.empty((M, K), dtype=torch.int8, device=dev) if xq is None else xq
+    scale = torch.empty(M, dtype=torch.float32, device=dev) if scale is None else scale
+    rowsum = torch.empty(M, dtype=torch.int32, device=dev) if rowsum is None else rowsum
+    norm = torch.empty_like(x) if x_norm is True else (x_norm if isinstance(x_norm, torch.Tensor) else None)
+    _check(lib().bitlinear_rmsnorm_quant(_ptr(x), _dtype_code(x.dtype), M, K, _ptr(gain), float(eps), _ptr(norm),
+                                         _ptr(xq), _ptr(scale), _ptr(rowsum), _stream(stream)))
+    return (norm, xq, scale, rowsum) if norm is not None else (xq, scale, rowsum)
 
 
 def forward(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, out_dtype=torch.bfloat16,

@@ -171,6 +171,184 @@ __global__ void __launch_bounds__(kQuantMaxThreads) act_quant_kernel(const __gri
   }
 }
 
+// ---------------------------------------------------------------------------
+// RMSNorm fused with the quantisation: the normalisation that precedes a
+// BitLinear ("BitNet's Real Bet: Designing the Whole Inference Stack",
+// native-training section: RMSNorm, sub-layer normalisation).  Reading (no
+// formula on the pages): v = x * r * g, r = 1 / sqrt(mean(x^2) + eps); the
+// squares are summed in double (exact squares, one rounding per add, so the
+// order changes r only in double's last bits), r is rounded once to fp32,
+// x * r then * g are fp32 multiplies, and v is rounded to the activation
+// type exactly as an unfused norm would store it; then the same per-token
+// quantisation as above.  One block per token, the token held in registers.
+// ---------------------------------------------------------------------------
+struct NormParams {
+  const void* x;
+  const float* gain;  // [K] or null
+  float eps;
+  void* x_norm;       // [M][K] in the activation type, or null
+  int8_t* xq;         // [M][K]
+  float* scale;
+  int32_t* rowsum;    // or null
+  int K;
+};
+
+// v = round_to_TX(x * r [* g]) for the 16 inputs of chunk c.
+template <typename TX>
+__device__ __forceinline__ void norm_chunk(const Chunk16& raw, float r, const float* gain, int c, float (&v)[16]) {
+  float gv[16];
+  if (gain) {
+    const float4* gp = reinterpret_cast<const float4*>(gain + 16 * c);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 t = __ldg(gp + i);
+      gv[4 * i] = t.x;
+      gv[4 * i + 1] = t.y;
+      gv[4 * i + 2] = t.z;
+      gv[4 * i + 3] = t.w;
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    float t = __fmul_rn(elem<TX>(raw, e), r);
+    if (gain) t = __fmul_rn(t, gv[e]);
+    if constexpr (sizeof(TX) == 2) t = __bfloat162float(__float2bfloat16_rn(t));
+    v[e] = t;
+  }
+}
+
+template <typename TX>
+__global__ void __launch_bounds__(kQuantMaxThreads) rmsnorm_quant_kernel(const __grid_constant__ NormParams P) {
+  __shared__ double red_d[kQuantMaxThreads / 32];
+  __shared__ float red_f[kQuantMaxThreads / 32];
+  __shared__ int red_i[kQuantMaxThreads / 32];
+  griddep_launch_dependents();
+  griddep_wait();  // x may be the preceding kernel's output; q may still be read by it
+
+  const int m = blockIdx.x, K = P.K, chunks = K >> 4, T = blockDim.x;
+  const TX* xr = static_cast<const TX*>(P.x) + static_cast<size_t>(m) * K;
+  int8_t* qr = P.xq + static_cast<size_t>(m) * K;
+  TX* nr = P.x_norm ? static_cast<TX*>(P.x_norm) + static_cast<size_t>(m) * K : nullptr;
+  const bool in_regs = chunks <= T * kQuantRegChunks;
+  Chunk16 reg[kQuantRegChunks];
+  if (in_regs) {
+#pragma unroll
+    for (int i = 0; i < kQuantRegChunks; ++i) {
+      const int c = threadIdx.x + i * T;
+      if (c < chunks) load16<TX>(xr + c * 16, reg[i]);
+    }
+  }
+  // fn(chunk, c) over this thread's chunks: from registers, or read again.
+  auto for_each_chunk = [&](auto&& fn) {
+    if (in_regs) {
+#pragma unroll
+      for (int i = 0; i < kQuantRegChunks; ++i) {
+        const int c = threadIdx.x + i * T;
+        if (c < chunks) fn(reg[i], c);
+      }
+    } else {
+      for (int c = threadIdx.x; c < chunks; c += T) {
+        Chunk16 raw;
+        load16<TX>(xr + c * 16, raw);
+        fn(raw, c);
+      }
+    }
+  };
+
+  // Mean of squares, in double (each square exact, one rounding per add).
+  double ss = 0.0;
+  for_each_chunk([&](const Chunk16& ch, int) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const double v = static_cast<double>(elem<TX>(ch, e));
+      ss = __fma_rn(v, v, ss);
+    }
+  });
+  ss = block_reduce(ss, [](double a, double b) { return __dadd_rn(a, b); }, red_d);
+  const double ms = __ddiv_rn(ss, static_cast<double>(K));
+  const float r = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(ms, static_cast<double>(P.eps)))));
+
+  // Absmax of the normalised token.  When the token is in registers the
+  // normalised values of the thread's first kNormKeep chunks stay there too.
+  constexpr int kNormKeep = 2;
+  float vkeep[kNormKeep][16];
+  float amax = 0.0f;
+  for_each_chunk([&](const Chunk16& ch, int c) {
+    float v[16];
+    norm_chunk<TX>(ch, r, P.gain, c, v);
+    const int i = (c - static_cast<int>(threadIdx.x)) / T;
+#pragma unroll
+    for (int k = 0; k < kNormKeep; ++k)
+      if (in_regs && i == k) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) vkeep[k][e] = v[e];
+      }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
+  });
+  amax = block_reduce(amax, [](float a, float b) { return fmaxf(a, b); }, red_f);
+  const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
+
+  // Codes (and the normalised activations when asked for).
+  int sum = 0;
+  for_each_chunk([&](const Chunk16& ch, int c) {
+    float v[16];
+    const int i = (c - static_cast<int>(threadIdx.x)) / T;
+    if (in_regs && i < kNormKeep) {
+#pragma unroll
+      for (int k = 0; k < kNormKeep; ++k)
+        if (i == k) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = vkeep[k][e];
+        }
+    } else {
+      norm_chunk<TX>(ch, r, P.gain, c, v);
+    }
+    uint32_t w[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      int q[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) q[e] = min(max(__float2int_rn(__fmul_rn(v[4 * b + e], s)), -128), 127);
+      w[b] = pack4(q[0], q[1], q[2], q[3]);
+      sum = __dp4a(static_cast<int>(w[b]), 0x01010101, sum);
+    }
+    *reinterpret_cast<uint4*>(qr + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    if (nr) {
+      if constexpr (sizeof(TX) == 2) {
+        uint32_t h[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          h[e] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * e]))) |
+                 (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * e + 1]))) << 16);
+        uint4* dst = reinterpret_cast<uint4*>(nr + c * 16);
+        dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
+        dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
+      } else {
+        float4* dst = reinterpret_cast<float4*>(nr + c * 16);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+      }
+    }
+  });
+  sum = block_reduce(sum, [](int a, int b) { return a + b; }, red_i);
+  if (threadIdx.x == 0) {
+    P.scale[m] = s;
+    if (P.rowsum) P.rowsum[m] = sum;
+  }
+}
+
+cudaError_t launch_rmsnorm_quant(const void* x, int x_bf16, int M, int K, const float* gain, float eps, void* x_norm,
+                                 int8_t* xq, float* scale, int32_t* rowsum, cudaStream_t stream, bool pdl) {
+  if (M <= 0) return cudaSuccess;
+  const NormParams P{x, gain, eps, x_norm, xq, scale, rowsum, K};
+  int threads = ((K / 16 + 1) / 2 + 31) / 32 * 32;  // about two chunks per thread, 64 .. 512
+  if (threads < 64) threads = 64;
+  if (threads > kQuantMaxThreads) threads = kQuantMaxThreads;
+  if (x_bf16) return launch(rmsnorm_quant_kernel<__nv_bfloat16>, dim3(M), dim3(threads), 0, stream, pdl, P);
+  return launch(rmsnorm_quant_kernel<float>, dim3(M), dim3(threads), 0, stream, pdl, P);
+}
+
 cudaError_t launch_act_quant_group(const QuantArgs* items, int n_items, int M, int x_bf16, cudaStream_t stream,
                                    bool pdl) {
   if (M <= 0 || n_items <= 0) return cudaSuccess;

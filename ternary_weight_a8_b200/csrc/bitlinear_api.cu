@@ -2,6 +2,7 @@
 // dispatch to the kernels, and the layer chain.  The declarations and their
 // contracts are in include/bitlinear.h.
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
 
@@ -214,6 +215,25 @@ int bitlinear_quant_act(const void* x, int x_dtype, int M, int K, int8_t* xq, fl
   cudaError_t e = bl::launch_act_quant(x, x_dtype == BL_BF16, M, K, K, xq, scale, rowsum,
                                        static_cast<cudaStream_t>(stream), true);
   if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+  return BL_OK;
+}
+
+int bitlinear_rmsnorm_quant(const void* x, int x_dtype, int M, int K, const float* gain, float eps, void* x_norm,
+                            int8_t* xq, float* scale, int32_t* rowsum, void* stream) {
+  BL_TRY(check_dtype(x_dtype, "x_dtype"));
+  if (M < 0) return fail(BL_ERR_INVALID_ARG, "M = %d < 0", M);
+  if (K < 64 || K % 64 != 0) return fail(BL_ERR_UNSUPPORTED_SHAPE, "K = %d: need K >= 64 and K %% 64 == 0", K);
+  if (!(eps >= 0.0f) || !(eps < INFINITY)) return fail(BL_ERR_INVALID_ARG, "eps = %g: need a finite eps >= 0", eps);
+  if (M == 0) return BL_OK;
+  BL_TRY(check_ptr(x, "x", 16));
+  BL_TRY(check_ptr(gain, "gain", 16, true));
+  BL_TRY(check_ptr(x_norm, "x_norm", 16, true));
+  BL_TRY(check_ptr(xq, "xq", 16));
+  BL_TRY(check_ptr(scale, "scale", 4));
+  BL_TRY(check_ptr(rowsum, "rowsum", 4, true));
+  cudaError_t e = bl::launch_rmsnorm_quant(x, x_dtype == BL_BF16, M, K, gain, eps, x_norm, xq, scale, rowsum,
+                                           static_cast<cudaStream_t>(stream), true);
+  if (e != cudaSuccess) return cuda_fail(e, "rmsnorm_quant launch");
   return BL_OK;
 }
 

@@ -49,6 +49,11 @@ cudaError_t launch_act_quant(const void* x, int x_bf16, int M, int K, int ldq, i
 cudaError_t launch_act_quant_group(const QuantArgs* items, int n_items, int M, int x_bf16, cudaStream_t stream,
                                    bool pdl);
 
+// RMSNorm (gain optional) fused with the per-token quantisation; x_norm
+// (optional) receives the normalised activations in the input type.
+cudaError_t launch_rmsnorm_quant(const void* x, int x_bf16, int M, int K, const float* gain, float eps, void* x_norm,
+                                 int8_t* xq, float* scale, int32_t* rowsum, cudaStream_t stream, bool pdl);
+
 enum InType { kInInt8 = 0, kInBF16 = 1, kInF32 = 2 };
 
 // Tensor-core GEMM on quantised activations (many tokens).

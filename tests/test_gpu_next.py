@@ -1,0 +1,84 @@
+"""GPU parity of the rows built beyond the forward itself, against the oracle.
+
+Fused pre-norm: RMSNorm (gain optional) fused with the per-token
+quantisation, compared with the oracle's RMSNorm followed by its
+quantisation.  The normalised activations, codes, scales and code sums are
+compared bit for bit (the norm's mean of squares is summed in double on both
+sides, so its order changes only double's last bits and, in practice, never
+the fp32 factor derived from it).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import ternary_weight_a8_b200 as tb
+from parity import activations, assert_y_matches, bf16_bits, dev, f32_bits, weights
+
+pytestmark = pytest.mark.gpu
+
+
+def _gain(K, seed):
+    """A per-channel gain around 1 (what a trained norm weight looks like)."""
+    return (1.0 + 0.1 * synth.activations_f32(1, K, seed=seed)[0]).astype(np.float32)
+
+
+@pytest.mark.parametrize("M,K,dtype,with_gain,eps", [
+    (1, 2560, "bf16", True, 1e-6), (4, 64, "f32", False, 1e-5), (16, 8640, "bf16", True, 1e-6),
+    (2048, 2560, "bf16", True, 1e-6), (3, 28672, "bf16", False, 1e-6), (5, 8192, "f32", True, 0.0),
+    (7, 32768 + 1024, "bf16", True, 1e-6),  # longer than a block holds in registers: read twice
+])
+def test_rmsnorm_quant_parity(M, K, dtype, with_gain, eps):
+    x, xf = activations(M, K, seed=M * 3 + K, dtype=dtype)
+    g = _gain(K, seed=K) if with_gain else None
+    v_ref, q_ref, s_ref, r_ref = oracle.rmsnorm_quant(xf, g, eps, dtype == "bf16")
+    v, q, s, r = tb.rmsnorm_quant(x, None if g is None else dev(g), eps=eps, x_norm=True)
+    if dtype == "bf16":
+        want = (f32_bits(v_ref) >> 16).astype(np.uint16)
+        assert np.array_equal(bf16_bits(v), want)
+    else:
+        assert np.array_equal(f32_bits(v.cpu().numpy()), f32_bits(v_ref))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(f32_bits(s.cpu().numpy()), f32_bits(s_ref))
+    assert np.array_equal(r.cpu().numpy(), r_ref)
+
+
+def test_rmsnorm_quant_degenerate_tokens():
+    """A zero token, a one-hot token and a constant token."""
+    K = 256
+    xf = np.zeros((3, K), np.float32)
+    xf[1, 17] = -3.0
+    xf[2, :] = 0.5
+    x = dev(xf)
+    v_ref, q_ref, s_ref, r_ref = oracle.rmsnorm_quant(xf, None, 1e-6, False)
+    v, q, s, r = tb.rmsnorm_quant(x, eps=1e-6, x_norm=True)
+    assert np.array_equal(f32_bits(v.cpu().numpy()), f32_bits(v_ref))
+    assert np.array_equal(q.cpu().numpy(), q_ref) and np.array_equal(r.cpu().numpy(), r_ref)
+    assert np.array_equal(f32_bits(s.cpu().numpy()), f32_bits(s_ref))
+    assert not q.cpu().numpy()[0].any()
+
+
+def test_rmsnorm_codes_feed_the_product():
+    """Normalised codes into the product: the same result as the oracle's norm, quantisation and product."""
+    M, N, K = 3, 700, 2560
+    W = weights(N, K, seed=11)
+    packed_ref, gamma_ref, T = oracle.pack_weights(W)
+    x, xf = activations(M, K, seed=12, dtype="bf16")
+    g = _gain(K, seed=13)
+    v_ref, q_ref, s_ref, r_ref = oracle.rmsnorm_quant(xf, g, 1e-6, True)
+    acc_ref = oracle.accumulate(q_ref, T)
+    y_ref = oracle.dequant(acc_ref, gamma_ref, s_ref)
+    xq, s, r = tb.rmsnorm_quant(x, dev(g), eps=1e-6)
+    y, acc = tb.forward_quantized(dev(packed_ref), dev(np.array([gamma_ref], np.float32)), xq, s, r,
+                                  out_dtype=torch.bfloat16, acc_out=True)
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert_y_matches(y, y_ref, acc_ref)
+
+
+def test_rmsnorm_rejects_bad_eps():
+    x = torch.zeros((1, 64), dtype=torch.float32, device="cuda")
+    for eps in (-1.0, float("inf"), float("nan")):
+        with pytest.raises(tb.BitLinearError) as e:
+            tb.rmsnorm_quant(x, eps=eps)
+        assert e.value.code == tb.BL_ERR_INVALID_ARG
