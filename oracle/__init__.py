@@ -65,6 +65,8 @@ def _lib():
         lib.oracle_round_bf16.restype = None
         lib.oracle_rmsnorm.argtypes = [vp, i64, i64, vp, ctypes.c_float, ctypes.c_int, vp]
         lib.oracle_rmsnorm.restype = None
+        lib.oracle_glu.argtypes = [vp, vp, i64, ctypes.c_int, ctypes.c_int, vp]
+        lib.oracle_glu.restype = None
         _handle = lib
     return _handle
 
@@ -192,3 +194,23 @@ def rmsnorm_quant(x: np.ndarray, gain: np.ndarray | None, eps: float, out_bf16: 
     v = rmsnorm(x, gain, eps, out_bf16)
     q, s, r = quant_act(v)
     return v, q, s, r
+
+
+GLU_RELU2, GLU_SILU = 0, 1
+
+
+def glu(gate: np.ndarray, up: np.ndarray, act: int, out_bf16: bool) -> np.ndarray:
+    """h = act(gate) * up (act GLU_RELU2 or GLU_SILU), rounded to bf16 when ``out_bf16``."""
+    gate = _c(gate, np.float32)
+    up = _c(up, np.float32)
+    assert gate.shape == up.shape
+    out = np.empty(gate.shape, dtype=np.float32)
+    _lib().oracle_glu(gate.ctypes.data, up.ctypes.data, gate.size, int(act), 1 if out_bf16 else 0, out.ctypes.data)
+    return out
+
+
+def glu_quant(gate: np.ndarray, up: np.ndarray, act: int, out_bf16: bool):
+    """The FFN's gated activation then per-token quantisation; returns (h, q, s, rowsum)."""
+    h = glu(gate, up, act, out_bf16)
+    q, s, r = quant_act(h)
+    return h, q, s, r

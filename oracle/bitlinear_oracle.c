@@ -24,6 +24,11 @@
  *            (W1.58A8); the GPU path stores four ternary values in one int8.
  *  [Energy]  same blog as [AbsMean], section "The Energy Revolution": the
  *            product reduces to integer additions of 8-bit activations.
+ *  [GLU]     "BitNet's Real Bet: Designing the Whole Inference Stack" (native
+ *            training section: the 2024 model uses SwiGLU, the 2B4T model
+ *            squared ReLU) and "A Two-Billion Ternary Bet" (squared-ReLU-style
+ *            activations tame gradient scale): the gated activation between
+ *            the gate/up BitLinears and the down BitLinear of the FFN.
  *  [Norm]    "BitNet's Real Bet: Designing the Whole Inference Stack" (native
  *            training section: the 2024 model uses RMSNorm, the 2B4T model
  *            sub-layer normalisation) and "A Two-Billion Ternary Bet"
@@ -49,6 +54,12 @@
  *    and rounded once to fp32, the products x * r then * g are fp32, and v
  *    is rounded to the activation type (bf16 round-to-nearest-even for bf16
  *    inputs), as an unfused norm that writes its output would store it.
+ *  - Gated activation (named, no formula): h = act(gate) * up with
+ *    act = ReLU(z)^2 (2B4T) or SiLU(z) = z / (1 + e^-z) (SwiGLU); gate and up
+ *    are the BitLinear outputs as stored (activation type); h is rounded to
+ *    the activation type.  Squared ReLU is two fp32 multiplies, (g * g) * u
+ *    with g = max(gate, 0); SiLU is evaluated exactly (double) and rounded
+ *    once, the GPU's fp32 evaluation being held to a stated bar.
  */
 #include <math.h>
 #include <stdint.h>
@@ -230,5 +241,27 @@ void oracle_rmsnorm(const float* x, int64_t M, int64_t K, const float* g, float 
       }
       out[m * K + k] = v;
     }
+  }
+}
+
+/* [GLU]: h = act(gate) * up, rounded to the activation type (values as fp32).
+ * act 0: squared ReLU in fp32; act 1: SiLU, exact then rounded once. */
+void oracle_glu(const float* gate, const float* up, int64_t count, int act, int out_bf16, float* out) {
+  for (int64_t i = 0; i < count; ++i) {
+    float h;
+    if (act == 0) {
+      float g = gate[i] > 0.0f ? gate[i] : 0.0f;
+      h = (g * g) * up[i];
+    } else {
+      double z = (double)gate[i];
+      h = (float)(z / (1.0 + exp(-z)) * (double)up[i]);
+    }
+    if (out_bf16) {
+      uint16_t b = oracle_bf16_of(act == 0 ? (double)h : (double)gate[i] / (1.0 + exp(-(double)gate[i])) *
+                                                            (double)up[i]);
+      uint32_t u = (uint32_t)b << 16;
+      memcpy(&h, &u, 4);
+    }
+    out[i] = h;
   }
 }

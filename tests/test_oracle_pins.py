@@ -18,6 +18,9 @@ Passages (web pages on BitNet b1.58):
             training: RMSNorm, sub-layer normalisation) and "BitNet b1.58 and
             the 1-Bit AI Architecture Revolution", section "Empirical
             Performance and The New Scaling Law" (RMSNorm).
+  [GLU]     "BitNet's Real Bet: Designing the Whole Inference Stack" (native
+            training: SwiGLU, squared ReLU) and "A Two-Billion Ternary Bet"
+            (squared-ReLU-style activations).
 """
 import math
 from fractions import Fraction
@@ -410,3 +413,60 @@ def test_rmsnorm_bf16_output_is_the_rounded_fp32_output():
 def test_rmsnorm_quant_of_a_zero_token():
     v, q, s, r = oracle.rmsnorm_quant(np.zeros((1, 64), np.float32), None, 1e-6, True)
     assert not v.any() and not q.any() and r[0] == 0 and s[0] == np.float32(127.0) / EPS32
+
+
+# ----------------------------------------------------------------------------
+# The FFN's gated activation before the down BitLinear  [GLU]
+# ----------------------------------------------------------------------------
+
+def test_glu_golden_cases():
+    rows = read_golden("glu.txt")
+    n = 0
+    for i in range(0, len(rows), 5):
+        (ka, a), (kg, g), (ku, u), (kh, h), (kl, ul) = rows[i:i + 5]
+        assert (ka, kg, ku, kh, kl) == ("act", "gate", "up", "h", "ulps")
+        act = {"relu2": oracle.GLU_RELU2, "silu": oracle.GLU_SILU}[a[0]]
+        got = oracle.glu(np.array([[float(t) for t in g]], np.float32), np.array([[float(t) for t in u]], np.float32),
+                         act, False)[0]
+        for x, want in zip(got, (float(t) for t in h)):
+            assert abs(float(x) - want) <= int(ul[0]) * max(ulp32(want), 1e-45), (a, got, h)
+        n += 1
+    assert n == 3
+
+
+def test_silu_odd_part_is_the_identity():
+    """silu(z) - silu(-z) = z * (sigma(z) + sigma(-z)) = z."""
+    z = synth.activations_f32(1, 4096, seed=21)[0] * np.float32(3.0)
+    one = np.ones_like(z)
+    d = oracle.glu(z[None], one[None], oracle.GLU_SILU, False)[0].astype(np.float64) - \
+        oracle.glu(-z[None], one[None], oracle.GLU_SILU, False)[0].astype(np.float64)
+    tol = np.array([ulp32(t) for t in z]) * 2
+    assert (np.abs(d - z.astype(np.float64)) <= tol).all()
+
+
+def test_silu_limits():
+    """Far right silu(z) = z in fp32; far left it is z * e^z to first order."""
+    one = np.ones((1, 2), np.float32)
+    hi = oracle.glu(np.array([[30.0, 60.0]], np.float32), one, oracle.GLU_SILU, False)[0]
+    assert hi[0] == np.float32(30.0) and hi[1] == np.float32(60.0)
+    lo = oracle.glu(np.array([[-30.0, -60.0]], np.float32), one, oracle.GLU_SILU, False)[0]
+    for z, v in zip((-30.0, -60.0), lo):
+        assert abs(float(v) - z * math.exp(z)) <= 1e-6 * abs(z * math.exp(z))
+
+
+def test_relu2_scales_by_powers_of_four():
+    g = synth.activations_f32(2, 512, seed=22)
+    u = synth.activations_f32(2, 512, seed=23)
+    base = oracle.glu(g, u, oracle.GLU_RELU2, False)
+    for j in (-2, 3):
+        got = oracle.glu(g * np.float32(2.0 ** j), u, oracle.GLU_RELU2, False)
+        assert np.array_equal(got, base * np.float32(4.0 ** j))
+    assert (base[g <= 0] == 0).all()
+
+
+def test_glu_bf16_output_rounds_the_relu2_product():
+    g = synth.activations_f32(3, 2048, seed=24)
+    u = synth.activations_f32(3, 2048, seed=25)
+    f32 = oracle.glu(g, u, oracle.GLU_RELU2, False)
+    b16 = oracle.glu(g, u, oracle.GLU_RELU2, True)
+    assert np.array_equal(b16, (_bf16_rne_bits(f32).astype(np.uint32) << 16).view(np.float32))
