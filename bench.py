@@ -492,6 +492,33 @@ def run_next(args, world, peaks, L2):
         usecs, _ = timed_graph_run(unfused, steps, 20, world, chunk=100)
         res["unfused_torch_norm_then_quant_us"] = round(usecs / steps * 1e6, 3)
         out["rmsnorm_quant_%dx%d" % (M, K)] = res
+    # The FFN's gated activation + quantisation of the down BitLinear's input.
+    for M, N in ((2048, 6912), (1, 28672)):
+        n_in = max(2, int(4 * L2 // (M * N * 4)) + 1)
+        gs, us = [], []
+        for i in range(min(n_in, 32)):
+            gs.append(torch.from_numpy(synth.activations_bf16(M, N, seed=600 + i)[0].view("int16")).cuda()
+                      .view(torch.bfloat16))
+            us.append(torch.from_numpy(synth.activations_bf16(M, N, seed=700 + i)[0].view("int16")).cuda()
+                      .view(torch.bfloat16))
+        xq = torch.empty((M, N), dtype=torch.int8, device="cuda")
+        sc = torch.empty(M, dtype=torch.float32, device="cuda")
+        rs = torch.empty(M, dtype=torch.int32, device="cuda")
+        steps = 400
+        secs, _ = timed_graph_run(lambda i: tb.glu_quant(gs[i % len(gs)], us[i % len(us)], tb.GLU_RELU2, None, xq, sc,
+                                                         rs), steps, 20, world, chunk=100)
+        nb = M * N * 5 + M * 8
+        gbs = nb / (secs / steps) / 1e9
+        res = {"us": round(secs / steps * 1e6, 3), "GB/s": round(gbs, 1),
+               "pct_hbm_measured": round(100 * gbs / peaks["hbm"], 2), "bytes_per_call": nb, "act": "relu2"}
+
+        def unfused(i):
+            g, u = gs[i % len(gs)], us[i % len(us)]
+            h = (torch.relu(g.float()).square() * u.float()).to(torch.bfloat16)
+            tb.quant_act(h, xq, sc, rs)
+        usecs, _ = timed_graph_run(unfused, steps, 20, world, chunk=100)
+        res["unfused_torch_glu_then_quant_us"] = round(usecs / steps * 1e6, 3)
+        out["glu_quant_%dx%d" % (M, N)] = res
     return out
 
 

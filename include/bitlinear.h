@@ -126,6 +126,31 @@ int bitlinear_quant_act(const void* x, int x_dtype, int M, int K, int8_t* xq, fl
 int bitlinear_rmsnorm_quant(const void* x, int x_dtype, int M, int K, const float* gain, float eps, void* x_norm,
                             int8_t* xq, float* scale, int32_t* rowsum, void* stream);
 
+/* The FFN's gated activation (see bitlinear_glu_quant). */
+typedef enum { BL_GLU_RELU2 = 0, BL_GLU_SILU = 1 } bl_glu;
+
+/*
+ * The FFN's gated activation between the gate/up BitLinears and the down
+ * BitLinear, fused with the quantisation of the down BitLinear's input:
+ * squared ReLU (the 2B4T model) or SwiGLU (the 2024 model), "BitNet's Real
+ * Bet: Designing the Whole Inference Stack", native training section; "A
+ * Two-Billion Ternary Bet" (squared-ReLU-style activations).  The pages give
+ * no formula; the reading is h = act(gate) * up on the stored gate and up
+ * values, in fp32: BL_GLU_RELU2 (g * g) * up with g = max(gate, 0),
+ * BL_GLU_SILU gate / (1 + expf(-gate)) * up; h is rounded to x_dtype and
+ * quantised exactly as bitlinear_quant_act does.  One pass per token.
+ *   gate, up device [M][N] of x_dtype (BL_F32 or BL_BF16), e.g. the y of the
+ *           gate and up BitLinears; read only; 16-byte aligned.
+ *   act     BL_GLU_RELU2 or BL_GLU_SILU.
+ *   h       device [M][N] of x_dtype out, or NULL: h itself.
+ *   xq, scale, rowsum: as bitlinear_quant_act with K = N (rowsum may be NULL);
+ *           they feed bitlinear_forward_quantized of the down BitLinear.
+ * N >= 64 and N % 64 == 0 (the down BitLinear's K).  Errors: as
+ * bitlinear_quant_act; BL_ERR_INVALID_ARG for an unknown act.
+ */
+int bitlinear_glu_quant(const void* gate, const void* up, int x_dtype, int M, int N, int act, void* h,
+                        int8_t* xq, float* scale, int32_t* rowsum, void* stream);
+
 /* Workspace bytes bitlinear_forward needs (status word + q, s, rowsum). */
 size_t bitlinear_workspace_bytes(int M, int N, int K);
 

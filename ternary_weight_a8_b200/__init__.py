@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
             "bitlinear_pack_weights": (i32, [vp, i32, i32, vp, vp, vp, sz, vp]),
             "bitlinear_quant_act": (i32, [vp, i32, i32, i32, vp, vp, vp, vp]),
             "bitlinear_rmsnorm_quant": (i32, [vp, i32, i32, i32, vp, ctypes.c_float, vp, vp, vp, vp, vp]),
+            "bitlinear_glu_quant": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
             "bitlinear_workspace_bytes": (sz, [i32, i32, i32]),
             "bitlinear_forward": (i32, [vp, vp, i32, i32, vp, i32, i32, vp, i32, vp, vp, sz, vp]),
             "bitlinear_forward_quantized": (i32, [vp, vp, i32, i32, vp, vp, vp, i32, vp, i32, vp, vp, sz, vp]),
@@ -190,6 +191,26 @@ def rmsnorm_quant(x: torch.Tensor, gain: torch.Tensor | None = None, eps: float 
     _check(lib().bitlinear_rmsnorm_quant(_ptr(x), _dtype_code(x.dtype), M, K, _ptr(gain), float(eps), _ptr(norm),
                                          _ptr(xq), _ptr(scale), _ptr(rowsum), _stream(stream)))
     return (norm, xq, scale, rowsum) if norm is not None else (xq, scale, rowsum)
+
+
+GLU_RELU2, GLU_SILU = 0, 1
+
+
+def glu_quant(gate: torch.Tensor, up: torch.Tensor, act: int = GLU_RELU2, h=None, xq=None, scale=None, rowsum=None,
+              stream=None):
+    """h = act(gate) * up fused with its per-token quantisation (the down BitLinear's input):
+    returns (xq, scale, rowsum), and h first when ``h`` is True or a tensor."""
+    if gate.shape != up.shape or gate.dtype != up.dtype:
+        raise ValueError("gate and up must have the same shape and dtype")
+    M, N = gate.shape
+    dev = gate.device
+    xq = torch.empty((M, N), dtype=torch.int8, device=dev) if xq is None else xq
+    scale = torch.empty(M, dtype=torch.float32, device=dev) if scale is None else scale
+    rowsum = torch.empty(M, dtype=torch.int32, device=dev) if rowsum is None else rowsum
+    hout = torch.empty_like(gate) if h is True else (h if isinstance(h, torch.Tensor) else None)
+    _check(lib().bitlinear_glu_quant(_ptr(gate), _ptr(up), _dtype_code(gate.dtype), M, N, int(act), _ptr(hout),
+                                     _ptr(xq), _ptr(scale), _ptr(rowsum), _stream(stream)))
+    return (hout, xq, scale, rowsum) if hout is not None else (xq, scale, rowsum)
 
 
 def forward(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, out_dtype=torch.bfloat16,

@@ -217,6 +217,40 @@ __device__ __forceinline__ void norm_chunk(const Chunk16& raw, float r, const fl
   }
 }
 
+// Codes of 16 values (one 16-byte store), and the values themselves in the
+// activation type when `vout` is set; returns the sum of the codes.
+template <typename TX>
+__device__ __forceinline__ int quant_store16(const float (&v)[16], float s, int8_t* dst, TX* vout) {
+  uint32_t w[4];
+  int sum = 0;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    int q[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) q[e] = min(max(__float2int_rn(__fmul_rn(v[4 * b + e], s)), -128), 127);
+    w[b] = pack4(q[0], q[1], q[2], q[3]);
+    sum = __dp4a(static_cast<int>(w[b]), 0x01010101, sum);
+  }
+  *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  if (vout) {
+    if constexpr (sizeof(TX) == 2) {
+      uint32_t h[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        h[e] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * e]))) |
+               (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * e + 1]))) << 16);
+      uint4* d = reinterpret_cast<uint4*>(vout);
+      d[0] = make_uint4(h[0], h[1], h[2], h[3]);
+      d[1] = make_uint4(h[4], h[5], h[6], h[7]);
+    } else {
+      float4* d = reinterpret_cast<float4*>(vout);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) d[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+    }
+  }
+  return sum;
+}
+
 template <typename TX>
 __global__ void __launch_bounds__(kQuantMaxThreads) rmsnorm_quant_kernel(const __grid_constant__ NormParams P) {
   __shared__ double red_d[kQuantMaxThreads / 32];
@@ -304,32 +338,7 @@ __global__ void __launch_bounds__(kQuantMaxThreads) rmsnorm_quant_kernel(const _
     } else {
       norm_chunk<TX>(ch, r, P.gain, c, v);
     }
-    uint32_t w[4];
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      int q[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) q[e] = min(max(__float2int_rn(__fmul_rn(v[4 * b + e], s)), -128), 127);
-      w[b] = pack4(q[0], q[1], q[2], q[3]);
-      sum = __dp4a(static_cast<int>(w[b]), 0x01010101, sum);
-    }
-    *reinterpret_cast<uint4*>(qr + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-    if (nr) {
-      if constexpr (sizeof(TX) == 2) {
-        uint32_t h[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          h[e] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * e]))) |
-                 (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * e + 1]))) << 16);
-        uint4* dst = reinterpret_cast<uint4*>(nr + c * 16);
-        dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
-        dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
-      } else {
-        float4* dst = reinterpret_cast<float4*>(nr + c * 16);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-      }
-    }
+    sum += quant_store16<TX>(v, s, qr + c * 16, nr ? nr + c * 16 : nullptr);
   });
   sum = block_reduce(sum, [](int a, int b) { return a + b; }, red_i);
   if (threadIdx.x == 0) {
@@ -347,6 +356,116 @@ cudaError_t launch_rmsnorm_quant(const void* x, int x_bf16, int M, int K, const 
   if (threads > kQuantMaxThreads) threads = kQuantMaxThreads;
   if (x_bf16) return launch(rmsnorm_quant_kernel<__nv_bfloat16>, dim3(M), dim3(threads), 0, stream, pdl, P);
   return launch(rmsnorm_quant_kernel<float>, dim3(M), dim3(threads), 0, stream, pdl, P);
+}
+
+// ---------------------------------------------------------------------------
+// The FFN's gated activation fused with the quantisation of the down
+// BitLinear's input ("BitNet's Real Bet: Designing the Whole Inference
+// Stack", native-training section: SwiGLU, squared ReLU; "A Two-Billion
+// Ternary Bet": squared-ReLU-style activations).  Reading (no formula on the
+// pages): h = act(gate) * up on the stored gate/up values, in fp32, rounded
+// to the activation type; act = max(z, 0)^2 as (g * g) * u, or SiLU as
+// z / (1 + expf(-z)) * u; then the per-token quantisation.  One block per
+// token, h kept in registers between its absmax and its codes.
+// ---------------------------------------------------------------------------
+struct GluParams {
+  const void* gate;
+  const void* up;
+  int act;         // kGluRelu2 or kGluSilu
+  void* h;         // [M][N] in the activation type, or null
+  int8_t* xq;      // [M][N]
+  float* scale;
+  int32_t* rowsum; // or null
+  int N;
+};
+
+template <typename TX>
+__device__ __forceinline__ void glu_chunk(const Chunk16& g, const Chunk16& u, int act, float (&h)[16]) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float z = elem<TX>(g, e), w = elem<TX>(u, e);
+    float t;
+    if (act == kGluRelu2) {
+      const float p = z > 0.0f ? z : 0.0f;
+      t = __fmul_rn(__fmul_rn(p, p), w);
+    } else {
+      t = __fmul_rn(__fdiv_rn(z, __fadd_rn(1.0f, expf(-z))), w);
+    }
+    if constexpr (sizeof(TX) == 2) t = __bfloat162float(__float2bfloat16_rn(t));
+    h[e] = t;
+  }
+}
+
+template <typename TX>
+__global__ void __launch_bounds__(kQuantMaxThreads) glu_quant_kernel(const __grid_constant__ GluParams P) {
+  __shared__ float red_f[kQuantMaxThreads / 32];
+  __shared__ int red_i[kQuantMaxThreads / 32];
+  griddep_launch_dependents();
+  griddep_wait();  // gate and up are the preceding kernel's outputs
+
+  const int m = blockIdx.x, N = P.N, chunks = N >> 4, T = blockDim.x;
+  const TX* gr = static_cast<const TX*>(P.gate) + static_cast<size_t>(m) * N;
+  const TX* ur = static_cast<const TX*>(P.up) + static_cast<size_t>(m) * N;
+  int8_t* qr = P.xq + static_cast<size_t>(m) * N;
+  TX* hr = P.h ? static_cast<TX*>(P.h) + static_cast<size_t>(m) * N : nullptr;
+  constexpr int kKeep = 2;  // chunks per thread whose h stays in registers
+  const bool keep = chunks <= T * kKeep;
+  float hk[kKeep][16];
+
+  float amax = 0.0f;
+  for (int i = 0, c = threadIdx.x; c < chunks; ++i, c += T) {
+    Chunk16 g, u;
+    load16<TX>(gr + c * 16, g);
+    load16<TX>(ur + c * 16, u);
+    float h[16];
+    glu_chunk<TX>(g, u, P.act, h);
+#pragma unroll
+    for (int k = 0; k < kKeep; ++k)
+      if (keep && i == k) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) hk[k][e] = h[e];
+      }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(h[e]));
+  }
+  amax = block_reduce(amax, [](float a, float b) { return fmaxf(a, b); }, red_f);
+  const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
+
+  int sum = 0;
+  for (int i = 0, c = threadIdx.x; c < chunks; ++i, c += T) {
+    float h[16];
+    if (keep) {
+#pragma unroll
+      for (int k = 0; k < kKeep; ++k)
+        if (i == k) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) h[e] = hk[k][e];
+        }
+    } else {
+      Chunk16 g, u;
+      load16<TX>(gr + c * 16, g);
+      load16<TX>(ur + c * 16, u);
+      glu_chunk<TX>(g, u, P.act, h);
+    }
+    sum += quant_store16<TX>(h, s, qr + c * 16, hr ? hr + c * 16 : nullptr);
+  }
+  sum = block_reduce(sum, [](int a, int b) { return a + b; }, red_i);
+  if (threadIdx.x == 0) {
+    P.scale[m] = s;
+    if (P.rowsum) P.rowsum[m] = sum;
+  }
+}
+
+cudaError_t launch_glu_quant(const void* gate, const void* up, int x_bf16, int M, int N, int act, void* h,
+                             int8_t* xq, float* scale, int32_t* rowsum, cudaStream_t stream, bool pdl) {
+  if (M <= 0) return cudaSuccess;
+  if (act != kGluRelu2 && act != kGluSilu) return cudaErrorInvalidValue;
+  const GluParams P{gate, up, act, h, xq, scale, rowsum, N};
+  int threads = ((N / 16 + 1) / 2 + 31) / 32 * 32;  // about two chunks per thread, 64 .. 512
+  if (threads < 64) threads = 64;
+  if (threads > kQuantMaxThreads) threads = kQuantMaxThreads;
+  if (x_bf16) return launch(glu_quant_kernel<__nv_bfloat16>, dim3(M), dim3(threads), 0, stream, pdl, P);
+  return launch(glu_quant_kernel<float>, dim3(M), dim3(threads), 0, stream, pdl, P);
 }
 
 cudaError_t launch_act_quant_group(const QuantArgs* items, int n_items, int M, int x_bf16, cudaStream_t stream,

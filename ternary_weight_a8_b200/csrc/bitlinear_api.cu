@@ -218,6 +218,26 @@ int bitlinear_quant_act(const void* x, int x_dtype, int M, int K, int8_t* xq, fl
   return BL_OK;
 }
 
+int bitlinear_glu_quant(const void* gate, const void* up, int x_dtype, int M, int N, int act, void* h,
+                        int8_t* xq, float* scale, int32_t* rowsum, void* stream) {
+  BL_TRY(check_dtype(x_dtype, "x_dtype"));
+  if (M < 0) return fail(BL_ERR_INVALID_ARG, "M = %d < 0", M);
+  if (N < 64 || N % 64 != 0) return fail(BL_ERR_UNSUPPORTED_SHAPE, "N = %d: need N >= 64 and N %% 64 == 0", N);
+  if (act != BL_GLU_RELU2 && act != BL_GLU_SILU) return fail(BL_ERR_INVALID_ARG, "act = %d: unknown", act);
+  if (M == 0) return BL_OK;
+  BL_TRY(check_ptr(gate, "gate", 16));
+  BL_TRY(check_ptr(up, "up", 16));
+  BL_TRY(check_ptr(h, "h", 16, true));
+  BL_TRY(check_ptr(xq, "xq", 16));
+  BL_TRY(check_ptr(scale, "scale", 4));
+  BL_TRY(check_ptr(rowsum, "rowsum", 4, true));
+  cudaError_t e = bl::launch_glu_quant(gate, up, x_dtype == BL_BF16, M, N, act == BL_GLU_RELU2 ? bl::kGluRelu2
+                                                                                             : bl::kGluSilu,
+                                       h, xq, scale, rowsum, static_cast<cudaStream_t>(stream), true);
+  if (e != cudaSuccess) return cuda_fail(e, "glu_quant launch");
+  return BL_OK;
+}
+
 int bitlinear_rmsnorm_quant(const void* x, int x_dtype, int M, int K, const float* gain, float eps, void* x_norm,
                             int8_t* xq, float* scale, int32_t* rowsum, void* stream) {
   BL_TRY(check_dtype(x_dtype, "x_dtype"));

@@ -54,6 +54,13 @@ cudaError_t launch_act_quant_group(const QuantArgs* items, int n_items, int M, i
 cudaError_t launch_rmsnorm_quant(const void* x, int x_bf16, int M, int K, const float* gain, float eps, void* x_norm,
                                  int8_t* xq, float* scale, int32_t* rowsum, cudaStream_t stream, bool pdl);
 
+// The FFN's gated activation h = act(gate) * up fused with the per-token
+// quantisation of h (the down BitLinear's input); h (optional) written in the
+// activation type.
+enum GluAct { kGluRelu2 = 0, kGluSilu = 1 };
+cudaError_t launch_glu_quant(const void* gate, const void* up, int x_bf16, int M, int N, int act, void* h,
+                             int8_t* xq, float* scale, int32_t* rowsum, cudaStream_t stream, bool pdl);
+
 enum InType { kInInt8 = 0, kInBF16 = 1, kInF32 = 2 };
 
 // Tensor-core GEMM on quantised activations (many tokens).

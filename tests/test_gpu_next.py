@@ -2,7 +2,8 @@
 
 Fused pre-norm: RMSNorm (gain optional) fused with the per-token
 quantisation, compared with the oracle's RMSNorm followed by its
-quantisation.  The normalised activations, codes, scales and code sums are
+quantisation.  Gated activation: h = act(gate) * up fused with the
+quantisation of the down BitLinear's input (bars below).  The normalised activations, codes, scales and code sums are
 compared bit for bit (the norm's mean of squares is summed in double on both
 sides, so its order changes only double's last bits and, in practice, never
 the fp32 factor derived from it).
@@ -14,7 +15,7 @@ import torch
 import oracle
 import synth
 import ternary_weight_a8_b200 as tb
-from parity import activations, assert_y_matches, bf16_bits, dev, f32_bits, weights
+from parity import activations, assert_y_matches, bf16_bits, bf16_ordered, dev, f32_bits, weights
 
 pytestmark = pytest.mark.gpu
 
@@ -82,3 +83,83 @@ def test_rmsnorm_rejects_bad_eps():
         with pytest.raises(tb.BitLinearError) as e:
             tb.rmsnorm_quant(x, eps=eps)
         assert e.value.code == tb.BL_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------------------
+# The FFN's gated activation fused with the down BitLinear's quantisation.
+# Squared ReLU is exact fp32 arithmetic: h, codes, scales and sums bit for
+# bit.  SiLU calls the device expf (a few fp32 ulps from the exact value):
+# h within 1 bf16 ulp (fp32: 8 ulps) of the oracle's one rounding of the
+# exact value, and the codes exactly those of the oracle's quantisation of
+# the kernel's own h (the integer decision taken on the same values).
+# ----------------------------------------------------------------------------
+
+def _gate_up(M, N, dtype, seed):
+    g, gf = activations(M, N, seed=seed, dtype=dtype)
+    u, uf = activations(M, N, seed=seed + 1, dtype=dtype)
+    return g, gf, u, uf
+
+
+@pytest.mark.parametrize("M,N,dtype", [(1, 6912, "bf16"), (16, 28672, "bf16"), (2048, 6912, "bf16"),
+                                       (5, 640, "f32"), (3, 33792, "bf16")])
+def test_glu_relu2_quant_parity(M, N, dtype):
+    g, gf, u, uf = _gate_up(M, N, dtype, seed=N + M)
+    h_ref, q_ref, s_ref, r_ref = oracle.glu_quant(gf, uf, oracle.GLU_RELU2, dtype == "bf16")
+    h, q, s, r = tb.glu_quant(g, u, tb.GLU_RELU2, h=True)
+    if dtype == "bf16":
+        assert np.array_equal(bf16_bits(h), (f32_bits(h_ref) >> 16).astype(np.uint16))
+    else:
+        assert np.array_equal(f32_bits(h.cpu().numpy()), f32_bits(h_ref))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(f32_bits(s.cpu().numpy()), f32_bits(s_ref))
+    assert np.array_equal(r.cpu().numpy(), r_ref)
+
+
+@pytest.mark.parametrize("M,N,dtype", [(1, 6912, "bf16"), (64, 2560, "bf16"), (4, 1024, "f32")])
+def test_glu_silu_quant_parity(M, N, dtype):
+    g, gf, u, uf = _gate_up(M, N, dtype, seed=N + 2 * M)
+    h_ref = oracle.glu(gf, uf, oracle.GLU_SILU, dtype == "bf16")
+    h, q, s, r = tb.glu_quant(g, u, tb.GLU_SILU, h=True)
+    if dtype == "bf16":
+        hv = (bf16_bits(h).astype(np.uint32) << 16).view(np.float32)
+        d = np.abs(bf16_ordered(bf16_bits(h)) - bf16_ordered((f32_bits(h_ref) >> 16).astype(np.uint16)))
+        assert d.max() <= 1 and (d == 0).mean() > 0.99
+    else:
+        hv = h.cpu().numpy()
+        err = np.abs(hv.astype(np.float64) - h_ref.astype(np.float64))
+        assert (err <= 8 * np.spacing(np.abs(h_ref)) + 1e-45).all()
+    q_ref, s_ref, r_ref = oracle.quant_act(hv)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(f32_bits(s.cpu().numpy()), f32_bits(s_ref))
+    assert np.array_equal(r.cpu().numpy(), r_ref)
+
+
+def test_ffn_gate_up_glu_down_matches_the_oracle():
+    """x -> gate, up (one launch, shared quantisation) -> squared-ReLU GLU + quantisation -> down."""
+    M, D, F = 4, 1024, 2816
+    x, xf = activations(M, D, seed=31, dtype="bf16")
+    Wg, Wu, Wd = weights(F, D, seed=32), weights(F, D, seed=33), weights(D, F, seed=34)
+    (pg, gg, Tg), (pu, gu, Tu), (pd, gd, Td) = (oracle.pack_weights(W) for W in (Wg, Wu, Wd))
+    yg = torch.empty((M, F), dtype=torch.bfloat16, device="cuda")
+    yu = torch.empty((M, F), dtype=torch.bfloat16, device="cuda")
+    layers = [tb.Layer(dev(pg), dev(np.array([gg], np.float32)), x, yg),
+              tb.Layer(dev(pu), dev(np.array([gu], np.float32)), x, yu)]
+    tb.layer_chain(layers)
+    xq, s, r = tb.glu_quant(yg, yu, tb.GLU_RELU2)
+    y, acc = tb.forward_quantized(dev(pd), dev(np.array([gd], np.float32)), xq, s, r, out_dtype=torch.bfloat16,
+                                  acc_out=True)
+    # oracle: the two products, stored as bf16, the gated activation, its codes, the down product
+    _, yg_ref, *_ = oracle.forward(Tg, gg, xf)
+    _, yu_ref, *_ = oracle.forward(Tu, gu, xf)
+    to_bf16 = lambda v: (oracle.round_bf16(v).astype(np.uint32) << 16).view(np.float32)
+    h_ref, q_ref, s_ref, r_ref = oracle.glu_quant(to_bf16(yg_ref), to_bf16(yu_ref), oracle.GLU_RELU2, True)
+    acc_ref = oracle.accumulate(q_ref, Td)
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert_y_matches(y, oracle.dequant(acc_ref, gd, s_ref), acc_ref)
+
+
+def test_glu_rejects_unknown_activation():
+    g = torch.zeros((1, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(tb.BitLinearError) as e:
+        tb.glu_quant(g, g, 7)
+    assert e.value.code == tb.BL_ERR_INVALID_ARG
