@@ -519,6 +519,26 @@ def run_next(args, world, peaks, L2):
         usecs, _ = timed_graph_run(unfused, steps, 20, world, chunk=100)
         res["unfused_torch_glu_then_quant_us"] = round(usecs / steps * 1e6, 3)
         out["glu_quant_%dx%d" % (M, N)] = res
+    # The lookup-table decode product against the tensor-core decode kernel, same codes, one token.
+    for K, N in ((2560, 6912), (8192, 10240)):
+        sets, set_bytes = make_layer_sets([(K, N)], seed=800, min_bytes=4 * L2)
+        bits, _ = synth.activations_bf16(1, K, seed=801)
+        xq, sc, rs = tb.quant_act(torch.from_numpy(bits.view("int16")).cuda().view(torch.bfloat16))
+        y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+        ws = tb.new_workspace(tb.workspace_bytes(1, N, K))
+        steps = 400
+        res = {"weight_bytes": set_bytes}
+        for name, fn in (("lut", lambda i: tb.forward_lut(sets[i % len(sets)][0][0], sets[i % len(sets)][0][1], xq,
+                                                           sc, rs, y=y)),
+                         ("tensor_core_gemv", lambda i: tb.forward_quantized(sets[i % len(sets)][0][0],
+                                                                             sets[i % len(sets)][0][1], xq, sc, rs,
+                                                                             y=y, workspace=ws))):
+            secs, _ = timed_graph_run(fn, steps, 20, world, chunk=100)
+            gbs = set_bytes / (secs / steps) / 1e9
+            res[name] = {"us": round(secs / steps * 1e6, 3), "GB/s": round(gbs, 1),
+                         "pct_hbm_measured": round(100 * gbs / peaks["hbm"], 2)}
+        out["lut_vs_gemv_%dx%d" % (K, N)] = res
+        del sets
     return out
 
 

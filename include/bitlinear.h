@@ -151,6 +151,30 @@ typedef enum { BL_GLU_RELU2 = 0, BL_GLU_SILU = 1 } bl_glu;
 int bitlinear_glu_quant(const void* gate, const void* up, int x_dtype, int M, int N, int act, void* h,
                         int8_t* xq, float* scale, int32_t* rowsum, void* stream);
 
+/*
+ * The product and dequantisation of one token by table lookup instead of
+ * multiplication: the T-MAC approach ("BitNet b1.58 and the 1-Bit AI
+ * Architecture Revolution", section "The CPU Revival: bitnet.cpp and T-MAC":
+ * four ternary weights leave few partial sums, precomputed and looked up,
+ * with the sign structure reducing the tables to 16 binary combinations).
+ * Here each 16-entry table holds the subset sums of the 4 codes of q that
+ * share a packed byte, and a byte's two bit planes index it
+ * (sum c*q = T[lo] + 2 T[hi]).  The result equals bitlinear_forward_quantized's
+ * bit for bit (acc) and at its bars (y); it exists to compare the two
+ * decode algorithms.
+ *   packed, gamma, N, K: as bitlinear_forward; K % 64 == 0 and K <= 24576
+ *           (the tables take 8 bytes of shared memory per input).
+ *   xq, scale, rowsum: one token's codes [K], scale [1], code sum [1] as
+ *           bitlinear_quant_act wrote them (rowsum required).
+ *   M       must be 1.
+ *   y, y_dtype, acc_out: as bitlinear_forward_quantized.
+ * No workspace.  Errors: BL_ERR_UNSUPPORTED_SHAPE for M != 1 or K out of
+ * range; the rest as bitlinear_forward_quantized.
+ */
+int bitlinear_forward_lut(const uint8_t* packed, const float* gamma, int N, int K, const int8_t* xq,
+                          const float* scale, const int32_t* rowsum, int M, void* y, int y_dtype, int32_t* acc_out,
+                          void* stream);
+
 /* Workspace bytes bitlinear_forward needs (status word + q, s, rowsum). */
 size_t bitlinear_workspace_bytes(int M, int N, int K);
 

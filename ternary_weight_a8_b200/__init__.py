@@ -70,6 +70,7 @@ def lib() -> ctypes.CDLL:
             "bitlinear_quant_act": (i32, [vp, i32, i32, i32, vp, vp, vp, vp]),
             "bitlinear_rmsnorm_quant": (i32, [vp, i32, i32, i32, vp, ctypes.c_float, vp, vp, vp, vp, vp]),
             "bitlinear_glu_quant": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
+            "bitlinear_forward_lut": (i32, [vp, vp, i32, i32, vp, vp, vp, i32, vp, i32, vp, vp]),
             "bitlinear_workspace_bytes": (sz, [i32, i32, i32]),
             "bitlinear_forward": (i32, [vp, vp, i32, i32, vp, i32, i32, vp, i32, vp, vp, sz, vp]),
             "bitlinear_forward_quantized": (i32, [vp, vp, i32, i32, vp, vp, vp, i32, vp, i32, vp, vp, sz, vp]),
@@ -191,6 +192,21 @@ def rmsnorm_quant(x: torch.Tensor, gain: torch.Tensor | None = None, eps: float 
     _check(lib().bitlinear_rmsnorm_quant(_ptr(x), _dtype_code(x.dtype), M, K, _ptr(gain), float(eps), _ptr(norm),
                                          _ptr(xq), _ptr(scale), _ptr(rowsum), _stream(stream)))
     return (norm, xq, scale, rowsum) if norm is not None else (xq, scale, rowsum)
+
+
+def forward_lut(packed: torch.Tensor, gamma: torch.Tensor, xq: torch.Tensor, scale: torch.Tensor,
+                rowsum: torch.Tensor, out_dtype=torch.bfloat16, y: torch.Tensor | None = None,
+                acc_out: torch.Tensor | bool | None = None, stream=None):
+    """One token's product by table lookup (the T-MAC-style decode), on codes from ``quant_act``."""
+    N = packed.shape[0]
+    M, K = xq.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    acc = torch.empty((M, N), dtype=torch.int32, device=xq.device) if acc_out is True else (
+        acc_out if isinstance(acc_out, torch.Tensor) else None)
+    _check(lib().bitlinear_forward_lut(_ptr(packed), _ptr(gamma), N, K, _ptr(xq), _ptr(scale), _ptr(rowsum), M,
+                                       _ptr(y), _dtype_code(y.dtype), _ptr(acc), _stream(stream)))
+    return (y, acc) if acc is not None else y
 
 
 GLU_RELU2, GLU_SILU = 0, 1

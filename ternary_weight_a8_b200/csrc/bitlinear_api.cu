@@ -218,6 +218,28 @@ int bitlinear_quant_act(const void* x, int x_dtype, int M, int K, int8_t* xq, fl
   return BL_OK;
 }
 
+int bitlinear_forward_lut(const uint8_t* packed, const float* gamma, int N, int K, const int8_t* xq,
+                          const float* scale, const int32_t* rowsum, int M, void* y, int y_dtype, int32_t* acc_out,
+                          void* stream) {
+  BL_TRY(check_nk(N, K));
+  BL_TRY(check_dtype(y_dtype, "y_dtype"));
+  if (M != 1) return fail(BL_ERR_UNSUPPORTED_SHAPE, "M = %d: the lookup-table product takes one token", M);
+  if (K > bl::kLutMaxK)
+    return fail(BL_ERR_UNSUPPORTED_SHAPE, "K = %d: the lookup tables need K <= %d", K, bl::kLutMaxK);
+  BL_TRY(check_ptr(packed, "packed", 16));
+  BL_TRY(check_ptr(gamma, "gamma", 4));
+  BL_TRY(check_ptr(xq, "xq", 16));
+  BL_TRY(check_ptr(scale, "scale", 4));
+  BL_TRY(check_ptr(rowsum, "rowsum", 4));
+  BL_TRY(check_ptr(y, "y", 4));
+  BL_TRY(check_ptr(acc_out, "acc_out", 4, true));
+  cudaError_t e = bl::launch_lut_gemv(packed, gamma, N, K, xq, scale, rowsum, y,
+                                      y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32, acc_out,
+                                      static_cast<cudaStream_t>(stream), true);
+  if (e != cudaSuccess) return cuda_fail(e, "lookup-table product launch");
+  return BL_OK;
+}
+
 int bitlinear_glu_quant(const void* gate, const void* up, int x_dtype, int M, int N, int act, void* h,
                         int8_t* xq, float* scale, int32_t* rowsum, void* stream) {
   BL_TRY(check_dtype(x_dtype, "x_dtype"));

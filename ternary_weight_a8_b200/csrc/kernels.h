@@ -108,6 +108,14 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 void* tensor_map_encoder();
 cudaError_t launch_gemm(const ProductArgs& a, cudaStream_t stream, bool pdl);
 
+// Lookup-table decode product for one token (the T-MAC-style alternative):
+// codes of one token [K], K % 64 == 0 and K <= kLutMaxK (its tables fill
+// shared memory: 8 bytes per input).
+constexpr int kLutMaxK = 24576;
+cudaError_t launch_lut_gemv(const uint8_t* packed, const float* gamma, int N, int K, const int8_t* xq,
+                            const float* scale, const int32_t* rowsum, void* y, int y_type, int32_t* acc_out,
+                            cudaStream_t stream, bool pdl);
+
 // Self-test of the bounded device wait.
 cudaError_t launch_wait_timeout_selftest(uint32_t* status, int limit_us, cudaStream_t stream);
 

@@ -163,3 +163,54 @@ def test_glu_rejects_unknown_activation():
     with pytest.raises(tb.BitLinearError) as e:
         tb.glu_quant(g, g, 7)
     assert e.value.code == tb.BL_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------------------
+# The lookup-table decode product: the same exact accumulators as the
+# forward (bit for bit), y at the forward's bars, and equal to the
+# tensor-core decode kernel's output on the same codes.
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K", [(6912, 2560), (2560, 2560), (1000, 8192), (300, 24576), (17, 64), (333, 8640)])
+def test_lut_product_parity(N, K):
+    W = weights(N, K, seed=N + K)
+    packed_ref, gamma_ref, T = oracle.pack_weights(W)
+    x, xf = activations(1, K, seed=K, dtype="bf16")
+    acc_ref, y_ref, *_ = oracle.forward(T, gamma_ref, xf)
+    p, g = dev(packed_ref), dev(np.array([gamma_ref], np.float32))
+    xq, s, r = tb.quant_act(x)
+    for ydt in (torch.bfloat16, torch.float32):
+        y, acc = tb.forward_lut(p, g, xq, s, r, out_dtype=ydt, acc_out=True)
+        assert np.array_equal(acc.cpu().numpy(), acc_ref)
+        assert_y_matches(y, y_ref, acc_ref)
+    if K % 128 == 0:
+        y2 = tb.forward_quantized(p, g, xq, s, r, out_dtype=torch.bfloat16)
+        y1 = tb.forward_lut(p, g, xq, s, r, out_dtype=torch.bfloat16)
+        assert torch.equal(y1, y2)
+
+
+def test_lut_product_extremes():
+    """All weights +1 or -1 and a token at +-127: |acc| = 127 K through the tables."""
+    N, K = 64, 4096
+    for sign in (1, -1):
+        T = np.full((N, K), sign, np.int8)
+        packed = dev(oracle.pack(T))
+        xq = torch.full((1, K), 127, dtype=torch.int8, device="cuda")
+        s = torch.ones(1, dtype=torch.float32, device="cuda")
+        r = torch.full((1,), 127 * K, dtype=torch.int32, device="cuda")
+        g = torch.ones(1, dtype=torch.float32, device="cuda")
+        y, acc = tb.forward_lut(packed, g, xq, s, r, out_dtype=torch.float32, acc_out=True)
+        assert (acc.cpu().numpy() == sign * 127 * K).all()
+
+
+def test_lut_product_rejects_unsupported_shapes():
+    p = torch.zeros((8, 64), dtype=torch.uint8, device="cuda")
+    g = torch.ones(1, dtype=torch.float32, device="cuda")
+    for M, K in ((2, 256), (1, 24576 + 64)):
+        xq = torch.zeros((M, K), dtype=torch.int8, device="cuda")
+        pk = torch.zeros((8, K // 4), dtype=torch.uint8, device="cuda")
+        s = torch.ones(M, dtype=torch.float32, device="cuda")
+        r = torch.zeros(M, dtype=torch.int32, device="cuda")
+        with pytest.raises(tb.BitLinearError) as e:
+            tb.forward_lut(pk, g, xq, s, r)
+        assert e.value.code == tb.BL_ERR_UNSUPPORTED_SHAPE
