@@ -67,6 +67,12 @@ def _lib():
         lib.oracle_rmsnorm.restype = None
         lib.oracle_glu.argtypes = [vp, vp, i64, ctypes.c_int, ctypes.c_int, vp]
         lib.oracle_glu.restype = None
+        lib.oracle_ste_grad_input.argtypes = [vp, vp, ctypes.c_float, i64, i64, i64, vp]
+        lib.oracle_ste_grad_input.restype = None
+        lib.oracle_ste_xhat.argtypes = [vp, vp, i64, i64, vp]
+        lib.oracle_ste_xhat.restype = None
+        lib.oracle_ste_grad_weight.argtypes = [vp, vp, i64, i64, i64, vp]
+        lib.oracle_ste_grad_weight.restype = None
         _handle = lib
     return _handle
 
@@ -214,3 +220,37 @@ def glu_quant(gate: np.ndarray, up: np.ndarray, act: int, out_bf16: bool):
     h = glu(gate, up, act, out_bf16)
     q, s, r = quant_act(h)
     return h, q, s, r
+
+
+def ste_grad_input(dy: np.ndarray, T: np.ndarray, gamma) -> np.ndarray:
+    """Straight-through dx = gamma * (dy . t), double ``[M][K]``."""
+    dy = _c(dy, np.float32)
+    T = _c(T, np.int8)
+    M, N = dy.shape
+    K = T.shape[1]
+    assert T.shape[0] == N
+    dx = np.empty((M, K), dtype=np.float64)
+    _lib().oracle_ste_grad_input(dy.ctypes.data, T.ctypes.data, float(np.float32(gamma)), M, N, K, dx.ctypes.data)
+    return dx
+
+
+def ste_xhat(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """The stored dequantised activations bf16(q / s), as fp32 values ``[M][K]``."""
+    q = _c(q, np.int8)
+    s = _c(s, np.float32)
+    M, K = q.shape
+    out = np.empty((M, K), dtype=np.float32)
+    _lib().oracle_ste_xhat(q.ctypes.data, s.ctypes.data, M, K, out.ctypes.data)
+    return out
+
+
+def ste_grad_weight(dy: np.ndarray, xhat: np.ndarray) -> np.ndarray:
+    """Straight-through dW = dy^T . xhat, double ``[N][K]``."""
+    dy = _c(dy, np.float32)
+    xhat = _c(xhat, np.float32)
+    M, N = dy.shape
+    K = xhat.shape[1]
+    assert xhat.shape[0] == M
+    dw = np.empty((N, K), dtype=np.float64)
+    _lib().oracle_ste_grad_weight(dy.ctypes.data, xhat.ctypes.data, M, N, K, dw.ctypes.data)
+    return dw

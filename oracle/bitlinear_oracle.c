@@ -29,6 +29,11 @@
  *            squared ReLU) and "A Two-Billion Ternary Bet" (squared-ReLU-style
  *            activations tame gradient scale): the gated activation between
  *            the gate/up BitLinears and the down BitLinear of the FFN.
+ *  [STE]     "BitNet b1.58 and the 1-Bit AI Architecture Revolution", section
+ *            "Training Dynamics: The Straight-Through Estimator": the backward
+ *            pass treats the quantisation as the identity, so gradients pass
+ *            through the quantised weights to the high-precision shadow
+ *            weights, which are quantised again before the next forward.
  *  [Norm]    "BitNet's Real Bet: Designing the Whole Inference Stack" (native
  *            training section: the 2024 model uses RMSNorm, the 2B4T model
  *            sub-layer normalisation) and "A Two-Billion Ternary Bet"
@@ -60,6 +65,11 @@
  *    the activation type.  Squared ReLU is two fp32 multiplies, (g * g) * u
  *    with g = max(gate, 0); SiLU is evaluated exactly (double) and rounded
  *    once, the GPU's fp32 evaluation being held to a stated bar.
+ *  - Straight-through backward: the forward is y = xhat . What^T with
+ *    xhat = q / s (per token) and What = gamma * t; the quantisers pass
+ *    gradients unchanged, so dx = dy . What = gamma * (dy . t) and
+ *    dW = dy^T . xhat.  xhat enters as the backward stores it: q / s in fp32
+ *    rounded to bf16.  Both products are evaluated in double.
  */
 #include <math.h>
 #include <stdint.h>
@@ -263,5 +273,41 @@ void oracle_glu(const float* gate, const float* up, int64_t count, int act, int 
       memcpy(&h, &u, 4);
     }
     out[i] = h;
+  }
+}
+
+/* [STE]: dx[m][k] = gamma * sum_n dy[m][n] * t[n][k], in double. */
+void oracle_ste_grad_input(const float* dy, const int8_t* T, float gamma, int64_t M, int64_t N, int64_t K,
+                           double* dx) {
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t k = 0; k < K; ++k) {
+      double sum = 0.0;
+      for (int64_t n = 0; n < N; ++n) sum += (double)dy[m * N + n] * (double)T[n * K + k];
+      dx[m * K + k] = (double)gamma * sum;
+    }
+  }
+}
+
+/* [STE]: the stored dequantised activations, xhat = bf16(fp32(q / s)), as fp32 values. */
+void oracle_ste_xhat(const int8_t* q, const float* s, int64_t M, int64_t K, float* xhat) {
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t k = 0; k < K; ++k) {
+      float v = (float)q[m * K + k] / s[m];
+      uint16_t h = oracle_bf16_of((double)v);
+      uint32_t u = (uint32_t)h << 16;
+      memcpy(&v, &u, 4);
+      xhat[m * K + k] = v;
+    }
+  }
+}
+
+/* [STE]: dW[n][k] = sum_m dy[m][n] * xhat[m][k], in double. */
+void oracle_ste_grad_weight(const float* dy, const float* xhat, int64_t M, int64_t N, int64_t K, double* dw) {
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t k = 0; k < K; ++k) {
+      double sum = 0.0;
+      for (int64_t m = 0; m < M; ++m) sum += (double)dy[m * N + n] * (double)xhat[m * K + k];
+      dw[n * K + k] = sum;
+    }
   }
 }

@@ -43,6 +43,11 @@ MUTANTS = {
     "glu_silu_wrong_sign": ("h = (float)(z / (1.0 + exp(-z)) * (double)up[i]);",
                             "h = (float)(z / (1.0 + exp(z)) * (double)up[i]);"),
     "glu_silu_ignores_up": ("h = (float)(z / (1.0 + exp(-z)) * (double)up[i]);", "h = (float)(z / (1.0 + exp(-z)));"),
+    "ste_input_without_gamma": ("dx[m * K + k] = (double)gamma * sum;", "dx[m * K + k] = sum;"),
+    "ste_xhat_multiplies_scale": ("float v = (float)q[m * K + k] / s[m];", "float v = (float)q[m * K + k] * s[m];"),
+    "ste_xhat_not_rounded": ("xhat[m * K + k] = v;", "xhat[m * K + k] = (float)q[m * K + k] / s[m];"),
+    "ste_weight_reversed_k": ("sum += (double)dy[m * N + n] * (double)xhat[m * K + k];",
+                              "sum += (double)dy[m * N + n] * (double)xhat[m * K + (K - 1 - k)];"),
 }
 
 

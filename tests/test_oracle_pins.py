@@ -18,6 +18,8 @@ Passages (web pages on BitNet b1.58):
             training: RMSNorm, sub-layer normalisation) and "BitNet b1.58 and
             the 1-Bit AI Architecture Revolution", section "Empirical
             Performance and The New Scaling Law" (RMSNorm).
+  [STE]     "BitNet b1.58 and the 1-Bit AI Architecture Revolution", section
+            "Training Dynamics: The Straight-Through Estimator".
   [GLU]     "BitNet's Real Bet: Designing the Whole Inference Stack" (native
             training: SwiGLU, squared ReLU) and "A Two-Billion Ternary Bet"
             (squared-ReLU-style activations).
@@ -470,3 +472,62 @@ def test_glu_bf16_output_rounds_the_relu2_product():
     f32 = oracle.glu(g, u, oracle.GLU_RELU2, False)
     b16 = oracle.glu(g, u, oracle.GLU_RELU2, True)
     assert np.array_equal(b16, (_bf16_rne_bits(f32).astype(np.uint32) << 16).view(np.float32))
+
+
+# ----------------------------------------------------------------------------
+# The straight-through backward  [STE]
+# ----------------------------------------------------------------------------
+
+def _ste_case(M, N, K, seed):
+    W = synth.latent_weights(N, K, seed=seed)
+    _, gamma, T = oracle.pack_weights(W)
+    _, x = synth.activations_bf16(M, K, seed=seed + 1)
+    q, s, _ = oracle.quant_act(x)
+    dy = synth.activations_f32(M, N, seed=seed + 2)
+    return T, gamma, q, s, dy
+
+
+@pytest.mark.parametrize("M,N,K,seed", [(4, 48, 64, 0), (16, 96, 128, 1), (7, 33, 256, 2)])
+def test_ste_grads_match_float64_products(M, N, K, seed):
+    """dx = gamma (dy . t) and dW = dy^T . xhat, against numpy's float64 products."""
+    T, gamma, q, s, dy = _ste_case(M, N, K, seed)
+    dx = oracle.ste_grad_input(dy, T, gamma)
+    want = float(gamma) * (dy.astype(np.float64) @ T.astype(np.float64))
+    assert np.allclose(dx, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+    xhat = oracle.ste_xhat(q, s)
+    dw = oracle.ste_grad_weight(dy, xhat)
+    want = dy.astype(np.float64).T @ xhat.astype(np.float64)
+    assert np.allclose(dw, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+
+
+def test_ste_one_hot_gradients_select_rows():
+    """A one-hot dy picks one row of gamma * t for dx and one token of xhat for dW."""
+    T, gamma, q, s, dy = _ste_case(3, 20, 64, 3)
+    dy = np.zeros_like(dy)
+    dy[1, 7] = 1.0
+    dx = oracle.ste_grad_input(dy, T, gamma)
+    assert np.array_equal(dx[1], float(gamma) * T[7].astype(np.float64)) and not dx[0].any() and not dx[2].any()
+    xhat = oracle.ste_xhat(q, s)
+    dw = oracle.ste_grad_weight(dy, xhat)
+    assert np.array_equal(dw[7], xhat[1].astype(np.float64)) and not np.delete(dw, 7, axis=0).any()
+
+
+def test_ste_xhat_is_the_bf16_rounding_of_q_over_s():
+    T, gamma, q, s, dy = _ste_case(5, 8, 256, 4)
+    xhat = oracle.ste_xhat(q, s)
+    f32 = (q.astype(np.float32) / s[:, None]).astype(np.float32)
+    assert np.array_equal(xhat, (_bf16_rne_bits(f32).astype(np.uint32) << 16).view(np.float32))
+
+
+def test_ste_grads_share_the_bilinear_form():
+    """<dx, xhat> = <dW, gamma t> = <dy, xhat . (gamma t)^T> (Euler's identity for a bilinear form)."""
+    T, gamma, q, s, dy = _ste_case(6, 40, 128, 5)
+    xhat = oracle.ste_xhat(q, s)
+    dx = oracle.ste_grad_input(dy, T, gamma)
+    dw = oracle.ste_grad_weight(dy, xhat)
+    a = math.fsum((dx * xhat.astype(np.float64)).ravel())
+    b = math.fsum((dw * (float(gamma) * T.astype(np.float64))).ravel())
+    y = xhat.astype(np.float64) @ (float(gamma) * T.astype(np.float64)).T
+    c = math.fsum((dy.astype(np.float64) * y).ravel())
+    scale = math.fsum(np.abs(dy.astype(np.float64) * y).ravel())
+    assert abs(a - c) <= 1e-12 * scale and abs(b - c) <= 1e-12 * scale
