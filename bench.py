@@ -539,6 +539,25 @@ def run_next(args, world, peaks, L2):
                          "pct_hbm_measured": round(100 * gbs / peaks["hbm"], 2)}
         out["lut_vs_gemv_%dx%d" % (K, N)] = res
         del sets
+    # The straight-through backward at the prefill shape: two bf16 tensor-core products.
+    M, K, N = PREFILL["M"], PREFILL["K"], PREFILL["N"]
+    codes = torch.randint(0, 3, (N, K // 4, 4), dtype=torch.int32, device="cuda")  # 2-bit codes 0..2
+    packed = (codes[..., 0] | (codes[..., 1] << 2) | (codes[..., 2] << 4) | (codes[..., 3] << 6)).to(torch.uint8)
+    gamma = torch.full((1,), 0.02, dtype=torch.float32, device="cuda")
+    bits, _ = synth.activations_bf16(M, K, seed=900)
+    xq, sc, _ = tb.quant_act(torch.from_numpy(bits.view("int16")).cuda().view(torch.bfloat16))
+    dy = torch.from_numpy(synth.activations_bf16(M, N, seed=901)[0].view("int16")).cuda().view(torch.bfloat16)
+    dx = torch.empty((M, K), dtype=torch.float32, device="cuda")
+    dw = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    ws = tb.new_workspace(tb.ste_workspace_bytes(M, N, K))
+    steps = 50
+    secs, _ = timed_graph_run(lambda i: tb.ste_backward(packed, gamma, K, dy, xq, sc, dx=dx, dw=dw, workspace=ws),
+                              steps, 5, world, chunk=50)
+    flops = 2 * 2.0 * M * N * K
+    tf = flops / (secs / steps) / 1e12
+    out["ste_backward_2048x2560x6912"] = {"us": round(secs / steps * 1e6, 2), "TFLOP/s": round(tf, 1),
+                                          "pct_bf16_measured": round(100 * tf / peaks["bf16"], 2),
+                                          "flops_per_call": flops, "device_status": tb.device_status(ws)}
     return out
 
 

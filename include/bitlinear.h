@@ -175,6 +175,31 @@ int bitlinear_forward_lut(const uint8_t* packed, const float* gamma, int N, int 
                           const float* scale, const int32_t* rowsum, int M, void* y, int y_dtype, int32_t* acc_out,
                           void* stream);
 
+/* Workspace bytes bitlinear_ste_backward needs for M tokens of an N x K BitLinear. */
+size_t bitlinear_ste_workspace_bytes(int M, int N, int K);
+
+/*
+ * The straight-through backward of a BitLinear, for training on latent
+ * ("shadow") weights: "BitNet b1.58 and the 1-Bit AI Architecture
+ * Revolution", section "Training Dynamics: The Straight-Through Estimator"
+ * (the backward treats the quantisation as the identity; gradients reach the
+ * high-precision shadow weights, which are quantised again, with
+ * bitlinear_pack_weights, before the next forward).  With the forward
+ * y = xhat . What^T, xhat = q / s and What = gamma * t:
+ *   dx = gamma * (dy . t)   and   dW = dy^T . xhat,
+ * xhat taken as the backward stores it, bf16(q / s).  Both products run on
+ * the tensor cores (bf16 operands, fp32 accumulation).
+ *   packed, gamma, N, K: the weights of the forward (N % 64 == 0, K % 64 == 0).
+ *   dy      device bf16 [M][N]: the output gradient; M % 8 == 0.
+ *   xq, scale: the forward's codes [M][K] and scales [M] (bitlinear_quant_act).
+ *   dx      device [M][K] of dx_dtype out, or NULL to skip.
+ *   dw      device fp32 [N][K] out, or NULL to skip (the gradient of the latent weights).
+ *   workspace / workspace_bytes: >= bitlinear_ste_workspace_bytes(M, N, K), first 256 bytes zero.
+ */
+int bitlinear_ste_backward(const uint8_t* packed, const float* gamma, int N, int K, const void* dy,
+                           const int8_t* xq, const float* scale, int M, void* dx, int dx_dtype, float* dw,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
 /* Workspace bytes bitlinear_forward needs (status word + q, s, rowsum). */
 size_t bitlinear_workspace_bytes(int M, int N, int K);
 

@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
             "bitlinear_rmsnorm_quant": (i32, [vp, i32, i32, i32, vp, ctypes.c_float, vp, vp, vp, vp, vp]),
             "bitlinear_glu_quant": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
             "bitlinear_forward_lut": (i32, [vp, vp, i32, i32, vp, vp, vp, i32, vp, i32, vp, vp]),
+            "bitlinear_ste_workspace_bytes": (sz, [i32, i32, i32]),
+            "bitlinear_ste_backward": (i32, [vp, vp, i32, i32, vp, vp, vp, i32, vp, i32, vp, vp, sz, vp]),
             "bitlinear_workspace_bytes": (sz, [i32, i32, i32]),
             "bitlinear_forward": (i32, [vp, vp, i32, i32, vp, i32, i32, vp, i32, vp, vp, sz, vp]),
             "bitlinear_forward_quantized": (i32, [vp, vp, i32, i32, vp, vp, vp, i32, vp, i32, vp, vp, sz, vp]),
@@ -207,6 +209,27 @@ def forward_lut(packed: torch.Tensor, gamma: torch.Tensor, xq: torch.Tensor, sca
     _check(lib().bitlinear_forward_lut(_ptr(packed), _ptr(gamma), N, K, _ptr(xq), _ptr(scale), _ptr(rowsum), M,
                                        _ptr(y), _dtype_code(y.dtype), _ptr(acc), _stream(stream)))
     return (y, acc) if acc is not None else y
+
+
+def ste_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().bitlinear_ste_workspace_bytes(M, N, K))
+
+
+def ste_backward(packed: torch.Tensor, gamma: torch.Tensor, K: int, dy: torch.Tensor, xq: torch.Tensor,
+                 scale: torch.Tensor, dx=True, dx_dtype=torch.float32, dw=True, workspace=None, stream=None):
+    """The straight-through backward: returns (dx [M][K] or None, dW [N][K] fp32 or None)."""
+    M, N = dy.shape
+    if dy.dtype != torch.bfloat16:
+        raise ValueError("dy must be bf16")
+    dev = dy.device
+    dxt = torch.empty((M, K), dtype=dx_dtype, device=dev) if dx is True else (dx if isinstance(dx, torch.Tensor) else None)
+    dwt = torch.empty((N, K), dtype=torch.float32, device=dev) if dw is True else (dw if isinstance(dw, torch.Tensor) else None)
+    if workspace is None:
+        workspace = new_workspace(ste_workspace_bytes(M, N, K), device=dev)
+    _check(lib().bitlinear_ste_backward(_ptr(packed), _ptr(gamma), N, K, _ptr(dy), _ptr(xq), _ptr(scale), M, _ptr(dxt),
+                                        _dtype_code(dxt.dtype) if dxt is not None else 0, _ptr(dwt), _ptr(workspace),
+                                        workspace.numel(), _stream(stream)))
+    return dxt, dwt
 
 
 GLU_RELU2, GLU_SILU = 0, 1

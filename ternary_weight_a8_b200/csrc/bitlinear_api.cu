@@ -218,6 +218,39 @@ int bitlinear_quant_act(const void* x, int x_dtype, int M, int K, int8_t* xq, fl
   return BL_OK;
 }
 
+size_t bitlinear_ste_workspace_bytes(int M, int N, int K) {
+  if (M < 0 || N < 0 || K < 0) return 0;
+  return kStatusBytes + bl::ste_scratch_bytes(M, N, K);
+}
+
+int bitlinear_ste_backward(const uint8_t* packed, const float* gamma, int N, int K, const void* dy,
+                           const int8_t* xq, const float* scale, int M, void* dx, int dx_dtype, float* dw,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  BL_TRY(check_nk(N, K));
+  if (N % 64 != 0) return fail(BL_ERR_UNSUPPORTED_SHAPE, "N = %d: the backward needs N %% 64 == 0", N);
+  if (M < 0) return fail(BL_ERR_INVALID_ARG, "M = %d < 0", M);
+  if (M % 8 != 0) return fail(BL_ERR_UNSUPPORTED_SHAPE, "M = %d: the backward needs M %% 8 == 0", M);
+  BL_TRY(check_dtype(dx_dtype, "dx_dtype"));
+  if (M == 0 || (!dx && !dw)) return BL_OK;
+  BL_TRY(check_ptr(packed, "packed", 16));
+  BL_TRY(check_ptr(gamma, "gamma", 4));
+  BL_TRY(check_ptr(dy, "dy", 16));
+  BL_TRY(check_ptr(xq, "xq", 16));
+  BL_TRY(check_ptr(scale, "scale", 4));
+  BL_TRY(check_ptr(dx, "dx", 16, true));
+  BL_TRY(check_ptr(dw, "dw", 16, true));
+  BL_TRY(check_ptr(workspace, "workspace", 256));
+  const size_t need = bitlinear_ste_workspace_bytes(M, N, K);
+  if (workspace_bytes < need)
+    return fail(BL_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, need);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaError_t e = bl::launch_ste_backward(packed, gamma, N, K, dy, xq, scale, M, dx, dx_dtype == BL_BF16, dw,
+                                          ws + kStatusBytes, reinterpret_cast<uint32_t*>(ws),
+                                          static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "straight-through backward launch");
+  return BL_OK;
+}
+
 int bitlinear_forward_lut(const uint8_t* packed, const float* gamma, int N, int K, const int8_t* xq,
                           const float* scale, const int32_t* rowsum, int M, void* y, int y_dtype, int32_t* acc_out,
                           void* stream) {

@@ -116,6 +116,15 @@ cudaError_t launch_lut_gemv(const uint8_t* packed, const float* gamma, int N, in
                             const float* scale, const int32_t* rowsum, void* y, int y_type, int32_t* acc_out,
                             cudaStream_t stream, bool pdl);
 
+// The straight-through backward: dx = gamma (dy . t) [M][K] (fp32 or bf16,
+// null to skip) and dW = dy^T . bf16(q / s) [N][K] fp32 (null to skip), from
+// the packed weights, bf16 dy [M][N] and the forward's codes and scales.
+// scratch: ste_scratch_bytes(M, N, K) bytes, 256-byte aligned.
+size_t ste_scratch_bytes(int M, int N, int K);
+cudaError_t launch_ste_backward(const uint8_t* packed, const float* gamma, int N, int K, const void* dy, const int8_t* xq,
+                                const float* scale, int M, void* dx, bool dx_bf16, float* dw, uint8_t* scratch,
+                                uint32_t* status, cudaStream_t stream);
+
 // Self-test of the bounded device wait.
 cudaError_t launch_wait_timeout_selftest(uint32_t* status, int limit_us, cudaStream_t stream);
 

@@ -15,7 +15,7 @@ import torch
 import oracle
 import synth
 import ternary_weight_a8_b200 as tb
-from parity import activations, assert_y_matches, bf16_bits, bf16_ordered, dev, f32_bits, weights
+from parity import activations, assert_y_matches, bf16_bits, bf16_dev, bf16_ordered, dev, f32_bits, weights
 
 pytestmark = pytest.mark.gpu
 
@@ -214,3 +214,84 @@ def test_lut_product_rejects_unsupported_shapes():
         with pytest.raises(tb.BitLinearError) as e:
             tb.forward_lut(pk, g, xq, s, r)
         assert e.value.code == tb.BL_ERR_UNSUPPORTED_SHAPE
+
+
+# ----------------------------------------------------------------------------
+# The straight-through backward.  The operands are exact on both sides (bf16
+# dy as given, t in {-1, 0, 1}, xhat = bf16(q / s) formed the same way), the
+# products of bf16 pairs are exact in fp32, so the only error is the fp32
+# accumulation over the R summed terms: |err| <= R * 2^-24 * sum|terms| for
+# any order of the sums (each partial sum rounded once).
+# ----------------------------------------------------------------------------
+
+def _ste_inputs(M, N, K, seed):
+    W = weights(N, K, seed=seed)
+    packed_ref, gamma_ref, T = oracle.pack_weights(W)
+    x, xf = activations(M, K, seed=seed + 1, dtype="bf16")
+    dy_bits, dyf = synth.activations_bf16(M, N, seed=seed + 2)
+    return packed_ref, gamma_ref, T, x, xf, bf16_dev(dy_bits), dyf
+
+
+def _assert_within_accumulation_bound(got, ref, absterms, R):
+    bound = max(R * 2.0 ** -24, 1e-6) * absterms + 1e-30
+    err = np.abs(got.astype(np.float64) - ref)
+    assert (err <= bound).all(), "max err/bound %.3g" % float((err / bound).max())
+
+
+@pytest.mark.parametrize("M,N,K", [(8, 64, 64), (64, 640, 1024), (256, 512, 2560), (136, 320, 192)])
+def test_ste_backward_parity(M, N, K):
+    packed_ref, gamma_ref, T, x, xf, dy, dyf = _ste_inputs(M, N, K, seed=M + N + K)
+    p, g = dev(packed_ref), dev(np.array([gamma_ref], np.float32))
+    xq, s, _ = tb.quant_act(x)
+    dx, dw = tb.ste_backward(p, g, K, dy, xq, s)
+    q_ref, s_ref, _ = oracle.quant_act(xf)
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    dx_ref = oracle.ste_grad_input(dyf, T, gamma_ref)
+    absx = float(gamma_ref) * (np.abs(dyf).astype(np.float64) @ np.abs(T).astype(np.float64))
+    _assert_within_accumulation_bound(dx.cpu().numpy(), dx_ref, absx, N)
+    xhat = oracle.ste_xhat(q_ref, s_ref)
+    dw_ref = oracle.ste_grad_weight(dyf, xhat)
+    absw = np.abs(dyf).astype(np.float64).T @ np.abs(xhat).astype(np.float64)
+    _assert_within_accumulation_bound(dw.cpu().numpy(), dw_ref, absw, M)
+
+
+def test_ste_backward_bf16_dx_and_skips():
+    M, N, K = 64, 256, 512
+    packed_ref, gamma_ref, T, x, xf, dy, dyf = _ste_inputs(M, N, K, seed=5)
+    p, g = dev(packed_ref), dev(np.array([gamma_ref], np.float32))
+    xq, s, _ = tb.quant_act(x)
+    dx32, _ = tb.ste_backward(p, g, K, dy, xq, s, dw=False)
+    dx16, none = tb.ste_backward(p, g, K, dy, xq, s, dx_dtype=torch.bfloat16, dw=False)
+    assert none is None
+    # bf16 dx is the kernel's fp32 dx rounded once
+    want = (f32_bits(dx32.cpu().numpy()) >> 16) + ((f32_bits(dx32.cpu().numpy()) >> 15) & 1)
+    d = np.abs(bf16_bits(dx16).astype(np.int64) - want.astype(np.int64))
+    assert d.max() <= 1
+    _, dw_only = tb.ste_backward(p, g, K, dy, xq, s, dx=False)
+    assert dw_only is not None and dw_only.shape == (N, K)
+
+
+def test_ste_gradient_matches_the_forward():
+    """<dx, xhat> = <dy, y_acc * gamma / s>: the backward of the forward's own bilinear form."""
+    M, N, K = 64, 768, 2560
+    packed_ref, gamma_ref, T, x, xf, dy, dyf = _ste_inputs(M, N, K, seed=9)
+    p, g = dev(packed_ref), dev(np.array([gamma_ref], np.float32))
+    xq, s, r = tb.quant_act(x)
+    y = tb.forward_quantized(p, g, xq, s, r, out_dtype=torch.float32)
+    dx, _ = tb.ste_backward(p, g, K, dy, xq, s, dw=False)
+    q_ref, s_ref, _ = oracle.quant_act(xf)
+    xhat = (q_ref.astype(np.float64) / s_ref[:, None].astype(np.float64))
+    lhs = float(np.sum(dx.cpu().numpy().astype(np.float64) * xhat))
+    rhs = float(np.sum(dyf.astype(np.float64) * y.cpu().numpy().astype(np.float64)))
+    assert abs(lhs - rhs) <= 1e-4 * float(np.sum(np.abs(dyf.astype(np.float64) * y.cpu().numpy().astype(np.float64))))
+
+
+def test_ste_rejects_unsupported_shapes():
+    p = torch.zeros((96, 16), dtype=torch.uint8, device="cuda")
+    g = torch.ones(1, dtype=torch.float32, device="cuda")
+    dy = torch.zeros((8, 96), dtype=torch.bfloat16, device="cuda")
+    xq = torch.zeros((8, 64), dtype=torch.int8, device="cuda")
+    s = torch.ones(8, dtype=torch.float32, device="cuda")
+    with pytest.raises(tb.BitLinearError) as e:
+        tb.ste_backward(p, g, 64, dy, xq, s)  # N = 96 is not a multiple of 64
+    assert e.value.code == tb.BL_ERR_UNSUPPORTED_SHAPE
