@@ -16,7 +16,8 @@
 //    ordered largest-K layer first; each block takes its first unit by index
 //    and the rest from a ticket counter in the workspace, so the blocks end
 //    within a fraction of a unit of one another.  The block that finishes
-//    last resets the counter for the next launch.
+//    last resets the counter for the next launch.  With no more units than
+//    blocks, each block takes its own unit and the counter is not touched.
 //  * One producer thread streams the block's units with TMA in stages of 64
 //    rows x 256 bytes (1024 inputs, two 128-byte halves), in the 128-byte
 //    swizzle so that the lanes' 16-byte reads are conflict-free, through a deep ring of
@@ -91,6 +92,7 @@ struct GvParams {
   int n_layers, M, total_units, nring, x_pitch;
   uint32_t* status;
   uint32_t* tickets;  // [0] next ticket, [1] blocks done
+  int one_unit;       // as many blocks as units: each block takes its own unit, no tickets
 };
 
 __device__ __forceinline__ void mma_u8s8_16x8x32(int (&d)[4], uint32_t a0, uint32_t a1,
@@ -376,12 +378,16 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           ++issued;
           if (++slot == nring) { slot = 0; phase ^= 1; }
         }
-        if (!waited) {
-          griddep_wait();  // the ticket counter is reset by the preceding launch
-          waited = true;
-        }
         st0 = 0;
-        unit = static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(P.tickets, 1u));
+        if (P.one_unit) {
+          unit = P.total_units;
+        } else {
+          if (!waited) {
+            griddep_wait();  // the ticket counter is reset by the preceding launch
+            waited = true;
+          }
+          unit = static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(P.tickets, 1u));
+        }
       }
       if (ok) {
         // End marker: one more phase on the next slot, with no data.
@@ -535,6 +541,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
   }
 
   // The block that finishes last resets the ticket counter for the next launch.
+  if (P.one_unit) return;
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
@@ -676,6 +683,7 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   const int smem = gemv_smem_bytes(M, k_max, nring, stream_x);
   const int slots = kGvBlocksPerSM * num_sms();
   const int grid = units < slots ? units : slots;
+  P.one_unit = units <= slots ? 1 : 0;
   return y_type == kOutBF16 ? launch_group_y<__nv_bfloat16>(x_type, P, grid, smem, stream, pdl)
                             : launch_group_y<float>(x_type, P, grid, smem, stream, pdl);
 }
