@@ -422,6 +422,16 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
     }
     int staged = -1;  // layer whose activations are in shared memory
     int slot = 0, phase = 0;
+    if constexpr (!kStream) {
+      // The first unit is the block's index, so its activations can be
+      // quantised while its first weight stage is still on the way.
+      if (static_cast<int>(blockIdx.x) < P.total_units) {
+        int l = 0;
+        while (l + 1 < P.n_layers && static_cast<int>(blockIdx.x) >= P.layer[l + 1].unit0) ++l;
+        stage_activations<TT, TX>(P.layer[l], M, xs, P.x_pitch, s_tok, rs_tok, scratch);
+        staged = l;
+      }
+    }
     while (true) {
       const bool got0 = mbar_wait(bar0 + 8 * slot, phase, ctl);
       if (!__all_sync(0xffffffffu, got0)) break;
