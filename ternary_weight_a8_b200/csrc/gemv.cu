@@ -449,6 +449,25 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         }
       }
 
+      // The epilogue's scalars, loaded now so their latency hides behind the products.
+      const float gamma = __ldg(L.gamma);
+      int rsum_m[TG][2];
+      float s_m[TG][2];
+#pragma unroll
+      for (int tg = 0; tg < TG; ++tg)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int m = tg * 8 + 2 * t + e;
+          rsum_m[tg][e] = 0;
+          s_m[tg][e] = 1.0f;
+          if constexpr (kStream) {
+            if (m < M) {
+              rsum_m[tg][e] = __ldcg(L.rowsum + m);
+              s_m[tg][e] = __ldcg(L.scale + m);
+            }
+          }
+        }
+
       int d[TG][4][4];
 #pragma unroll
       for (int tg = 0; tg < TG; ++tg)
@@ -528,7 +547,6 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       if (!ok) break;
 
       // Finish the unit: y = (sum c*q - sum q) * (gamma / s).
-      const float gamma = __ldg(L.gamma);
       const int n_base = (unit - L.unit0) * kGvRows;
       TY* y = static_cast<TY*>(L.y);
 #pragma unroll
@@ -538,8 +556,8 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           const int n = n_base + r_lo + ((c & 2) ? 8 : 0);
           const int m = tg * 8 + 2 * t + (c & 1);
           if (n < L.N && m < M) {
-            const int rsum = kStream ? __ldcg(L.rowsum + m) : rs_tok[m];
-            const float sm = kStream ? __ldcg(L.scale + m) : s_tok[m];
+            const int rsum = kStream ? rsum_m[tg][c & 1] : rs_tok[m];
+            const float sm = kStream ? s_m[tg][c & 1] : s_tok[m];
             const int a = d[tg][0][c] + (d[tg][1][c] >> 2) + (d[tg][2][c] >> 4) + (d[tg][3][c] >> 6) - rsum;
             const float v = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, sm));
             const size_t o = static_cast<size_t>(m) * L.N + n;
