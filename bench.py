@@ -157,7 +157,12 @@ class ClockSampler:
 # distributed plumbing (replicas: no data-path collective)
 # ----------------------------------------------------------------------------
 
+_BACKEND = None  # process-group backend of this run (None: one rank)
+
+
 def dist_init():
+    """One process per GPU (NCCL); without a GPU (host-side tests) the ranks use gloo."""
+    global _BACKEND
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -167,9 +172,14 @@ def dist_init():
         import torch
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+            _BACKEND = "nccl"
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+            _BACKEND = "gloo"
     return world, rank, local
 
 
@@ -186,7 +196,7 @@ def max_over_ranks(v: float, world: int) -> float:
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device="cpu" if _BACKEND == "gloo" else "cuda")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
