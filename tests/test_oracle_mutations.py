@@ -37,7 +37,7 @@ MUTANTS = {
                              "float r = (float)(1.0 / (sqrt(ms) + (double)eps));"),
     "rms_gain_ignored": ("if (g) v = v * g[k];", ";"),
     "rms_sum_of_abs": ("ss += v * v;", "ss += fabs(v);"),
-    "rms_no_bf16_rounding": ("if (out_bf16) {", "if (0) {"),
+    "rms_no_bf16_rounding": ("if (g) v = v * g[k];\n      if (out_bf16) {", "if (g) v = v * g[k];\n      if (0) {"),
     "glu_relu_not_squared": ("h = (g * g) * up[i];", "h = g * up[i];"),
     "glu_relu_not_clamped": ("float g = gate[i] > 0.0f ? gate[i] : 0.0f;", "float g = gate[i];"),
     "glu_silu_wrong_sign": ("h = (float)(z / (1.0 + exp(-z)) * (double)up[i]);",
