@@ -65,6 +65,35 @@ def test_host_side_validation(L):
     assert L.bitlinear_quant_act(vp(16), 0, 0, 256, vp(16), vp(16), None, None) == tb.BL_OK
 
 
+def test_host_side_validation_of_the_next_rows(L):
+    vp, f = ctypes.c_void_p, ctypes.c_float
+    # fused norm: K, dtype and eps are checked before any pointer
+    assert L.bitlinear_rmsnorm_quant(None, 0, 1, 48, None, f(1e-6), None, None, None, None, None) == tb.BL_ERR_UNSUPPORTED_SHAPE
+    assert L.bitlinear_rmsnorm_quant(None, 5, 1, 64, None, f(1e-6), None, None, None, None, None) == tb.BL_ERR_INVALID_ARG
+    for eps in (-1.0, float("inf"), float("nan")):
+        assert L.bitlinear_rmsnorm_quant(None, 0, 1, 64, None, f(eps), None, None, None, None, None) == tb.BL_ERR_INVALID_ARG
+    assert "eps" in tb.last_error()
+    assert L.bitlinear_rmsnorm_quant(vp(16), 0, 0, 64, None, f(1e-6), None, vp(16), vp(16), None, None) == tb.BL_OK
+    # gated activation: the width is the down BitLinear's K; unknown activations are refused
+    assert L.bitlinear_glu_quant(None, None, 0, 1, 96, 0, None, None, None, None, None) == tb.BL_ERR_UNSUPPORTED_SHAPE
+    assert L.bitlinear_glu_quant(None, None, 0, 1, 128, 2, None, None, None, None, None) == tb.BL_ERR_INVALID_ARG
+    # lookup-table product: one token, K within the tables' shared memory
+    assert L.bitlinear_forward_lut(None, None, 8, 256, None, None, None, 2, None, 0, None, None) == tb.BL_ERR_UNSUPPORTED_SHAPE
+    assert L.bitlinear_forward_lut(None, None, 8, 24576 + 64, None, None, None, 1, None, 0, None, None) == \
+        tb.BL_ERR_UNSUPPORTED_SHAPE
+    # straight-through backward: N % 64, M % 8, dtype; nothing to do is a no-op
+    assert L.bitlinear_ste_backward(None, None, 96, 64, None, None, None, 8, None, 0, None, None, 0, None) == \
+        tb.BL_ERR_UNSUPPORTED_SHAPE
+    assert L.bitlinear_ste_backward(None, None, 64, 64, None, None, None, 12, None, 0, None, None, 0, None) == \
+        tb.BL_ERR_UNSUPPORTED_SHAPE
+    assert L.bitlinear_ste_backward(None, None, 64, 64, None, None, None, 8, None, 9, None, None, 0, None) == \
+        tb.BL_ERR_INVALID_ARG
+    assert L.bitlinear_ste_backward(None, None, 64, 64, None, None, None, 8, None, 0, None, None, 0, None) == tb.BL_OK
+    # its workspace: status block + t^T [K][N] + dy^T [N][M] + xhat^T [K][M] in bf16, each 256-rounded
+    assert tb.ste_workspace_bytes(2048, 6912, 2560) == 256 + 2560 * 6912 * 2 + 6912 * 2048 * 2 + 2560 * 2048 * 2
+    assert tb.ste_workspace_bytes(8, 64, 64) == 256 + 64 * 64 * 2 + 64 * 8 * 2 + 64 * 8 * 2
+
+
 def test_workspace_layout(L):
     # status block (256) + q (M rows of K rounded up to 128, 256-rounded) + scale and
     # rowsum (4*M each, 256-rounded)
