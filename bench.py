@@ -11,8 +11,8 @@ at load time (absmean + ternarise + pack), as a deployed checkpoint is; that
 offline path is timed separately under ``pack``.
 
 Also reported in the same line: the 2B prefill GEMM (2048 tokens) in int8
-TOPS against the tensor-core roofline, and the 70B-class decode layer chain
-at 1 and 8 tokens in GB/s.  Inputs are seeded and synthetic with the pages'
+TOPS against the tensor-core roofline, the 70B-class decode layer chain
+at 1 and 8 tokens and the 3B-class decode layers at 1 to 16 tokens in GB/s.  Inputs are seeded and synthetic with the pages'
 shapes and distributions; weights rotate over enough copies that every step
 reads them from HBM (more than 4x the L2 size).
 
@@ -52,7 +52,7 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-extras", action="store_true", help="skip prefill / 70B chain / pack lines")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--only", choices=["prefill", "chain70b", "next"], default=None,
+    p.add_argument("--only", choices=["prefill", "chain70b", "decode3b", "next"], default=None,
                    help="run one secondary workload alone and print its own line (a small case for profiling)")
     return p.parse_args()
 
@@ -380,6 +380,7 @@ def run_ours(args, world, rank, local):
     if not args.no_extras:
         out["prefill"] = run_prefill(args, world, peaks, L2)
         out["chain_70b"] = run_chain(args, world, peaks, L2)
+        out["decode_3b"] = run_decode_3b(args, world, peaks, L2)
         out["pack"] = run_pack(world)
         out["next"] = run_next(args, world, peaks, L2)
 
@@ -446,6 +447,41 @@ def run_prefill(args, world, peaks, L2):
                          "traffic": profiled_traffic("prefill_2b", "gemm"),
                          "algorithmic_bytes_per_launch": M * K + N * K // 4 + M * N * 2 + 8 * M},
             "pct_int8_nominal_4500": round(100 * tops / world / 4500.0, 2), "device_status": status}
+
+
+DECODE_3B = [(3200, 8640), (8640, 3200)]  # (K in, N out)
+DECODE_3B_TOKENS = (1, 2, 4, 8, 16)
+
+
+def run_decode_3b(args, world, peaks, L2):
+    """The 3B-class decode sweep: one BitLinear per step through the public
+    single-layer call (quantisation and product), 1 to 16 tokens."""
+    import torch
+
+    import ternary_weight_a8_b200 as tb
+
+    res = {"workload": "decode_3b: BitLinear K=3200->N=8640 and K=8640->N=3200 alone, bf16 in/out, "
+                       "1/2/4/8/16 tokens, one forward call per step"}
+    for li, (K, N) in enumerate(DECODE_3B):
+        sets, set_bytes = make_layer_sets([(K, N)], seed=500 + li, min_bytes=4 * L2)
+        for M in DECODE_3B_TOKENS:
+            xs, ys = make_inputs([(K, N)], M, seed=500 + li)
+            x, y = xs[0], ys[0]
+            ws = tb.new_workspace(tb.workspace_bytes(M, N, K))
+
+            def step(i):
+                packed, gamma = sets[i % len(sets)][0]
+                tb.forward(packed, gamma, x, y=y, workspace=ws)
+
+            steps = 4000
+            secs, _ = timed_graph_run(step, steps, 200, world, chunk=500)
+            gbs = set_bytes * steps * world / secs / 1e9
+            res["k%d_n%d_m%d" % (K, N, M)] = {
+                "GB/s": round(gbs, 1), "pct_hbm_measured": round(100 * gbs / world / peaks["hbm"], 2),
+                "us_per_call": round(secs / steps * 1e6, 3), "tokens_per_s": round(M * steps * world / secs, 1),
+                "device_status": tb.device_status(ws)}
+        del sets
+    return res
 
 
 def run_chain(args, world, peaks, L2):
@@ -682,7 +718,7 @@ def main():
         import torch
 
         torch.cuda.set_device(local)
-        fn = {"prefill": run_prefill, "chain70b": run_chain, "next": run_next}[args.only]
+        fn = {"prefill": run_prefill, "chain70b": run_chain, "decode3b": run_decode_3b, "next": run_next}[args.only]
         res = fn(args, world, load_peaks(), l2_bytes())
         if rank == 0:
             print(json.dumps(res), flush=True)

@@ -8,7 +8,8 @@
 // 8-bit activations.  "BitNet b1.58 and the 1-Bit AI Architecture
 // Revolution", section "The Energy Revolution": the product is integer
 // additions; here they run on the tensor cores' int8 path (mma.sync
-// m16n8k32, u8 x s8 -> s32).
+// m16n8k32, u8 x s8 -> s32) for two or more tokens, and as byte dot products
+// (dp4a) for one token.
 //
 // Decode streams every weight byte once, so the kernel is built around one
 // uninterrupted weight stream per SM:
@@ -35,7 +36,7 @@
 //    (per-token absmax over all of K, s = 127 / max(amax, 1e-5),
 //    q = rint(x * s)) and staged whole, the 16-byte chunks of every 128-byte
 //    block rotated by twice the block index; that saves a launch.
-//  * Each lane takes 16-byte chunks 2t and 2t+1 of rows g and g+8 of its
+//  * Two or more tokens: each lane takes 16-byte chunks 2t and 2t+1 of rows g and g+8 of its
 //    warp's 16 rows into registers; a warp releases a stage once it has
 //    read everything it needs from it (at once when the activations are
 //    staged whole, after the stage's products when they stream with it).
@@ -45,6 +46,13 @@
 //    exact because each set is a multiple of 4^j.  The k order inside an mma
 //    is free as long as both operands agree, so lane (g, t) feeds its own
 //    words to the A fragment and the matching activation bytes to B.
+//  * One token: the mma's eight token columns would be seven-eighths idle, and
+//    one warp per SM sub-partition issues mma.sync too slowly for a short,
+//    latency-bound step.  Lane (rs, ch) instead takes 16-byte chunk ch of rows
+//    rs, rs+4, rs+8, rs+12 of its warp's 16 and the matching 64 codes: the
+//    same AND per four weights, then one dp4a (unsigned codes x signed codes)
+//    per four weights into the four accumulator sets; the eight lanes of a
+//    row group finish with a three-step butterfly.
 //  * Stored codes are c = t + 1: acc = sum c*q - sum q, and
 //    y = acc * (gamma / s) is stored straight from registers.
 //  * The kernel is specialised on the number of token slots (1, 2, 4, 8 or
@@ -67,6 +75,7 @@ constexpr int kGvConsumers = 32 * kGvWarps;
 constexpr int kGvBlocksPerSM = 3;
 constexpr int kGvSmemPerBlock = 75 * 1024;
 constexpr int kGvMaxRing = 16;
+constexpr int kGvMaxSplit = 4;        // CTAs of a cluster sharing one unit
 constexpr int kGvTagEnd = -1;
 constexpr int kGvFuseChunks = 2;      // 16-input chunks a consumer thread quantises itself
 constexpr int kGvFuseElems = 4096;    // M*K up to which the blocks quantise activations themselves
@@ -93,7 +102,18 @@ struct GvParams {
   uint32_t* status;
   uint32_t* tickets;  // [0] next ticket, [1] blocks done
   int one_unit;       // as many blocks as units: each block takes its own unit, no tickets
+  int ksplit;         // CTAs of a cluster that share one unit, each over its own range of stages
 };
+
+// Stages [sb, se) of a unit with nst stages taken by cluster rank `rank` of `ks`.
+__host__ __device__ inline void stage_range(int nst, int ks, int rank, int& sb, int& se) {
+  sb = rank * nst / ks;
+  se = (rank + 1) * nst / ks;
+}
+
+// Shared-memory bytes of one CTA's partial sums in a K-split launch: one
+// 16-byte vector per consumer thread and mma token group.
+__host__ __device__ constexpr int gv_part_bytes(int tt) { return ((tt + 7) / 8) * kGvConsumers * 16; }
 
 __device__ __forceinline__ void mma_u8s8_16x8x32(int (&d)[4], uint32_t a0, uint32_t a1,
                                                  uint32_t a2, uint32_t a3, uint32_t b0,
@@ -111,6 +131,19 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "r"(addr));
   return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// Sum of the four products of unsigned bytes of a with signed bytes of b, plus c.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
@@ -280,10 +313,11 @@ __device__ __forceinline__ void stage_activations(const GvLayer& L, int M, uint3
   consumer_sync();
 }
 
-template <int TT, typename TY, typename TX>
+template <int TT, typename TY, typename TX, bool kSplit>
 __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(const __grid_constant__ GvParams P) {
   constexpr int TG = (TT + 7) / 8;           // mma token groups of 8
   constexpr bool kStream = sizeof(TX) == 1;  // int8 codes stream with the weights
+  constexpr bool kAlu = TT == 1;             // one token: dp4a dot products instead of the mma path
   constexpr int kXHalf = x_half_bytes(TT);   // one half-stage activation tile
   constexpr int kSlot = kGvStageBytes + (kStream ? 2 * kXHalf : 0);
   extern __shared__ uint8_t smem_raw[];
@@ -292,14 +326,20 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
   const uint32_t sb = smem_u32(smem);
   const uint32_t ring = sb;
   const uint32_t xs = sb + nring * kSlot;  // whole-K activations (in-kernel quantisation only)
-  uint8_t* misc = smem + nring * kSlot + (kStream ? 0 : ((M * P.x_pitch + 127) / 128) * 128);
+  const int ks = kSplit ? P.ksplit : 1;    // CTAs sharing one unit (a cluster of ks)
+  const int x_bytes = kStream ? 0 : ((M * P.x_pitch + 127) / 128) * 128;
+  const uint32_t part = xs + x_bytes;      // this CTA's partial sums (K-split only)
+  uint8_t* misc = smem + nring * kSlot + x_bytes + (ks > 1 ? gv_part_bytes(TT) : 0);
   float* s_tok = reinterpret_cast<float*>(misc);          // [16]
   int* rs_tok = reinterpret_cast<int*>(misc + 64);         // [16]
   float* scratch = reinterpret_cast<float*>(misc + 128);   // [kGvWarps]
   int* tags = reinterpret_cast<int*>(misc + 160);          // [kGvMaxRing]: unit of each stage
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 224);
   volatile int* never = abort_flag + 1;
-  const uint32_t bar0 = smem_u32(misc + 256);              // full[nring], empty[nring]
+  const uint32_t bar0 = smem_u32(misc + 256);              // full[nring], empty[nring], then red
+  const uint32_t red_bar = bar0 + 16 * nring;              // K-split: the peers' partial sums are in place
+  const int rank = ks > 1 ? static_cast<int>(blockIdx.x) % ks : 0;
+  const int unit_first = static_cast<int>(blockIdx.x) / ks;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -307,11 +347,13 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       mbar_init(bar0 + 8 * i, 1);
       mbar_init(bar0 + 8 * (nring + i), kGvWarps);
     }
+    if (ks > 1) mbar_init(red_bar, (ks - 1) * kGvWarps);
     *abort_flag = 0;
     *never = 0;
     fence_barrier_init();
   }
   __syncthreads();
+  if (ks > 1) cluster_sync_all();  // the peers' barriers are initialised before any remote arrive
   griddep_launch_dependents();
   const WaitCtl ctl{P.status, abort_flag, kWaitLimitNs};
 
@@ -321,7 +363,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       int slot = 0, phase = 0, issued = 0;
       bool waited = false;  // grid dependency
       bool ok = true;
-      int unit = blockIdx.x;
+      int unit = unit_first;
       int st0 = 0;  // first stage of the current unit still to issue
       if constexpr (kStream) {
         // Before the grid dependency: the weights of the first unit's first
@@ -332,26 +374,29 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           while (l + 1 < P.n_layers && unit >= P.layer[l + 1].unit0) ++l;
           const GvLayer& L = P.layer[l];
           const int rb = unit - L.unit0;
-          const int nst = (L.K + kGvStageK - 1) / kGvStageK;
-          const int pre = nst < nring ? nst : nring;
-          for (int st = 0; st < pre; ++st) {  // fresh slots 0 .. pre-1
-            tags[st] = unit;
-            const uint32_t full = bar0 + 8 * st, dst = ring + st * kSlot;
+          int s0, s1;
+          stage_range((L.K + kGvStageK - 1) / kGvStageK, ks, rank, s0, s1);
+          const int pre = s1 - s0 < nring ? s1 - s0 : nring;
+          for (int j = 0; j < pre; ++j) {  // fresh slots 0 .. pre-1
+            const int st = s0 + j;
+            tags[j] = unit;
+            const uint32_t full = bar0 + 8 * j, dst = ring + j * kSlot;
             mbar_arrive_expect_tx(full, kGvStageBytes + 2 * TT * 4 * 128);
             tma_load_2d(dst, &L.tmap, st * 256, rb * kGvRows, full);
             tma_load_2d(dst + kGvStageBytes / 2, &L.tmap, st * 256 + 128, rb * kGvRows, full);
           }
           griddep_wait();  // the codes come from the preceding kernel
           waited = true;
-          for (int st = 0; st < pre; ++st) {
-            const uint32_t full = bar0 + 8 * st, dst = ring + st * kSlot;
+          for (int j = 0; j < pre; ++j) {
+            const int st = s0 + j;
+            const uint32_t full = bar0 + 8 * j, dst = ring + j * kSlot;
             tma_load_3d(dst + kGvStageBytes, &L.xmap, 0, 8 * st, 0, full);
             tma_load_3d(dst + kGvStageBytes + kXHalf, &L.xmap, 0, 8 * st + 4, 0, full);
           }
           issued = pre;
           slot = pre % nring;
           phase = pre == nring ? 1 : 0;
-          st0 = pre;
+          st0 = s0 + pre;
         }
       }
       while (ok && unit < P.total_units) {
@@ -359,8 +404,9 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         while (l + 1 < P.n_layers && unit >= P.layer[l + 1].unit0) ++l;
         const GvLayer& L = P.layer[l];
         const int rb = unit - L.unit0;
-        const int nst = (L.K + kGvStageK - 1) / kGvStageK;
-        for (int st = st0; st < nst; ++st) {
+        int s0, s1;
+        stage_range((L.K + kGvStageK - 1) / kGvStageK, ks, rank, s0, s1);
+        for (int st = st0 > s0 ? st0 : s0; st < s1; ++st) {
           if (!mbar_wait(bar0 + 8 * (nring + slot), phase ^ 1, ctl)) { ok = false; break; }
           tags[slot] = unit;
           const uint32_t full = bar0 + 8 * slot, dst = ring + slot * kSlot;
@@ -425,9 +471,9 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
     if constexpr (!kStream) {
       // The first unit is the block's index, so its activations can be
       // quantised while its first weight stage is still on the way.
-      if (static_cast<int>(blockIdx.x) < P.total_units) {
+      if (unit_first < P.total_units) {
         int l = 0;
-        while (l + 1 < P.n_layers && static_cast<int>(blockIdx.x) >= P.layer[l + 1].unit0) ++l;
+        while (l + 1 < P.n_layers && unit_first >= P.layer[l + 1].unit0) ++l;
         stage_activations<TT, TX>(P.layer[l], M, xs, P.x_pitch, s_tok, rs_tok, scratch);
         staged = l;
       }
@@ -440,7 +486,8 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       int l = 0;
       while (l + 1 < P.n_layers && unit >= P.layer[l + 1].unit0) ++l;
       const GvLayer& L = P.layer[l];
-      const int nst = (L.K + kGvStageK - 1) / kGvStageK;
+      int s0, s1;  // this CTA's stages of the unit
+      stage_range((L.K + kGvStageK - 1) / kGvStageK, ks, rank, s0, s1);
       if constexpr (!kStream) {
         if (l != staged) {
           consumer_sync();  // every warp is done with the previous layer's activations
@@ -460,7 +507,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           const int m = tg * 8 + 2 * t + e;
           rsum_m[tg][e] = 0;
           s_m[tg][e] = 1.0f;
-          if constexpr (kStream) {
+          if constexpr (kStream && !kAlu) {
             if (m < M) {
               rsum_m[tg][e] = __ldcg(L.rowsum + m);
               s_m[tg][e] = __ldcg(L.scale + m);
@@ -468,87 +515,205 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           }
         }
 
-      int d[TG][4][4];
+      int rsum1 = 0;  // the one-token path's epilogue scalars (every lane)
+      float s1tok = 1.0f;
+      if constexpr (kAlu && kStream) {
+        rsum1 = __ldcg(L.rowsum);
+        s1tok = __ldcg(L.scale);
+      }
+
+      int d[TG][4][4];      // mma path: accumulator fragments
+      int dr[kAlu ? 4 : 1][4];   // one-token path: rows warp*16 + (lane >> 3) + 4*it, one set per code position j
 #pragma unroll
       for (int tg = 0; tg < TG; ++tg)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
 #pragma unroll
           for (int c = 0; c < 4; ++c) d[tg][j][c] = 0;
+#pragma unroll
+      for (int r = 0; r < (kAlu ? 4 : 1); ++r)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dr[r][j] = 0;
       bool ok = true;
-      for (int i = 0; i < nst; ++i) {
-        if (i > 0) {
+      for (int i = s0; i < s1; ++i) {
+        if (i > s0) {
           const bool got = mbar_wait(bar0 + 8 * slot, phase, ctl);
           if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         }
         const uint32_t wt = ring + slot * kSlot;
-        uint4 w[2][4];  // [half][lo0, lo1, hi0, hi1]
+        if constexpr (kAlu) {
+          // Lane (rs, ch) = (lane >> 3, lane & 7) takes 16-byte chunk ch of rows
+          // warp*16 + rs + 4*it of each half (inputs 64ch .. 64ch+63 of the half) and the
+          // matching 64 codes: one AND and one dp4a per four weights, no idle mma
+          // columns.  Each 8-lane phase reads one 128-byte swizzled row.
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const uint32_t base = wt + hf * (kGvStageBytes / 2);
-          w[hf][0] = lds128(base + w_lo0);
-          w[hf][1] = lds128(base + w_lo1);
-          w[hf][2] = lds128(base + w_hi0);
-          w[hf][3] = lds128(base + w_hi1);
-        }
-        if constexpr (!kStream) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // the slot held only weights, now in registers
-        }
-        const uint32_t xt = wt + kGvStageBytes;
-
+          for (int hf = 0; hf < 2; ++hf) {
+            const int ch = lane & 7, rs = lane >> 3;
+            const int k0 = i * kGvStageK + hf * (kGvStageK / 2) + 64 * ch;
+            if (k0 < L.K) {  // inputs past K have zero weights (K is a multiple of 64)
+              uint4 xc[4];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int qblk = i * 8 + hf * 4 + t;  // this lane's 128-input block (whole-K staging)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint4 wl = w[hf][h], wh = w[hf][2 + h];
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-              const int c0 = 4 * h + 2 * p;  // activation chunks c0, c0+1 of the lane's block
-              uint4 xa[TG], xb[TG];
-#pragma unroll
-              for (int tg = 0; tg < TG; ++tg) {
-                const int m = tg * 8 + g;
-                if (m < M) {
-                  if constexpr (kStream) {
-                    const uint32_t row = xt + hf * kXHalf + x_row[tg];
-                    xa[tg] = lds128(row + ((c0 ^ x_sw[tg]) << 4));
-                    xb[tg] = lds128(row + (((c0 + 1) ^ x_sw[tg]) << 4));
-                  } else {
-                    const uint32_t row = xs + m * P.x_pitch + qblk * 128;
-                    xa[tg] = lds128(row + (((c0 + 2 * t) & 7) << 4));
-                    xb[tg] = lds128(row + (((c0 + 1 + 2 * t) & 7) << 4));
-                  }
+              for (int u = 0; u < 4; ++u) {
+                if constexpr (kStream) {
+                  const int q = ch >> 1, ci = 4 * (ch & 1) + u;  // 128-input block; token 0 owns rows 0..3
+                  xc[u] = lds128(wt + kGvStageBytes + hf * kXHalf + q * 128 + ((ci ^ q) << 4));
                 } else {
-                  xa[tg] = make_uint4(0, 0, 0, 0);
-                  xb[tg] = make_uint4(0, 0, 0, 0);
+                  xc[u] = lds128(xs + x_chunk_off((k0 >> 4) + u));
                 }
               }
-              const uint32_t lo0 = u4_get(wl, 2 * p), lo1 = u4_get(wl, 2 * p + 1);
-              const uint32_t hi0 = u4_get(wh, 2 * p), hi1 = u4_get(wh, 2 * p + 1);
+              const uint32_t base = wt + hf * (kGvStageBytes / 2);
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const uint32_t mask = 0x03030303u << (2 * j);
-                const uint32_t a0 = lo0 & mask, a1 = hi0 & mask, a2 = lo1 & mask, a3 = hi1 & mask;
+              for (int it = 0; it < 4; ++it) {
+                const int row = warp * 16 + rs + 4 * it;
+                const uint4 wv = lds128(base + row * 128 + ((ch ^ (row & 7)) << 4));
 #pragma unroll
-                for (int tg = 0; tg < TG; ++tg)
-                  mma_u8s8_16x8x32(d[tg][j], a0, a1, a2, a3, u4_get(xa[tg], j), u4_get(xb[tg], j));
+                for (int v = 0; v < 4; ++v)
+#pragma unroll
+                  for (int j = 0; j < 4; ++j)
+                    dr[it][j] = dp4a_us(u4_get(wv, v) & (0x03030303u << (2 * j)), u4_get(xc[v], j), dr[it][j]);
               }
             }
           }
-        }
-        if constexpr (kStream) {
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // done with the slot's activations too
+          if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // done with the slot
+        } else {
+          uint4 w[2][4];  // [half][lo0, lo1, hi0, hi1]
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const uint32_t base = wt + hf * (kGvStageBytes / 2);
+            w[hf][0] = lds128(base + w_lo0);
+            w[hf][1] = lds128(base + w_lo1);
+            w[hf][2] = lds128(base + w_hi0);
+            w[hf][3] = lds128(base + w_hi1);
+          }
+          if constexpr (!kStream) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // the slot held only weights, now in registers
+          }
+          const uint32_t xt = wt + kGvStageBytes;
+
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int qblk = i * 8 + hf * 4 + t;  // this lane's 128-input block (whole-K staging)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint4 wl = w[hf][h], wh = w[hf][2 + h];
+#pragma unroll
+              for (int p = 0; p < 2; ++p) {
+                const int c0 = 4 * h + 2 * p;  // activation chunks c0, c0+1 of the lane's block
+                uint4 xa[TG], xb[TG];
+#pragma unroll
+                for (int tg = 0; tg < TG; ++tg) {
+                  const int m = tg * 8 + g;
+                  if (m < M) {
+                    if constexpr (kStream) {
+                      const uint32_t row = xt + hf * kXHalf + x_row[tg];
+                      xa[tg] = lds128(row + ((c0 ^ x_sw[tg]) << 4));
+                      xb[tg] = lds128(row + (((c0 + 1) ^ x_sw[tg]) << 4));
+                    } else {
+                      const uint32_t row = xs + m * P.x_pitch + qblk * 128;
+                      xa[tg] = lds128(row + (((c0 + 2 * t) & 7) << 4));
+                      xb[tg] = lds128(row + (((c0 + 1 + 2 * t) & 7) << 4));
+                    }
+                  } else {
+                    xa[tg] = make_uint4(0, 0, 0, 0);
+                    xb[tg] = make_uint4(0, 0, 0, 0);
+                  }
+                }
+                const uint32_t lo0 = u4_get(wl, 2 * p), lo1 = u4_get(wl, 2 * p + 1);
+                const uint32_t hi0 = u4_get(wh, 2 * p), hi1 = u4_get(wh, 2 * p + 1);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const uint32_t mask = 0x03030303u << (2 * j);
+                  const uint32_t a0 = lo0 & mask, a1 = hi0 & mask, a2 = lo1 & mask, a3 = hi1 & mask;
+#pragma unroll
+                  for (int tg = 0; tg < TG; ++tg)
+                    mma_u8s8_16x8x32(d[tg][j], a0, a1, a2, a3, u4_get(xa[tg], j), u4_get(xb[tg], j));
+                }
+              }
+            }
+          }
+          if constexpr (kStream) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // done with the slot's activations too
+          }
         }
         if (++slot == nring) { slot = 0; phase ^= 1; }
       }
       if (!ok) break;
 
+      // This CTA's sums per lane: the four code-position sets shifted back (exact,
+      // each set being a multiple of 4^j).
+      int pc[TG][4];
+      if constexpr (kAlu) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) pc[0][r] = dr[r][0] + (dr[r][1] >> 2) + (dr[r][2] >> 4) + (dr[r][3] >> 6);
+      } else if constexpr (kSplit) {  // (the mma epilogue below combines them itself otherwise)
+#pragma unroll
+        for (int tg = 0; tg < TG; ++tg)
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            pc[tg][c] = d[tg][0][c] + (d[tg][1][c] >> 2) + (d[tg][2][c] >> 4) + (d[tg][3][c] >> 6);
+      }
+      if (ks > 1) {
+        // K-split: each CTA of the cluster holds the same lanes' sums over its own
+        // stages; rank 0 adds the others' (read from their shared memory) and
+        // finishes the unit.
+        const uint32_t mine = part + (warp * 32 + lane) * 16;
+        if (rank != 0) {
+#pragma unroll
+          for (int tg = 0; tg < TG; ++tg)
+            sts128(mine + tg * kGvConsumers * 16, make_uint4(pc[tg][0], pc[tg][1], pc[tg][2], pc[tg][3]));
+          __syncwarp();
+          if (lane == 0) mbar_arrive_release_cluster(mapa_shared(red_bar, 0));
+          continue;
+        }
+        const bool got = mbar_wait(red_bar, 0, ctl);
+        if (!__all_sync(0xffffffffu, got)) break;
+        fence_acq_rel_cluster();
+        for (int r = 1; r < ks; ++r)
+#pragma unroll
+          for (int tg = 0; tg < TG; ++tg) {
+            const uint4 v = ld_shared_cluster_v4(mapa_shared(mine + tg * kGvConsumers * 16, r));
+            pc[tg][0] += static_cast<int>(v.x);
+            pc[tg][1] += static_cast<int>(v.y);
+            pc[tg][2] += static_cast<int>(v.z);
+            pc[tg][3] += static_cast<int>(v.w);
+          }
+      }
+
       // Finish the unit: y = (sum c*q - sum q) * (gamma / s).
       const int n_base = (unit - L.unit0) * kGvRows;
       TY* y = static_cast<TY*>(L.y);
+      if constexpr (kAlu) {
+        // A butterfly over the 8 lanes of a row group leaves row
+        // warp*16 + (lane >> 3) + 4*((lane >> 1) & 3) summed in lanes 2r and 2r + 1.
+        int v[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) v[r] = pc[0][r];
+#pragma unroll
+        for (int st = 0; st < 2; ++st) {
+          const int off = 4 >> st, half = 2 >> st;
+          const bool upper = (lane & off) != 0;
+#pragma unroll
+          for (int r = 0; r < half; ++r) {
+            const int send = upper ? v[r] : v[r + half];
+            const int keep = upper ? v[r + half] : v[r];
+            v[r] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+          }
+        }
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+        const int n = n_base + warp * 16 + (lane >> 3) + 4 * ((lane >> 1) & 3);
+        if ((lane & 1) == 0 && n < L.N) {
+          const int rsum = kStream ? rsum1 : rs_tok[0];
+          const float sm = kStream ? s1tok : s_tok[0];
+          const int a = v[0] - rsum;
+          const float val = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, sm));
+          if constexpr (sizeof(TY) == 4) y[n] = val; else y[n] = __float2bfloat16_rn(val);
+          if (L.acc_out) L.acc_out[n] = a;
+        }
+        continue;
+      }
 #pragma unroll
       for (int tg = 0; tg < TG; ++tg)
 #pragma unroll
@@ -558,7 +723,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           if (n < L.N && m < M) {
             const int rsum = kStream ? rsum_m[tg][c & 1] : rs_tok[m];
             const float sm = kStream ? s_m[tg][c & 1] : s_tok[m];
-            const int a = d[tg][0][c] + (d[tg][1][c] >> 2) + (d[tg][2][c] >> 4) + (d[tg][3][c] >> 6) - rsum;
+            const int a = (kSplit ? pc[tg][c] : d[tg][0][c] + (d[tg][1][c] >> 2) + (d[tg][2][c] >> 4) + (d[tg][3][c] >> 6)) - rsum;
             const float v = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, sm));
             const size_t o = static_cast<size_t>(m) * L.N + n;
             if constexpr (sizeof(TY) == 4) y[o] = v; else y[o] = __float2bfloat16_rn(v);
@@ -568,6 +733,9 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
     }
   }
 
+  // No CTA of a K-split cluster leaves while a peer may still read its shared
+  // memory or arrive on its barrier.
+  if (ks > 1) cluster_sync_all();
   // The block that finishes last resets the ticket counter for the next launch.
   if (P.one_unit) return;
   __syncthreads();
@@ -588,11 +756,13 @@ static int token_slots(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M 
 int gemv_x_pitch(int K) { return ((K + 127) / 128) * 128 + 16; }
 
 // Shared memory of one block: the ring, then (in-kernel quantisation only) the
-// whole-K activations, then the small arrays and barriers.
-int gemv_smem_bytes(int M, int K_max, int nring, bool stream) {
+// whole-K activations, then (K-split only) the partial sums, then the small
+// arrays and barriers.
+int gemv_smem_bytes(int M, int K_max, int nring, bool stream, int ksplit = 1) {
   const int slot = kGvStageBytes + (stream ? 2 * x_half_bytes(token_slots(M)) : 0);
   const int staged = stream ? 0 : ((M * gemv_x_pitch(K_max) + 127) / 128) * 128;
-  return nring * slot + staged + 256 + 16 * nring + 1024;
+  const int part = ksplit > 1 ? gv_part_bytes(token_slots(M)) : 0;
+  return nring * slot + staged + part + 256 + 16 * nring + 16 + 1024;
 }
 
 bool gemv_fuses_quant(int M, int K, int x_bf16) {
@@ -607,14 +777,32 @@ bool gemv_fuses_quant(int M, int K, int x_bf16) {
 
 template <int TT, typename TY, typename TX>
 static cudaError_t launch_group_t(const GvParams& P, int grid, int smem, cudaStream_t stream, bool pdl) {
-  auto kernel = gemv_group_kernel<TT, TY, TX>;
-  static bool attr_set = false;  // per template instance
-  if (!attr_set) {
+  // Separate instances with and without the K-split, so that a launch that
+  // does not split runs none of its code.
+  static bool attr_set[2] = {false, false};  // per template instance
+  const int sp = P.ksplit > 1 ? 1 : 0;
+  auto kernel = sp ? gemv_group_kernel<TT, TY, TX, true> : gemv_group_kernel<TT, TY, TX, false>;
+  if (!attr_set[sp]) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemPerBlock);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[sp] = true;
   }
-  return launch(kernel, dim3(grid), dim3(kGvThreads), static_cast<size_t>(smem), stream, pdl, P);
+  if (!sp) return launch(kernel, dim3(grid), dim3(kGvThreads), static_cast<size_t>(smem), stream, pdl, P);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGvThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = P.ksplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kernel, P);
 }
 
 template <int TT, typename TY>
@@ -655,7 +843,7 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
     }
   GvParams P;
   memset(&P, 0, sizeof(P));
-  int units = 0, k_max = 64;
+  int units = 0, k_max = 64, nst_min = 1 << 30;
   for (int i = 0; i < n_layers; ++i) {
     const GemvLayerArgs& a = layers[order[i]];
     GvLayer& L = P.layer[i];
@@ -694,6 +882,8 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
     L.unit0 = units;
     units += (a.N + kGvRows - 1) / kGvRows;
     if (a.K > k_max) k_max = a.K;
+    const int nst = (a.K + kGvStageK - 1) / kGvStageK;
+    if (nst < nst_min) nst_min = nst;
   }
   P.n_layers = n_layers;
   P.M = M;
@@ -701,17 +891,30 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   P.x_pitch = gemv_x_pitch(k_max);
   P.status = status;
   P.tickets = tickets;
-  // Two blocks per SM, each with the deepest ring that fits beside its other data.
+  // Fewer units than SMs (a short, wide layer): a cluster of ks CTAs shares
+  // each unit, every CTA over its own contiguous range of the unit's stages,
+  // so that about every SM streams weights.  ks is the SM count over the unit
+  // count, rounded, at most 4 and at most the fewest stages of any layer.
+  const int sms = num_sms();
+  int ks = 1;
+  if (units < sms) {
+    ks = (sms + units / 2) / units;
+    if (ks > kGvMaxSplit) ks = kGvMaxSplit;
+    if (ks > nst_min) ks = nst_min;
+    if (ks < 1) ks = 1;
+  }
+  P.ksplit = ks;
+  // kGvBlocksPerSM blocks per SM, each with the deepest ring that fits beside its other data.
   const int slot = kGvStageBytes + (stream_x ? 2 * x_half_bytes(tt) : 0);
-  const int fixed = gemv_smem_bytes(M, k_max, 0, stream_x);
+  const int fixed = gemv_smem_bytes(M, k_max, 0, stream_x, ks);
   int nring = (kGvSmemPerBlock - fixed) / (slot + 16);
   if (nring > kGvMaxRing) nring = kGvMaxRing;
   if (nring < 2) return cudaErrorInvalidConfiguration;
   P.nring = nring;
-  const int smem = gemv_smem_bytes(M, k_max, nring, stream_x);
-  const int slots = kGvBlocksPerSM * num_sms();
-  const int grid = units < slots ? units : slots;
-  P.one_unit = units <= slots ? 1 : 0;
+  const int smem = gemv_smem_bytes(M, k_max, nring, stream_x, ks);
+  const int slots = kGvBlocksPerSM * sms;
+  const int grid = ks > 1 ? units * ks : (units < slots ? units : slots);
+  P.one_unit = ks > 1 || units <= slots ? 1 : 0;
   return y_type == kOutBF16 ? launch_group_y<__nv_bfloat16>(x_type, P, grid, smem, stream, pdl)
                             : launch_group_y<float>(x_type, P, grid, smem, stream, pdl);
 }

@@ -152,6 +152,31 @@ def test_forward_small_gemv(M, N, K, ydtype):
     _full_case(M, N, K, "bf16", ydtype, tb.PATH_GEMV, seed=M * N + K)
 
 
+# One token takes the dp4a path of the decode kernel: K from one 64-input chunk
+# to several 1024-input stages with a ragged last stage, N from one row to
+# ragged 64-row units; fp32 inputs of K <= 2048 and bf16 inputs of K <= 4096 are
+# quantised inside the kernel, longer ones by the quantisation kernel.
+ONE_TOKEN = [(1, 64), (63, 960), (65, 1024), (200, 1088), (130, 2048), (129, 4160), (64, 5120), (7, 8192)]
+
+
+@pytest.mark.parametrize("N,K", ONE_TOKEN)
+@pytest.mark.parametrize("xdtype", ["bf16", "f32"])
+def test_forward_one_token(N, K, xdtype):
+    _full_case(1, N, K, xdtype, torch.float32 if xdtype == "f32" else torch.bfloat16, tb.PATH_GEMV, seed=N + 7 * K)
+
+
+# Layers with fewer 64-row units than SMs are split along K over the CTAs of a
+# cluster (2 to 4, each a contiguous range of 1024-input stages) whose partial
+# sums meet in one CTA's shared memory: one to 16 tokens, ragged N and K.
+KSPLIT = [(130, 3072), (64, 8192), (300, 2112), (17, 4160)]
+
+
+@pytest.mark.parametrize("N,K", KSPLIT)
+@pytest.mark.parametrize("M", [1, 2, 5, 9, 16])
+def test_forward_ksplit(M, N, K):
+    _full_case(M, N, K, "bf16", torch.bfloat16, tb.PATH_GEMV, seed=M + N + K)
+
+
 @pytest.mark.parametrize("M,N,K", SMALL)
 @pytest.mark.parametrize("ydtype", [torch.float32, torch.bfloat16])
 def test_forward_small_gemm(M, N, K, ydtype):
