@@ -473,8 +473,8 @@ def run_decode_3b(args, world, peaks, L2):
                 packed, gamma = sets[i % len(sets)][0]
                 tb.forward(packed, gamma, x, y=y, workspace=ws)
 
-            steps = 4000
-            secs, _ = timed_graph_run(step, steps, 200, world, chunk=500)
+            steps = min(args.steps, 4000)
+            secs, _ = timed_graph_run(step, steps, min(args.warmup, 200), world, chunk=500)
             gbs = set_bytes * steps * world / secs / 1e9
             res["k%d_n%d_m%d" % (K, N, M)] = {
                 "GB/s": round(gbs, 1), "pct_hbm_measured": round(100 * gbs / world / peaks["hbm"], 2),

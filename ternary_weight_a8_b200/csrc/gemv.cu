@@ -891,18 +891,19 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   P.x_pitch = gemv_x_pitch(k_max);
   P.status = status;
   P.tickets = tickets;
-  // Fewer units than SMs (a short, wide layer): a cluster of ks CTAs shares
-  // each unit, every CTA over its own contiguous range of the unit's stages,
-  // so that about every SM streams weights.  ks is the SM count over the unit
-  // count, rounded, at most 4 and at most the fewest stages of any layer.
+  // Few units for the SMs (a short, wide layer): a cluster of ks CTAs shares
+  // each unit, every CTA over its own contiguous range of the unit's stages.
+  // One token: about one CTA per SM.  More tokens, where one warp per SM
+  // sub-partition issuing mma.sync is the limit: about two.  ks is that target
+  // over the unit count, rounded; at most 4, at most the fewest stages of any
+  // layer, and no more CTAs than are resident at once.
   const int sms = num_sms();
-  int ks = 1;
-  if (units < sms) {
-    ks = (sms + units / 2) / units;
-    if (ks > kGvMaxSplit) ks = kGvMaxSplit;
-    if (ks > nst_min) ks = nst_min;
-    if (ks < 1) ks = 1;
-  }
+  const int target = tt == 1 ? sms : 2 * sms;
+  int ks = units < target ? (target + units / 2) / units : 1;
+  while (ks > 1 && units * ks > kGvBlocksPerSM * sms) --ks;
+  if (ks > kGvMaxSplit) ks = kGvMaxSplit;
+  if (ks > nst_min) ks = nst_min;
+  if (ks < 1) ks = 1;
   P.ksplit = ks;
   // kGvBlocksPerSM blocks per SM, each with the deepest ring that fits beside its other data.
   const int slot = kGvStageBytes + (stream_x ? 2 * x_half_bytes(tt) : 0);
