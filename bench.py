@@ -584,7 +584,7 @@ def run_next(args, world, peaks, L2):
         res = {"weight_bytes": set_bytes}
         for name, fn in (("lut", lambda i: tb.forward_lut(sets[i % len(sets)][0][0], sets[i % len(sets)][0][1], xq,
                                                            sc, rs, y=y)),
-                         ("tensor_core_gemv", lambda i: tb.forward_quantized(sets[i % len(sets)][0][0],
+                         ("decode_kernel", lambda i: tb.forward_quantized(sets[i % len(sets)][0][0],
                                                                              sets[i % len(sets)][0][1], xq, sc, rs,
                                                                              y=y, workspace=ws))):
             secs, _ = timed_graph_run(fn, steps, 20, world, chunk=100)
