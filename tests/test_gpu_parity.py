@@ -166,7 +166,7 @@ def test_forward_one_token(N, K, xdtype):
 
 
 # Layers with fewer 64-row units than SMs are split along K over the CTAs of a
-# cluster (2 to 4, each a contiguous range of 1024-input stages) whose partial
+# cluster (2 to 8, each a contiguous range of 1024-input stages) whose partial
 # sums meet in one CTA's shared memory: one to 16 tokens, ragged N and K.
 KSPLIT = [(130, 3072), (64, 8192), (300, 2112), (17, 4160)]
 
