@@ -502,8 +502,8 @@ def run_chain(args, world, peaks, L2):
         def step(i):
             tb.layer_chain(layer_sets[i % len(layer_sets)], workspace=ws)
 
-        steps = 300
-        secs, _ = timed_graph_run(step, steps, 10, world, chunk=100)
+        steps = min(args.steps, 300)
+        secs, _ = timed_graph_run(step, steps, min(args.warmup, 10), world, chunk=100)
         gbs = set_bytes * steps * world / secs / 1e9
         res["tokens_%d" % M] = {"GB/s": round(gbs, 1), "pct_hbm_measured": round(100 * gbs / world / peaks["hbm"], 2),
                                 "us_per_chain": round(secs / steps * 1e6, 2),
