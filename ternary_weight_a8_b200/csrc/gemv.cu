@@ -85,10 +85,6 @@ constexpr int kGvBlocksPerSM = 3;
 constexpr int kGvSmemPerBlock = 75 * 1024;
 constexpr int kGvMaxRing = 16;
 constexpr int kGvMaxSplit = 8;        // CTAs of a cluster sharing one unit (the portable cluster limit)
-// Token slots up to which the dp4a path replaces mma.sync.  The path handles
-// up to two; with two tokens it measured slower than mma.sync (3B layers:
-// 8.3 vs 7.3 us and 9.8 vs 8.3 us per call), so only one token takes it.
-constexpr int kGvAluTokens = 1;
 constexpr int kGvTagEnd = -1;
 constexpr int kGvFuseChunks = 2;      // 16-input chunks a consumer thread quantises itself
 constexpr int kGvFuseElems = 4096;    // M*K up to which the blocks quantise activations themselves
@@ -126,9 +122,7 @@ __host__ __device__ inline void stage_range(int nst, int ks, int rank, int& sb, 
 
 // Shared-memory bytes of one CTA's partial sums in a K-split launch: one
 // 16-byte vector per consumer thread and mma token group.
-__host__ __device__ constexpr int gv_part_bytes(int tt) {
-  return (tt <= kGvAluTokens ? tt : (tt + 7) / 8) * kGvConsumers * 16;
-}
+__host__ __device__ constexpr int gv_part_bytes(int tt) { return ((tt + 7) / 8) * kGvConsumers * 16; }
 
 __device__ __forceinline__ void mma_u8s8_16x8x32(int (&d)[4], uint32_t a0, uint32_t a1,
                                                  uint32_t a2, uint32_t a3, uint32_t b0,
@@ -332,9 +326,7 @@ template <int TT, typename TY, typename TX, bool kSplit>
 __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(const __grid_constant__ GvParams P) {
   constexpr int TG = (TT + 7) / 8;           // mma token groups of 8
   constexpr bool kStream = sizeof(TX) == 1;  // int8 codes stream with the weights
-  constexpr bool kAlu = TT <= kGvAluTokens;  // one or two tokens: dp4a dot products instead of mma.sync
-  constexpr int TA = kAlu ? TT : 1;          // tokens of the dp4a path
-  constexpr int NV = kAlu ? TA : TG;         // 16-byte vectors of partial sums per lane (K-split)
+  constexpr bool kAlu = TT == 1;             // one token: dp4a dot products instead of the mma path
   constexpr int kXHalf = x_half_bytes(TT);   // one half-stage activation tile
   constexpr int kSlot = kGvStageBytes + (kStream ? 2 * kXHalf : 0);
   extern __shared__ uint8_t smem_raw[];
@@ -532,22 +524,15 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           }
         }
 
-      int rsum1[TA];  // the dp4a path's epilogue scalars (every lane)
-      float s1tok[TA];
-#pragma unroll
-      for (int m = 0; m < TA; ++m) {
-        rsum1[m] = 0;
-        s1tok[m] = 1.0f;
-        if constexpr (kAlu && kStream) {
-          if (m < M) {
-            rsum1[m] = __ldcg(L.rowsum + m);
-            s1tok[m] = __ldcg(L.scale + m);
-          }
-        }
+      int rsum1 = 0;  // the one-token path's epilogue scalars (every lane)
+      float s1tok = 1.0f;
+      if constexpr (kAlu && kStream) {
+        rsum1 = __ldcg(L.rowsum);
+        s1tok = __ldcg(L.scale);
       }
 
       int d[TG][4][4];      // mma path: accumulator fragments
-      int dr[TA][kAlu ? 4 : 1][4];  // dp4a path: token m, rows warp*16 + (lane >> 3) + 4*it, code position j
+      int dr[kAlu ? 4 : 1][4];   // one-token path: rows warp*16 + (lane >> 3) + 4*it, one set per code position j
 #pragma unroll
       for (int tg = 0; tg < TG; ++tg)
 #pragma unroll
@@ -555,11 +540,9 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
 #pragma unroll
           for (int c = 0; c < 4; ++c) d[tg][j][c] = 0;
 #pragma unroll
-      for (int m = 0; m < TA; ++m)
+      for (int r = 0; r < (kAlu ? 4 : 1); ++r)
 #pragma unroll
-        for (int r = 0; r < (kAlu ? 4 : 1); ++r)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) dr[m][r][j] = 0;
+        for (int j = 0; j < 4; ++j) dr[r][j] = 0;
       bool ok = true;
       for (int i = s0; i < s1; ++i) {
         if (i > s0) {
@@ -570,31 +553,23 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         if constexpr (kAlu) {
           // Lane (rs, ch) = (lane >> 3, lane & 7) takes 16-byte chunk ch of rows
           // warp*16 + rs + 4*it of each half (inputs 64ch .. 64ch+63 of the half) and the
-          // matching 64 codes of each token: one AND per four weights and one dp4a per
-          // four weights and token, no idle mma columns.  Each 8-lane phase reads one
-          // 128-byte swizzled row.
+          // matching 64 codes: one AND and one dp4a per four weights, no idle mma
+          // columns.  Each 8-lane phase reads one 128-byte swizzled row.
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
             const int ch = lane & 7, rs = lane >> 3;
             const int k0 = i * kGvStageK + hf * (kGvStageK / 2) + 64 * ch;
             if (k0 < L.K) {  // inputs past K have zero weights (K is a multiple of 64)
-              uint4 xc[TA][4];
+              uint4 xc[4];
 #pragma unroll
-              for (int m = 0; m < TA; ++m)
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  if (m < M) {
-                    if constexpr (kStream) {
-                      // 128-input block q of token m is row 4m + q of the half tile
-                      const int row = 4 * m + (ch >> 1), ci = 4 * (ch & 1) + u;
-                      xc[m][u] = lds128(wt + kGvStageBytes + hf * kXHalf + row * 128 + ((ci ^ (row & 7)) << 4));
-                    } else {
-                      xc[m][u] = lds128(xs + m * P.x_pitch + x_chunk_off((k0 >> 4) + u));
-                    }
-                  } else {
-                    xc[m][u] = make_uint4(0, 0, 0, 0);
-                  }
+              for (int u = 0; u < 4; ++u) {
+                if constexpr (kStream) {
+                  const int q = ch >> 1, ci = 4 * (ch & 1) + u;  // 128-input block; token 0 owns rows 0..3
+                  xc[u] = lds128(wt + kGvStageBytes + hf * kXHalf + q * 128 + ((ci ^ q) << 4));
+                } else {
+                  xc[u] = lds128(xs + x_chunk_off((k0 >> 4) + u));
                 }
+              }
               const uint32_t base = wt + hf * (kGvStageBytes / 2);
 #pragma unroll
               for (int it = 0; it < 4; ++it) {
@@ -603,11 +578,8 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
 #pragma unroll
                 for (int v = 0; v < 4; ++v)
 #pragma unroll
-                  for (int j = 0; j < 4; ++j) {
-                    const uint32_t a = u4_get(wv, v) & (0x03030303u << (2 * j));
-#pragma unroll
-                    for (int m = 0; m < TA; ++m) dr[m][it][j] = dp4a_us(a, u4_get(xc[m][v], j), dr[m][it][j]);
-                  }
+                  for (int j = 0; j < 4; ++j)
+                    dr[it][j] = dp4a_us(u4_get(wv, v) & (0x03030303u << (2 * j)), u4_get(xc[v], j), dr[it][j]);
               }
             }
           }
@@ -681,13 +653,10 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
 
       // This CTA's sums per lane: the four code-position sets shifted back (exact,
       // each set being a multiple of 4^j).
-      int pc[NV][4];
+      int pc[TG][4];
       if constexpr (kAlu) {
 #pragma unroll
-        for (int m = 0; m < TA; ++m)
-#pragma unroll
-          for (int r = 0; r < 4; ++r)
-            pc[m][r] = dr[m][r][0] + (dr[m][r][1] >> 2) + (dr[m][r][2] >> 4) + (dr[m][r][3] >> 6);
+        for (int r = 0; r < 4; ++r) pc[0][r] = dr[r][0] + (dr[r][1] >> 2) + (dr[r][2] >> 4) + (dr[r][3] >> 6);
       } else if constexpr (kSplit) {  // (the mma epilogue below combines them itself otherwise)
 #pragma unroll
         for (int tg = 0; tg < TG; ++tg)
@@ -702,8 +671,8 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         const uint32_t mine = part + (warp * 32 + lane) * 16;
         if (rank != 0) {
 #pragma unroll
-          for (int pv = 0; pv < NV; ++pv)
-            sts128(mine + pv * kGvConsumers * 16, make_uint4(pc[pv][0], pc[pv][1], pc[pv][2], pc[pv][3]));
+          for (int tg = 0; tg < TG; ++tg)
+            sts128(mine + tg * kGvConsumers * 16, make_uint4(pc[tg][0], pc[tg][1], pc[tg][2], pc[tg][3]));
           __syncwarp();
           if (lane == 0) mbar_arrive_release_cluster(mapa_shared(red_bar, 0));
           continue;
@@ -713,12 +682,12 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         fence_acq_rel_cluster();
         for (int r = 1; r < ks; ++r)
 #pragma unroll
-          for (int pv = 0; pv < NV; ++pv) {
-            const uint4 v = ld_shared_cluster_v4(mapa_shared(mine + pv * kGvConsumers * 16, r));
-            pc[pv][0] += static_cast<int>(v.x);
-            pc[pv][1] += static_cast<int>(v.y);
-            pc[pv][2] += static_cast<int>(v.z);
-            pc[pv][3] += static_cast<int>(v.w);
+          for (int tg = 0; tg < TG; ++tg) {
+            const uint4 v = ld_shared_cluster_v4(mapa_shared(mine + tg * kGvConsumers * 16, r));
+            pc[tg][0] += static_cast<int>(v.x);
+            pc[tg][1] += static_cast<int>(v.y);
+            pc[tg][2] += static_cast<int>(v.z);
+            pc[tg][3] += static_cast<int>(v.w);
           }
       }
 
@@ -726,35 +695,31 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       const int n_base = (unit - L.unit0) * kGvRows;
       TY* y = static_cast<TY*>(L.y);
       if constexpr (kAlu) {
-        // Per token, a butterfly over the 8 lanes of a row group leaves row
+        // A butterfly over the 8 lanes of a row group leaves row
         // warp*16 + (lane >> 3) + 4*((lane >> 1) & 3) summed in lanes 2r and 2r + 1.
+        int v[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) v[r] = pc[0][r];
+#pragma unroll
+        for (int st = 0; st < 2; ++st) {
+          const int off = 4 >> st, half = 2 >> st;
+          const bool upper = (lane & off) != 0;
+#pragma unroll
+          for (int r = 0; r < half; ++r) {
+            const int send = upper ? v[r] : v[r + half];
+            const int keep = upper ? v[r + half] : v[r];
+            v[r] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+          }
+        }
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
         const int n = n_base + warp * 16 + (lane >> 3) + 4 * ((lane >> 1) & 3);
-#pragma unroll
-        for (int m = 0; m < TA; ++m) {
-          int v[4];
-#pragma unroll
-          for (int r = 0; r < 4; ++r) v[r] = pc[m][r];
-#pragma unroll
-          for (int st = 0; st < 2; ++st) {
-            const int off = 4 >> st, half = 2 >> st;
-            const bool upper = (lane & off) != 0;
-#pragma unroll
-            for (int r = 0; r < half; ++r) {
-              const int send = upper ? v[r] : v[r + half];
-              const int keep = upper ? v[r + half] : v[r];
-              v[r] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-            }
-          }
-          v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
-          if ((lane & 1) == 0 && n < L.N && m < M) {
-            const int rsum = kStream ? rsum1[m] : rs_tok[m];
-            const float sm = kStream ? s1tok[m] : s_tok[m];
-            const int a = v[0] - rsum;
-            const float val = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, sm));
-            const size_t o = static_cast<size_t>(m) * L.N + n;
-            if constexpr (sizeof(TY) == 4) y[o] = val; else y[o] = __float2bfloat16_rn(val);
-            if (L.acc_out) L.acc_out[o] = a;
-          }
+        if ((lane & 1) == 0 && n < L.N) {
+          const int rsum = kStream ? rsum1 : rs_tok[0];
+          const float sm = kStream ? s1tok : s_tok[0];
+          const int a = v[0] - rsum;
+          const float val = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, sm));
+          if constexpr (sizeof(TY) == 4) y[n] = val; else y[n] = __float2bfloat16_rn(val);
+          if (L.acc_out) L.acc_out[n] = a;
         }
         continue;
       }
@@ -942,7 +907,7 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   // over the unit count, rounded; at most 8, at most the fewest stages of any
   // layer, and no more CTAs than are resident at once.
   const int sms = num_sms();
-  const int target = tt <= kGvAluTokens ? sms : 2 * sms;
+  const int target = tt == 1 ? sms : 2 * sms;
   int ks = units < target ? (target + units / 2) / units : 1;
   while (ks > 1 && units * ks > kGvBlocksPerSM * sms) --ks;
   if (ks > kGvMaxSplit) ks = kGvMaxSplit;
