@@ -48,6 +48,14 @@
  *  - A workspace starts with a 256-byte status word, which must be zero
  *    before first use (zero the workspace once after allocating it).  Calls
  *    that overlap on the GPU must not share a workspace.
+ *  - The product kernels are launched as programmatic dependents of the
+ *    kernel before them on the stream: they start loading the packed
+ *    weights while that kernel finishes, and wait for it before reading
+ *    anything else (activations, codes, scales, gamma) or writing.  So the
+ *    packed weights must not be written by the kernel launched immediately
+ *    before the call, unless that kernel makes its writes visible before it
+ *    exits, as bitlinear_pack_weights does.  Weights written by earlier work
+ *    on the stream, or copied in by a memory copy, need nothing more.
  */
 #ifndef BITLINEAR_H
 #define BITLINEAR_H

@@ -86,6 +86,11 @@ __global__ void __launch_bounds__(256) ternary_pack_kernel(const float* __restri
     }
     packed[g] = word;
   }
+  // The forward kernels, launched as programmatic dependents of the kernel
+  // before them, start loading packed weights before their grid-dependency
+  // wait.  The fence makes this kernel's words visible device-wide before its
+  // blocks exit, which is the earliest a dependent launch can begin.
+  __threadfence();
 }
 
 cudaError_t launch_gamma(const float* W, int N, int K, double* row_sums, float* gamma,
