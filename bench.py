@@ -645,9 +645,8 @@ def run_pack(world):
 # the oracle (CPU) on the same workload
 # ----------------------------------------------------------------------------
 
-def oracle_decode_setup():
-    import numpy as np
-
+def oracle_decode_layers():
+    """The decode_2b layers as the oracle takes them: (packed, gamma, K, x) per layer."""
     import oracle
     import synth
 
@@ -657,15 +656,31 @@ def oracle_decode_setup():
         packed, gamma, _ = oracle.pack_weights(W)
         _, xf = synth.activations_bf16(1, K, seed=100 + i)
         layers.append((packed, gamma, K, xf))
-    set_bytes = sum(p.size for p, *_ in layers)
+    return layers, sum(p.size for p, *_ in layers)
 
-    def step():
+
+def oracle_decode_steps(layers, reps):
+    """reps decode steps of the oracle over `layers` (any subset of rows); returns seconds."""
+    import oracle
+
+    t0 = time.perf_counter()
+    for _ in range(reps):
         for packed, gamma, K, xf in layers:
             T, ok = oracle.unpack(packed, K)
             acc, y, *_ = oracle.forward(T, gamma, xf)
             oracle.round_bf16(y)
+    return time.perf_counter() - t0
 
-    return step, set_bytes
+
+def oracle_decode_setup():
+    layers, set_bytes = oracle_decode_layers()
+    return (lambda: oracle_decode_steps(layers, 1)), set_bytes
+
+
+def _oracle_rows_worker(task):
+    layers, reps = task
+    oracle_decode_steps(layers, 1)  # load the oracle library before timing
+    return oracle_decode_steps(layers, reps)
 
 
 def cpu_baseline(target_s=10.0):
@@ -681,6 +696,40 @@ def cpu_baseline(target_s=10.0):
     return {"value": round(reps * set_bytes / secs / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": "%d full decode_2b steps (unpack + quantise + accumulate + dequantise + bf16 round, "
                       "both layers) on one host core, %.1f s" % (reps, secs)}
+
+
+def cpu_baseline_all_cores(cpu_work_s=20.0):
+    """The same oracle decode steps spread over the host's cores: each process
+    takes a contiguous slice of every layer's output rows (rows are independent,
+    so the slices together compute the whole step).  The pool is started with
+    `spawn`, so no process inherits the CUDA context."""
+    import multiprocessing
+
+    layers, set_bytes = oracle_decode_layers()
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    cores = max(1, min(cores, 128))
+    one = oracle_decode_steps(layers, 1)
+    reps = max(2, int(cpu_work_s / max(one, 1e-6)))  # about cpu_work_s of CPU work in total
+    tasks = []
+    for c in range(cores):
+        shard = []
+        for packed, gamma, K, xf in layers:
+            N = packed.shape[0]
+            n0, n1 = N * c // cores, N * (c + 1) // cores
+            if n1 > n0:
+                shard.append((packed[n0:n1], gamma, K, xf))
+        tasks.append((shard, reps))
+    with multiprocessing.get_context("spawn").Pool(cores) as pool:
+        pool.map(_oracle_rows_worker, [(t[0], 1) for t in tasks])  # start every worker
+        t0 = time.perf_counter()
+        pool.map(_oracle_rows_worker, tasks, chunksize=1)
+        secs = time.perf_counter() - t0
+    return {"value": round(reps * set_bytes / secs / 1e9, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": "%d full decode_2b steps, each process of %d taking 1/%d of every layer's rows, %.2f s wall"
+                      % (reps, cores, cores, secs)}
 
 
 def run_reference(args, world, rank):
@@ -726,6 +775,7 @@ def main():
     res = run_ours(args, world, rank, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline()
+        res["cpu_baseline_all_cores"] = cpu_baseline_all_cores()
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:
