@@ -677,6 +677,11 @@ def oracle_decode_setup():
     return (lambda: oracle_decode_steps(layers, 1)), set_bytes
 
 
+def row_slices(n_rows, parts):
+    """Contiguous, disjoint [n0, n1) slices of n_rows rows, one per part, sizes within one."""
+    return [(n_rows * c // parts, n_rows * (c + 1) // parts) for c in range(parts)]
+
+
 def _oracle_rows_worker(task):
     layers, reps = task
     oracle_decode_steps(layers, 1)  # load the oracle library before timing
@@ -717,8 +722,7 @@ def cpu_baseline_all_cores(cpu_work_s=20.0):
     for c in range(cores):
         shard = []
         for packed, gamma, K, xf in layers:
-            N = packed.shape[0]
-            n0, n1 = N * c // cores, N * (c + 1) // cores
+            n0, n1 = row_slices(packed.shape[0], cores)[c]
             if n1 > n0:
                 shard.append((packed[n0:n1], gamma, K, xf))
         tasks.append((shard, reps))
