@@ -53,9 +53,9 @@
  *    weights while that kernel finishes, and wait for it before reading
  *    anything else (activations, codes, scales, gamma) or writing.  So the
  *    packed weights must not be written by the kernel launched immediately
- *    before the call, unless that kernel makes its writes visible before it
- *    exits, as bitlinear_pack_weights does.  Weights written by earlier work
- *    on the stream, or copied in by a memory copy, need nothing more.
+ *    before the call.  bitlinear_pack_weights ends with a memory operation
+ *    (not a kernel) for this reason; weights written by earlier work on the
+ *    stream, or copied in by a memory copy, need nothing more.
  */
 #ifndef BITLINEAR_H
 #define BITLINEAR_H
@@ -159,6 +159,40 @@ typedef enum { BL_GLU_RELU2 = 0, BL_GLU_SILU = 1 } bl_glu;
 int bitlinear_glu_quant(const void* gate, const void* up, int x_dtype, int M, int N, int act, void* h,
                         int8_t* xq, float* scale, int32_t* rowsum, void* stream);
 
+/* Workspace bytes bitlinear_gate_up_glu needs for M tokens, gate/up N x K. */
+size_t bitlinear_gate_up_glu_workspace_bytes(int M, int N, int K);
+
+/*
+ * The FFN's gate and up BitLinears, the gated activation between them and the
+ * down BitLinear, and the quantisation of its result for the down BitLinear,
+ * as one call ("BitNet's Real Bet: Designing the Whole Inference Stack",
+ * native training section: SwiGLU for the 2024 model, squared ReLU for 2B4T;
+ * "A Two-Billion Ternary Bet": squared-ReLU-style activations).  The result
+ * equals, bit for bit, bitlinear_layer_chain of the gate and up BitLinears
+ * on x (outputs in x_dtype) followed by bitlinear_glu_quant of their outputs.
+ *   packed_gate, gamma_gate, packed_up, gamma_up: the two BitLinears (each its
+ *           own gamma), N x K each; N % 64 == 0 (N is the down BitLinear's K).
+ *   x       device [M][K] of x_dtype, the FFN's (normalised) input.
+ *   act     BL_GLU_RELU2 or BL_GLU_SILU, as bitlinear_glu_quant.
+ *   h       device [M][N] of x_dtype out, or NULL: h itself.
+ *   xq, scale, rowsum: device int8 [M][N], fp32 [M], int32 [M] out: the
+ *           codes of h, as bitlinear_quant_act would make them; they feed the
+ *           down BitLinear (bitlinear_forward_quantized, or a chain layer's
+ *           xq / scale / rowsum).
+ *   workspace / workspace_bytes: >= bitlinear_gate_up_glu_workspace_bytes(M, N, K),
+ *           its first 256 bytes zero.
+ * M <= 16: one quantisation launch and one decode launch that computes gate
+ * and up, forms h as soon as both halves of a group of rows are in, keeps
+ * the per-token maxima of |h| and, once every row is in, quantises h with
+ * the final scales (no further launch).  Larger M: the quantisation of x,
+ * one tensor-core GEMM whose tiles pair 128 gate rows with the same 128 up
+ * rows so that its epilogue writes h, then the quantisation of h.
+ */
+int bitlinear_gate_up_glu(const uint8_t* packed_gate, const float* gamma_gate, const uint8_t* packed_up,
+                          const float* gamma_up, int N, int K, const void* x, int x_dtype, int M, int act, void* h,
+                          int8_t* xq, float* scale, int32_t* rowsum, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
 /*
  * The product and dequantisation of one token by table lookup instead of
  * multiplication: the T-MAC approach ("BitNet b1.58 and the 1-Bit AI
@@ -219,6 +253,8 @@ size_t bitlinear_workspace_bytes(int M, int N, int K);
  *   y       device [M][N] of y_dtype out.
  *   acc_out device int32 [M][N] out, or NULL: the exact accumulators
  *           sum_k q*t (for parity checks).
+ *   workspace / workspace_bytes: >= bitlinear_workspace_bytes(M, N, K), its
+ *           first 256 bytes zero.
  * M <= 16 runs the decode GEMV kernel (which quantises small activations
  * itself); larger M the quantisation kernel and the tcgen05 tensor-core GEMM.
  */
@@ -236,7 +272,17 @@ int bitlinear_forward_quantized(const uint8_t* packed, const float* gamma, int N
                                 int M, void* y, int y_dtype, int32_t* acc_out, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
-/* One BitLinear of a chain: weights, gamma, shape, input [M][K], output [M][N]. */
+/*
+ * One BitLinear of a chain: weights, gamma, shape, input [M][K], output [M][N].
+ *   x       device [M][K] activations of the chain's x_dtype; ignored (may be
+ *           NULL) when xq is set.
+ *   xq, scale, rowsum: NULL, or the layer's input already quantised, as
+ *           bitlinear_quant_act or bitlinear_glu_quant wrote it (codes
+ *           [M][K], scales [M], code sums [M]): the chain then quantises
+ *           nothing for this layer.
+ *   acc_out NULL, or device int32 [M][N] out: the layer's exact accumulators
+ *           (for parity checks).
+ */
 typedef struct {
   const uint8_t* packed;
   const float* gamma;
@@ -244,6 +290,10 @@ typedef struct {
   int K;
   const void* x;
   void* y;
+  const int8_t* xq;
+  const float* scale;
+  const int32_t* rowsum;
+  int32_t* acc_out;
 } bl_layer;
 
 /* Workspace bytes bitlinear_layer_chain needs for these layers at M tokens. */
@@ -252,8 +302,12 @@ size_t bitlinear_chain_workspace_bytes(const bl_layer* layers, int n_layers, int
 /*
  * Runs n_layers BitLinear forwards back to back on one stream.  Consecutive
  * layers that read the same x pointer with the same K (e.g. FFN gate and up)
- * share one activation quantisation; each keeps its own gamma.  `layers` is a
- * host array, read during the call only.
+ * share one activation quantisation; each keeps its own gamma.  At decode
+ * sizes (M <= 16), consecutive layers that are independent of one another
+ * (no layer reads what another writes) run in one launch of the decode
+ * kernel.  `layers` is a host array, read during the call only; at most 64
+ * layers.  The workspace (>= bitlinear_chain_workspace_bytes) starts with a
+ * zero status block, as every workspace does.
  */
 int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dtype, int y_dtype,
                           void* workspace, size_t workspace_bytes, void* stream);
@@ -286,22 +340,44 @@ int bitlinear_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int
  *
  * The scratch is a fixed 1 MiB array in device memory that the library
  * declares once; every GPU that loads the library holds it until the
- * process exits.  A call needs 256 bytes plus about M * K bytes of it
- * (exactly bitlinear_workspace_bytes(M, N, K)); larger calls are refused
- * with BL_ERR_WORKSPACE_TOO_SMALL.  All calls share the array and each call
- * first clears its 256-byte control block, so calls in one stream are safe
- * but calls that overlap on the GPU (other streams, other host threads)
- * race on it.  The first call on a device looks up the array's device
- * address (with that device current) and caches it; make that first call
- * before any stream capture.  Device-side wait failures are recorded in the
- * shared array and are not reported; use bitlinear_forward with a
- * workspace and bitlinear_device_status to observe them.
+ * process exits.  What a call needs of it depends on the kernel that runs:
+ * 256 bytes when the decode kernel quantises the activations itself (M * K
+ * up to 4096), else 256 bytes plus about M * K bytes for the codes (exactly
+ * bitlinear_workspace_bytes(M, N, K)).  Larger calls are refused with
+ * BL_ERR_WORKSPACE_TOO_SMALL.  All calls share the array and each call first
+ * clears its 256-byte control block, so calls in one stream are safe but
+ * calls that overlap on the GPU (other streams, other host threads) race on
+ * it.  The first call on a device (and the first after the device's context
+ * changes, e.g. after cudaDeviceReset) looks up the array's device address
+ * with that device current and caches it per device and context; make that
+ * first call before any stream capture.  Device-side wait failures are
+ * recorded in the shared control block and wiped by the next call's clear:
+ * read them between calls with bitlinear_noalloc_status.
  */
 int bitlinear_forward_noalloc(const uint8_t* packed, const float* gamma, int N, int K, const void* x,
                               int x_dtype, int M, void* y, int y_dtype, int32_t* acc_out, void* stream);
 
+/*
+ * For bitlinear_forward_noalloc callers: synchronises `stream`, then returns
+ * BL_OK or BL_ERR_DEVICE_TIMEOUT from the shared control block's status word
+ * (as bitlinear_device_status does for a workspace) and clears the word.
+ * Call it after a no-allocation call and before the next one.  Allocates
+ * nothing.
+ */
+int bitlinear_noalloc_status(void* stream);
+
 /* Forces the product kernel: 0 = by M (default), 1 = GEMV (M <= 16 only), 2 = GEMM.  Per thread. */
 int bitlinear_set_path(int path);
+
+/*
+ * Forces how many CTAs (a thread-block cluster, 1 .. 8) share each unit of
+ * 64 weight rows in the decode kernel, each over its own range of K, on the
+ * calling thread: 0 (default) lets the kernel choose (it splits short, wide
+ * layers, whose units are too few for the SMs).  The split is capped by the
+ * layer's 1024-input stages and by the CTAs resident at once.  For tests and
+ * tuning; the fused gate/up call never splits.
+ */
+int bitlinear_set_decode_split(int ctas);
 
 /* Message of the most recent failure on the calling thread ("" if none). */
 const char* bitlinear_last_error(void);

@@ -45,11 +45,13 @@
  *    over k ascending, then the row sums over n ascending; the mean is that
  *    sum divided by N*K in double, rounded once to fp32.
  *  - The divide, round and clamp of the ternarisation run in fp32 (the
- *    listing's tensors are fp32); rounding is to nearest, ties to even.
+ *    section's weights are fp32 tensors); rounding is to nearest, ties to
+ *    even.  The divisor is gamma + 1e-5: the section fixes eps = 1e-5 as the
+ *    guard added to gamma (an all-zero matrix then ternarises to zeros).
  *  - Per-token 8-bit quantisation is symmetric absmax: s = 127 / max(amax,
  *    1e-5) in fp32, q = clamp(rint(x * s), -128, 127) (ties to even).
  *  - Dequantisation is y = acc * gamma / s, evaluated in double (gamma, not
- *    gamma + eps, because gamma is what the listing returns).
+ *    gamma + eps: the section keeps gamma itself beside the ternary matrix).
  *  - Storage: code c = t + 1 in {0, 1, 2}, two bits each, four to a byte;
  *    32-bit little-endian word g of a row holds elements 16g .. 16g+15, and
  *    element 16g + 4j + b sits in byte b at bits [2j, 2j+1].
@@ -77,7 +79,7 @@
 
 #define ORACLE_EPS 1e-5f
 
-/* [AbsMean]: gamma = mean(|W|) over the whole matrix. */
+/* [AbsMean]: gamma is the average absolute value of the entire weight matrix. */
 float oracle_absmean_gamma(const float* W, int64_t N, int64_t K, double* sum_out) {
   double total = 0.0;
   for (int64_t n = 0; n < N; ++n) {
@@ -92,7 +94,8 @@ float oracle_absmean_gamma(const float* W, int64_t N, int64_t K, double* sum_out
   return (float)(total / (double)(N * K));
 }
 
-/* [AbsMean]: t = clamp(round(w / (gamma + eps)), -1, 1). */
+/* [AbsMean]: every weight divided by the gamma scale (plus eps), rounded to the
+ * nearest integer, clamped so that no value leaves [-1, 1]. */
 void oracle_ternarize(const float* W, int64_t count, float gamma, int8_t* T) {
   float d = gamma + ORACLE_EPS;
   for (int64_t i = 0; i < count; ++i) {

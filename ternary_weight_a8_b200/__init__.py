@@ -48,6 +48,10 @@ class bl_layer(ctypes.Structure):
         ("K", ctypes.c_int),
         ("x", ctypes.c_void_p),
         ("y", ctypes.c_void_p),
+        ("xq", ctypes.c_void_p),
+        ("scale", ctypes.c_void_p),
+        ("rowsum", ctypes.c_void_p),
+        ("acc_out", ctypes.c_void_p),
     ]
 
 
@@ -70,6 +74,8 @@ def lib() -> ctypes.CDLL:
             "bitlinear_quant_act": (i32, [vp, i32, i32, i32, vp, vp, vp, vp]),
             "bitlinear_rmsnorm_quant": (i32, [vp, i32, i32, i32, vp, ctypes.c_float, vp, vp, vp, vp, vp]),
             "bitlinear_glu_quant": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
+            "bitlinear_gate_up_glu_workspace_bytes": (sz, [i32, i32, i32]),
+            "bitlinear_gate_up_glu": (i32, [vp, vp, vp, vp, i32, i32, vp, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]),
             "bitlinear_forward_lut": (i32, [vp, vp, i32, i32, vp, vp, vp, i32, vp, i32, vp, vp]),
             "bitlinear_ste_workspace_bytes": (sz, [i32, i32, i32]),
             "bitlinear_ste_backward": (i32, [vp, vp, i32, i32, vp, vp, vp, i32, vp, i32, vp, vp, sz, vp]),
@@ -81,6 +87,9 @@ def lib() -> ctypes.CDLL:
             "bitlinear_device_status": (i32, [vp, vp]),
             "bitlinear_selftest_wait_timeout": (i32, [vp, sz, i32, vp]),
             "bitlinear_set_path": (i32, [i32]),
+            "bitlinear_set_decode_split": (i32, [i32]),
+            "bitlinear_forward_noalloc": (i32, [vp, vp, i32, i32, vp, i32, i32, vp, i32, vp, vp]),
+            "bitlinear_noalloc_status": (i32, [vp]),
             "bitlinear_last_error": (ctypes.c_char_p, []),
             "bitlinear_version": (i32, []),
         }
@@ -129,6 +138,11 @@ def set_path(path: int) -> None:
     _check(lib().bitlinear_set_path(path))
 
 
+def set_decode_split(ctas: int) -> None:
+    """Force the decode kernel's K-split to ``ctas`` CTAs per unit on this thread (0: automatic)."""
+    _check(lib().bitlinear_set_decode_split(int(ctas)))
+
+
 def version() -> int:
     return lib().bitlinear_version()
 
@@ -150,6 +164,27 @@ def new_workspace(nbytes: int, device=None) -> torch.Tensor:
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
 
 
+_WS_CACHE: dict = {}
+
+
+def cached_workspace(nbytes: int, device=None, stream=None) -> torch.Tensor:
+    """The workspace a call without an explicit one uses: one zeroed buffer per
+    (device, stream), kept between calls and replaced by a larger one only
+    when a call needs more.  Calls on one stream are ordered, so they may share
+    it; the library leaves its zeroed parts zeroed."""
+    dev = torch.device(device if device is not None else "cuda")
+    if dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    key = (dev.index, s.cuda_stream)
+    ws = _WS_CACHE.get(key)
+    if ws is None or ws.numel() < nbytes:
+        with torch.cuda.stream(s):
+            ws = new_workspace(nbytes, dev)
+        _WS_CACHE[key] = ws
+    return ws
+
+
 # ----------------------------------------------------------------------------
 # Calls
 # ----------------------------------------------------------------------------
@@ -163,7 +198,7 @@ def pack_weights(W: torch.Tensor, packed: torch.Tensor | None = None, gamma: tor
     if gamma is None:
         gamma = torch.empty(1, dtype=torch.float32, device=W.device)
     if workspace is None:
-        workspace = new_workspace(pack_workspace_bytes(N, K), W.device)
+        workspace = cached_workspace(pack_workspace_bytes(N, K), W.device, stream)
     _check(lib().bitlinear_pack_weights(_ptr(W), N, K, _ptr(packed), _ptr(gamma), _ptr(workspace),
                                         workspace.numel(), _stream(stream)))
     return packed, gamma
@@ -225,7 +260,7 @@ def ste_backward(packed: torch.Tensor, gamma: torch.Tensor, K: int, dy: torch.Te
     dxt = torch.empty((M, K), dtype=dx_dtype, device=dev) if dx is True else (dx if isinstance(dx, torch.Tensor) else None)
     dwt = torch.empty((N, K), dtype=torch.float32, device=dev) if dw is True else (dw if isinstance(dw, torch.Tensor) else None)
     if workspace is None:
-        workspace = new_workspace(ste_workspace_bytes(M, N, K), device=dev)
+        workspace = cached_workspace(ste_workspace_bytes(M, N, K), dev, stream)
     _check(lib().bitlinear_ste_backward(_ptr(packed), _ptr(gamma), N, K, _ptr(dy), _ptr(xq), _ptr(scale), M, _ptr(dxt),
                                         _dtype_code(dxt.dtype) if dxt is not None else 0, _ptr(dwt), _ptr(workspace),
                                         workspace.numel(), _stream(stream)))
@@ -252,6 +287,30 @@ def glu_quant(gate: torch.Tensor, up: torch.Tensor, act: int = GLU_RELU2, h=None
     return (hout, xq, scale, rowsum) if hout is not None else (xq, scale, rowsum)
 
 
+def gate_up_glu_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().bitlinear_gate_up_glu_workspace_bytes(M, N, K))
+
+
+def gate_up_glu(packed_gate: torch.Tensor, gamma_gate: torch.Tensor, packed_up: torch.Tensor,
+                gamma_up: torch.Tensor, x: torch.Tensor, act: int = GLU_RELU2, h=None, xq=None, scale=None,
+                rowsum=None, workspace=None, stream=None):
+    """The FFN's gate and up BitLinears, h = act(gate) * up and h's quantisation for the down
+    BitLinear in one call: returns (xq, scale, rowsum), and h first when ``h`` is True or a tensor."""
+    N = packed_gate.shape[0]
+    M, K = x.shape
+    dev = x.device
+    xq = torch.empty((M, N), dtype=torch.int8, device=dev) if xq is None else xq
+    scale = torch.empty(M, dtype=torch.float32, device=dev) if scale is None else scale
+    rowsum = torch.empty(M, dtype=torch.int32, device=dev) if rowsum is None else rowsum
+    hout = torch.empty((M, N), dtype=x.dtype, device=dev) if h is True else (h if isinstance(h, torch.Tensor) else None)
+    if workspace is None:
+        workspace = cached_workspace(gate_up_glu_workspace_bytes(M, N, K), dev, stream)
+    _check(lib().bitlinear_gate_up_glu(_ptr(packed_gate), _ptr(gamma_gate), _ptr(packed_up), _ptr(gamma_up), N, K,
+                                       _ptr(x), _dtype_code(x.dtype), M, int(act), _ptr(hout), _ptr(xq), _ptr(scale),
+                                       _ptr(rowsum), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return (hout, xq, scale, rowsum) if hout is not None else (xq, scale, rowsum)
+
+
 def forward(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, out_dtype=torch.bfloat16,
             y: torch.Tensor | None = None, acc_out: torch.Tensor | bool | None = None,
             workspace: torch.Tensor | None = None, stream=None):
@@ -266,7 +325,7 @@ def forward(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, out_dtyp
     elif isinstance(acc_out, torch.Tensor):
         acc = acc_out
     if workspace is None:
-        workspace = new_workspace(workspace_bytes(M, N, K), x.device)
+        workspace = cached_workspace(workspace_bytes(M, N, K), x.device, stream)
     _check(lib().bitlinear_forward(_ptr(packed), _ptr(gamma), N, K, _ptr(x), _dtype_code(x.dtype), M,
                                    _ptr(y), _dtype_code(y.dtype), _ptr(acc), _ptr(workspace),
                                    workspace.numel(), _stream(stream)))
@@ -288,7 +347,7 @@ def forward_quantized(packed: torch.Tensor, gamma: torch.Tensor, xq: torch.Tenso
     elif isinstance(acc_out, torch.Tensor):
         acc = acc_out
     if workspace is None:
-        workspace = new_workspace(workspace_bytes(M, N, K), xq.device)
+        workspace = cached_workspace(workspace_bytes(M, N, K), xq.device, stream)
     _check(lib().bitlinear_forward_quantized(_ptr(packed), _ptr(gamma), N, K, _ptr(xq), _ptr(scale),
                                              _ptr(rowsum), M, _ptr(y), _dtype_code(y.dtype), _ptr(acc),
                                              _ptr(workspace), workspace.numel(), _stream(stream)))
@@ -297,16 +356,33 @@ def forward_quantized(packed: torch.Tensor, gamma: torch.Tensor, xq: torch.Tenso
 
 @dataclass
 class Layer:
+    """One BitLinear of a chain.  ``x`` is the input ``[M][K]``; or give
+    ``xq``/``scale``/``rowsum`` (codes from ``quant_act`` or ``glu_quant``)
+    instead, and ``x`` may be None.  ``acc_out`` (int32 ``[M][N]``) receives the
+    exact accumulators when given."""
     packed: torch.Tensor
     gamma: torch.Tensor
-    x: torch.Tensor
+    x: torch.Tensor | None
     y: torch.Tensor
+    xq: torch.Tensor | None = None
+    scale: torch.Tensor | None = None
+    rowsum: torch.Tensor | None = None
+    acc_out: torch.Tensor | None = None
+
+    @property
+    def tokens(self) -> int:
+        return (self.x if self.x is not None else self.xq).shape[0]
+
+    @property
+    def K(self) -> int:
+        return (self.x if self.x is not None else self.xq).shape[1]
 
 
 def _layer_array(layers: Sequence[Layer]):
     arr = (bl_layer * len(layers))()
     for i, L in enumerate(layers):
-        arr[i] = bl_layer(_ptr(L.packed), _ptr(L.gamma), L.packed.shape[0], L.x.shape[1], _ptr(L.x), _ptr(L.y))
+        arr[i] = bl_layer(_ptr(L.packed), _ptr(L.gamma), L.packed.shape[0], L.K, _ptr(L.x), _ptr(L.y),
+                          _ptr(L.xq), _ptr(L.scale), _ptr(L.rowsum), _ptr(L.acc_out))
     return arr
 
 
@@ -319,13 +395,28 @@ def layer_chain(layers: Sequence[Layer], workspace: torch.Tensor | None = None, 
     """Runs the layers back to back; each writes its ``y``.  Same-x neighbours share one quantisation."""
     if not layers:
         return
-    M = layers[0].x.shape[0]
+    M = layers[0].tokens
     arr = _layer_array(layers)
     if workspace is None:
-        workspace = new_workspace(lib().bitlinear_chain_workspace_bytes(arr, len(layers), M), layers[0].x.device)
-    _check(lib().bitlinear_layer_chain(arr, len(layers), M, _dtype_code(layers[0].x.dtype),
-                                       _dtype_code(layers[0].y.dtype), _ptr(workspace), workspace.numel(),
-                                       _stream(stream)))
+        workspace = cached_workspace(lib().bitlinear_chain_workspace_bytes(arr, len(layers), M), layers[0].y.device,
+                                     stream)
+    x_dtype = next((L.x.dtype for L in layers if L.x is not None), layers[0].y.dtype)
+    _check(lib().bitlinear_layer_chain(arr, len(layers), M, _dtype_code(x_dtype), _dtype_code(layers[0].y.dtype),
+                                       _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def forward_noalloc(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, y: torch.Tensor,
+                    acc_out: torch.Tensor | None = None, stream=None) -> None:
+    """The forward without a workspace (the library's fixed scratch): writes ``y`` (and ``acc_out``)."""
+    N = packed.shape[0]
+    M, K = x.shape
+    _check(lib().bitlinear_forward_noalloc(_ptr(packed), _ptr(gamma), N, K, _ptr(x), _dtype_code(x.dtype), M, _ptr(y),
+                                           _dtype_code(y.dtype), _ptr(acc_out), _stream(stream)))
+
+
+def noalloc_status(stream=None) -> int:
+    """Synchronises and returns BL_OK or BL_ERR_DEVICE_TIMEOUT for the no-allocation calls (clearing it)."""
+    return lib().bitlinear_noalloc_status(_stream(stream))
 
 
 def device_status(workspace: torch.Tensor, stream=None) -> int:

@@ -34,6 +34,8 @@ struct QuantItem {
 struct QuantParams {
   QuantItem item[kQuantMaxItems];
   int n_items;
+  uint4* zero;  // a region to clear (16-byte vectors), or null
+  long long zero_vecs;
 };
 
 struct Chunk16 {
@@ -119,6 +121,13 @@ __global__ void __launch_bounds__(kQuantMaxThreads) act_quant_kernel(const __gri
   griddep_launch_dependents();
   griddep_wait();  // x may be the preceding kernel's output; q may still be read by it
 
+  if (P.zero) {
+    // This block's slice of the region to clear (the following decode launch's split scratch).
+    const long long nb = static_cast<long long>(gridDim.x) * gridDim.y;
+    const long long b = static_cast<long long>(blockIdx.y) * gridDim.x + blockIdx.x;
+    const long long v0 = P.zero_vecs * b / nb, v1 = P.zero_vecs * (b + 1) / nb;
+    for (long long v = v0 + threadIdx.x; v < v1; v += blockDim.x) P.zero[v] = make_uint4(0, 0, 0, 0);
+  }
   const QuantItem& it = P.item[blockIdx.y];
   const int m = blockIdx.x, K = it.K, chunks = K >> 4, T = blockDim.x;
   const TX* xr = static_cast<const TX*>(it.x) + static_cast<size_t>(m) * K;
@@ -347,10 +356,16 @@ __global__ void __launch_bounds__(kQuantMaxThreads) rmsnorm_quant_kernel(const _
   }
 }
 
+static cudaError_t launch_rmsnorm_quant_cluster(const NormParams& P, int M, int x_bf16, cudaStream_t stream, bool pdl,
+                                                bool* done);
+
 cudaError_t launch_rmsnorm_quant(const void* x, int x_bf16, int M, int K, const float* gain, float eps, void* x_norm,
                                  int8_t* xq, float* scale, int32_t* rowsum, cudaStream_t stream, bool pdl) {
   if (M <= 0) return cudaSuccess;
   const NormParams P{x, gain, eps, x_norm, xq, scale, rowsum, K};
+  bool done = false;
+  cudaError_t ce = launch_rmsnorm_quant_cluster(P, M, x_bf16, stream, pdl, &done);
+  if (done || ce != cudaSuccess) return ce;
   int threads = ((K / 16 + 1) / 2 + 31) / 32 * 32;  // about two chunks per thread, 64 .. 512
   if (threads < 64) threads = 64;
   if (threads > kQuantMaxThreads) threads = kQuantMaxThreads;
@@ -456,11 +471,17 @@ __global__ void __launch_bounds__(kQuantMaxThreads) glu_quant_kernel(const __gri
   }
 }
 
+static cudaError_t launch_glu_quant_cluster(const GluParams& P, int M, int x_bf16, cudaStream_t stream, bool pdl,
+                                            bool* done);
+
 cudaError_t launch_glu_quant(const void* gate, const void* up, int x_bf16, int M, int N, int act, void* h,
                              int8_t* xq, float* scale, int32_t* rowsum, cudaStream_t stream, bool pdl) {
   if (M <= 0) return cudaSuccess;
   if (act != kGluRelu2 && act != kGluSilu) return cudaErrorInvalidValue;
   const GluParams P{gate, up, act, h, xq, scale, rowsum, N};
+  bool done = false;
+  cudaError_t ce = launch_glu_quant_cluster(P, M, x_bf16, stream, pdl, &done);
+  if (done || ce != cudaSuccess) return ce;
   int threads = ((N / 16 + 1) / 2 + 31) / 32 * 32;  // about two chunks per thread, 64 .. 512
   if (threads < 64) threads = 64;
   if (threads > kQuantMaxThreads) threads = kQuantMaxThreads;
@@ -468,17 +489,332 @@ cudaError_t launch_glu_quant(const void* gate, const void* up, int x_bf16, int M
   return launch(glu_quant_kernel<float>, dim3(M), dim3(threads), 0, stream, pdl, P);
 }
 
+// ---------------------------------------------------------------------------
+// Decode sizes: a token split over a thread-block cluster
+// ---------------------------------------------------------------------------
+// With few tokens one block per token leaves most SMs idle and serialises a
+// long token through one block's loads and reductions.  Here a cluster of
+// C <= 8 CTAs (128 threads each) shares a token: CTA c takes the contiguous
+// chunk range [c * chunks / C, (c + 1) * chunks / C), its chunks held in
+// registers; each reduction is a block reduction, then the C partial results
+// are read from the CTAs' shared memory (distributed shared memory) after a
+// cluster barrier, every CTA adding them in rank order.  One more barrier at
+// the end keeps every CTA's shared memory alive until its peers have read it.
+constexpr int kClusterThreads = 128;
+constexpr int kClusterMax = 8;
+constexpr int kClusterChunks = 4;  // 16-input chunks per thread, in registers
+
+__device__ __forceinline__ float ld_cluster_f32(const float* p, int rank) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(mapa_shared(smem_u32(p), rank)) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_cluster_s32(const int* p, int rank) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(mapa_shared(smem_u32(p), rank)) : "memory");
+  return v;
+}
+__device__ __forceinline__ double ld_cluster_f64(const double* p, int rank) {
+  double v;
+  asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(mapa_shared(smem_u32(p), rank)) : "memory");
+  return v;
+}
+
+// Cluster-wide reductions; `slot` is a shared variable used by this reduction only.
+__device__ __forceinline__ float cluster_max(float v, float* red, float* slot, int csize) {
+  v = block_reduce(v, [](float a, float b) { return fmaxf(a, b); }, red);
+  if (threadIdx.x == 0) *slot = v;
+  cluster_sync_all();
+  float r = 0.0f;
+  for (int c = 0; c < csize; ++c) r = fmaxf(r, ld_cluster_f32(slot, c));
+  return r;
+}
+__device__ __forceinline__ int cluster_sum(int v, int* red, int* slot, int csize) {
+  v = block_reduce(v, [](int a, int b) { return a + b; }, red);
+  if (threadIdx.x == 0) *slot = v;
+  cluster_sync_all();
+  int r = 0;
+  for (int c = 0; c < csize; ++c) r += ld_cluster_s32(slot, c);
+  return r;
+}
+__device__ __forceinline__ double cluster_sum(double v, double* red, double* slot, int csize) {
+  v = block_reduce(v, [](double a, double b) { return __dadd_rn(a, b); }, red);
+  if (threadIdx.x == 0) *slot = v;
+  cluster_sync_all();
+  double r = 0.0;
+  for (int c = 0; c < csize; ++c) r = __dadd_rn(r, ld_cluster_f64(slot, c));
+  return r;
+}
+
+// The chunk range of cluster rank `rank` (of csize) over `chunks` chunks, and
+// this thread's chunks in it: c0 + threadIdx.x + i * kClusterThreads.
+struct ClusterSlice {
+  int c0, c1;
+};
+__device__ __forceinline__ ClusterSlice cluster_slice(int chunks, int rank, int csize) {
+  return ClusterSlice{static_cast<int>(static_cast<long long>(chunks) * rank / csize),
+                      static_cast<int>(static_cast<long long>(chunks) * (rank + 1) / csize)};
+}
+
+// act_quant over a cluster per (item, token): blockIdx.x = token * C + rank, blockIdx.y = item.
+template <typename TX>
+__global__ void __launch_bounds__(kClusterThreads) act_quant_cluster_kernel(const __grid_constant__ QuantParams P) {
+  __shared__ float red_f[kClusterThreads / 32];
+  __shared__ int red_i[kClusterThreads / 32];
+  __shared__ float slot_max;
+  __shared__ int slot_sum;
+  griddep_launch_dependents();
+  griddep_wait();  // x may be the preceding kernel's output; q may still be read by it
+  const int csize = static_cast<int>(cluster_nctarank());
+  const int rank = static_cast<int>(cluster_ctarank());
+  if (P.zero) {
+    const long long nb = static_cast<long long>(gridDim.x) * gridDim.y;
+    const long long b = static_cast<long long>(blockIdx.y) * gridDim.x + blockIdx.x;
+    const long long v0 = P.zero_vecs * b / nb, v1 = P.zero_vecs * (b + 1) / nb;
+    for (long long v = v0 + threadIdx.x; v < v1; v += blockDim.x) P.zero[v] = make_uint4(0, 0, 0, 0);
+  }
+  const QuantItem& it = P.item[blockIdx.y];
+  const int m = blockIdx.x / csize, K = it.K, chunks = K >> 4;
+  const TX* xr = static_cast<const TX*>(it.x) + static_cast<size_t>(m) * K;
+  int8_t* qr = it.xq + static_cast<size_t>(m) * it.ldq;
+  if (rank == csize - 1)
+    for (int c = K + 16 * threadIdx.x; c < it.ldq; c += 16 * kClusterThreads)  // row padding
+      *reinterpret_cast<uint4*>(qr + c) = make_uint4(0, 0, 0, 0);
+  const ClusterSlice sl = cluster_slice(chunks, rank, csize);
+  Chunk16 reg[kClusterChunks];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kClusterChunks; ++i) {
+    const int c = sl.c0 + threadIdx.x + i * kClusterThreads;
+    if (c < sl.c1) load16<TX>(xr + c * 16, reg[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < kClusterChunks; ++i) {
+    const int c = sl.c0 + threadIdx.x + i * kClusterThreads;
+    if (c < sl.c1) amax = fmaxf(amax, chunk_absmax<TX>(reg[i]));
+  }
+  amax = cluster_max(amax, red_f, &slot_max, csize);
+  const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kClusterChunks; ++i) {
+    const int c = sl.c0 + threadIdx.x + i * kClusterThreads;
+    if (c < sl.c1) sum += quant_chunk<TX>(reg[i], s, qr + c * 16);
+  }
+  sum = cluster_sum(sum, red_i, &slot_sum, csize);
+  if (rank == 0 && threadIdx.x == 0) {
+    it.scale[m] = s;
+    if (it.rowsum) it.rowsum[m] = sum;
+  }
+  cluster_sync_all();  // peers may still read this CTA's slots
+}
+
+// RMSNorm + quantisation over a cluster per token (blockIdx.x = token * C + rank).
+template <typename TX>
+__global__ void __launch_bounds__(kClusterThreads) rmsnorm_quant_cluster_kernel(const __grid_constant__ NormParams P) {
+  __shared__ double red_d[kClusterThreads / 32];
+  __shared__ float red_f[kClusterThreads / 32];
+  __shared__ int red_i[kClusterThreads / 32];
+  __shared__ double slot_ss;
+  __shared__ float slot_max;
+  __shared__ int slot_sum;
+  griddep_launch_dependents();
+  griddep_wait();  // x may be the preceding kernel's output; q may still be read by it
+  const int csize = static_cast<int>(cluster_nctarank());
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int m = blockIdx.x / csize, K = P.K, chunks = K >> 4;
+  const TX* xr = static_cast<const TX*>(P.x) + static_cast<size_t>(m) * K;
+  int8_t* qr = P.xq + static_cast<size_t>(m) * K;
+  TX* nr = P.x_norm ? static_cast<TX*>(P.x_norm) + static_cast<size_t>(m) * K : nullptr;
+  const ClusterSlice sl = cluster_slice(chunks, rank, csize);
+  Chunk16 reg[kClusterChunks];
+#pragma unroll
+  for (int i = 0; i < kClusterChunks; ++i) {
+    const int c = sl.c0 + threadIdx.x + i * kClusterThreads;
+    if (c < sl.c1) load16<TX>(xr + c * 16, reg[i]);
+  }
+  double ss = 0.0;
+#pragma unroll
+  for (int i = 0; i < kClusterChunks; ++i) {
+    const int c = sl.c0 + threadIdx.x + i * kClusterThreads;
+    if (c < sl.c1) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const double v = static_cast<double>(elem<TX>(reg[i], e));
+        ss = __fma_rn(v, v, ss);
+      }
+    }
+  }
+  ss = cluster_sum(ss, red_d, &slot_ss, csize);
+  const double ms = __ddiv_rn(ss, static_cast<double>(K));
+  const float r = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(ms, static_cast<double>(P.eps)))));
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kClusterChunks; ++i) {
+    const int c = sl.c0 + threadIdx.x + i * kClusterThreads;
+    if (c < sl.c1) {
+      float v[16];
+      norm_chunk<TX>(reg[i], r, P.gain, c, v);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
+    }
+  }
+  amax = cluster_max(amax, red_f, &slot_max, csize);
+  const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kClusterChunks; ++i) {
+    const int c = sl.c0 + threadIdx.x + i * kClusterThreads;
+    if (c < sl.c1) {
+      float v[16];
+      norm_chunk<TX>(reg[i], r, P.gain, c, v);
+      sum += quant_store16<TX>(v, s, qr + c * 16, nr ? nr + c * 16 : nullptr);
+    }
+  }
+  sum = cluster_sum(sum, red_i, &slot_sum, csize);
+  if (rank == 0 && threadIdx.x == 0) {
+    P.scale[m] = s;
+    if (P.rowsum) P.rowsum[m] = sum;
+  }
+  cluster_sync_all();  // peers may still read this CTA's slots
+}
+
+// The gated activation + quantisation over a cluster per token.
+template <typename TX>
+__global__ void __launch_bounds__(kClusterThreads) glu_quant_cluster_kernel(const __grid_constant__ GluParams P) {
+  __shared__ float red_f[kClusterThreads / 32];
+  __shared__ int red_i[kClusterThreads / 32];
+  __shared__ float slot_max;
+  __shared__ int slot_sum;
+  griddep_launch_dependents();
+  griddep_wait();  // gate and up are the preceding kernel's outputs
+  const int csize = static_cast<int>(cluster_nctarank());
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int m = blockIdx.x / csize, N = P.N, chunks = N >> 4;
+  const TX* gr = static_cast<const TX*>(P.gate) + static_cast<size_t>(m) * N;
+  const TX* ur = static_cast<const TX*>(P.up) + static_cast<size_t>(m) * N;
+  int8_t* qr = P.xq + static_cast<size_t>(m) * N;
+  TX* hr = P.h ? static_cast<TX*>(P.h) + static_cast<size_t>(m) * N : nullptr;
+  const ClusterSlice sl = cluster_slice(chunks, rank, csize);
+  constexpr int kKeep = 2;  // chunks per thread whose h stays in registers
+  float hk[kKeep][16];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kClusterChunks; ++i) {
+    const int c = sl.c0 + threadIdx.x + i * kClusterThreads;
+    if (c < sl.c1) {
+      Chunk16 g, u;
+      load16<TX>(gr + c * 16, g);
+      load16<TX>(ur + c * 16, u);
+      float h[16];
+      glu_chunk<TX>(g, u, P.act, h);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(h[e]));
+      if (i < kKeep) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) hk[i < kKeep ? i : 0][e] = h[e];
+      }
+    }
+  }
+  amax = cluster_max(amax, red_f, &slot_max, csize);
+  const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kClusterChunks; ++i) {
+    const int c = sl.c0 + threadIdx.x + i * kClusterThreads;
+    if (c < sl.c1) {
+      float h[16];
+      if (i < kKeep) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) h[e] = hk[i < kKeep ? i : 0][e];
+      } else {
+        Chunk16 g, u;
+        load16<TX>(gr + c * 16, g);
+        load16<TX>(ur + c * 16, u);
+        glu_chunk<TX>(g, u, P.act, h);
+      }
+      sum += quant_store16<TX>(h, s, qr + c * 16, hr ? hr + c * 16 : nullptr);
+    }
+  }
+  sum = cluster_sum(sum, red_i, &slot_sum, csize);
+  if (rank == 0 && threadIdx.x == 0) {
+    P.scale[m] = s;
+    if (P.rowsum) P.rowsum[m] = sum;
+  }
+  cluster_sync_all();  // peers may still read this CTA's slots
+}
+
+// CTAs per token for the cluster form (0: use one block per token).  Only
+// tokens longer than one block holds at two chunks per thread (512 threads)
+// gain: below that the cluster's launch and barriers cost more than they save
+// (measured: a one-token RMSNorm at K = 8192 went from 4.3 to 6.7 us as two
+// CTAs, the gated activation at N = 28672 from 7.6 to 5.1 us as seven).
+static int cluster_size_for(int M, int k_max) {
+  const int chunks = k_max / 16;
+  if (M > 16 || chunks <= 2 * kQuantMaxThreads) return 0;
+  int c = (chunks + 2 * kClusterThreads - 1) / (2 * kClusterThreads);  // about two chunks per thread
+  if (c > kClusterMax) c = kClusterMax;
+  if (chunks > c * kClusterThreads * kClusterChunks) return 0;  // does not fit the registers
+  return c;
+}
+
+template <typename Kern, typename Params>
+static cudaError_t launch_cluster(Kern kernel, dim3 grid, int csize, cudaStream_t stream, bool pdl, const Params& P) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kClusterThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(csize);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kernel, P);
+}
+
+static cudaError_t launch_rmsnorm_quant_cluster(const NormParams& P, int M, int x_bf16, cudaStream_t stream, bool pdl,
+                                                bool* done) {
+  const int csize = cluster_size_for(M, P.K);
+  *done = csize > 0;
+  if (csize == 0) return cudaSuccess;
+  if (x_bf16) return launch_cluster(rmsnorm_quant_cluster_kernel<__nv_bfloat16>, dim3(M * csize), csize, stream, pdl, P);
+  return launch_cluster(rmsnorm_quant_cluster_kernel<float>, dim3(M * csize), csize, stream, pdl, P);
+}
+
+static cudaError_t launch_glu_quant_cluster(const GluParams& P, int M, int x_bf16, cudaStream_t stream, bool pdl,
+                                            bool* done) {
+  const int csize = cluster_size_for(M, P.N);
+  *done = csize > 0;
+  if (csize == 0) return cudaSuccess;
+  if (x_bf16) return launch_cluster(glu_quant_cluster_kernel<__nv_bfloat16>, dim3(M * csize), csize, stream, pdl, P);
+  return launch_cluster(glu_quant_cluster_kernel<float>, dim3(M * csize), csize, stream, pdl, P);
+}
+
 cudaError_t launch_act_quant_group(const QuantArgs* items, int n_items, int M, int x_bf16, cudaStream_t stream,
-                                   bool pdl) {
+                                   bool pdl, void* zero, size_t zero_bytes) {
   if (M <= 0 || n_items <= 0) return cudaSuccess;
   if (n_items > kQuantMaxItems) return cudaErrorInvalidValue;
+  if ((reinterpret_cast<uintptr_t>(zero) | zero_bytes) % 16 != 0) return cudaErrorInvalidValue;
   QuantParams P = {};
+  P.zero = zero_bytes ? static_cast<uint4*>(zero) : nullptr;
+  P.zero_vecs = static_cast<long long>(zero_bytes / 16);
   int k_max = 0;
   for (int i = 0; i < n_items; ++i) {
     P.item[i] = QuantItem{items[i].x, items[i].xq, items[i].scale, items[i].rowsum, items[i].K, items[i].ldq};
     if (items[i].K > k_max) k_max = items[i].K;
   }
   P.n_items = n_items;
+  const int csize = cluster_size_for(M, k_max);
+  if (csize > 0) {
+    const dim3 grid(M * csize, n_items);
+    if (x_bf16) return launch_cluster(act_quant_cluster_kernel<__nv_bfloat16>, grid, csize, stream, pdl, P);
+    return launch_cluster(act_quant_cluster_kernel<float>, grid, csize, stream, pdl, P);
+  }
   // About two chunks per thread, in whole warps, 64 .. 512 threads.
   int threads = ((k_max / 16 + 1) / 2 + 31) / 32 * 32;
   if (threads < 64) threads = 64;
@@ -489,9 +825,9 @@ cudaError_t launch_act_quant_group(const QuantArgs* items, int n_items, int M, i
 }
 
 cudaError_t launch_act_quant(const void* x, int x_bf16, int M, int K, int ldq, int8_t* xq, float* scale,
-                             int32_t* rowsum, cudaStream_t stream, bool pdl) {
+                             int32_t* rowsum, cudaStream_t stream, bool pdl, void* zero, size_t zero_bytes) {
   const QuantArgs a{x, xq, scale, rowsum, K, ldq};
-  return launch_act_quant_group(&a, 1, M, x_bf16, stream, pdl);
+  return launch_act_quant_group(&a, 1, M, x_bf16, stream, pdl, zero, zero_bytes);
 }
 
 }  // namespace bl

@@ -1,6 +1,7 @@
 // C ABI of the BitLinear W1.58A8 forward: argument checks, workspace layout,
 // dispatch to the kernels, and the layer chain.  The declarations and their
 // contracts are in include/bitlinear.h.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdarg.h>
@@ -199,6 +200,13 @@ int bitlinear_pack_weights(const float* W, int N, int K, uint8_t* packed, float*
   if (e != cudaSuccess) return cuda_fail(e, "gamma launch");
   e = bl::launch_ternary_pack(W, N, K, gamma, packed, s);
   if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  // The forward kernels start loading packed weights before waiting for the
+  // kernel before them (programmatic dependent launch), which makes only that
+  // kernel's writes visible after the wait.  A stream operation that is not a
+  // kernel ends the pack (rewriting the status word's zero), so the next
+  // kernel on the stream starts only once the packed weights are complete.
+  e = cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s);
+  if (e != cudaSuccess) return cuda_fail(e, "pack completion");
   return BL_OK;
 }
 
@@ -318,6 +326,12 @@ size_t bitlinear_workspace_bytes(int M, int N, int K) {
   return forward_layout(M, K).total;
 }
 
+int bitlinear_set_decode_split(int ctas) {
+  if (ctas < 0 || ctas > 8) return fail(BL_ERR_INVALID_ARG, "ctas = %d not in [0, 8]", ctas);
+  bl::gemv_force_ksplit(ctas);
+  return BL_OK;
+}
+
 int bitlinear_forward_quantized(const uint8_t* packed, const float* gamma, int N, int K,
                                 const int8_t* xq, const float* scale, const int32_t* rowsum,
                                 int M, void* y, int y_dtype, int32_t* acc_out, void* workspace,
@@ -354,6 +368,36 @@ int bitlinear_forward_quantized(const uint8_t* packed, const float* gamma, int N
   return launch_gemm_q(packed, gamma, N, K, M, xq, K, scale, rowsum, y, y_dtype, acc_out, status, s);
 }
 
+// The forward on a caller-supplied scratch laid out as forward_layout(M, K)
+// (the status block included).
+static int forward_on(const uint8_t* packed, const float* gamma, int N, int K, const void* x, int x_dtype, int M,
+                      void* y, int y_dtype, int32_t* acc_out, uint8_t* ws, cudaStream_t s) {
+  const FwdLayout l = forward_layout(M, K);
+  bool gemv = false;
+  BL_TRY(choose_gemv(M, K, &gemv));
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  const int yt = y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32;
+  if (gemv && bl::gemv_fuses_quant(M, K, x_dtype == BL_BF16)) {
+    // Small activations: the decode kernel quantises them itself (one launch).
+    const bl::GemvLayerArgs L{packed, gamma, N, K, x, nullptr, nullptr, 0, y, acc_out};
+    cudaError_t e = bl::launch_gemv_group(&L, 1, M, x_dtype == BL_BF16 ? bl::kInBF16 : bl::kInF32, yt, status,
+                                          tickets_of(ws), s, true);
+    return e == cudaSuccess ? BL_OK : gemv_fail(e);
+  }
+  int8_t* xq = reinterpret_cast<int8_t*>(ws + l.xq);
+  float* scale = reinterpret_cast<float*>(ws + l.scale);
+  int32_t* rowsum = reinterpret_cast<int32_t*>(ws + l.rowsum);
+  const int ldq = code_pitch(K);
+  cudaError_t e = bl::launch_act_quant(x, x_dtype == BL_BF16, M, K, ldq, xq, scale, rowsum, s, true);
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+  if (gemv) {
+    const bl::GemvLayerArgs L{packed, gamma, N, K, xq, scale, rowsum, ldq, y, acc_out};
+    e = bl::launch_gemv_group(&L, 1, M, bl::kInInt8, yt, status, tickets_of(ws), s, true);
+    return e == cudaSuccess ? BL_OK : gemv_fail(e);
+  }
+  return launch_gemm_q(packed, gamma, N, K, M, xq, ldq, scale, rowsum, y, y_dtype, acc_out, status, s);
+}
+
 int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, const void* x,
                       int x_dtype, int M, void* y, int y_dtype, int32_t* acc_out, void* workspace,
                       size_t workspace_bytes, void* stream) {
@@ -371,34 +415,11 @@ int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, c
   const FwdLayout l = forward_layout(M, K);
   if (workspace_bytes < l.total)
     return fail(BL_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, l.total);
-  bool gemv = false;
-  BL_TRY(choose_gemv(M, K, &gemv));
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int yt = y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32;
-  if (gemv && bl::gemv_fuses_quant(M, K, x_dtype == BL_BF16)) {
-    // Small activations: the decode kernel quantises them itself (one launch).
-    const bl::GemvLayerArgs L{packed, gamma, N, K, x, nullptr, nullptr, 0, y, acc_out};
-    cudaError_t e = bl::launch_gemv_group(&L, 1, M, x_dtype == BL_BF16 ? bl::kInBF16 : bl::kInF32, yt, status,
-                                          tickets_of(workspace), s, true);
-    return e == cudaSuccess ? BL_OK : gemv_fail(e);
-  }
-  int8_t* xq = reinterpret_cast<int8_t*>(ws + l.xq);
-  float* scale = reinterpret_cast<float*>(ws + l.scale);
-  int32_t* rowsum = reinterpret_cast<int32_t*>(ws + l.rowsum);
-  const int ldq = code_pitch(K);
-  cudaError_t e = bl::launch_act_quant(x, x_dtype == BL_BF16, M, K, ldq, xq, scale, rowsum, s, true);
-  if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
-  if (gemv) {
-    const bl::GemvLayerArgs L{packed, gamma, N, K, xq, scale, rowsum, ldq, y, acc_out};
-    e = bl::launch_gemv_group(&L, 1, M, bl::kInInt8, yt, status, tickets_of(workspace), s, true);
-    return e == cudaSuccess ? BL_OK : gemv_fail(e);
-  }
-  return launch_gemm_q(packed, gamma, N, K, M, xq, ldq, scale, rowsum, y, y_dtype, acc_out, status, s);
+  return forward_on(packed, gamma, N, K, x, x_dtype, M, y, y_dtype, acc_out, static_cast<uint8_t*>(workspace),
+                    static_cast<cudaStream_t>(stream));
 }
 
-// Every layer of a chain has its own activation region (the layers of one
+// Every layer of a chain has its own region of codes (the layers of one
 // decode group are live together): status block, then per layer q, s, rowsum.
 static size_t chain_region_bytes(int M, int K) { return forward_layout(M, K).total - kStatusBytes; }
 
@@ -422,14 +443,22 @@ int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dty
   BL_TRY(check_dtype(y_dtype, "y_dtype"));
   if (M < 0) return fail(BL_ERR_INVALID_ARG, "M = %d < 0", M);
   if (M == 0 || n_layers == 0) return BL_OK;
+  if (n_layers > 64) return fail(BL_ERR_INVALID_ARG, "n_layers = %d > 64", n_layers);
   BL_TRY(check_ptr(workspace, "workspace", 256));
   for (int i = 0; i < n_layers; ++i) {
     const bl_layer& L = layers[i];
     BL_TRY(check_nk(L.N, L.K));
     BL_TRY(check_ptr(L.packed, "layer.packed", 16));
     BL_TRY(check_ptr(L.gamma, "layer.gamma", 4));
-    BL_TRY(check_ptr(L.x, "layer.x", 16));
+    if (L.xq) {
+      BL_TRY(check_ptr(L.xq, "layer.xq", 16));
+      BL_TRY(check_ptr(L.scale, "layer.scale", 4));
+      BL_TRY(check_ptr(L.rowsum, "layer.rowsum", 4));
+    } else {
+      BL_TRY(check_ptr(L.x, "layer.x", 16));
+    }
     BL_TRY(check_ptr(L.y, "layer.y", 16));
+    BL_TRY(check_ptr(L.acc_out, "layer.acc_out", 16, true));
   }
   const size_t need = bitlinear_chain_workspace_bytes(layers, n_layers, M);
   if (workspace_bytes < need)
@@ -441,9 +470,8 @@ int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dty
   const size_t xsz = x_bf16 ? 2 : 4, ysz = y_dtype == BL_BF16 ? 2 : 4;
   const int yt = y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32;
 
-  // Activation region of each layer.
+  // Region of each layer.
   size_t off[64];
-  if (n_layers > 64) return fail(BL_ERR_INVALID_ARG, "n_layers = %d > 64", n_layers);
   {
     size_t o = kStatusBytes;
     for (int i = 0; i < n_layers; ++i) {
@@ -457,54 +485,89 @@ int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dty
     *sc = reinterpret_cast<float*>(ws + off[i] + (l.scale - kStatusBytes));
     *rs = reinterpret_cast<int32_t*>(ws + off[i] + (l.rowsum - kStatusBytes));
   };
-  // quant_src[i]: the layer whose region holds layer i's quantised input.
+  // The codes of layer i: the caller's, or those quantised into a region.
+  // quant_src[i]: the layer whose region holds layer i's quantised input (-1: the caller's codes).
   int quant_src[64];
-  for (int i = 0; i < n_layers; ++i) quant_src[i] = -1;
-  auto quantise = [&](int i) -> int {
+  for (int i = 0; i < n_layers; ++i) quant_src[i] = -2;
+  auto codes_of = [&](int i, const int8_t** xq, const float** sc, const int32_t** rs, int* ld) {
+    if (layers[i].xq) {
+      *xq = layers[i].xq;
+      *sc = layers[i].scale;
+      *rs = layers[i].rowsum;
+      *ld = layers[i].K;
+      return;
+    }
+    int8_t* q;
+    float* c;
+    int32_t* r;
+    region(quant_src[i], &q, &c, &r);
+    *xq = q;
+    *sc = c;
+    *rs = r;
+    *ld = code_pitch(layers[i].K);
+  };
+  // Same input already quantised earlier in this call?
+  auto shared_src = [&](int i) -> int {
     for (int j = 0; j < i; ++j)
-      if (quant_src[j] == j && layers[j].x == layers[i].x && layers[j].K == layers[i].K) {
-        quant_src[i] = j;  // same input already quantised earlier in this call
-        return BL_OK;
-      }
-    int8_t* xq;
-    float* sc;
-    int32_t* rsum;
-    region(i, &xq, &sc, &rsum);
-    cudaError_t e = bl::launch_act_quant(layers[i].x, x_bf16, M, layers[i].K, code_pitch(layers[i].K), xq, sc, rsum,
-                                         s, true);
-    if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
-    quant_src[i] = i;
-    return BL_OK;
+      if (quant_src[j] == j && !layers[j].xq && layers[j].x == layers[i].x && layers[j].K == layers[i].K) return j;
+    return i;
   };
 
   int i = 0;
   while (i < n_layers) {
     bool gemv = false;
     BL_TRY(choose_gemv(M, layers[i].K, &gemv));
+    // Caller codes reach the decode kernel only in 128-byte blocks.
+    if (gemv && layers[i].xq && layers[i].K % 128 != 0) gemv = false;
     if (!gemv) {
-      BL_TRY(quantise(i));
-      int8_t* xq;
-      float* sc;
-      int32_t* rsum;
-      region(quant_src[i], &xq, &sc, &rsum);
-      BL_TRY(launch_gemm_q(layers[i].packed, layers[i].gamma, layers[i].N, layers[i].K, M, xq,
-                           code_pitch(layers[i].K), sc, rsum, layers[i].y, y_dtype, nullptr, status, s));
+      if (!layers[i].xq) {
+        quant_src[i] = shared_src(i);
+        if (quant_src[i] == i) {
+          int8_t* xq;
+          float* sc;
+          int32_t* rsum;
+          region(i, &xq, &sc, &rsum);
+          cudaError_t e = bl::launch_act_quant(layers[i].x, x_bf16, M, layers[i].K, code_pitch(layers[i].K), xq, sc,
+                                               rsum, s, true);
+          if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+        }
+      }
+      const int8_t* xq;
+      const float* sc;
+      const int32_t* rsum;
+      int ld;
+      codes_of(i, &xq, &sc, &rsum, &ld);
+      BL_TRY(launch_gemm_q(layers[i].packed, layers[i].gamma, layers[i].N, layers[i].K, M, xq, ld, sc, rsum,
+                           layers[i].y, y_dtype, layers[i].acc_out, status, s));
       ++i;
       continue;
     }
     // A decode group: following layers that also take the GEMV path the same way
     // and neither read what the group writes nor write what it reads.
-    const bool fused = bl::gemv_fuses_quant(M, layers[i].K, x_bf16);
+    auto fused_of = [&](int k) { return !layers[k].xq && bl::gemv_fuses_quant(M, layers[k].K, x_bf16); };
+    const bool fused = fused_of(i);
     int j = i + 1;
     while (j < n_layers && j - i < bl::kGvMaxLayers) {
       bool gj = false;
       if (choose_gemv(M, layers[j].K, &gj) != BL_OK || !gj) break;
-      if (bl::gemv_fuses_quant(M, layers[j].K, x_bf16) != fused) break;
+      if (layers[j].xq && layers[j].K % 128 != 0) break;
+      if (fused_of(j) != fused) break;
+      // Input (activations or caller codes) and output byte ranges of a layer.
+      auto in_of = [&](int k, const void** p, size_t* n) {
+        *p = layers[k].xq ? static_cast<const void*>(layers[k].xq) : layers[k].x;
+        *n = static_cast<size_t>(M) * layers[k].K * (layers[k].xq ? 1 : xsz);
+      };
       bool independent = true;
-      const size_t xj = static_cast<size_t>(M) * layers[j].K * xsz, yj = static_cast<size_t>(M) * layers[j].N * ysz;
+      const void* xj;
+      size_t nxj;
+      in_of(j, &xj, &nxj);
+      const size_t yj = static_cast<size_t>(M) * layers[j].N * ysz;
       for (int k = i; k < j && independent; ++k) {
-        const size_t xk = static_cast<size_t>(M) * layers[k].K * xsz, yk = static_cast<size_t>(M) * layers[k].N * ysz;
-        if (ranges_overlap(layers[j].x, xj, layers[k].y, yk) || ranges_overlap(layers[j].y, yj, layers[k].x, xk) ||
+        const void* xk;
+        size_t nxk;
+        in_of(k, &xk, &nxk);
+        const size_t yk = static_cast<size_t>(M) * layers[k].N * ysz;
+        if (ranges_overlap(xj, nxj, layers[k].y, yk) || ranges_overlap(layers[j].y, yj, xk, nxk) ||
             ranges_overlap(layers[j].y, yj, layers[k].y, yk))
           independent = false;
       }
@@ -512,36 +575,35 @@ int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dty
       ++j;
     }
     bl::GemvLayerArgs args[bl::kGvMaxLayers];
-    if (!fused) {
-      // Quantise the group's distinct inputs once, in one launch.
-      bl::QuantArgs qa[bl::kGvMaxLayers];
-      int nq = 0;
-      for (int k = i; k < j; ++k) {
-        int src = k;
-        for (int p = 0; p < k; ++p)
-          if (quant_src[p] == p && layers[p].x == layers[k].x && layers[p].K == layers[k].K) { src = p; break; }
-        quant_src[k] = src;
-        if (src == k) {
-          int8_t* xq;
-          float* sc;
-          int32_t* rsum;
-          region(k, &xq, &sc, &rsum);
-          qa[nq++] = bl::QuantArgs{layers[k].x, xq, sc, rsum, layers[k].K, code_pitch(layers[k].K)};
-        }
-      }
-      cudaError_t e = bl::launch_act_quant_group(qa, nq, M, x_bf16, s, true);
-      if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
-    }
     for (int k = i; k < j; ++k) {
       const bl_layer& L = layers[k];
       if (fused) {
-        args[k - i] = bl::GemvLayerArgs{L.packed, L.gamma, L.N, L.K, L.x, nullptr, nullptr, 0, L.y, nullptr};
+        args[k - i] = bl::GemvLayerArgs{L.packed, L.gamma, L.N, L.K, L.x, nullptr, nullptr, 0, L.y, L.acc_out};
       } else {
+        if (!L.xq) quant_src[k] = shared_src(k);
+        const int8_t* xq;
+        const float* sc;
+        const int32_t* rsum;
+        int ld;
+        codes_of(k, &xq, &sc, &rsum, &ld);
+        args[k - i] = bl::GemvLayerArgs{L.packed, L.gamma, L.N, L.K, xq, sc, rsum, ld, L.y, L.acc_out};
+      }
+    }
+    if (!fused) {
+      // Quantise the group's distinct raw inputs once, in one launch.
+      bl::QuantArgs qa[bl::kGvMaxLayers];
+      int nq = 0;
+      for (int k = i; k < j; ++k) {
+        if (layers[k].xq || quant_src[k] != k) continue;
         int8_t* xq;
         float* sc;
         int32_t* rsum;
-        region(quant_src[k], &xq, &sc, &rsum);
-        args[k - i] = bl::GemvLayerArgs{L.packed, L.gamma, L.N, L.K, xq, sc, rsum, code_pitch(L.K), L.y, nullptr};
+        region(k, &xq, &sc, &rsum);
+        qa[nq++] = bl::QuantArgs{layers[k].x, xq, sc, rsum, layers[k].K, code_pitch(layers[k].K)};
+      }
+      if (nq > 0) {
+        cudaError_t e = bl::launch_act_quant_group(qa, nq, M, x_bf16, s, true);
+        if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
       }
     }
     const int xt = fused ? (x_bf16 ? bl::kInBF16 : bl::kInF32) : bl::kInInt8;
@@ -549,6 +611,113 @@ int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dty
     if (e != cudaSuccess) return gemv_fail(e);
     i = j;
   }
+  return BL_OK;
+}
+
+// ---------------------------------------------------------------------------
+// The FFN's gate and up BitLinears with the gated activation and the down
+// BitLinear's input quantisation.  Workspace: status block, the codes of x,
+// the gate and up outputs y_g, y_u [M][N] and h [M][N] (elements of 4 bytes
+// at most, each region 256-rounded), then (decode sizes) the fused launch's
+// counters, zeroed before it.
+// ---------------------------------------------------------------------------
+struct GluLayout {
+  size_t yg, yu, h, zero, total;
+};
+
+static GluLayout glu_layout(int M, int N, int K) {
+  GluLayout g;
+  const FwdLayout f = forward_layout(M, K);
+  const size_t act = round_up(static_cast<size_t>(M) * N * 4, 256);
+  g.yg = f.total;
+  g.yu = g.yg + act;
+  g.h = g.yu + act;
+  g.zero = g.h + act;
+  g.total = g.zero + (M >= 1 && M <= 16 ? bl::gemv_glu_scratch_bytes(N) : 0);
+  return g;
+}
+
+size_t bitlinear_gate_up_glu_workspace_bytes(int M, int N, int K) {
+  if (M < 0 || N < 0 || K < 0) return 0;
+  return glu_layout(M, N, K).total;
+}
+
+int bitlinear_gate_up_glu(const uint8_t* packed_gate, const float* gamma_gate, const uint8_t* packed_up,
+                          const float* gamma_up, int N, int K, const void* x, int x_dtype, int M, int act, void* h,
+                          int8_t* xq, float* scale, int32_t* rowsum, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  BL_TRY(check_nk(N, K));
+  if (N % 64 != 0) return fail(BL_ERR_UNSUPPORTED_SHAPE, "N = %d: h is the down BitLinear's input, N %% 64 == 0", N);
+  BL_TRY(check_dtype(x_dtype, "x_dtype"));
+  if (act != BL_GLU_RELU2 && act != BL_GLU_SILU) return fail(BL_ERR_INVALID_ARG, "act = %d: unknown", act);
+  if (M < 0) return fail(BL_ERR_INVALID_ARG, "M = %d < 0", M);
+  if (M == 0) return BL_OK;
+  BL_TRY(check_ptr(packed_gate, "packed_gate", 16));
+  BL_TRY(check_ptr(gamma_gate, "gamma_gate", 4));
+  BL_TRY(check_ptr(packed_up, "packed_up", 16));
+  BL_TRY(check_ptr(gamma_up, "gamma_up", 4));
+  BL_TRY(check_ptr(x, "x", 16));
+  BL_TRY(check_ptr(h, "h", 16, true));
+  BL_TRY(check_ptr(xq, "xq", 16));
+  BL_TRY(check_ptr(scale, "scale", 4));
+  BL_TRY(check_ptr(rowsum, "rowsum", 4));
+  BL_TRY(check_ptr(workspace, "workspace", 256));
+  const GluLayout g = glu_layout(M, N, K);
+  if (workspace_bytes < g.total)
+    return fail(BL_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, g.total);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool x_bf16 = x_dtype == BL_BF16;
+  const int at = x_bf16 ? bl::kOutBF16 : bl::kOutF32;  // gate/up outputs and h in the activation type
+  void* yg = ws + g.yg;
+  void* yu = ws + g.yu;
+  void* hh = h ? h : static_cast<void*>(ws + g.h);
+  const FwdLayout f = forward_layout(M, K);
+  int8_t* cq = reinterpret_cast<int8_t*>(ws + f.xq);
+  float* cs = reinterpret_cast<float*>(ws + f.scale);
+  int32_t* cr = reinterpret_cast<int32_t*>(ws + f.rowsum);
+  const int ldq = code_pitch(K);
+  bool gemv = false;
+  BL_TRY(choose_gemv(M, K, &gemv));
+  if (gemv) {
+    // One decode launch: gate, up, h and its codes (after the quantisation of x,
+    // which also clears the launch's counters).
+    const bool fused = bl::gemv_fuses_quant(M, K, x_bf16);
+    bl::GemvLayerArgs L[2];
+    if (fused) {
+      L[0] = bl::GemvLayerArgs{packed_gate, gamma_gate, N, K, x, nullptr, nullptr, 0, yg, nullptr};
+      L[1] = bl::GemvLayerArgs{packed_up, gamma_up, N, K, x, nullptr, nullptr, 0, yu, nullptr};
+    } else {
+      L[0] = bl::GemvLayerArgs{packed_gate, gamma_gate, N, K, cq, cs, cr, ldq, yg, nullptr};
+      L[1] = bl::GemvLayerArgs{packed_up, gamma_up, N, K, cq, cs, cr, ldq, yu, nullptr};
+    }
+    cudaError_t e;
+    if (fused) {
+      e = cudaMemsetAsync(ws + g.zero, 0, g.total - g.zero, s);
+      if (e != cudaSuccess) return cuda_fail(e, "clearing the fused launch's counters");
+    } else {
+      e = bl::launch_act_quant(x, x_bf16, M, K, ldq, cq, cs, cr, s, true, ws + g.zero, g.total - g.zero);
+      if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+    }
+    const bl::GemvGluArgs G{act == BL_GLU_RELU2 ? bl::kGluRelu2 : bl::kGluSilu, hh, xq, scale, rowsum,
+                            reinterpret_cast<uint32_t*>(ws + g.zero)};
+    e = bl::launch_gemv_group(L, 2, M, fused ? (x_bf16 ? bl::kInBF16 : bl::kInF32) : bl::kInInt8, at, status,
+                              tickets_of(ws), s, true, &G);
+    return e == cudaSuccess ? BL_OK : gemv_fail(e);
+  }
+  // Many tokens: the quantisation of x, one tensor-core GEMM over the gate and
+  // up weights whose epilogue writes h, then the quantisation of h.
+  cudaError_t e = bl::launch_act_quant(x, x_bf16, M, K, ldq, cq, cs, cr, s, true);
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+  bl::ProductArgs a{packed_gate, gamma_gate, N, K, M, cq, ldq, cs, cr, hh, at, nullptr, status};
+  a.packed2 = packed_up;
+  a.gamma2 = gamma_up;
+  a.glu_act = act == BL_GLU_RELU2 ? bl::kGluRelu2 : bl::kGluSilu;
+  e = bl::launch_gemm(a, s, true);
+  if (e != cudaSuccess) return cuda_fail(e, "GEMM launch (gate and up with the gated activation)");
+  e = bl::launch_act_quant(hh, x_bf16, M, N, N, xq, scale, rowsum, s, true);
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant launch (h)");
   return BL_OK;
 }
 
@@ -608,23 +777,56 @@ constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB
 // never an address to give a kernel; noalloc_scratch() looks the address up.
 __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Identity of the current context (0 if the driver cannot tell): the cached
+// address is valid only in the context it was looked up in, and a device
+// reset or a released primary context gives the device a new one.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    looked_up = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, &id) == CUDA_SUCCESS) return id;
+  return 0;
+}
+
 std::mutex g_noalloc_mutex;
 void* g_noalloc_ptr[64] = {nullptr};
+unsigned long long g_noalloc_ctx[64] = {0};
 
 // Device address of the scratch on the current device: looked up once per
-// device, with that device current, then cached.
+// device and context, with that device current, then cached.  (Before the
+// first CUDA call of the process no context is current yet; the lookup then
+// creates it and is repeated once on the next call, under its identity.)
 int noalloc_scratch(uint8_t** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= 64) return fail(BL_ERR_CUDA, "device index %d out of range", dev);
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_ptr[dev]) {
+  if (!g_noalloc_ptr[dev] || ctx == 0 || g_noalloc_ctx[dev] != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
     if (p == nullptr) return fail(BL_ERR_CUDA, "cudaGetSymbolAddress(scratch) returned NULL");
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = ctx;
   }
   *out = static_cast<uint8_t*>(g_noalloc_ptr[dev]);
   return BL_OK;
@@ -645,38 +847,40 @@ extern "C" int bitlinear_forward_noalloc(const uint8_t* packed, const float* gam
   BL_TRY(check_ptr(x, "x", 16));
   BL_TRY(check_ptr(y, "y", 16));
   BL_TRY(check_ptr(acc_out, "acc_out", 16, true));
-  // Same layout as a bitlinear_forward workspace: control block, then q, s, rowsum.
+  // Same layout as a bitlinear_forward workspace: control block, then q, s,
+  // rowsum.  What the call needs depends on its path: the decode kernel
+  // quantising in-kernel needs only the control block, the others the codes too.
   const FwdLayout l = forward_layout(M, K);
-  if (l.total > kNoAllocScratchBytes)
+  bool gemv = false;
+  BL_TRY(choose_gemv(M, K, &gemv));
+  const bool fused = gemv && bl::gemv_fuses_quant(M, K, x_dtype == BL_BF16);
+  const size_t need = fused ? kStatusBytes : l.total;
+  if (need > kNoAllocScratchBytes)
     return fail(BL_ERR_WORKSPACE_TOO_SMALL,
                 "M = %d, K = %d needs %zu bytes of scratch but the fixed scratch holds %zu; "
                 "use bitlinear_forward with a workspace",
-                M, K, l.total, kNoAllocScratchBytes);
+                M, K, need, kNoAllocScratchBytes);
   uint8_t* scratch = nullptr;
   BL_TRY(noalloc_scratch(&scratch));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(scratch, 0, kStatusBytes, s);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the scratch control block");
-  bool gemv = false;
-  BL_TRY(choose_gemv(M, K, &gemv));
-  uint32_t* status = reinterpret_cast<uint32_t*>(scratch);
-  const int yt = y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32;
-  if (gemv && bl::gemv_fuses_quant(M, K, x_dtype == BL_BF16)) {
-    const bl::GemvLayerArgs L{packed, gamma, N, K, x, nullptr, nullptr, 0, y, acc_out};
-    e = bl::launch_gemv_group(&L, 1, M, x_dtype == BL_BF16 ? bl::kInBF16 : bl::kInF32, yt, status,
-                              tickets_of(scratch), s, true);
-    return e == cudaSuccess ? BL_OK : gemv_fail(e);
+  return forward_on(packed, gamma, N, K, x, x_dtype, M, y, y_dtype, acc_out, scratch, s);
+}
+
+extern "C" int bitlinear_noalloc_status(void* stream) {
+  uint8_t* scratch = nullptr;
+  BL_TRY(noalloc_scratch(&scratch));
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  uint32_t word = 0;
+  e = cudaMemcpy(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (word != 0) {
+    e = cudaMemset(scratch, 0, sizeof(word));
+    if (e != cudaSuccess) return cuda_fail(e, "status clear");
+    return fail(BL_ERR_DEVICE_TIMEOUT, "a device-side wait of a no-allocation call ran out of time (status 0x%x)",
+                word);
   }
-  int8_t* xq = reinterpret_cast<int8_t*>(scratch + l.xq);
-  float* scale = reinterpret_cast<float*>(scratch + l.scale);
-  int32_t* rowsum = reinterpret_cast<int32_t*>(scratch + l.rowsum);
-  const int ldq = code_pitch(K);
-  e = bl::launch_act_quant(x, x_dtype == BL_BF16, M, K, ldq, xq, scale, rowsum, s, true);
-  if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
-  if (gemv) {
-    const bl::GemvLayerArgs L{packed, gamma, N, K, xq, scale, rowsum, ldq, y, acc_out};
-    e = bl::launch_gemv_group(&L, 1, M, bl::kInInt8, yt, status, tickets_of(scratch), s, true);
-    return e == cudaSuccess ? BL_OK : gemv_fail(e);
-  }
-  return launch_gemm_q(packed, gamma, N, K, M, xq, ldq, scale, rowsum, y, y_dtype, acc_out, status, s);
+  return BL_OK;
 }

@@ -5,6 +5,7 @@
 // instructions, plus the workspace status word that bounded waits report to.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -259,6 +260,11 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
 
 // The shared::cluster address of `addr` (a shared::cta address of this CTA's
 // layout) in the CTA of the cluster with the given rank.
@@ -353,6 +359,35 @@ __device__ __forceinline__ void tc_commit_pair_mc(uint32_t bar, uint16_t cta_mas
           bar),
       "h"(cta_mask)
       : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// The FFN's gated activation
+// ---------------------------------------------------------------------------
+// h = act(g) * u in fp32 on the stored gate and up values, rounded to the
+// activation type TY: act 0 (squared ReLU) as (p * p) * u with p = max(g, 0),
+// act 1 (SiLU) as g / (1 + e^-g) * u.
+template <typename TY>
+__device__ __forceinline__ float glu_value(float g, float u, int act) {
+  float t;
+  if (act == 0) {
+    const float p = g > 0.0f ? g : 0.0f;
+    t = __fmul_rn(__fmul_rn(p, p), u);
+  } else {
+    t = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+  }
+  if constexpr (sizeof(TY) == 2) t = __uint_as_float(static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(t))) << 16);
+  return t;
+}
+
+// A value rounded to TY (bf16 or fp32), returned as fp32.
+template <typename TY>
+__device__ __forceinline__ float round_to(float v) {
+  if constexpr (sizeof(TY) == 2) {
+    return __uint_as_float(static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v))) << 16);
+  } else {
+    return v;
+  }
 }
 
 // ---------------------------------------------------------------------------

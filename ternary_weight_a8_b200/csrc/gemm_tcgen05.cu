@@ -174,6 +174,33 @@ __device__ __forceinline__ void stage_y(uint8_t* buf, int lane, const uint32_t (
   }
 }
 
+// Output values already computed in fp32 (held as bits): a staged box, or direct stores.
+template <typename TY>
+__device__ __forceinline__ void stage_vals(uint8_t* buf, int lane, const uint32_t (&v)[32]) {
+  if constexpr (sizeof(TY) == 2) {
+    uint32_t p[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      p[i] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[2 * i])))) |
+             (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[2 * i + 1])))) << 16);
+    stage_box_b16(buf, lane, p);
+  } else {
+    stage_box_b32(buf, lane, v);
+  }
+}
+
+template <typename TY>
+__device__ __forceinline__ void store_vals32(TY* __restrict__ y, size_t row_off, int n0, int N, const uint32_t (&v)[32]) {
+  for (int i = 0; i < 32; ++i)
+    if (n0 + i < N) {
+      if constexpr (sizeof(TY) == 2) {
+        y[row_off + n0 + i] = __float2bfloat16_rn(__uint_as_float(v[i]));
+      } else {
+        y[row_off + n0 + i] = __uint_as_float(v[i]);
+      }
+    }
+}
+
 // Bounded wait for the GEMM: as mbar_wait, and in the pair form a wait that
 // gives up raises the abort flag of the peer CTA too.
 template <int CG>
@@ -212,10 +239,22 @@ __device__ __forceinline__ void commit_to(uint32_t bar) {
   }
 }
 
+// The FFN's gate and up products in one GEMM (glu_act >= 0): a tile holds
+// 128 rows of the gate weights (tmap_b) in accumulator columns 0..127 and the
+// same 128 rows of the up weights (tmap_b2) in columns 128..255 (in the pair
+// form the even CTA loads the gate half, the odd one the up half), and the
+// epilogue stores h = act(gate) * up (each output rounded to TY first, as
+// stored BitLinear outputs are, then h rounded to TY) instead of y.
+struct GemmGlu {
+  int act;              // -1: plain GEMM; else the GluAct of h
+  const float* gamma2;  // the up BitLinear's gamma
+};
+
 template <typename TY, int CG>
 __global__ void __maxnreg__(128) gemm_kernel(
     const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-    const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_acc, int tma_out,
+    const __grid_constant__ CUtensorMap tmap_b2, const __grid_constant__ CUtensorMap tmap_y,
+    const __grid_constant__ CUtensorMap tmap_acc, int tma_out, const GemmGlu glu,
     const float* __restrict__ gamma_ptr, int N, int K, int M, const float* __restrict__ scale,
     const int32_t* __restrict__ rowsum, TY* __restrict__ y, int32_t* __restrict__ acc_out,
     uint32_t* status) {
@@ -262,8 +301,12 @@ __global__ void __maxnreg__(128) gemm_kernel(
     *never = 0;
     fence_barrier_init();
   }
+  const bool is_glu = glu.act >= 0;
   if (warp == 0 && lane == 0) tma_prefetch_desc(&tmap_a);
-  if (warp == 2 && lane == 0) tma_prefetch_desc(&tmap_b);
+  if (warp == 2 && lane == 0) {
+    tma_prefetch_desc(&tmap_b);
+    if (is_glu) tma_prefetch_desc(&tmap_b2);
+  }
   if (warp == 1) {
     if constexpr (CG == 1) {
       tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -290,7 +333,8 @@ __global__ void __maxnreg__(128) gemm_kernel(
 
   const WaitCtl ctl{status, abort_flag, kWaitLimitNs};
   const int m_tiles = (M + kBM * CG - 1) / (kBM * CG);
-  const int n_tiles = (N + kBN - 1) / kBN;
+  const int tile_n = is_glu ? kBN / 2 : kBN;  // output columns per tile
+  const int n_tiles = (N + tile_n - 1) / tile_n;
   const int tiles = m_tiles * n_tiles;
   const int kblocks = (K + kBK - 1) / kBK;
   const int cluster_id = blockIdx.x / CG, n_clusters = gridDim.x / CG;
@@ -323,8 +367,16 @@ __global__ void __maxnreg__(128) gemm_kernel(
             }
           } else {
             mbar_arrive_expect_tx(pfull_bar(s), C::kBPBytes);
-            tma_load_2d(sb + C::kOffBP + s * C::kBPBytes, &tmap_b, kb * (kBK / 4),
-                        nt * kBN + static_cast<int>(rank) * C::kRowsB, pfull_bar(s));
+            const uint32_t dst = sb + C::kOffBP + s * C::kBPBytes;
+            if (!is_glu) {
+              tma_load_2d(dst, &tmap_b, kb * (kBK / 4), nt * kBN + static_cast<int>(rank) * C::kRowsB, pfull_bar(s));
+            } else if constexpr (CG == 1) {
+              // 128 gate rows, then the same 128 rows of up.
+              tma_load_2d(dst, &tmap_b, kb * (kBK / 4), nt * (kBN / 2), pfull_bar(s));
+              tma_load_2d(dst + (kBN / 2) * (kBK / 4), &tmap_b2, kb * (kBK / 4), nt * (kBN / 2), pfull_bar(s));
+            } else {
+              tma_load_2d(dst, rank == 0 ? &tmap_b : &tmap_b2, kb * (kBK / 4), nt * (kBN / 2), pfull_bar(s));
+            }
           }
           if (++s == nst) { s = 0; ph ^= 1; }
         }
@@ -437,6 +489,7 @@ __global__ void __maxnreg__(128) gemm_kernel(
     const int q = warp & 3;  // tensor-memory lane quarter this warp may read
     griddep_wait();          // scales and row sums come from the preceding kernel; y may be read by it
     const float gamma = __ldg(gamma_ptr);
+    const float gamma2 = is_glu ? __ldg(glu.gamma2) : 0.0f;
     const bool staged = C::kOutWarpBytes > 0 && tma_out;
     uint8_t* obuf = smem + C::kOffOut + (warp - C::kEpiWarp0) * C::kOutWarpBytes;
     int ob = 0;  // staging buffer of the next box
@@ -455,11 +508,52 @@ __global__ void __maxnreg__(128) gemm_kernel(
       const int m0 = mt * kBM * CG + static_cast<int>(rank) * kBM + q * 32;  // first row of this warp
       const int m = m0 + lane;
       const bool mvalid = m < M;
-      float gs = 0.0f;
+      float gs = 0.0f, gs2 = 0.0f;
       int rs = 0;
       if (mvalid) {
         gs = __fdiv_rn(gamma, __ldg(scale + m));
+        if (is_glu) gs2 = __fdiv_rn(gamma2, __ldg(scale + m));
         rs = __ldg(rowsum + m);
+      }
+      if (is_glu) {
+        // 32 output columns at a time: the gate accumulators at column c, the
+        // up accumulators at column c + 128.
+#pragma unroll 1
+        for (int c = 0; c < kBN / 64; ++c) {
+          uint32_t r[32], r2[32];
+          const uint32_t t0 = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kBN + c * 32;
+          tmem_ld_32x32b_x32(t0, r);
+          tmem_ld_32x32b_x32(t0 + kBN / 2, r2);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float g = round_to<TY>(__fmul_rn(static_cast<float>(static_cast<int>(r[i]) - rs), gs));
+            const float u = round_to<TY>(__fmul_rn(static_cast<float>(static_cast<int>(r2[i]) - rs), gs2));
+            r[i] = __float_as_uint(glu_value<TY>(g, u, glu.act));
+          }
+          const int n0 = nt * (kBN / 2) + c * 32;
+          if (staged) {
+            if (n0 < N && m0 < M) {  // warp-uniform
+              if (lane == 0) bulk_wait_group_read<1>();
+              __syncwarp();
+              uint8_t* b = obuf + ob * 4096;
+              stage_vals<TY>(b, lane, r);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmap_y, smem_u32(b), n0, m0);
+                bulk_commit_group();
+              }
+              ob ^= 1;
+            }
+          } else if (mvalid && n0 < N) {
+            store_vals32<TY>(y, static_cast<size_t>(m) * N, n0, N, r);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_leader<CG>(tempty_bar(a));
+        continue;
       }
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
@@ -561,11 +655,17 @@ static bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint
 template <typename TY, int CG>
 static cudaError_t launch_gemm_t(const ProductArgs& a, cudaStream_t stream, bool pdl) {
   using C = GemmCfg<CG>;
-  CUtensorMap ta, tb;
+  const bool glu = a.glu_act >= 0;
+  if (glu && (!a.packed2 || !a.gamma2 || a.acc_out)) return cudaErrorInvalidValue;
+  // A GLU tile takes 128 rows of each weight tensor (one load each, or one per CTA of the pair).
+  const uint32_t rows_b = glu ? kBN / 2 : C::kRowsB;
+  CUtensorMap ta, tb, tb2 = {};
   if (!make_map_2d(&ta, a.xq, static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M), kBK, kBM,
                    CU_TENSOR_MAP_SWIZZLE_128B, static_cast<uint64_t>(a.ldx)) ||
-      !make_map_2d(&tb, a.packed, static_cast<uint64_t>(a.K / 4), static_cast<uint64_t>(a.N), kBK / 4,
-                   C::kRowsB, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+      !make_map_2d(&tb, a.packed, static_cast<uint64_t>(a.K / 4), static_cast<uint64_t>(a.N), kBK / 4, rows_b,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      (glu && !make_map_2d(&tb2, a.packed2, static_cast<uint64_t>(a.K / 4), static_cast<uint64_t>(a.N), kBK / 4,
+                           rows_b, CU_TENSOR_MAP_SWIZZLE_NONE))) {
     return cudaErrorInvalidValue;
   }
   // The pair form writes its outputs by TMA when the rows are 16-byte
@@ -610,7 +710,8 @@ static cudaError_t launch_gemm_t(const ProductArgs& a, cudaStream_t stream, bool
     }
     max_clusters = n > 0 ? n : 1;
   }
-  const int tiles = ((a.M + kBM * CG - 1) / (kBM * CG)) * ((a.N + kBN - 1) / kBN);
+  const int tile_n = glu ? kBN / 2 : kBN;
+  const int tiles = ((a.M + kBM * CG - 1) / (kBM * CG)) * ((a.N + tile_n - 1) / tile_n);
   const int clusters = tiles < max_clusters ? tiles : max_clusters;
 
   cudaLaunchConfig_t cfg = {};
@@ -634,7 +735,8 @@ static cudaError_t launch_gemm_t(const ProductArgs& a, cudaStream_t stream, bool
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, gemm_kernel<TY, CG>, ta, tb, ty, tacc, tma_out, a.gamma, a.N, a.K, a.M,
+  const GemmGlu gg{a.glu_act, a.gamma2};
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<TY, CG>, ta, tb, tb2, ty, tacc, tma_out, gg, a.gamma, a.N, a.K, a.M,
                             a.scale, a.rowsum, static_cast<TY*>(a.y), a.acc_out, a.status);
 }
 

@@ -66,6 +66,8 @@
 //    y = acc * (gamma / s) is stored straight from registers.
 //  * The kernel is specialised on the number of token slots (1, 2, 4, 8 or
 //    16), so a one-token decode does no work for absent tokens.
+//  * The FFN's gate and up BitLinears can run as one launch that also forms
+//    h = act(gate) * up and quantises it for the down BitLinear (GvGlu below).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <string.h>
@@ -105,6 +107,36 @@ struct GvLayer {
 // rounded to the 1024-byte period of the 128-byte swizzle.
 __host__ __device__ constexpr int x_half_bytes(int tt) { return ((tt * 4 * 128 + 1023) / 1024) * 1024; }
 
+// The FFN's gate and up BitLinears in one launch, with the gated activation
+// and the quantisation of its result (the down BitLinear's input) done by the
+// same launch: layers glu.gate and glu.up store their outputs (rounded to the
+// activation type) in scratch; the warp that stores the second of a pair of
+// 16-row groups computes h for those rows, keeps a per-token running max of
+// |h| and counts the group done.  After the pair's units the tickets hand out
+// quantisation units, each a range of h's elements: they wait until every
+// group is done (the pair's units were all handed out before them, to running
+// blocks), then quantise with the final per-token scale; the last one writes
+// the scales and code sums.
+struct GvGlu {
+  int on;
+  int act;                // kGluRelu2 or kGluSilu
+  int gate, up;           // their layer slots
+  int q_unit0;            // first quantisation unit
+  int q_elems;            // elements of h per quantisation unit (a multiple of 16)
+  int groups;             // 16-row groups of h: units * kGvWarps
+  int q_warps;            // quantisation units * kGvWarps
+  const void* yg;         // [M][N] gate output, activation type
+  const void* yu;         // [M][N] up output
+  void* h;                // [M][N] h, activation type
+  int8_t* xq;             // [M][N] codes of h
+  float* scale;           // [M]
+  int32_t* rowsum;        // [M]
+  uint32_t* pair_cnt;     // [units][kGvWarps], zero at launch
+  uint32_t* amax;         // [16] float bits, zero at launch
+  int32_t* rsum;          // [16] zero at launch
+  uint32_t* done;         // [2] zero at launch: groups with h, quantisation warps finished
+};
+
 struct GvParams {
   GvLayer layer[kGvMaxLayers];
   int n_layers, M, total_units, nring, x_pitch;
@@ -112,6 +144,7 @@ struct GvParams {
   uint32_t* tickets;  // [0] next ticket, [1] blocks done
   int one_unit;       // as many blocks as units: each block takes its own unit, no tickets
   int ksplit;         // CTAs of a cluster that share one unit, each over its own range of stages
+  GvGlu glu;          // the fused gate/up launch (ksplit is 1 then)
 };
 
 // Stages [sb, se) of a unit with nst stages taken by cluster rank `rank` of `ks`.
@@ -322,8 +355,146 @@ __device__ __forceinline__ void stage_activations(const GvLayer& L, int M, uint3
   consumer_sync();
 }
 
-template <int TT, typename TY, typename TX, bool kSplit>
+// Counts this warp on an arrival counter in global memory (after its earlier
+// stores).  Returns true (warp-uniform) in the warp that arrives as the
+// `expected`-th, which may then read what the others stored.
+__device__ __forceinline__ bool arrive_last(uint32_t* cnt, int expected) {
+  __threadfence();  // this lane's stores are visible before the count
+  __syncwarp();
+  uint32_t old = 0;
+  if ((threadIdx.x & 31) == 0) old = atomicAdd(cnt, 1u);
+  old = __shfl_sync(0xffffffffu, old, 0);
+  if (static_cast<int>(old) != expected - 1) return false;
+  __threadfence();  // the other warps' stores are read after their counts
+  __syncwarp();
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// The gated activation and its quantisation inside the gate/up launch
+// ---------------------------------------------------------------------------
+template <typename TY>
+__device__ __forceinline__ float ld_act(const void* p, size_t i) {
+  if constexpr (sizeof(TY) == 4) {
+    return __ldcg(static_cast<const float*>(p) + i);
+  } else {
+    const unsigned short b = __ldcg(static_cast<const unsigned short*>(p) + i);
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+  }
+}
+
+static_assert(kGluRelu2 == 0 && kGluSilu == 1, "glu_value's activation codes");
+
+// Polls a counter in global memory (lane 0) until it reaches `target`;
+// bounded like every wait.  Warp-uniform result.
+__device__ __forceinline__ bool wait_count(const uint32_t* p, uint32_t target, const WaitCtl& ctl) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) {
+    const uint64_t t0 = global_ns();
+    while (true) {
+      uint32_t v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+      if (v >= target) break;
+      if (*ctl.abort) { ok = false; break; }
+      if (global_ns() - t0 > ctl.limit_ns) {
+        *ctl.abort = 1;
+        if (ctl.status) atomicOr(ctl.status, kStatusTimeout);
+        ok = false;
+        break;
+      }
+      __nanosleep(256);
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  __syncwarp();
+  return ok;
+}
+
+// After a warp of the gate or up layer stored its 16 rows of y: if the other
+// layer's warp has stored the same rows, compute h for them (all tokens),
+// fold |h| into the per-token maxima and count the group done.
+template <typename TY>
+__device__ __noinline__ void glu_rows(const GvParams& P, int rb, int warp, int N) {
+  const GvGlu& G = P.glu;
+  if (!arrive_last(G.pair_cnt + rb * kGvWarps + warp, 2)) return;
+  const int lane = threadIdx.x & 31, M = P.M;
+  const int n0 = rb * kGvRows + warp * 16;
+  // Element e = 16 m + r of the group: token m, row n0 + r.  Lanes 0..15 and
+  // 16..31 take one token each per step.
+  for (int base = 0; base < 16 * M; base += 32) {
+    const int e = base + lane, m = e >> 4, n = n0 + (e & 15);
+    float a = 0.0f;
+    if (m < M && n < N) {
+      const size_t o = static_cast<size_t>(m) * N + n;
+      const float h = glu_value<TY>(ld_act<TY>(G.yg, o), ld_act<TY>(G.yu, o), G.act);
+      if constexpr (sizeof(TY) == 4) {
+        __stcg(static_cast<float*>(G.h) + o, h);
+      } else {
+        __stcg(static_cast<unsigned short*>(G.h) + o, __bfloat16_as_ushort(__float2bfloat16_rn(h)));
+      }
+      a = fabsf(h);
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((lane & 15) == 0 && m < M && a > 0.0f) atomicMax(G.amax + m, __float_as_uint(a));
+  }
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) atomicAdd(G.done, 1u);
+}
+
+// One quantisation unit: elements [q * q_elems, (q + 1) * q_elems) of h
+// ([M][N], N % 16 == 0, so no 16-element chunk crosses a token), once every
+// group of h is done.  Codes as the quantisation kernel makes them:
+// s = 127 / max(amax, 1e-5), q = clamp(rint(h * s), -128, 127).
+template <typename TY>
+__device__ __noinline__ bool glu_quant_unit(const GvParams& P, int q, int N, const WaitCtl& ctl) {
+  const GvGlu& G = P.glu;
+  if (!wait_count(G.done, static_cast<uint32_t>(G.groups), ctl)) return false;
+  const int lane = threadIdx.x & 31, M = P.M;
+  const long long total = static_cast<long long>(M) * N;
+  const long long e0 = static_cast<long long>(q) * G.q_elems;
+  const long long e1 = e0 + G.q_elems < total ? e0 + G.q_elems : total;
+  for (long long e = e0 + 16LL * threadIdx.x; e < e1; e += 16LL * kGvConsumers) {
+    const int m = static_cast<int>(e / N);
+    const float s = __fdiv_rn(127.0f, fmaxf(__uint_as_float(__ldcg(G.amax + m)), 1e-5f));
+    uint32_t w[4];
+    int sum = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      int c[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        c[k] = __float2int_rn(__fmul_rn(ld_act<TY>(G.h, static_cast<size_t>(e) + 4 * b + k), s));
+        c[k] = min(max(c[k], -128), 127);
+      }
+      w[b] = pack4_s8(c[0], c[1], c[2], c[3]);
+      sum = __dp4a(static_cast<int>(w[b]), 0x01010101, sum);
+    }
+    *reinterpret_cast<uint4*>(G.xq + e) = make_uint4(w[0], w[1], w[2], w[3]);
+    atomicAdd(G.rsum + m, sum);
+  }
+  // The warp that finishes the last quantisation work writes the scales and code sums.
+  __threadfence();
+  __syncwarp();
+  uint32_t old = 0;
+  if (lane == 0) old = atomicAdd(G.done + 1, 1u);
+  old = __shfl_sync(0xffffffffu, old, 0);
+  if (static_cast<int>(old) == G.q_warps - 1) {
+    __threadfence();
+    if (lane < M) {
+      G.scale[lane] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(__ldcg(G.amax + lane)), 1e-5f));
+      G.rowsum[lane] = __ldcg(G.rsum + lane);
+    }
+  }
+  return true;
+}
+
+// kMode: 0 plain, 1 K-split over clusters, 2 the fused gate/up launch.
+template <int TT, typename TY, typename TX, int kMode>
 __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(const __grid_constant__ GvParams P) {
+  constexpr bool kSplit = kMode == 1;
+  constexpr bool kGlu = kMode == 2;
   constexpr int TG = (TT + 7) / 8;           // mma token groups of 8
   constexpr bool kStream = sizeof(TX) == 1;  // int8 codes stream with the weights
   constexpr bool kAlu = TT == 1;             // one token: dp4a dot products instead of the mma path
@@ -378,7 +549,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         // Before the grid dependency: the weights of the first unit's first
         // stages (a whole ring of them); their activation tiles, written by
         // the preceding kernel, follow once it has finished.
-        if (unit < P.total_units) {
+        if (unit < P.total_units && !(kGlu && unit >= P.glu.q_unit0)) {
           int l = 0;
           while (l + 1 < P.n_layers && unit >= P.layer[l + 1].unit0) ++l;
           const GvLayer& L = P.layer[l];
@@ -409,6 +580,25 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         }
       }
       while (ok && unit < P.total_units) {
+        if (kGlu && unit >= P.glu.q_unit0) {
+          // A quantisation unit: a slot with no data, only the tag.
+          if (!mbar_wait(bar0 + 8 * (nring + slot), phase ^ 1, ctl)) { ok = false; break; }
+          tags[slot] = unit;
+          mbar_arrive(bar0 + 8 * slot);
+          ++issued;
+          if (++slot == nring) { slot = 0; phase ^= 1; }
+          st0 = 0;
+          if (P.one_unit) {
+            unit = P.total_units;
+          } else {
+            if (!waited) {
+              griddep_wait();  // the ticket counter is reset by the preceding launch
+              waited = true;
+            }
+            unit = static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(P.tickets, 1u));
+          }
+          continue;
+        }
         int l = 0;
         while (l + 1 < P.n_layers && unit >= P.layer[l + 1].unit0) ++l;
         const GvLayer& L = P.layer[l];
@@ -475,16 +665,18 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       x_row[tg] = (4 * m + t) * 128;
       x_sw[tg] = (4 * m + t) & 7;
     }
-    int staged = -1;  // layer whose activations are in shared memory
+    const void* staged = nullptr;  // input whose activations are in shared memory (layers may share one)
+    int staged_k = 0;
     int slot = 0, phase = 0;
     if constexpr (!kStream) {
       // The first unit is the block's index, so its activations can be
       // quantised while its first weight stage is still on the way.
-      if (unit_first < P.total_units) {
+      if (unit_first < P.total_units && !(kGlu && unit_first >= P.glu.q_unit0)) {
         int l = 0;
         while (l + 1 < P.n_layers && unit_first >= P.layer[l + 1].unit0) ++l;
         stage_activations<TT, TX>(P.layer[l], M, xs, P.x_pitch, s_tok, rs_tok, scratch);
-        staged = l;
+        staged = P.layer[l].x;
+        staged_k = P.layer[l].K;
       }
     }
     while (true) {
@@ -492,16 +684,25 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       if (!__all_sync(0xffffffffu, got0)) break;
       const int unit = tags[slot];
       if (unit == kGvTagEnd) break;
+      if (kGlu && unit >= P.glu.q_unit0) {
+        // A quantisation unit: release the (empty) slot, then quantise.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));
+        if (++slot == nring) { slot = 0; phase ^= 1; }
+        if (!glu_quant_unit<TY>(P, unit - P.glu.q_unit0, P.layer[P.glu.gate].N, ctl)) break;
+        continue;
+      }
       int l = 0;
       while (l + 1 < P.n_layers && unit >= P.layer[l + 1].unit0) ++l;
       const GvLayer& L = P.layer[l];
       int s0, s1;  // this CTA's stages of the unit
       stage_range((L.K + kGvStageK - 1) / kGvStageK, ks, rank, s0, s1);
       if constexpr (!kStream) {
-        if (l != staged) {
-          consumer_sync();  // every warp is done with the previous layer's activations
+        if (L.x != staged || L.K != staged_k) {
+          consumer_sync();  // every warp is done with the previous input's activations
           stage_activations<TT, TX>(L, M, xs, P.x_pitch, s_tok, rs_tok, scratch);
-          staged = l;
+          staged = L.x;
+          staged_k = L.K;
         }
       }
 
@@ -721,6 +922,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           if constexpr (sizeof(TY) == 4) y[n] = val; else y[n] = __float2bfloat16_rn(val);
           if (L.acc_out) L.acc_out[n] = a;
         }
+        if constexpr (kGlu) glu_rows<TY>(P, unit - L.unit0, warp, L.N);
         continue;
       }
 #pragma unroll
@@ -739,6 +941,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
             if (L.acc_out) L.acc_out[o] = a;
           }
         }
+      if constexpr (kGlu) glu_rows<TY>(P, unit - L.unit0, warp, L.N);
     }
   }
 
@@ -786,16 +989,19 @@ bool gemv_fuses_quant(int M, int K, int x_bf16) {
 
 template <int TT, typename TY, typename TX>
 static cudaError_t launch_group_t(const GvParams& P, int grid, int smem, cudaStream_t stream, bool pdl) {
-  // Separate instances with and without the K-split, so that a launch that
-  // does not split runs none of its code.
-  static bool attr_set[2] = {false, false};  // per template instance
-  const int sp = P.ksplit > 1 ? 1 : 0;
-  auto kernel = sp ? gemv_group_kernel<TT, TY, TX, true> : gemv_group_kernel<TT, TY, TX, false>;
-  if (!attr_set[sp]) {
+  // Separate instances for the plain launch, the K-split and the fused
+  // gate/up launch, so that each runs none of the others' code.
+  static bool attr_set[3] = {false, false, false};  // per template instance
+  const int mode = P.glu.on ? 2 : P.ksplit > 1 ? 1 : 0;
+  auto kernel = mode == 2   ? gemv_group_kernel<TT, TY, TX, 2>
+                : mode == 1 ? gemv_group_kernel<TT, TY, TX, 1>
+                            : gemv_group_kernel<TT, TY, TX, 0>;
+  if (!attr_set[mode]) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemPerBlock);
     if (e != cudaSuccess) return e;
-    attr_set[sp] = true;
+    attr_set[mode] = true;
   }
+  const int sp = mode == 1 ? 1 : 0;
   if (!sp) return launch(kernel, dim3(grid), dim3(kGvThreads), static_cast<size_t>(smem), stream, pdl, P);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -834,9 +1040,26 @@ static cudaError_t launch_group_y(int x_type, const GvParams& P, int grid, int s
   }
 }
 
+thread_local int g_force_ksplit = 0;  // 0: automatic
+
+void gemv_force_ksplit(int ks) { g_force_ksplit = ks > 0 ? ks : 0; }
+
+constexpr int kGluQuantElems = 2048;  // elements of h per quantisation unit
+
+// Zeroed scratch of a fused gate/up launch: the pair counters (one per 16-row
+// group), then amax[16], rsum[16], done[2].
+size_t gemv_glu_scratch_bytes(int N) {
+  const size_t groups = static_cast<size_t>((N + kGvRows - 1) / kGvRows) * kGvWarps;
+  return (groups * 4 + 255) / 256 * 256 + 256;
+}
+
 cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, int x_type, int y_type,
-                              uint32_t* status, uint32_t* tickets, cudaStream_t stream, bool pdl) {
+                              uint32_t* status, uint32_t* tickets, cudaStream_t stream, bool pdl,
+                              const GemvGluArgs* glu) {
   if (n_layers < 1 || n_layers > kGvMaxLayers || M < 1 || M > 16) return cudaErrorInvalidValue;
+  if (glu && (n_layers != 2 || layers[0].N != layers[1].N || layers[0].K != layers[1].K || layers[0].N % 16 != 0 ||
+              !glu->zeroed || !glu->h || !glu->xq || !glu->scale || !glu->rowsum))
+    return cudaErrorInvalidValue;
   EncodeTiledFn enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
   if (!enc) return cudaErrorNotSupported;
   const bool stream_x = x_type == kInInt8;
@@ -909,11 +1132,42 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   const int sms = num_sms();
   const int target = tt == 1 ? sms : 2 * sms;
   int ks = units < target ? (target + units / 2) / units : 1;
+  if (g_force_ksplit > 0) ks = g_force_ksplit;
   while (ks > 1 && units * ks > kGvBlocksPerSM * sms) --ks;
   if (ks > kGvMaxSplit) ks = kGvMaxSplit;
   if (ks > nst_min) ks = nst_min;
-  if (ks < 1) ks = 1;
+  if (ks < 1 || glu) ks = 1;  // the fused gate/up launch hands its quantisation units out by ticket
   P.ksplit = ks;
+  if (glu) {
+    GvGlu& G = P.glu;
+    const int N = layers[0].N;
+    const long long elems = static_cast<long long>(M) * N;
+    const int q_units = static_cast<int>((elems + kGluQuantElems - 1) / kGluQuantElems);
+    G.on = 1;
+    G.act = glu->act;
+    for (int i = 0; i < n_layers; ++i) {
+      if (order[i] == 0) G.gate = i;
+      if (order[i] == 1) G.up = i;
+    }
+    G.q_unit0 = units;
+    G.q_elems = kGluQuantElems;
+    G.groups = ((N + kGvRows - 1) / kGvRows) * kGvWarps;
+    G.q_warps = q_units * kGvWarps;
+    G.yg = layers[0].y;
+    G.yu = layers[1].y;
+    G.h = glu->h;
+    G.xq = glu->xq;
+    G.scale = glu->scale;
+    G.rowsum = glu->rowsum;
+    G.pair_cnt = glu->zeroed;
+    uint32_t* small =
+        reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(glu->zeroed) + gemv_glu_scratch_bytes(N) - 256);
+    G.amax = small;
+    G.rsum = reinterpret_cast<int32_t*>(small + 16);
+    G.done = small + 32;
+    units += q_units;
+    P.total_units = units;
+  }
   // kGvBlocksPerSM blocks per SM, each with the deepest ring that fits beside its other data.
   const int slot = kGvStageBytes + (stream_x ? 2 * x_half_bytes(tt) : 0);
   const int fixed = gemv_smem_bytes(M, k_max, 0, stream_x, ks);

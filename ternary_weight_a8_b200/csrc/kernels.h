@@ -44,10 +44,14 @@ struct QuantArgs {
   int K, ldq;
 };
 constexpr int kQuantMaxItems = 8;
+// zero / zero_bytes (16-byte aligned, a multiple of 16; may be null / 0): a
+// region the launch also clears, once the preceding kernel has finished
+// (the split scratch of the decode launch that follows).
 cudaError_t launch_act_quant(const void* x, int x_bf16, int M, int K, int ldq, int8_t* xq, float* scale,
-                             int32_t* rowsum, cudaStream_t stream, bool pdl);
+                             int32_t* rowsum, cudaStream_t stream, bool pdl, void* zero = nullptr,
+                             size_t zero_bytes = 0);
 cudaError_t launch_act_quant_group(const QuantArgs* items, int n_items, int M, int x_bf16, cudaStream_t stream,
-                                   bool pdl);
+                                   bool pdl, void* zero = nullptr, size_t zero_bytes = 0);
 
 // RMSNorm (gain optional) fused with the per-token quantisation; x_norm
 // (optional) receives the normalised activations in the input type.
@@ -76,6 +80,13 @@ struct ProductArgs {
   int y_type;  // OutType
   int32_t* acc_out;
   uint32_t* status;
+  // The FFN's gate and up products in one launch (glu_act >= 0): packed /
+  // gamma are the gate BitLinear's, packed2 / gamma2 the up BitLinear's (same
+  // N and K), and y receives h = act(gate) * up [M][N] in y_type; acc_out
+  // must be null.  glu_act = -1: a plain product.
+  const uint8_t* packed2 = nullptr;
+  const float* gamma2 = nullptr;
+  int glu_act = -1;
 };
 
 // Decode GEMV (M <= 16) over a group of independent layers in one launch.
@@ -94,9 +105,29 @@ struct GemvLayerArgs {
 };
 constexpr int kGvMaxLayers = 8;
 bool gemv_fuses_quant(int M, int K, int x_bf16);
+// CTAs per unit of the decode kernel's K-split (a cluster): 0 lets the kernel
+// choose (by the unit count), else forced (1 .. 8, capped by the stages).  Per thread.
+void gemv_force_ksplit(int ks);
+
+// The FFN's gated activation fused into the launch of its gate and up
+// BitLinears (layers[0] = gate, layers[1] = up, same N and K, their y in
+// scratch): h = act(gate) * up [M][N] in the activation type, and its
+// per-token quantisation (codes [M][N], scales, code sums) for the down
+// BitLinear.  `zeroed`: gemv_glu_scratch_bytes(N) bytes, zero at launch.
+struct GemvGluArgs {
+  int act;  // GluAct
+  void* h;
+  int8_t* xq;
+  float* scale;
+  int32_t* rowsum;
+  uint32_t* zeroed;
+};
+size_t gemv_glu_scratch_bytes(int N);
+
 // tickets: two zero-initialised uint32 in device memory (reset by the kernel after use).
 cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, int x_type, int y_type,
-                              uint32_t* status, uint32_t* tickets, cudaStream_t stream, bool pdl);
+                              uint32_t* status, uint32_t* tickets, cudaStream_t stream, bool pdl,
+                              const GemvGluArgs* glu = nullptr);
 
 // cuTensorMapEncodeTiled from the driver (no link-time dependency on libcuda).
 #ifdef CUDA_VERSION

@@ -14,27 +14,36 @@
 
 namespace bl {
 
-// One thread per row: sum_k |W[n][k]| in double, k ascending.  Each thread
-// reads its row 128 bytes (one cache line) at a time.
-__global__ void __launch_bounds__(128) gamma_row_sums_kernel(const float* __restrict__ W, int N,
-                                                             int K, double* __restrict__ row_sums) {
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
-  const float4* row = reinterpret_cast<const float4*>(W + static_cast<size_t>(n) * K);
+// Row sums sum_k |W[n][k]| in double, each in the fixed order k = 0, 1, ...
+// A warp takes 32 rows: it reads them 32 columns at a time, lane l loading
+// column l of each row (one 128-byte line per load, all 32 in flight), and
+// after a transpose through shared memory lane r adds row r's 32 values in
+// column order.
+constexpr int kRowWarps = 4;
+
+__global__ void __launch_bounds__(32 * kRowWarps) gamma_row_sums_kernel(const float* __restrict__ W, int N,
+                                                                       int K, double* __restrict__ row_sums) {
+  __shared__ float tile[kRowWarps][32][33];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = (blockIdx.x * kRowWarps + warp) * 32;
+  if (row0 >= N) return;  // warp-uniform
+  float (*t)[33] = tile[warp];
   double acc = 0.0;
-  for (int i = 0; i < K / 4; i += 8) {  // K % 64 == 0: whole lines
-    float4 v[8];
+  for (int k0 = 0; k0 < K; k0 += 32) {  // K % 64 == 0: whole 32-column blocks
+    float v[32];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = __ldg(row + i + u);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      acc = __dadd_rn(acc, fabs(static_cast<double>(v[u].x)));
-      acc = __dadd_rn(acc, fabs(static_cast<double>(v[u].y)));
-      acc = __dadd_rn(acc, fabs(static_cast<double>(v[u].z)));
-      acc = __dadd_rn(acc, fabs(static_cast<double>(v[u].w)));
+    for (int r = 0; r < 32; ++r) {
+      const int n = row0 + r;
+      v[r] = n < N ? __ldg(W + static_cast<size_t>(n) * K + k0 + lane) : 0.0f;
     }
+#pragma unroll
+    for (int r = 0; r < 32; ++r) t[r][lane] = v[r];
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 32; ++c) acc = __dadd_rn(acc, fabs(static_cast<double>(t[lane][c])));
+    __syncwarp();
   }
-  row_sums[n] = acc;
+  if (row0 + lane < N) row_sums[row0 + lane] = acc;
 }
 
 // One block: the row sums are staged through shared memory a chunk at a
@@ -86,16 +95,12 @@ __global__ void __launch_bounds__(256) ternary_pack_kernel(const float* __restri
     }
     packed[g] = word;
   }
-  // The forward kernels, launched as programmatic dependents of the kernel
-  // before them, start loading packed weights before their grid-dependency
-  // wait.  The fence makes this kernel's words visible device-wide before its
-  // blocks exit, which is the earliest a dependent launch can begin.
-  __threadfence();
 }
 
 cudaError_t launch_gamma(const float* W, int N, int K, double* row_sums, float* gamma,
                          cudaStream_t stream) {
-  gamma_row_sums_kernel<<<(N + 127) / 128, 128, 0, stream>>>(W, N, K, row_sums);
+  gamma_row_sums_kernel<<<(N + 32 * kRowWarps - 1) / (32 * kRowWarps), 32 * kRowWarps, 0, stream>>>(W, N, K,
+                                                                                                 row_sums);
   gamma_finalize_kernel<<<1, 256, 0, stream>>>(row_sums, N, static_cast<long long>(N) * K, gamma);
   return cudaGetLastError();
 }

@@ -4,6 +4,7 @@
   kernel's sources hash as they did at capture time.
 - The all-cores CPU baseline splits every layer's output rows into contiguous,
   disjoint slices; the oracle on the slices reproduces the whole decode step.
+- The timed-block count covers the minimum timed region.
 """
 import os
 import sys
@@ -49,11 +50,26 @@ def test_source_hash_covers_the_kernel_files(tmp_path, monkeypatch):
     assert bench.kernel_source_hash("probe") != h1
 
 
+def test_rep_plan_covers_the_minimum_region():
+    assert bench.rep_plan(20, 0.8e-3, 0.5) == 625
+    assert bench.rep_plan(20, 1.0, 0.05) == 1
+    assert bench.rep_plan(20, 1e-9, 0.05, max_reps=100) == 100
+    assert bench.rep_plan(20, 0.0, 0.05, max_reps=7) == 7
+
+
+def test_chain_sample_rows_and_shared_input():
+    layers, set_bytes = bench.oracle_chain_layers(rows_div=256)
+    assert len(layers) == len(bench.CHAIN_70B)
+    assert set_bytes == sum(-(-N // 256) * K // 4 for K, N in bench.CHAIN_70B)
+    for (packed, gamma, K, xf), (K2, N) in zip(layers, bench.CHAIN_70B):
+        assert packed.shape == (-(-N // 256), K // 4) and K == K2 and xf.shape == (1, K)
+    assert layers[3][3] is layers[2][3]  # gate and up take one input
+
+
 def test_oracle_row_slices_reassemble_the_decode_step():
     import oracle
 
-    layers, set_bytes = bench.oracle_decode_layers()
-    assert set_bytes == sum(N * K // 4 for K, N in bench.DECODE_LAYERS)
+    layers, set_bytes = bench.oracle_chain_layers(rows_div=256)
     for packed, gamma, K, xf in layers:
         T, ok = oracle.unpack(packed, K)
         acc, y, *_ = oracle.forward(T, gamma, xf)

@@ -97,7 +97,9 @@ def test_pack_special_matrices():
                                        (2048, 2560, "bf16"), (8, 28672, "bf16"), (5, 8640, "f32"),
                                        # many tokens, short and long rows
                                        (700, 2048, "f32"), (600, 576, "bf16"), (640, 4096, "bf16"),
-                                       (600, 4160, "bf16"), (1200, 64, "f32")])
+                                       (600, 4160, "bf16"), (1200, 64, "f32"),
+                                       # few long tokens: one token over a cluster of 2 to 8 CTAs
+                                       (1, 20480, "f32"), (2, 65536, "bf16"), (16, 16448, "bf16")])
 def test_quant_parity(M, K, dtype):
     x, xf = activations(M, K, seed=M * 7 + K, dtype=dtype)
     q_ref, s_ref, r_ref = oracle.quant_act(xf)
@@ -175,6 +177,43 @@ KSPLIT = [(130, 3072), (64, 8192), (300, 2112), (17, 4160)]
 @pytest.mark.parametrize("M", [1, 2, 5, 9, 16])
 def test_forward_ksplit(M, N, K):
     _full_case(M, N, K, "bf16", torch.bfloat16, tb.PATH_GEMV, seed=M + N + K)
+
+
+@pytest.fixture
+def forced_split():
+    """The K-split forced to `ctas` CTAs per unit, reset afterwards."""
+    def force(ctas):
+        tb.set_decode_split(ctas)
+    yield force
+    tb.set_decode_split(0)
+
+
+# The K-split forced on shapes the automatic choice leaves whole: both decode
+# paths (dp4a for one token, mma.sync for more), activations quantised inside
+# the kernel or streamed as codes, fp32 and bf16, up to the 8-CTA cluster.
+FORCED = [(1, 640, 2048, "f32"), (1, 1000, 9216, "bf16"), (3, 2000, 4160, "bf16"), (8, 3000, 5120, "bf16"),
+          (16, 1200, 8192, "f32"), (12, 1300, 2560, "bf16")]
+
+
+@pytest.mark.parametrize("M,N,K,xdt", FORCED)
+@pytest.mark.parametrize("ctas", [2, 3, 8])
+def test_forward_forced_split(M, N, K, xdt, ctas, forced_split):
+    forced_split(ctas)
+    _full_case(M, N, K, xdt, torch.float32 if xdt == "f32" else torch.bfloat16, tb.PATH_GEMV, seed=M * K + ctas)
+
+
+def test_forced_split_matches_unsplit_bit_for_bit(forced_split):
+    """The split changes the order of integer sums only: acc and y are identical."""
+    W = weights(700, 8192, seed=11)
+    packed, gamma = tb.pack_weights(dev(W))
+    for M in (1, 4, 16):
+        x, _ = activations(M, 8192, seed=M + 3, dtype="bf16")
+        forced_split(1)
+        y1, a1 = tb.forward(packed, gamma, x, acc_out=True, out_dtype=torch.float32)
+        for ctas in (2, 5, 8):
+            forced_split(ctas)
+            y2, a2 = tb.forward(packed, gamma, x, acc_out=True, out_dtype=torch.float32)
+            assert torch.equal(a1, a2) and torch.equal(y1, y2)
 
 
 @pytest.mark.parametrize("M,N,K", SMALL)
@@ -306,8 +345,11 @@ def test_forward_zero_tokens_and_weights():
 # 70B-class layer chain at decode
 # ----------------------------------------------------------------------------
 
-@pytest.mark.parametrize("M", [1, 8])
+@pytest.mark.parametrize("M", [1, 8, 16])
 def test_layer_chain_70b_sampled(M):
+    """The five BitLinears of a 70B-class block in one grouped launch (split into
+    items of a few stages), with every layer's int32 accumulators compared bit
+    for bit on sampled rows."""
     layers_shape = synth.CHAIN_70B
     shared = synth.CHAIN_70B_SHARED_INPUT
     rng = np.random.default_rng(M)
@@ -326,8 +368,9 @@ def test_layer_chain_70b_sampled(M):
             x, xf = activations(M, K, seed=2000 + li, dtype="bf16")
         x_prev = (x, xf)
         y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-        layers.append(tb.Layer(packed, gamma, x, y))
-        rows = np.unique(np.concatenate([rng.choice(N, 48, replace=False), [0, N - 1]]))
+        acc = torch.full((M, N), -7, dtype=torch.int32, device="cuda")
+        layers.append(tb.Layer(packed, gamma, x, y, acc_out=acc))
+        rows = np.unique(np.concatenate([rng.choice(N, 48, replace=False), [0, 63, 64, N - 1]]))
         T_rows = oracle.ternarize(W[rows], gamma_ref)
         acc_ref, y_ref, *_ = oracle.forward(T_rows, gamma_ref, xf)
         refs.append((rows, acc_ref, y_ref))
@@ -335,8 +378,49 @@ def test_layer_chain_70b_sampled(M):
     tb.layer_chain(layers)
     torch.cuda.synchronize()
     for L, (rows, acc_ref, y_ref) in zip(layers, refs):
-        assert_y_matches(L.y[:, torch.as_tensor(rows, device="cuda")].contiguous(), y_ref, acc_ref)
+        idx = torch.as_tensor(rows, device="cuda")
+        assert np.array_equal(L.acc_out[:, idx].cpu().numpy(), acc_ref)
+        assert_y_matches(L.y[:, idx].contiguous(), y_ref, acc_ref)
         assert torch.isfinite(L.y.float()).all()
+        assert ((L.acc_out == 0) == (L.y.float() == 0)).all()
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_layer_chain_3b_full(M):
+    """Both 3B-class BitLinears as one chain call, every output and accumulator compared."""
+    layers, refs = [], []
+    for li, (K, N) in enumerate([(3200, 8640), (8640, 3200)]):
+        W = weights(N, K, seed=3000 + li)
+        packed_ref, gamma_ref, T = oracle.pack_weights(W)
+        x, xf = activations(M, K, seed=3100 + li, dtype="bf16")
+        acc_ref, y_ref, *_ = oracle.forward(T, gamma_ref, xf)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+        layers.append(tb.Layer(dev(packed_ref), dev(np.array([gamma_ref], np.float32)), x, y, acc_out=acc))
+        refs.append((acc_ref, y_ref))
+    tb.layer_chain(layers)
+    for L, (acc_ref, y_ref) in zip(layers, refs):
+        assert np.array_equal(L.acc_out.cpu().numpy(), acc_ref)
+        assert_y_matches(L.y, y_ref, acc_ref)
+
+
+@pytest.mark.parametrize("M", [1, 2, 16])
+def test_layer_chain_on_caller_codes(M):
+    """A chain layer given its input as codes (xq, scale, rowsum) equals forward_quantized."""
+    K = 2048
+    x, _ = activations(M, K, seed=5, dtype="bf16")
+    xq, sc, rs = tb.quant_act(x)
+    specs = [(K, 900), (K, 300)]
+    layers, singles = [], []
+    for i, (k, n) in enumerate(specs):
+        packed, gamma = tb.pack_weights(dev(weights(n, k, seed=60 + i)))
+        y = torch.empty((M, n), dtype=torch.bfloat16, device="cuda")
+        acc = torch.empty((M, n), dtype=torch.int32, device="cuda")
+        layers.append(tb.Layer(packed, gamma, None, y, xq=xq, scale=sc, rowsum=rs, acc_out=acc))
+        singles.append(tb.forward_quantized(packed, gamma, xq, sc, rs, acc_out=True))
+    tb.layer_chain(layers)
+    for L, (y, a) in zip(layers, singles):
+        assert torch.equal(L.acc_out, a) and torch.equal(L.y, y)
 
 
 def test_layer_chain_matches_separate_forwards():
@@ -362,6 +446,6 @@ def test_shared_workspace_across_shapes_stays_consistent():
         packed, gamma = tb.pack_weights(dev(weights(N, K, seed=70 + i)))
         x, _ = activations(M, K, seed=80 + i, dtype="bf16")
         y1, a1 = tb.forward(packed, gamma, x, acc_out=True, workspace=ws)
-        y2, a2 = tb.forward(packed, gamma, x, acc_out=True)  # fresh workspace
+        y2, a2 = tb.forward(packed, gamma, x, acc_out=True, workspace=tb.new_workspace(tb.workspace_bytes(M, N, K)))
         assert torch.equal(a1, a2) and torch.equal(y1, y2)
     assert int(ws[:256].count_nonzero().item()) == 0
