@@ -66,8 +66,10 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-extras", action="store_true", help="headline only (no decode / prefill / pack / next)")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--only", choices=["chain70b", "decode2b", "prefill", "decode3b", "next"], default=None,
+    p.add_argument("--only", choices=["chain70b", "decode2b", "prefill", "decode3b", "next", "ffn"], default=None,
                    help="run one workload alone and print its own line (a small case for profiling)")
+    p.add_argument("--tokens", type=str, default=None,
+                   help="with --only chain70b / ffn: the token counts to run, comma-separated")
     return p.parse_args(argv)
 
 
@@ -618,6 +620,56 @@ def run_decode_3b(args, world, peaks, L2):
     return res
 
 
+def run_ffn(args, world, peaks, L2, tokens=(1, 8, 2048)):
+    """The FFN's gate and up BitLinears with the gated activation and the
+    quantisation of h: one call (gate_up_glu) against the same work as the
+    chain of the two products followed by the gated-activation kernel."""
+    import torch
+
+    import synth
+    import ternary_weight_a8_b200 as tb
+
+    out = {}
+    shapes = {1: (1, 8192, 28672), 8: (8, 8192, 28672), 16: (16, 8192, 28672), 2048: (2048, 2560, 6912)}
+    for M, K, N in (shapes[t] for t in tokens):
+        wsets, wbytes = make_layer_sets([(K, N), (K, N)], seed=1100, min_bytes=3 * L2)
+        x = torch.from_numpy(synth.activations_bf16(M, K, seed=1101)[0].view("int16")).cuda().view(torch.bfloat16)
+        yg = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        yu = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        xq = torch.empty((M, N), dtype=torch.int8, device="cuda")
+        sc = torch.empty(M, dtype=torch.float32, device="cuda")
+        rs = torch.empty(M, dtype=torch.int32, device="cuda")
+        ws_f = tb.new_workspace(tb.gate_up_glu_workspace_bytes(M, N, K))
+        lsets = [[tb.Layer(p, g, x, yg if j == 0 else yu) for j, (p, g) in enumerate(S)] for S in wsets]
+        ws_c = tb.new_workspace(tb.chain_workspace_bytes(lsets[0], M))
+
+        def fused(i):
+            (pg, gg), (pu, gu) = wsets[i % len(wsets)]
+            tb.gate_up_glu(pg, gg, pu, gu, x, tb.GLU_RELU2, xq=xq, scale=sc, rowsum=rs, workspace=ws_f)
+
+        def unfused(i):
+            tb.layer_chain(lsets[i % len(lsets)], workspace=ws_c)
+            tb.glu_quant(yg, yu, tb.GLU_RELU2, None, xq, sc, rs)
+
+        steps = 20
+        res = {"weight_bytes": wbytes}
+        for name, fn in (("fused_one_call", fused), ("chain_then_glu_quant", unfused)):
+            secs, _, _ = timed_graph_run(fn, steps, 5, world, chunk=steps, min_region_s=0.05)
+            us = secs / steps * 1e6
+            res[name] = {"us": round(us, 3)}
+            if M <= 16:
+                gbs = wbytes / (us * 1e-6) / 1e9
+                res[name].update({"GB/s": round(gbs, 1), "pct_hbm_measured": round(100 * gbs / peaks["hbm"], 2)})
+            else:
+                tops = 2 * 2.0 * M * N * K / (us * 1e-6) / 1e12
+                res[name].update({"TOPS": round(tops, 1)})
+        res["launches"] = {"fused_one_call": 2 if M <= 16 else 3, "chain_then_glu_quant": 3 if M <= 16 else 4}
+        res["device_status"] = tb.device_status(ws_f)
+        out["ffn_gate_up_glu_%dx%dx%d" % (M, K, N)] = res
+        del wsets, lsets
+    return out
+
+
 def run_next(args, world, peaks, L2):
     """The rows beyond the forward: fused RMSNorm + quantisation, gated activation +
     quantisation, the lookup-table decode product and the straight-through backward."""
@@ -682,45 +734,7 @@ def run_next(args, world, peaks, L2):
         usecs, _, _ = timed_graph_run(unfused, steps, 20, world, chunk=200, min_region_s=0.02)
         res["unfused_torch_glu_then_quant_us"] = round(usecs / steps * 1e6, 3)
         out["glu_quant_%dx%d" % (M, N)] = res
-    # The FFN's gate and up BitLinears with the gated activation and the
-    # quantisation of h: one call (gate_up_glu) against the same work as the
-    # chain of the two products followed by the gated-activation kernel.
-    for M, K, N in ((1, 8192, 28672), (8, 8192, 28672), (2048, 2560, 6912)):
-        wsets, wbytes = make_layer_sets([(K, N), (K, N)], seed=1100, min_bytes=3 * L2)
-        x = torch.from_numpy(synth.activations_bf16(M, K, seed=1101)[0].view("int16")).cuda().view(torch.bfloat16)
-        yg = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-        yu = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-        xq = torch.empty((M, N), dtype=torch.int8, device="cuda")
-        sc = torch.empty(M, dtype=torch.float32, device="cuda")
-        rs = torch.empty(M, dtype=torch.int32, device="cuda")
-        ws_f = tb.new_workspace(tb.gate_up_glu_workspace_bytes(M, N, K))
-        lsets = [[tb.Layer(p, g, x, yg if j == 0 else yu) for j, (p, g) in enumerate(S)] for S in wsets]
-        ws_c = tb.new_workspace(tb.chain_workspace_bytes(lsets[0], M))
-
-        def fused(i):
-            (pg, gg), (pu, gu) = wsets[i % len(wsets)]
-            tb.gate_up_glu(pg, gg, pu, gu, x, tb.GLU_RELU2, xq=xq, scale=sc, rowsum=rs, workspace=ws_f)
-
-        def unfused(i):
-            tb.layer_chain(lsets[i % len(lsets)], workspace=ws_c)
-            tb.glu_quant(yg, yu, tb.GLU_RELU2, None, xq, sc, rs)
-
-        steps = 20
-        res = {"weight_bytes": wbytes}
-        for name, fn in (("fused_one_call", fused), ("chain_then_glu_quant", unfused)):
-            secs, _, _ = timed_graph_run(fn, steps, 5, world, chunk=steps, min_region_s=0.05)
-            us = secs / steps * 1e6
-            res[name] = {"us": round(us, 3)}
-            if M <= 16:
-                gbs = wbytes / (us * 1e-6) / 1e9
-                res[name].update({"GB/s": round(gbs, 1), "pct_hbm_measured": round(100 * gbs / peaks["hbm"], 2)})
-            else:
-                tops = 2 * 2.0 * M * N * K / (us * 1e-6) / 1e12
-                res[name].update({"TOPS": round(tops, 1)})
-        res["launches"] = {"fused_one_call": 2 if M <= 16 else 3, "chain_then_glu_quant": 3 if M <= 16 else 4}
-        res["device_status"] = tb.device_status(ws_f)
-        out["ffn_gate_up_glu_%dx%dx%d" % (M, K, N)] = res
-        del wsets, lsets
+    out.update(run_ffn(args, world, peaks, L2))
     # The lookup-table decode product against the tensor-core decode kernel, same codes, one token.
     for K, N in ((2560, 6912), (8192, 10240)):
         sets, set_bytes = make_layer_sets([(K, N)], seed=800, min_bytes=4 * L2)
@@ -987,8 +1001,12 @@ def main():
 
         torch.cuda.set_device(local)
         peaks, L2 = load_peaks(), l2_bytes()
+        tokens = tuple(int(t) for t in args.tokens.split(",")) if args.tokens else None
         if args.only == "chain70b":
-            res, _, _ = run_chain(args, world, peaks, L2, steps=args.steps, warmup=args.warmup)
+            res, _, _ = run_chain(args, world, peaks, L2, steps=args.steps, warmup=args.warmup,
+                                  **({"tokens": tokens} if tokens else {}))
+        elif args.only == "ffn":
+            res = run_ffn(args, world, peaks, L2, **({"tokens": tokens} if tokens else {}))
         else:
             fn = {"decode2b": run_decode_2b, "prefill": run_prefill, "decode3b": run_decode_3b,
                   "next": run_next}[args.only]

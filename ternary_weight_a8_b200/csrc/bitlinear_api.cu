@@ -617,22 +617,18 @@ int bitlinear_layer_chain(const bl_layer* layers, int n_layers, int M, int x_dty
 // ---------------------------------------------------------------------------
 // The FFN's gate and up BitLinears with the gated activation and the down
 // BitLinear's input quantisation.  Workspace: status block, the codes of x,
-// the gate and up outputs y_g, y_u [M][N] and h [M][N] (elements of 4 bytes
-// at most, each region 256-rounded), then (decode sizes) the fused launch's
+// h [M][N] (for callers that do not want h; elements of 4 bytes at most,
+// 256-rounded), then (decode sizes) the fused launch's 256 bytes of
 // counters, zeroed before it.
 // ---------------------------------------------------------------------------
 struct GluLayout {
-  size_t yg, yu, h, zero, total;
+  size_t h, zero, total;
 };
 
 static GluLayout glu_layout(int M, int N, int K) {
   GluLayout g;
-  const FwdLayout f = forward_layout(M, K);
-  const size_t act = round_up(static_cast<size_t>(M) * N * 4, 256);
-  g.yg = f.total;
-  g.yu = g.yg + act;
-  g.h = g.yu + act;
-  g.zero = g.h + act;
+  g.h = forward_layout(M, K).total;
+  g.zero = g.h + round_up(static_cast<size_t>(M) * N * 4, 256);
   g.total = g.zero + (M >= 1 && M <= 16 ? bl::gemv_glu_scratch_bytes(N) : 0);
   return g;
 }
@@ -670,8 +666,6 @@ int bitlinear_gate_up_glu(const uint8_t* packed_gate, const float* gamma_gate, c
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool x_bf16 = x_dtype == BL_BF16;
   const int at = x_bf16 ? bl::kOutBF16 : bl::kOutF32;  // gate/up outputs and h in the activation type
-  void* yg = ws + g.yg;
-  void* yu = ws + g.yu;
   void* hh = h ? h : static_cast<void*>(ws + g.h);
   const FwdLayout f = forward_layout(M, K);
   int8_t* cq = reinterpret_cast<int8_t*>(ws + f.xq);
@@ -686,11 +680,11 @@ int bitlinear_gate_up_glu(const uint8_t* packed_gate, const float* gamma_gate, c
     const bool fused = bl::gemv_fuses_quant(M, K, x_bf16);
     bl::GemvLayerArgs L[2];
     if (fused) {
-      L[0] = bl::GemvLayerArgs{packed_gate, gamma_gate, N, K, x, nullptr, nullptr, 0, yg, nullptr};
-      L[1] = bl::GemvLayerArgs{packed_up, gamma_up, N, K, x, nullptr, nullptr, 0, yu, nullptr};
+      L[0] = bl::GemvLayerArgs{packed_gate, gamma_gate, N, K, x, nullptr, nullptr, 0, nullptr, nullptr};
+      L[1] = bl::GemvLayerArgs{packed_up, gamma_up, N, K, x, nullptr, nullptr, 0, nullptr, nullptr};
     } else {
-      L[0] = bl::GemvLayerArgs{packed_gate, gamma_gate, N, K, cq, cs, cr, ldq, yg, nullptr};
-      L[1] = bl::GemvLayerArgs{packed_up, gamma_up, N, K, cq, cs, cr, ldq, yu, nullptr};
+      L[0] = bl::GemvLayerArgs{packed_gate, gamma_gate, N, K, cq, cs, cr, ldq, nullptr, nullptr};
+      L[1] = bl::GemvLayerArgs{packed_up, gamma_up, N, K, cq, cs, cr, ldq, nullptr, nullptr};
     }
     cudaError_t e;
     if (fused) {

@@ -109,32 +109,34 @@ __host__ __device__ constexpr int x_half_bytes(int tt) { return ((tt * 4 * 128 +
 
 // The FFN's gate and up BitLinears in one launch, with the gated activation
 // and the quantisation of its result (the down BitLinear's input) done by the
-// same launch: layers glu.gate and glu.up store their outputs (rounded to the
-// activation type) in scratch; the warp that stores the second of a pair of
-// 16-row groups computes h for those rows, keeps a per-token running max of
-// |h| and counts the group done.  After the pair's units the tickets hand out
-// quantisation units, each a range of h's elements: they wait until every
-// group is done (the pair's units were all handed out before them, to running
-// blocks), then quantise with the final per-token scale; the last one writes
-// the scales and code sums.
+// same launch.  A ticket below q_unit0 is a unit of 32 output rows: each
+// half-stage of its weights holds those 32 gate rows, then the same 32 up
+// rows, so that a lane's mma fragment (rows g and g + 8 of its warp's 16), or
+// a dp4a lane and its partner lane ^ 4, holds the gate and up sums of one
+// output row.  The lane rounds both outputs to the activation type, as
+// stored outputs are, forms h = act(gate) * up, stores h and keeps the
+// warp's running maximum of |h| per token in registers.  Each warp
+// publishes its maxima (one atomic max per token, each token's word on a
+// 128-byte line of its own) and counts itself done, once, with a fence, when
+// it meets its first quantisation unit or the end;
+// the tickets from q_unit0 on are quantisation units, each a range of h's
+// elements, which wait until every warp of the grid is done (all units were
+// handed out before them, to running blocks), then quantise with the final
+// per-token scale; the last one writes the scales and code sums.
 struct GvGlu {
   int on;
   int act;                // kGluRelu2 or kGluSilu
   int gate, up;           // their layer slots
-  int q_unit0;            // first quantisation unit
+  int q_unit0;            // first quantisation ticket (= the units of 32 output rows)
   int q_elems;            // elements of h per quantisation unit (a multiple of 16)
-  int groups;             // 16-row groups of h: units * kGvWarps
   int q_warps;            // quantisation units * kGvWarps
-  const void* yg;         // [M][N] gate output, activation type
-  const void* yu;         // [M][N] up output
   void* h;                // [M][N] h, activation type
   int8_t* xq;             // [M][N] codes of h
   float* scale;           // [M]
   int32_t* rowsum;        // [M]
-  uint32_t* pair_cnt;     // [units][kGvWarps], zero at launch
-  uint32_t* amax;         // [16] float bits, zero at launch
-  int32_t* rsum;          // [16] zero at launch
-  uint32_t* done;         // [2] zero at launch: groups with h, quantisation warps finished
+  uint32_t* amax;         // per token m, word 32 m: max |h| as float bits; zero at launch
+  int32_t* rsum;          // per token m, word 32 m: sum of h's codes; zero at launch
+  uint32_t* done;         // [2] zero at launch: warps done with units, quantisation warps finished
 };
 
 struct GvParams {
@@ -355,21 +357,6 @@ __device__ __forceinline__ void stage_activations(const GvLayer& L, int M, uint3
   consumer_sync();
 }
 
-// Counts this warp on an arrival counter in global memory (after its earlier
-// stores).  Returns true (warp-uniform) in the warp that arrives as the
-// `expected`-th, which may then read what the others stored.
-__device__ __forceinline__ bool arrive_last(uint32_t* cnt, int expected) {
-  __threadfence();  // this lane's stores are visible before the count
-  __syncwarp();
-  uint32_t old = 0;
-  if ((threadIdx.x & 31) == 0) old = atomicAdd(cnt, 1u);
-  old = __shfl_sync(0xffffffffu, old, 0);
-  if (static_cast<int>(old) != expected - 1) return false;
-  __threadfence();  // the other warps' stores are read after their counts
-  __syncwarp();
-  return true;
-}
-
 // ---------------------------------------------------------------------------
 // The gated activation and its quantisation inside the gate/up launch
 // ---------------------------------------------------------------------------
@@ -410,54 +397,51 @@ __device__ __forceinline__ bool wait_count(const uint32_t* p, uint32_t target, c
   return ok;
 }
 
-// After a warp of the gate or up layer stored its 16 rows of y: if the other
-// layer's warp has stored the same rows, compute h for them (all tokens),
-// fold |h| into the per-token maxima and count the group done.
-template <typename TY>
-__device__ __noinline__ void glu_rows(const GvParams& P, int rb, int warp, int N) {
-  const GvGlu& G = P.glu;
-  if (!arrive_last(G.pair_cnt + rb * kGvWarps + warp, 2)) return;
-  const int lane = threadIdx.x & 31, M = P.M;
-  const int n0 = rb * kGvRows + warp * 16;
-  // Element e = 16 m + r of the group: token m, row n0 + r.  Lanes 0..15 and
-  // 16..31 take one token each per step.
-  for (int base = 0; base < 16 * M; base += 32) {
-    const int e = base + lane, m = e >> 4, n = n0 + (e & 15);
-    float a = 0.0f;
-    if (m < M && n < N) {
-      const size_t o = static_cast<size_t>(m) * N + n;
-      const float h = glu_value<TY>(ld_act<TY>(G.yg, o), ld_act<TY>(G.yu, o), G.act);
-      if constexpr (sizeof(TY) == 4) {
-        __stcg(static_cast<float*>(G.h) + o, h);
-      } else {
-        __stcg(static_cast<unsigned short*>(G.h) + o, __bfloat16_as_ushort(__float2bfloat16_rn(h)));
-      }
-      a = fabsf(h);
-    }
+// Token m's word of a per-token array of the fused gate/up launch: one
+// 128-byte line each, so that atomics on different tokens meet in different
+// L2 slices.
+constexpr int kGluTokStride = 32;
+
+// A consumer warp's units of the fused gate/up launch are done: its
+// per-token maxima of |h| are folded into the grid's (one atomic max per
+// token, from the lanes that hold them), then its h stores and those maxima
+// are made visible and the warp is counted.
+template <int TG, bool kAlu>
+__device__ __forceinline__ void glu_warp_done(const GvParams& P, const float (&hmax)[TG][2]) {
+  const int lane = threadIdx.x & 31;
+  if constexpr (kAlu) {
+    if (lane == 0 && hmax[0][0] > 0.0f) atomicMax(P.glu.amax, __float_as_uint(hmax[0][0]));
+  } else {
+    const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    if ((lane & 15) == 0 && m < M && a > 0.0f) atomicMax(G.amax + m, __float_as_uint(a));
+    for (int tg = 0; tg < TG; ++tg)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int m = tg * 8 + 2 * t + e;
+        if (g == 0 && m < P.M && hmax[tg][e] > 0.0f)
+          atomicMax(P.glu.amax + kGluTokStride * m, __float_as_uint(hmax[tg][e]));
+      }
   }
   __threadfence();
   __syncwarp();
-  if (lane == 0) atomicAdd(G.done, 1u);
+  if (lane == 0) atomicAdd(P.glu.done, 1u);
 }
 
 // One quantisation unit: elements [q * q_elems, (q + 1) * q_elems) of h
 // ([M][N], N % 16 == 0, so no 16-element chunk crosses a token), once every
-// group of h is done.  Codes as the quantisation kernel makes them:
+// consumer warp of the grid is done with its units.  Codes as the quantisation kernel makes them:
 // s = 127 / max(amax, 1e-5), q = clamp(rint(h * s), -128, 127).
 template <typename TY>
 __device__ __noinline__ bool glu_quant_unit(const GvParams& P, int q, int N, const WaitCtl& ctl) {
   const GvGlu& G = P.glu;
-  if (!wait_count(G.done, static_cast<uint32_t>(G.groups), ctl)) return false;
+  if (!wait_count(G.done, gridDim.x * kGvWarps, ctl)) return false;
   const int lane = threadIdx.x & 31, M = P.M;
   const long long total = static_cast<long long>(M) * N;
   const long long e0 = static_cast<long long>(q) * G.q_elems;
   const long long e1 = e0 + G.q_elems < total ? e0 + G.q_elems : total;
   for (long long e = e0 + 16LL * threadIdx.x; e < e1; e += 16LL * kGvConsumers) {
     const int m = static_cast<int>(e / N);
-    const float s = __fdiv_rn(127.0f, fmaxf(__uint_as_float(__ldcg(G.amax + m)), 1e-5f));
+    const float s = __fdiv_rn(127.0f, fmaxf(__uint_as_float(__ldcg(G.amax + kGluTokStride * m)), 1e-5f));
     uint32_t w[4];
     int sum = 0;
 #pragma unroll
@@ -472,7 +456,17 @@ __device__ __noinline__ bool glu_quant_unit(const GvParams& P, int q, int N, con
       sum = __dp4a(static_cast<int>(w[b]), 0x01010101, sum);
     }
     *reinterpret_cast<uint4*>(G.xq + e) = make_uint4(w[0], w[1], w[2], w[3]);
-    atomicAdd(G.rsum + m, sum);
+    // One atomic per warp when the warp's chunks are of one token.
+    const unsigned active = __activemask();
+    const int lead = __ffs(active) - 1;
+    const int m0 = __shfl_sync(active, m, lead);
+    if (__all_sync(active, m == m0)) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(active, sum, o);
+      if ((threadIdx.x & 31) == lead) atomicAdd(G.rsum + kGluTokStride * m, sum);
+    } else {
+      atomicAdd(G.rsum + kGluTokStride * m, sum);
+    }
   }
   // The warp that finishes the last quantisation work writes the scales and code sums.
   __threadfence();
@@ -483,8 +477,8 @@ __device__ __noinline__ bool glu_quant_unit(const GvParams& P, int q, int N, con
   if (static_cast<int>(old) == G.q_warps - 1) {
     __threadfence();
     if (lane < M) {
-      G.scale[lane] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(__ldcg(G.amax + lane)), 1e-5f));
-      G.rowsum[lane] = __ldcg(G.rsum + lane);
+      G.scale[lane] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(__ldcg(G.amax + kGluTokStride * lane)), 1e-5f));
+      G.rowsum[lane] = __ldcg(G.rsum + kGluTokStride * lane);
     }
   }
   return true;
@@ -544,35 +538,70 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       bool waited = false;  // grid dependency
       bool ok = true;
       int unit = unit_first;
-      int st0 = 0;  // first stage of the current unit still to issue
+      // The layer, row block and stage range of a unit.  A unit of the fused
+      // gate/up launch is 32 output rows: each half-stage holds those 32 gate
+      // rows, then the same 32 up rows.
+      auto locate = [&](int u, const GvLayer*& Lp, int& rb, int& s0, int& s1) {
+        if constexpr (kGlu) {
+          Lp = &P.layer[P.glu.gate];
+          rb = u;
+          s0 = 0;
+          s1 = (Lp->K + kGvStageK - 1) / kGvStageK;
+        } else {
+          int l = 0;
+          while (l + 1 < P.n_layers && u >= P.layer[l + 1].unit0) ++l;
+          Lp = &P.layer[l];
+          rb = u - Lp->unit0;
+          stage_range((Lp->K + kGvStageK - 1) / kGvStageK, ks, rank, s0, s1);
+        }
+      };
+      auto load_weights = [&](const GvLayer& L, int rb, int st, uint32_t full, uint32_t dst) {
+        if constexpr (kGlu) {
+          const GvLayer& LU = P.layer[P.glu.up];
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const uint32_t d = dst + hf * (kGvStageBytes / 2);
+            tma_load_2d(d, &L.tmap, st * 256 + hf * 128, rb * (kGvRows / 2), full);
+            tma_load_2d(d + (kGvRows / 2) * 128, &LU.tmap, st * 256 + hf * 128, rb * (kGvRows / 2), full);
+          }
+        } else {
+          tma_load_2d(dst, &L.tmap, st * 256, rb * kGvRows, full);
+          tma_load_2d(dst + kGvStageBytes / 2, &L.tmap, st * 256 + 128, rb * kGvRows, full);
+        }
+      };
+      // The stage's activation tiles (streamed codes), in the same slot after the weights.
+      auto load_act = [&](const GvLayer& L, int st, uint32_t full, uint32_t dst) {
+        tma_load_3d(dst + kGvStageBytes, &L.xmap, 0, 8 * st, 0, full);
+        tma_load_3d(dst + kGvStageBytes + kXHalf, &L.xmap, 0, 8 * st + 4, 0, full);
+      };
+      constexpr uint32_t kStageTx = kGvStageBytes + (kStream ? 2 * TT * 4 * 128 : 0);
+      // The next ticket (none when each block takes only its own unit).
+      auto next_unit = [&]() {
+        if (P.one_unit) return P.total_units;
+        if (!waited) {
+          griddep_wait();  // the ticket counter is reset by the preceding launch
+          waited = true;
+        }
+        return static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(P.tickets, 1u));
+      };
+      int st0 = -1;  // first stage of the current unit still to issue (-1: all)
       if constexpr (kStream) {
         // Before the grid dependency: the weights of the first unit's first
         // stages (a whole ring of them); their activation tiles, written by
         // the preceding kernel, follow once it has finished.
         if (unit < P.total_units && !(kGlu && unit >= P.glu.q_unit0)) {
-          int l = 0;
-          while (l + 1 < P.n_layers && unit >= P.layer[l + 1].unit0) ++l;
-          const GvLayer& L = P.layer[l];
-          const int rb = unit - L.unit0;
-          int s0, s1;
-          stage_range((L.K + kGvStageK - 1) / kGvStageK, ks, rank, s0, s1);
+          const GvLayer* Lp;
+          int rb, s0, s1;
+          locate(unit, Lp, rb, s0, s1);
           const int pre = s1 - s0 < nring ? s1 - s0 : nring;
           for (int j = 0; j < pre; ++j) {  // fresh slots 0 .. pre-1
-            const int st = s0 + j;
             tags[j] = unit;
-            const uint32_t full = bar0 + 8 * j, dst = ring + j * kSlot;
-            mbar_arrive_expect_tx(full, kGvStageBytes + 2 * TT * 4 * 128);
-            tma_load_2d(dst, &L.tmap, st * 256, rb * kGvRows, full);
-            tma_load_2d(dst + kGvStageBytes / 2, &L.tmap, st * 256 + 128, rb * kGvRows, full);
+            mbar_arrive_expect_tx(bar0 + 8 * j, kStageTx);
+            load_weights(*Lp, rb, s0 + j, bar0 + 8 * j, ring + j * kSlot);
           }
           griddep_wait();  // the codes come from the preceding kernel
           waited = true;
-          for (int j = 0; j < pre; ++j) {
-            const int st = s0 + j;
-            const uint32_t full = bar0 + 8 * j, dst = ring + j * kSlot;
-            tma_load_3d(dst + kGvStageBytes, &L.xmap, 0, 8 * st, 0, full);
-            tma_load_3d(dst + kGvStageBytes + kXHalf, &L.xmap, 0, 8 * st + 4, 0, full);
-          }
+          for (int j = 0; j < pre; ++j) load_act(*Lp, s0 + j, bar0 + 8 * j, ring + j * kSlot);
           issued = pre;
           slot = pre % nring;
           phase = pre == nring ? 1 : 0;
@@ -587,52 +616,31 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           mbar_arrive(bar0 + 8 * slot);
           ++issued;
           if (++slot == nring) { slot = 0; phase ^= 1; }
-          st0 = 0;
-          if (P.one_unit) {
-            unit = P.total_units;
-          } else {
-            if (!waited) {
-              griddep_wait();  // the ticket counter is reset by the preceding launch
-              waited = true;
-            }
-            unit = static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(P.tickets, 1u));
-          }
+          unit = next_unit();
           continue;
         }
-        int l = 0;
-        while (l + 1 < P.n_layers && unit >= P.layer[l + 1].unit0) ++l;
-        const GvLayer& L = P.layer[l];
-        const int rb = unit - L.unit0;
-        int s0, s1;
-        stage_range((L.K + kGvStageK - 1) / kGvStageK, ks, rank, s0, s1);
-        for (int st = st0 > s0 ? st0 : s0; st < s1; ++st) {
+        const GvLayer* Lp;
+        int rb, s0, s1;
+        locate(unit, Lp, rb, s0, s1);
+        for (int st = st0 >= 0 ? st0 : s0; st < s1; ++st) {
           if (!mbar_wait(bar0 + 8 * (nring + slot), phase ^ 1, ctl)) { ok = false; break; }
           tags[slot] = unit;
           const uint32_t full = bar0 + 8 * slot, dst = ring + slot * kSlot;
-          mbar_arrive_expect_tx(full, kStream ? kGvStageBytes + 2 * TT * 4 * 128 : kGvStageBytes);
-          tma_load_2d(dst, &L.tmap, st * 256, rb * kGvRows, full);
-          tma_load_2d(dst + kGvStageBytes / 2, &L.tmap, st * 256 + 128, rb * kGvRows, full);
+          mbar_arrive_expect_tx(full, kStageTx);
+          load_weights(*Lp, rb, st, full, dst);
           if constexpr (kStream) {
             if (!waited) {
               griddep_wait();  // the codes come from the preceding kernel
               waited = true;
             }
-            tma_load_3d(dst + kGvStageBytes, &L.xmap, 0, 8 * st, 0, full);
-            tma_load_3d(dst + kGvStageBytes + kXHalf, &L.xmap, 0, 8 * st + 4, 0, full);
+            load_act(*Lp, st, full, dst);
           }
           ++issued;
           if (++slot == nring) { slot = 0; phase ^= 1; }
         }
-        st0 = 0;
-        if (P.one_unit) {
-          unit = P.total_units;
-        } else {
-          if (!waited) {
-            griddep_wait();  // the ticket counter is reset by the preceding launch
-            waited = true;
-          }
-          unit = static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(P.tickets, 1u));
-        }
+        st0 = -1;
+        if (!ok) break;
+        unit = next_unit();
       }
       if (ok) {
         // End marker: one more phase on the next slot, with no data.
@@ -651,11 +659,15 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
     // ---- consumers ----
     griddep_wait();  // activations may be the preceding kernel's output
     const int g = lane >> 2, t = lane & 3;
-    const int r_lo = warp * 16 + g;  // rows of this lane within the unit (and + 8)
-    // Byte offsets of this lane's weight chunks 2t, 2t+1 of rows r_lo, r_lo+8 within a
+    // The lane's two rows of the stage in the mma path: g and g + 8 of the
+    // warp's 16; in the fused gate/up launch, gate row 8 * warp + g and the
+    // same up row, 32 rows further on.
+    const int row_lo = kGlu ? warp * 8 + g : warp * 16 + g;
+    const int row_hi = kGlu ? 32 + warp * 8 + g : row_lo + 8;
+    // Byte offsets of this lane's weight chunks 2t, 2t+1 of those rows within a
     // 128-byte-swizzled half-stage: chunk c of row r sits at chunk position c ^ (r & 7).
-    const uint32_t w_lo0 = r_lo * 128 + (((2 * t) ^ g) << 4), w_lo1 = r_lo * 128 + (((2 * t + 1) ^ g) << 4);
-    const uint32_t w_hi0 = w_lo0 + 8 * 128, w_hi1 = w_lo1 + 8 * 128;
+    const uint32_t w_lo0 = row_lo * 128 + (((2 * t) ^ g) << 4), w_lo1 = row_lo * 128 + (((2 * t + 1) ^ g) << 4);
+    const uint32_t w_hi0 = row_hi * 128 + (((2 * t) ^ g) << 4), w_hi1 = row_hi * 128 + (((2 * t + 1) ^ g) << 4);
     // Streamed activations: row 4m + t of a half tile holds block t of token m.
     uint32_t x_row[TG];
     int x_sw[TG];
@@ -672,28 +684,47 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       // The first unit is the block's index, so its activations can be
       // quantised while its first weight stage is still on the way.
       if (unit_first < P.total_units && !(kGlu && unit_first >= P.glu.q_unit0)) {
-        int l = 0;
-        while (l + 1 < P.n_layers && unit_first >= P.layer[l + 1].unit0) ++l;
+        int l = kGlu ? P.glu.gate : 0;
+        if constexpr (!kGlu) {
+          while (l + 1 < P.n_layers && unit_first >= P.layer[l + 1].unit0) ++l;
+        }
         stage_activations<TT, TX>(P.layer[l], M, xs, P.x_pitch, s_tok, rs_tok, scratch);
         staged = P.layer[l].x;
         staged_k = P.layer[l].K;
       }
     }
+    bool glu_done = !kGlu;  // this warp has counted itself done with its units
+    float hmax[TG][2];      // the fused gate/up launch: this lane's running max of |h| per token
+#pragma unroll
+    for (int tg = 0; tg < TG; ++tg) hmax[tg][0] = hmax[tg][1] = 0.0f;
     while (true) {
       const bool got0 = mbar_wait(bar0 + 8 * slot, phase, ctl);
       if (!__all_sync(0xffffffffu, got0)) break;
       const int unit = tags[slot];
-      if (unit == kGvTagEnd) break;
-      if (kGlu && unit >= P.glu.q_unit0) {
-        // A quantisation unit: release the (empty) slot, then quantise.
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));
-        if (++slot == nring) { slot = 0; phase ^= 1; }
-        if (!glu_quant_unit<TY>(P, unit - P.glu.q_unit0, P.layer[P.glu.gate].N, ctl)) break;
-        continue;
+      if (unit == kGvTagEnd) {
+        if constexpr (kGlu) {
+          if (!glu_done) glu_warp_done<TG, kAlu>(P, hmax);
+        }
+        break;
       }
-      int l = 0;
-      while (l + 1 < P.n_layers && unit >= P.layer[l + 1].unit0) ++l;
+      if constexpr (kGlu) {
+        if (unit >= P.glu.q_unit0) {
+          // A quantisation unit: release the (empty) slot, then quantise.
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));
+          if (++slot == nring) { slot = 0; phase ^= 1; }
+          if (!glu_done) {
+            glu_warp_done<TG, kAlu>(P, hmax);
+            glu_done = true;
+          }
+          if (!glu_quant_unit<TY>(P, unit - P.glu.q_unit0, P.layer[P.glu.gate].N, ctl)) break;
+          continue;
+        }
+      }
+      int l = kGlu ? P.glu.gate : 0;
+      if constexpr (!kGlu) {
+        while (l + 1 < P.n_layers && unit >= P.layer[l + 1].unit0) ++l;
+      }
       const GvLayer& L = P.layer[l];
       int s0, s1;  // this CTA's stages of the unit
       stage_range((L.K + kGvStageK - 1) / kGvStageK, ks, rank, s0, s1);
@@ -708,6 +739,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
 
       // The epilogue's scalars, loaded now so their latency hides behind the products.
       const float gamma = __ldg(L.gamma);
+      const float gamma_up = kGlu ? __ldg(P.layer[P.glu.up].gamma) : 0.0f;
       int rsum_m[TG][2];
       float s_m[TG][2];
 #pragma unroll
@@ -733,7 +765,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       }
 
       int d[TG][4][4];      // mma path: accumulator fragments
-      int dr[kAlu ? 4 : 1][4];   // one-token path: rows warp*16 + (lane >> 3) + 4*it, one set per code position j
+      int dr[kAlu ? 4 : 1][4];   // one-token path: the lane's four rows, one set per code position j
 #pragma unroll
       for (int tg = 0; tg < TG; ++tg)
 #pragma unroll
@@ -745,20 +777,36 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
 #pragma unroll
         for (int j = 0; j < 4; ++j) dr[r][j] = 0;
       bool ok = true;
-      for (int i = s0; i < s1; ++i) {
+      for (int i = s0; i < s1 && ok; ++i) {
         if (i > s0) {
           const bool got = mbar_wait(bar0 + 8 * slot, phase, ctl);
           if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         }
         const uint32_t wt = ring + slot * kSlot;
         if constexpr (kAlu) {
-          // Lane (rs, ch) = (lane >> 3, lane & 7) takes 16-byte chunk ch of rows
-          // warp*16 + rs + 4*it of each half (inputs 64ch .. 64ch+63 of the half) and the
-          // matching 64 codes: one AND and one dp4a per four weights, no idle mma
-          // columns.  Each 8-lane phase reads one 128-byte swizzled row.
+          // Lane (rs, ch) = (lane >> 3, lane & 7) takes 16-byte chunk ch of four
+          // rows of its warp in each half (inputs 64ch .. 64ch+63 of the half)
+          // and the matching 64 codes: one AND and one dp4a per four weights,
+          // no idle mma columns.  Each 8-lane phase reads one 128-byte swizzled
+          // row.  Rows: warp*16 + rs + 4*it; in the fused gate/up launch the
+          // first two are gate rows warp*8 + rs + 4*it, the last two the same
+          // up rows.
+          const int ch = lane & 7, rs = lane >> 3;
+          uint4 wv[2][4];
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int row = kGlu ? (it < 2 ? warp * 8 + rs + 4 * it : 32 + warp * 8 + rs + 4 * (it - 2))
+                                   : warp * 16 + rs + 4 * it;
+              wv[hf][it] = lds128(wt + hf * (kGvStageBytes / 2) + row * 128 + ((ch ^ (row & 7)) << 4));
+            }
+          if constexpr (!kStream) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // the slot held only weights, now in registers
+          }
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
-            const int ch = lane & 7, rs = lane >> 3;
             const int k0 = i * kGvStageK + hf * (kGvStageK / 2) + 64 * ch;
             if (k0 < L.K) {  // inputs past K have zero weights (K is a multiple of 64)
               uint4 xc[4];
@@ -771,21 +819,19 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
                   xc[u] = lds128(xs + x_chunk_off((k0 >> 4) + u));
                 }
               }
-              const uint32_t base = wt + hf * (kGvStageBytes / 2);
 #pragma unroll
-              for (int it = 0; it < 4; ++it) {
-                const int row = warp * 16 + rs + 4 * it;
-                const uint4 wv = lds128(base + row * 128 + ((ch ^ (row & 7)) << 4));
+              for (int it = 0; it < 4; ++it)
 #pragma unroll
                 for (int v = 0; v < 4; ++v)
 #pragma unroll
                   for (int j = 0; j < 4; ++j)
-                    dr[it][j] = dp4a_us(u4_get(wv, v) & (0x03030303u << (2 * j)), u4_get(xc[v], j), dr[it][j]);
-              }
+                    dr[it][j] = dp4a_us(u4_get(wv[hf][it], v) & (0x03030303u << (2 * j)), u4_get(xc[v], j), dr[it][j]);
             }
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // done with the slot
+          if constexpr (kStream) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // done with the slot's activations too
+          }
         } else {
           uint4 w[2][4];  // [half][lo0, lo1, hi0, hi1]
 #pragma unroll
@@ -800,11 +846,11 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
             __syncwarp();
             if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));  // the slot held only weights, now in registers
           }
-          const uint32_t xt = wt + kGvStageBytes;
 
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
-            const int qblk = i * 8 + hf * 4 + t;  // this lane's 128-input block (whole-K staging)
+            const uint32_t xt = wt + kGvStageBytes + hf * kXHalf;  // streamed: this half's tile
+            const int qblk = i * 8 + hf * 4 + t;                   // this lane's 128-input block (whole-K staging)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const uint4 wl = w[hf][h], wh = w[hf][2 + h];
@@ -817,7 +863,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
                   const int m = tg * 8 + g;
                   if (m < M) {
                     if constexpr (kStream) {
-                      const uint32_t row = xt + hf * kXHalf + x_row[tg];
+                      const uint32_t row = xt + x_row[tg];
                       xa[tg] = lds128(row + ((c0 ^ x_sw[tg]) << 4));
                       xb[tg] = lds128(row + (((c0 + 1) ^ x_sw[tg]) << 4));
                     } else {
@@ -892,12 +938,17 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           }
       }
 
-      // Finish the unit: y = (sum c*q - sum q) * (gamma / s).
-      const int n_base = (unit - L.unit0) * kGvRows;
+      // Finish the unit: y = (sum c*q - sum q) * (gamma / s).  The fused
+      // gate/up launch instead forms h = act(gate) * up from the lane's gate
+      // and up sums of the same output row (each output rounded to the
+      // activation type first, as a stored output is), stores h and folds
+      // |h| into the per-token maxima.
+      const int n_base = (kGlu ? unit : unit - L.unit0) * (kGlu ? kGvRows / 2 : kGvRows);
       TY* y = static_cast<TY*>(L.y);
       if constexpr (kAlu) {
-        // A butterfly over the 8 lanes of a row group leaves row
-        // warp*16 + (lane >> 3) + 4*((lane >> 1) & 3) summed in lanes 2r and 2r + 1.
+        // A butterfly over the 8 lanes of a row group leaves the lane's row
+        // number (lane >> 3) + 4*((lane >> 1) & 3) of the warp's 16 summed in
+        // lanes 2r and 2r + 1.
         int v[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) v[r] = pc[0][r];
@@ -908,28 +959,77 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
 #pragma unroll
           for (int r = 0; r < half; ++r) {
             const int send = upper ? v[r] : v[r + half];
-            const int keep = upper ? v[r + half] : v[r];
-            v[r] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+            const int keep_v = upper ? v[r + half] : v[r];
+            v[r] = keep_v + __shfl_xor_sync(0xffffffffu, send, off);
           }
         }
         v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
-        const int n = n_base + warp * 16 + (lane >> 3) + 4 * ((lane >> 1) & 3);
-        if ((lane & 1) == 0 && n < L.N) {
-          const int rsum = kStream ? rsum1 : rs_tok[0];
-          const float sm = kStream ? s1tok : s_tok[0];
-          const int a = v[0] - rsum;
-          const float val = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, sm));
-          if constexpr (sizeof(TY) == 4) y[n] = val; else y[n] = __float2bfloat16_rn(val);
-          if (L.acc_out) L.acc_out[n] = a;
+        const int rsum = kStream ? rsum1 : rs_tok[0];
+        const float sm = kStream ? s1tok : s_tok[0];
+        if constexpr (kGlu) {
+          // Row numbers 0..7 of the warp's 16 are gate rows, 8..15 the same up
+          // rows: a gate lane finds its up sum in lane ^ 4.
+          const int vu = __shfl_xor_sync(0xffffffffu, v[0], 4);
+          const int n = n_base + warp * 8 + (lane >> 3) + 4 * ((lane >> 1) & 1);
+          float habs = 0.0f;
+          if ((lane & 5) == 0 && n < L.N) {
+            const float g_v = round_to<TY>(__fmul_rn(static_cast<float>(v[0] - rsum), __fdiv_rn(gamma, sm)));
+            const float u_v = round_to<TY>(__fmul_rn(static_cast<float>(vu - rsum), __fdiv_rn(gamma_up, sm)));
+            const float h = glu_value<TY>(g_v, u_v, P.glu.act);
+            TY* hp = static_cast<TY*>(P.glu.h);
+            if constexpr (sizeof(TY) == 4) hp[n] = h; else hp[n] = __float2bfloat16_rn(h);
+            habs = fabsf(h);
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) habs = fmaxf(habs, __shfl_xor_sync(0xffffffffu, habs, o));
+          hmax[0][0] = fmaxf(hmax[0][0], habs);
+        } else {
+          const int n = n_base + warp * 16 + (lane >> 3) + 4 * ((lane >> 1) & 3);
+          if ((lane & 1) == 0 && n < L.N) {
+            const int a = v[0] - rsum;
+            const float val = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, sm));
+            if constexpr (sizeof(TY) == 4) y[n] = val; else y[n] = __float2bfloat16_rn(val);
+            if (L.acc_out) L.acc_out[n] = a;
+          }
         }
-        if constexpr (kGlu) glu_rows<TY>(P, unit - L.unit0, warp, L.N);
+        continue;
+      }
+      if constexpr (kGlu) {
+        // Fragment c holds row g (c < 2: a gate row) or g + 8 (the same up row)
+        // for token 2t + (c & 1).
+#pragma unroll
+        for (int tg = 0; tg < TG; ++tg)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int n = n_base + warp * 8 + g;
+            const int m = tg * 8 + 2 * t + e;
+            float habs = 0.0f;
+            if (n < L.N && m < M) {
+              const int rsum = kStream ? rsum_m[tg][e] : rs_tok[m];
+              const float sm = kStream ? s_m[tg][e] : s_tok[m];
+              const int ag = d[tg][0][e] + (d[tg][1][e] >> 2) + (d[tg][2][e] >> 4) + (d[tg][3][e] >> 6) - rsum;
+              const int au = d[tg][0][e + 2] + (d[tg][1][e + 2] >> 2) + (d[tg][2][e + 2] >> 4) +
+                             (d[tg][3][e + 2] >> 6) - rsum;
+              const float g_v = round_to<TY>(__fmul_rn(static_cast<float>(ag), __fdiv_rn(gamma, sm)));
+              const float u_v = round_to<TY>(__fmul_rn(static_cast<float>(au), __fdiv_rn(gamma_up, sm)));
+              const float h = glu_value<TY>(g_v, u_v, P.glu.act);
+              TY* hp = static_cast<TY*>(P.glu.h);
+              const size_t o = static_cast<size_t>(m) * L.N + n;
+              if constexpr (sizeof(TY) == 4) hp[o] = h; else hp[o] = __float2bfloat16_rn(h);
+              habs = fabsf(h);
+            }
+            // Per token: the 8 lanes (g) holding it.
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) habs = fmaxf(habs, __shfl_xor_sync(0xffffffffu, habs, o));
+            hmax[tg][e] = fmaxf(hmax[tg][e], habs);
+          }
         continue;
       }
 #pragma unroll
       for (int tg = 0; tg < TG; ++tg)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const int n = n_base + r_lo + ((c & 2) ? 8 : 0);
+          const int n = n_base + row_lo + ((c & 2) ? 8 : 0);
           const int m = tg * 8 + 2 * t + (c & 1);
           if (n < L.N && m < M) {
             const int rsum = kStream ? rsum_m[tg][c & 1] : rs_tok[m];
@@ -941,7 +1041,6 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
             if (L.acc_out) L.acc_out[o] = a;
           }
         }
-      if constexpr (kGlu) glu_rows<TY>(P, unit - L.unit0, warp, L.N);
     }
   }
 
@@ -1046,11 +1145,11 @@ void gemv_force_ksplit(int ks) { g_force_ksplit = ks > 0 ? ks : 0; }
 
 constexpr int kGluQuantElems = 2048;  // elements of h per quantisation unit
 
-// Zeroed scratch of a fused gate/up launch: the pair counters (one per 16-row
-// group), then amax[16], rsum[16], done[2].
+// Zeroed scratch of a fused gate/up launch: amax and rsum (one 128-byte line
+// per token, 16 tokens each), then done[2].
 size_t gemv_glu_scratch_bytes(int N) {
-  const size_t groups = static_cast<size_t>((N + kGvRows - 1) / kGvRows) * kGvWarps;
-  return (groups * 4 + 255) / 256 * 256 + 256;
+  (void)N;
+  return 2 * 16 * kGluTokStride * 4 + 256;
 }
 
 cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, int x_type, int y_type,
@@ -1080,9 +1179,10 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
     const GemvLayerArgs& a = layers[order[i]];
     GvLayer& L = P.layer[i];
     {
+      // The fused gate/up launch loads 32 rows of each layer per half-stage.
       const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K / 4), static_cast<cuuint64_t>(a.N)};
       const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K / 4)};
-      const cuuint32_t box[2] = {128, kGvRows};
+      const cuuint32_t box[2] = {128, glu ? kGvRows / 2 : kGvRows};
       const cuuint32_t estr[2] = {1, 1};
       if (enc(&L.tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.packed), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
@@ -1139,8 +1239,10 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   if (ks < 1 || glu) ks = 1;  // the fused gate/up launch hands its quantisation units out by ticket
   P.ksplit = ks;
   if (glu) {
+    // Tickets: one per unit of 64 rows of both layers, then the quantisation units.
     GvGlu& G = P.glu;
     const int N = layers[0].N;
+    const int row_units = (N + kGvRows / 2 - 1) / (kGvRows / 2);  // 32 output rows each
     const long long elems = static_cast<long long>(M) * N;
     const int q_units = static_cast<int>((elems + kGluQuantElems - 1) / kGluQuantElems);
     G.on = 1;
@@ -1149,26 +1251,21 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
       if (order[i] == 0) G.gate = i;
       if (order[i] == 1) G.up = i;
     }
-    G.q_unit0 = units;
+    G.q_unit0 = row_units;
     G.q_elems = kGluQuantElems;
-    G.groups = ((N + kGvRows - 1) / kGvRows) * kGvWarps;
     G.q_warps = q_units * kGvWarps;
-    G.yg = layers[0].y;
-    G.yu = layers[1].y;
     G.h = glu->h;
     G.xq = glu->xq;
     G.scale = glu->scale;
     G.rowsum = glu->rowsum;
-    G.pair_cnt = glu->zeroed;
-    uint32_t* small =
-        reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(glu->zeroed) + gemv_glu_scratch_bytes(N) - 256);
-    G.amax = small;
-    G.rsum = reinterpret_cast<int32_t*>(small + 16);
-    G.done = small + 32;
-    units += q_units;
+    uint32_t* z = glu->zeroed;
+    G.amax = z;
+    G.rsum = reinterpret_cast<int32_t*>(z + 16 * kGluTokStride);
+    G.done = z + 2 * 16 * kGluTokStride;
+    units = row_units + q_units;
     P.total_units = units;
   }
-  // kGvBlocksPerSM blocks per SM, each with the deepest ring that fits beside its other data.
+  // kGvBlocksPerSM blocks per SM, each with the deepest weight ring that fits beside its other data.
   const int slot = kGvStageBytes + (stream_x ? 2 * x_half_bytes(tt) : 0);
   const int fixed = gemv_smem_bytes(M, k_max, 0, stream_x, ks);
   int nring = (kGvSmemPerBlock - fixed) / (slot + 16);

@@ -110,10 +110,10 @@ bool gemv_fuses_quant(int M, int K, int x_bf16);
 void gemv_force_ksplit(int ks);
 
 // The FFN's gated activation fused into the launch of its gate and up
-// BitLinears (layers[0] = gate, layers[1] = up, same N and K, their y in
-// scratch): h = act(gate) * up [M][N] in the activation type, and its
-// per-token quantisation (codes [M][N], scales, code sums) for the down
-// BitLinear.  `zeroed`: gemv_glu_scratch_bytes(N) bytes, zero at launch.
+// BitLinears (layers[0] = gate, layers[1] = up, same N and K; their y are
+// not written): h = act(gate) * up [M][N] in the activation type (y_type),
+// and its per-token quantisation (codes [M][N], scales, code sums) for the
+// down BitLinear.  `zeroed`: gemv_glu_scratch_bytes(N) bytes, zero at launch.
 struct GemvGluArgs {
   int act;  // GluAct
   void* h;
