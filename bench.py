@@ -69,7 +69,7 @@ def parse_args(argv=None):
     p.add_argument("--only", choices=["chain70b", "decode2b", "prefill", "decode3b", "next", "ffn"], default=None,
                    help="run one workload alone and print its own line (a small case for profiling)")
     p.add_argument("--tokens", type=str, default=None,
-                   help="with --only chain70b / ffn: the token counts to run, comma-separated")
+                   help="with --only chain70b / ffn / decode3b: the token counts to run, comma-separated")
     return p.parse_args(argv)
 
 
@@ -590,7 +590,7 @@ DECODE_3B = [(3200, 8640), (8640, 3200)]  # (K in, N out)
 DECODE_3B_TOKENS = (1, 2, 4, 8, 16)
 
 
-def run_decode_3b(args, world, peaks, L2):
+def run_decode_3b(args, world, peaks, L2, tokens=None):
     """The 3B-class decode sweep: one BitLinear per step through the public
     single-layer call (quantisation and product), 1 to 16 tokens."""
     import ternary_weight_a8_b200 as tb
@@ -599,7 +599,7 @@ def run_decode_3b(args, world, peaks, L2):
                        "1/2/4/8/16 tokens, one forward call per step"}
     for li, (K, N) in enumerate(DECODE_3B):
         sets, set_bytes = make_layer_sets([(K, N)], seed=500 + li, min_bytes=4 * L2)
-        for M in DECODE_3B_TOKENS:
+        for M in (tokens or DECODE_3B_TOKENS):
             xs, ys = make_inputs([(K, N)], M, seed=500 + li)
             x, y = xs[0], ys[0]
             ws = tb.new_workspace(tb.workspace_bytes(M, N, K))
@@ -1007,9 +1007,10 @@ def main():
                                   **({"tokens": tokens} if tokens else {}))
         elif args.only == "ffn":
             res = run_ffn(args, world, peaks, L2, **({"tokens": tokens} if tokens else {}))
+        elif args.only == "decode3b":
+            res = run_decode_3b(args, world, peaks, L2, tokens=tokens)
         else:
-            fn = {"decode2b": run_decode_2b, "prefill": run_prefill, "decode3b": run_decode_3b,
-                  "next": run_next}[args.only]
+            fn = {"decode2b": run_decode_2b, "prefill": run_prefill, "next": run_next}[args.only]
             res = fn(args, world, peaks, L2)
         if rank == 0:
             print(json.dumps(res), flush=True)

@@ -202,28 +202,35 @@ struct NormParams {
   int K;
 };
 
-// v = round_to_TX(x * r [* g]) for the 16 inputs of chunk c.
-template <typename TX>
-__device__ __forceinline__ void norm_chunk(const Chunk16& raw, float r, const float* gain, int c, float (&v)[16]) {
-  float gv[16];
-  if (gain) {
-    const float4* gp = reinterpret_cast<const float4*>(gain + 16 * c);
+// The gains of chunk c (16 floats).
+__device__ __forceinline__ void load_gain16(const float* gain, int c, float4 (&g)[4]) {
+  const float4* gp = reinterpret_cast<const float4*>(gain + 16 * c);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 t = __ldg(gp + i);
-      gv[4 * i] = t.x;
-      gv[4 * i + 1] = t.y;
-      gv[4 * i + 2] = t.z;
-      gv[4 * i + 3] = t.w;
-    }
-  }
+  for (int i = 0; i < 4; ++i) g[i] = __ldg(gp + i);
+}
+
+// v = round_to_TX(x * r [* g]) for the 16 inputs of a chunk, g its gains.
+template <typename TX>
+__device__ __forceinline__ void norm_vals(const Chunk16& raw, float r, bool has_gain, const float4 (&g)[4],
+                                          float (&v)[16]) {
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
     float t = __fmul_rn(elem<TX>(raw, e), r);
-    if (gain) t = __fmul_rn(t, gv[e]);
+    if (has_gain) {
+      const float4 q = g[e >> 2];
+      t = __fmul_rn(t, (e & 3) == 0 ? q.x : (e & 3) == 1 ? q.y : (e & 3) == 2 ? q.z : q.w);
+    }
     if constexpr (sizeof(TX) == 2) t = __bfloat162float(__float2bfloat16_rn(t));
     v[e] = t;
   }
+}
+
+// The same, loading the gains of chunk c.
+template <typename TX>
+__device__ __forceinline__ void norm_chunk(const Chunk16& raw, float r, const float* gain, int c, float (&v)[16]) {
+  float4 g[4];
+  if (gain) load_gain16(gain, c, g);
+  norm_vals<TX>(raw, r, gain != nullptr, g, v);
 }
 
 // Codes of 16 values (one 16-byte store), and the values themselves in the
@@ -274,11 +281,23 @@ __global__ void __launch_bounds__(kQuantMaxThreads) rmsnorm_quant_kernel(const _
   TX* nr = P.x_norm ? static_cast<TX*>(P.x_norm) + static_cast<size_t>(m) * K : nullptr;
   const bool in_regs = chunks <= T * kQuantRegChunks;
   Chunk16 reg[kQuantRegChunks];
+  // When the token is in registers, the gains of the thread's first kNormKeep
+  // chunks are fetched with it (off the path between the two reductions), and
+  // the normalised values of those chunks are kept for the codes.
+  constexpr int kNormKeep = 2;
+  float4 gpre[kNormKeep][4];
   if (in_regs) {
 #pragma unroll
     for (int i = 0; i < kQuantRegChunks; ++i) {
       const int c = threadIdx.x + i * T;
       if (c < chunks) load16<TX>(xr + c * 16, reg[i]);
+    }
+    if (P.gain) {
+#pragma unroll
+      for (int k = 0; k < kNormKeep; ++k) {
+        const int c = threadIdx.x + k * T;
+        if (c < chunks) load_gain16(P.gain, c, gpre[k]);
+      }
     }
   }
   // fn(chunk, c) over this thread's chunks: from registers, or read again.
@@ -311,15 +330,24 @@ __global__ void __launch_bounds__(kQuantMaxThreads) rmsnorm_quant_kernel(const _
   const double ms = __ddiv_rn(ss, static_cast<double>(K));
   const float r = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(ms, static_cast<double>(P.eps)))));
 
-  // Absmax of the normalised token.  When the token is in registers the
-  // normalised values of the thread's first kNormKeep chunks stay there too.
-  constexpr int kNormKeep = 2;
+  // Absmax of the normalised token.
   float vkeep[kNormKeep][16];
   float amax = 0.0f;
   for_each_chunk([&](const Chunk16& ch, int c) {
     float v[16];
-    norm_chunk<TX>(ch, r, P.gain, c, v);
     const int i = (c - static_cast<int>(threadIdx.x)) / T;
+    if (in_regs && P.gain && i < kNormKeep) {
+      float4 g[4];
+#pragma unroll
+      for (int k = 0; k < kNormKeep; ++k)
+        if (i == k) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) g[q] = gpre[k][q];
+        }
+      norm_vals<TX>(ch, r, true, g, v);
+    } else {
+      norm_chunk<TX>(ch, r, P.gain, c, v);
+    }
 #pragma unroll
     for (int k = 0; k < kNormKeep; ++k)
       if (in_regs && i == k) {

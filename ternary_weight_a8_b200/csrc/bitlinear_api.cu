@@ -377,7 +377,7 @@ static int forward_on(const uint8_t* packed, const float* gamma, int N, int K, c
   BL_TRY(choose_gemv(M, K, &gemv));
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   const int yt = y_dtype == BL_BF16 ? bl::kOutBF16 : bl::kOutF32;
-  if (gemv && bl::gemv_fuses_quant(M, K, x_dtype == BL_BF16)) {
+  if (gemv && bl::gemv_fuses_quant(M, K, x_dtype == BL_BF16, true)) {
     // Small activations: the decode kernel quantises them itself (one launch).
     const bl::GemvLayerArgs L{packed, gamma, N, K, x, nullptr, nullptr, 0, y, acc_out};
     cudaError_t e = bl::launch_gemv_group(&L, 1, M, x_dtype == BL_BF16 ? bl::kInBF16 : bl::kInF32, yt, status,
@@ -847,7 +847,7 @@ extern "C" int bitlinear_forward_noalloc(const uint8_t* packed, const float* gam
   const FwdLayout l = forward_layout(M, K);
   bool gemv = false;
   BL_TRY(choose_gemv(M, K, &gemv));
-  const bool fused = gemv && bl::gemv_fuses_quant(M, K, x_dtype == BL_BF16);
+  const bool fused = gemv && bl::gemv_fuses_quant(M, K, x_dtype == BL_BF16, true);
   const size_t need = fused ? kStatusBytes : l.total;
   if (need > kNoAllocScratchBytes)
     return fail(BL_ERR_WORKSPACE_TOO_SMALL,

@@ -89,6 +89,7 @@ constexpr int kGvMaxRing = 16;
 constexpr int kGvMaxSplit = 8;        // CTAs of a cluster sharing one unit (the portable cluster limit)
 constexpr int kGvTagEnd = -1;
 constexpr int kGvFuseChunks = 2;      // 16-input chunks a consumer thread quantises itself
+constexpr int kGvFuseChunks1 = 5;     // the same for one bf16 token of a single layer
 constexpr int kGvFuseElems = 4096;    // M*K up to which the blocks quantise activations themselves
 
 struct GvLayer {
@@ -109,34 +110,33 @@ __host__ __device__ constexpr int x_half_bytes(int tt) { return ((tt * 4 * 128 +
 
 // The FFN's gate and up BitLinears in one launch, with the gated activation
 // and the quantisation of its result (the down BitLinear's input) done by the
-// same launch.  A ticket below q_unit0 is a unit of 32 output rows: each
-// half-stage of its weights holds those 32 gate rows, then the same 32 up
-// rows, so that a lane's mma fragment (rows g and g + 8 of its warp's 16), or
-// a dp4a lane and its partner lane ^ 4, holds the gate and up sums of one
-// output row.  The lane rounds both outputs to the activation type, as
-// stored outputs are, forms h = act(gate) * up, stores h and keeps the
-// warp's running maximum of |h| per token in registers.  Each warp
-// publishes its maxima (one atomic max per token, each token's word on a
-// 128-byte line of its own) and counts itself done, once, with a fence, when
-// it meets its first quantisation unit or the end;
-// the tickets from q_unit0 on are quantisation units, each a range of h's
-// elements, which wait until every warp of the grid is done (all units were
-// handed out before them, to running blocks), then quantise with the final
-// per-token scale; the last one writes the scales and code sums.
+// same launch.  A unit is 32 output rows: each half-stage of its weights
+// holds those 32 gate rows, then the same 32 up rows, so that a lane's mma
+// fragment (rows g and g + 8 of its warp's 16), or a dp4a lane and its
+// partner lane ^ 4, holds the gate and up sums of one output row.  The lane
+// rounds both outputs to the activation type, as stored outputs are, forms
+// h = act(gate) * up, stores h and keeps the warp's running maximum of |h|
+// per token in registers.  When the units run out, the block folds its
+// warps' maxima in shared memory, publishes them (one atomic max per token,
+// each token's word on a 128-byte line of its own) and counts itself done,
+// with one fence.  Then the quantisation is spread over the grid: global warp
+// w takes the 512-element slices w, w + W, ... of h (W warps in the grid);
+// its block waits until every block is done, quantises with the final
+// per-token scale and adds its code sums, then counts itself finished; the
+// last block to finish writes the scales and code sums.
 struct GvGlu {
   int on;
   int act;                // kGluRelu2 or kGluSilu
   int gate, up;           // their layer slots
-  int q_unit0;            // first quantisation ticket (= the units of 32 output rows)
-  int q_elems;            // elements of h per quantisation unit (a multiple of 16)
-  int q_warps;            // quantisation units * kGvWarps
+  int q_warps;            // warps with quantisation slices: min(slices, warps in the grid)
+  int q_blocks;           // blocks holding those warps
   void* h;                // [M][N] h, activation type
   int8_t* xq;             // [M][N] codes of h
   float* scale;           // [M]
   int32_t* rowsum;        // [M]
   uint32_t* amax;         // per token m, word 32 m: max |h| as float bits; zero at launch
   int32_t* rsum;          // per token m, word 32 m: sum of h's codes; zero at launch
-  uint32_t* done;         // [2] zero at launch: warps done with units, quantisation warps finished
+  uint32_t* done;         // [2] zero at launch: blocks done with units, quantisation blocks finished
 };
 
 struct GvParams {
@@ -146,6 +146,7 @@ struct GvParams {
   uint32_t* tickets;  // [0] next ticket, [1] blocks done
   int one_unit;       // as many blocks as units: each block takes its own unit, no tickets
   int ksplit;         // CTAs of a cluster that share one unit, each over its own range of stages
+  int narrow;         // 32-row units of 2048-input stages (one token, streamed codes, ksplit 1)
   GvGlu glu;          // the fused gate/up launch (ksplit is 1 then)
 };
 
@@ -202,6 +203,21 @@ __device__ __forceinline__ uint32_t u4_get(const uint4& v, int i) {
 
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kGvConsumers) : "memory");
+}
+
+// The same barrier, returning the OR of every consumer thread's `v` (one
+// decision for the whole block).
+__device__ __forceinline__ bool consumer_sync_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u), "n"(kGvConsumers)
+      : "memory");
+  return r != 0;
 }
 
 // Byte offset of activation chunk (16 bytes) `c` of a staged token row.
@@ -309,7 +325,7 @@ __device__ __forceinline__ void stage_activations(const GvLayer& L, int M, uint3
   const int chunks = K >> 4;
   {
     // At most kChunks chunks per thread (the host keeps M*K within that).
-    constexpr int kChunks = sizeof(TX) == 4 ? kGvFuseChunks / 2 : kGvFuseChunks;
+    constexpr int kChunks = sizeof(TX) == 4 ? kGvFuseChunks / 2 : TT == 1 ? kGvFuseChunks1 : kGvFuseChunks;
     RawChunk raw[kChunks];
     const TX* src = static_cast<const TX*>(L.x) + static_cast<size_t>(m) * K;
 #pragma unroll
@@ -402,15 +418,22 @@ __device__ __forceinline__ bool wait_count(const uint32_t* p, uint32_t target, c
 // L2 slices.
 constexpr int kGluTokStride = 32;
 
-// A consumer warp's units of the fused gate/up launch are done: its
-// per-token maxima of |h| are folded into the grid's (one atomic max per
-// token, from the lanes that hold them), then its h stores and those maxima
-// are made visible and the warp is counted.
+// The consumer warps of a block of the fused gate/up launch are done with
+// their units (every consumer warp calls this once, also after giving up, so
+// that the barriers match): their per-token maxima of |h| are folded through
+// `red` (64 floats of this block's shared memory, free once every consumer
+// warp is past its last stage) and published with one atomic max per token;
+// then the block's h stores and those maxima are made visible (the barrier
+// orders the other warps' stores before warp 0's fence) and the block is
+// counted.  A block that gave up publishes nothing (the others' waits run out).
 template <int TG, bool kAlu>
-__device__ __forceinline__ void glu_warp_done(const GvParams& P, const float (&hmax)[TG][2]) {
-  const int lane = threadIdx.x & 31;
+__device__ __forceinline__ void glu_block_done(const GvParams& P, const float (&hmax)[TG][2], float* red,
+                                               const WaitCtl& ctl) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Every consumer warp is past the ring before it is reused; one decision on giving up.
+  if (consumer_sync_or(*ctl.abort != 0)) return;
   if constexpr (kAlu) {
-    if (lane == 0 && hmax[0][0] > 0.0f) atomicMax(P.glu.amax, __float_as_uint(hmax[0][0]));
+    if (lane == 0) red[warp * 16] = hmax[0][0];
   } else {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
@@ -418,30 +441,73 @@ __device__ __forceinline__ void glu_warp_done(const GvParams& P, const float (&h
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int m = tg * 8 + 2 * t + e;
-        if (g == 0 && m < P.M && hmax[tg][e] > 0.0f)
-          atomicMax(P.glu.amax + kGluTokStride * m, __float_as_uint(hmax[tg][e]));
+        if (g == 0 && m < P.M) red[warp * 16 + m] = hmax[tg][e];
       }
   }
-  __threadfence();
-  __syncwarp();
-  if (lane == 0) atomicAdd(P.glu.done, 1u);
+  consumer_sync();
+  if (warp == 0) {
+    if (lane < P.M) {
+      float v = red[lane];
+#pragma unroll
+      for (int w = 1; w < kGvWarps; ++w) v = fmaxf(v, red[w * 16 + lane]);
+      if (v > 0.0f) atomicMax(P.glu.amax + kGluTokStride * lane, __float_as_uint(v));
+    }
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence();
+      atomicAdd(P.glu.done, 1u);
+    }
+  }
 }
 
-// One quantisation unit: elements [q * q_elems, (q + 1) * q_elems) of h
-// ([M][N], N % 16 == 0, so no 16-element chunk crosses a token), once every
-// consumer warp of the grid is done with its units.  Codes as the quantisation kernel makes them:
-// s = 127 / max(amax, 1e-5), q = clamp(rint(h * s), -128, 127).
+// The quantisation of h ([M][N], N % 16 == 0, so no 16-element chunk crosses
+// a token) by this warp: slices of 512 elements, one 16-element chunk per
+// lane, once every consumer warp of the grid is done with its units.  Codes
+// as the quantisation kernel makes them: s = 127 / max(amax, 1e-5),
+// q = clamp(rint(h * s), -128, 127).
+constexpr int kGluSlice = 512;
+
 template <typename TY>
-__device__ __noinline__ bool glu_quant_unit(const GvParams& P, int q, int N, const WaitCtl& ctl) {
+__device__ __noinline__ void glu_quant_slices(const GvParams& P, int N, const WaitCtl& ctl) {
   const GvGlu& G = P.glu;
-  if (!wait_count(G.done, gridDim.x * kGvWarps, ctl)) return false;
-  const int lane = threadIdx.x & 31, M = P.M;
+  if (static_cast<int>(blockIdx.x) >= G.q_blocks) return;  // block-uniform
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, M = P.M;
+  const int W = static_cast<int>(gridDim.x) * kGvWarps;
+  const int gw = static_cast<int>(blockIdx.x) * kGvWarps + warp;
+  // Warp 0 waits for every block; the barrier passes the outcome on (and
+  // orders warp 0's acquire before the other warps' loads of h).
+  bool bad = false;
+  if (warp == 0) bad = !wait_count(G.done, gridDim.x, ctl);
+  if (consumer_sync_or(bad || *ctl.abort != 0)) return;  // (every warp returns: no barrier follows)
   const long long total = static_cast<long long>(M) * N;
-  const long long e0 = static_cast<long long>(q) * G.q_elems;
-  const long long e1 = e0 + G.q_elems < total ? e0 + G.q_elems : total;
-  for (long long e = e0 + 16LL * threadIdx.x; e < e1; e += 16LL * kGvConsumers) {
+  for (long long e = static_cast<long long>(gw) * kGluSlice + 16 * lane; gw < G.q_warps && e < total;
+       e += static_cast<long long>(W) * kGluSlice) {
     const int m = static_cast<int>(e / N);
     const float s = __fdiv_rn(127.0f, fmaxf(__uint_as_float(__ldcg(G.amax + kGluTokStride * m)), 1e-5f));
+    float hv[16];
+    if constexpr (sizeof(TY) == 4) {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(G.h) + e);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const float4 v = __ldcg(src + b);
+        hv[4 * b] = v.x;
+        hv[4 * b + 1] = v.y;
+        hv[4 * b + 2] = v.z;
+        hv[4 * b + 3] = v.w;
+      }
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(G.h) + e);
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const uint4 v = __ldcg(src + b);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          hv[8 * b + 2 * k] = __uint_as_float(w4[k] << 16);
+          hv[8 * b + 2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u);
+        }
+      }
+    }
     uint32_t w[4];
     int sum = 0;
 #pragma unroll
@@ -449,7 +515,7 @@ __device__ __noinline__ bool glu_quant_unit(const GvParams& P, int q, int N, con
       int c[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        c[k] = __float2int_rn(__fmul_rn(ld_act<TY>(G.h, static_cast<size_t>(e) + 4 * b + k), s));
+        c[k] = __float2int_rn(__fmul_rn(hv[4 * b + k], s));
         c[k] = min(max(c[k], -128), 127);
       }
       w[b] = pack4_s8(c[0], c[1], c[2], c[3]);
@@ -463,37 +529,46 @@ __device__ __noinline__ bool glu_quant_unit(const GvParams& P, int q, int N, con
     if (__all_sync(active, m == m0)) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(active, sum, o);
-      if ((threadIdx.x & 31) == lead) atomicAdd(G.rsum + kGluTokStride * m, sum);
+      if (lane == lead) atomicAdd(G.rsum + kGluTokStride * m, sum);
     } else {
       atomicAdd(G.rsum + kGluTokStride * m, sum);
     }
   }
-  // The warp that finishes the last quantisation work writes the scales and code sums.
-  __threadfence();
-  __syncwarp();
-  uint32_t old = 0;
-  if (lane == 0) old = atomicAdd(G.done + 1, 1u);
-  old = __shfl_sync(0xffffffffu, old, 0);
-  if (static_cast<int>(old) == G.q_warps - 1) {
-    __threadfence();
-    if (lane < M) {
-      G.scale[lane] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(__ldcg(G.amax + kGluTokStride * lane)), 1e-5f));
-      G.rowsum[lane] = __ldcg(G.rsum + kGluTokStride * lane);
+  // The block that finishes the last quantisation work writes the scales and code sums.
+  consumer_sync();
+  if (warp == 0) {
+    uint32_t old = 0;
+    if (lane == 0) {
+      __threadfence();
+      old = atomicAdd(G.done + 1, 1u);
+    }
+    old = __shfl_sync(0xffffffffu, old, 0);
+    if (static_cast<int>(old) == G.q_blocks - 1) {
+      __threadfence();
+      if (lane < M) {
+        G.scale[lane] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(__ldcg(G.amax + kGluTokStride * lane)), 1e-5f));
+        G.rowsum[lane] = __ldcg(G.rsum + kGluTokStride * lane);
+      }
     }
   }
-  return true;
 }
 
-// kMode: 0 plain, 1 K-split over clusters, 2 the fused gate/up launch.
+// kMode: 0 plain, 1 K-split over clusters, 2 the fused gate/up launch,
+// 3 narrow units (one token, streamed codes).
 template <int TT, typename TY, typename TX, int kMode>
 __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(const __grid_constant__ GvParams P) {
   constexpr bool kSplit = kMode == 1;
   constexpr bool kGlu = kMode == 2;
+  constexpr bool kNarrow = kMode == 3;
   constexpr int TG = (TT + 7) / 8;           // mma token groups of 8
   constexpr bool kStream = sizeof(TX) == 1;  // int8 codes stream with the weights
   constexpr bool kAlu = TT == 1;             // one token: dp4a dot products instead of the mma path
+  static_assert(!kNarrow || (kAlu && kStream), "narrow units are a one-token, streamed-codes form");
+  // Inputs per stage: a narrow unit's stage is 32 rows of twice the inputs.
+  constexpr int kStageIn = kNarrow ? 2 * kGvStageK : kGvStageK;
   constexpr int kXHalf = x_half_bytes(TT);   // one half-stage activation tile
   constexpr int kSlot = kGvStageBytes + (kStream ? 2 * kXHalf : 0);
+  static_assert(!kNarrow || 2 * kXHalf >= 16 * 128, "a narrow stage's codes: 16 blocks of 128");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nring = P.nring, M = P.M;
@@ -540,7 +615,9 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       int unit = unit_first;
       // The layer, row block and stage range of a unit.  A unit of the fused
       // gate/up launch is 32 output rows: each half-stage holds those 32 gate
-      // rows, then the same 32 up rows.
+      // rows, then the same 32 up rows.  A narrow unit is 32 rows too: each
+      // half-stage holds them over one 512-input range, then over the range
+      // 1024 inputs further on.
       auto locate = [&](int u, const GvLayer*& Lp, int& rb, int& s0, int& s1) {
         if constexpr (kGlu) {
           Lp = &P.layer[P.glu.gate];
@@ -552,7 +629,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           while (l + 1 < P.n_layers && u >= P.layer[l + 1].unit0) ++l;
           Lp = &P.layer[l];
           rb = u - Lp->unit0;
-          stage_range((Lp->K + kGvStageK - 1) / kGvStageK, ks, rank, s0, s1);
+          stage_range((Lp->K + kStageIn - 1) / kStageIn, ks, rank, s0, s1);
         }
       };
       auto load_weights = [&](const GvLayer& L, int rb, int st, uint32_t full, uint32_t dst) {
@@ -564,17 +641,29 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
             tma_load_2d(d, &L.tmap, st * 256 + hf * 128, rb * (kGvRows / 2), full);
             tma_load_2d(d + (kGvRows / 2) * 128, &LU.tmap, st * 256 + hf * 128, rb * (kGvRows / 2), full);
           }
+        } else if constexpr (kNarrow) {
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int sb = 0; sb < 2; ++sb)
+              tma_load_2d(dst + hf * (kGvStageBytes / 2) + sb * (kGvRows / 2) * 128, &L.tmap,
+                          (2 * st + sb) * 256 + hf * 128, rb * (kGvRows / 2), full);
         } else {
           tma_load_2d(dst, &L.tmap, st * 256, rb * kGvRows, full);
           tma_load_2d(dst + kGvStageBytes / 2, &L.tmap, st * 256 + 128, rb * kGvRows, full);
         }
       };
-      // The stage's activation tiles (streamed codes), in the same slot after the weights.
+      // The stage's activation tiles (streamed codes), in the same slot after
+      // the weights; a narrow stage's 2048 codes are one 16-block tile.
       auto load_act = [&](const GvLayer& L, int st, uint32_t full, uint32_t dst) {
-        tma_load_3d(dst + kGvStageBytes, &L.xmap, 0, 8 * st, 0, full);
-        tma_load_3d(dst + kGvStageBytes + kXHalf, &L.xmap, 0, 8 * st + 4, 0, full);
+        if constexpr (kNarrow) {
+          tma_load_3d(dst + kGvStageBytes, &L.xmap, 0, 16 * st, 0, full);
+        } else {
+          tma_load_3d(dst + kGvStageBytes, &L.xmap, 0, 8 * st, 0, full);
+          tma_load_3d(dst + kGvStageBytes + kXHalf, &L.xmap, 0, 8 * st + 4, 0, full);
+        }
       };
-      constexpr uint32_t kStageTx = kGvStageBytes + (kStream ? 2 * TT * 4 * 128 : 0);
+      constexpr uint32_t kStageTx = kGvStageBytes + (kNarrow ? 16 * 128 : kStream ? 2 * TT * 4 * 128 : 0);
       // The next ticket (none when each block takes only its own unit).
       auto next_unit = [&]() {
         if (P.one_unit) return P.total_units;
@@ -589,7 +678,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         // Before the grid dependency: the weights of the first unit's first
         // stages (a whole ring of them); their activation tiles, written by
         // the preceding kernel, follow once it has finished.
-        if (unit < P.total_units && !(kGlu && unit >= P.glu.q_unit0)) {
+        if (unit < P.total_units) {
           const GvLayer* Lp;
           int rb, s0, s1;
           locate(unit, Lp, rb, s0, s1);
@@ -609,16 +698,6 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         }
       }
       while (ok && unit < P.total_units) {
-        if (kGlu && unit >= P.glu.q_unit0) {
-          // A quantisation unit: a slot with no data, only the tag.
-          if (!mbar_wait(bar0 + 8 * (nring + slot), phase ^ 1, ctl)) { ok = false; break; }
-          tags[slot] = unit;
-          mbar_arrive(bar0 + 8 * slot);
-          ++issued;
-          if (++slot == nring) { slot = 0; phase ^= 1; }
-          unit = next_unit();
-          continue;
-        }
         const GvLayer* Lp;
         int rb, s0, s1;
         locate(unit, Lp, rb, s0, s1);
@@ -683,7 +762,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
     if constexpr (!kStream) {
       // The first unit is the block's index, so its activations can be
       // quantised while its first weight stage is still on the way.
-      if (unit_first < P.total_units && !(kGlu && unit_first >= P.glu.q_unit0)) {
+      if (unit_first < P.total_units) {
         int l = kGlu ? P.glu.gate : 0;
         if constexpr (!kGlu) {
           while (l + 1 < P.n_layers && unit_first >= P.layer[l + 1].unit0) ++l;
@@ -693,7 +772,6 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         staged_k = P.layer[l].K;
       }
     }
-    bool glu_done = !kGlu;  // this warp has counted itself done with its units
     float hmax[TG][2];      // the fused gate/up launch: this lane's running max of |h| per token
 #pragma unroll
     for (int tg = 0; tg < TG; ++tg) hmax[tg][0] = hmax[tg][1] = 0.0f;
@@ -702,24 +780,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       if (!__all_sync(0xffffffffu, got0)) break;
       const int unit = tags[slot];
       if (unit == kGvTagEnd) {
-        if constexpr (kGlu) {
-          if (!glu_done) glu_warp_done<TG, kAlu>(P, hmax);
-        }
         break;
-      }
-      if constexpr (kGlu) {
-        if (unit >= P.glu.q_unit0) {
-          // A quantisation unit: release the (empty) slot, then quantise.
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar0 + 8 * (nring + slot));
-          if (++slot == nring) { slot = 0; phase ^= 1; }
-          if (!glu_done) {
-            glu_warp_done<TG, kAlu>(P, hmax);
-            glu_done = true;
-          }
-          if (!glu_quant_unit<TY>(P, unit - P.glu.q_unit0, P.layer[P.glu.gate].N, ctl)) break;
-          continue;
-        }
       }
       int l = kGlu ? P.glu.gate : 0;
       if constexpr (!kGlu) {
@@ -727,7 +788,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       }
       const GvLayer& L = P.layer[l];
       int s0, s1;  // this CTA's stages of the unit
-      stage_range((L.K + kGvStageK - 1) / kGvStageK, ks, rank, s0, s1);
+      stage_range((L.K + kStageIn - 1) / kStageIn, ks, rank, s0, s1);
       if constexpr (!kStream) {
         if (L.x != staged || L.K != staged_k) {
           consumer_sync();  // every warp is done with the previous input's activations
@@ -790,15 +851,16 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           // no idle mma columns.  Each 8-lane phase reads one 128-byte swizzled
           // row.  Rows: warp*16 + rs + 4*it; in the fused gate/up launch the
           // first two are gate rows warp*8 + rs + 4*it, the last two the same
-          // up rows.
+          // up rows; in a narrow unit the last two are the first two over the
+          // inputs 1024 further on.
           const int ch = lane & 7, rs = lane >> 3;
           uint4 wv[2][4];
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
             for (int it = 0; it < 4; ++it) {
-              const int row = kGlu ? (it < 2 ? warp * 8 + rs + 4 * it : 32 + warp * 8 + rs + 4 * (it - 2))
-                                   : warp * 16 + rs + 4 * it;
+              const int row = (kGlu || kNarrow) ? (it < 2 ? warp * 8 + rs + 4 * it : 32 + warp * 8 + rs + 4 * (it - 2))
+                                                : warp * 16 + rs + 4 * it;
               wv[hf][it] = lds128(wt + hf * (kGvStageBytes / 2) + row * 128 + ((ch ^ (row & 7)) << 4));
             }
           if constexpr (!kStream) {
@@ -807,6 +869,30 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           }
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
+            if constexpr (kNarrow) {
+              // Rows it < 2 over inputs (2i)*1024 + hf*512 + 64ch .. +63, rows
+              // it >= 2 over the same 1024 further on: code block b = sb*8 + hf*4
+              // + ch/2 of the stage's 16-block tile.
+#pragma unroll
+              for (int sb = 0; sb < 2; ++sb) {
+                const int k0 = (2 * i + sb) * kGvStageK + hf * (kGvStageK / 2) + 64 * ch;
+                if (k0 < L.K) {
+                  const int b = sb * 8 + hf * 4 + (ch >> 1);
+                  uint4 xc[4];
+#pragma unroll
+                  for (int u = 0; u < 4; ++u)
+                    xc[u] = lds128(wt + kGvStageBytes + b * 128 + (((4 * (ch & 1) + u) ^ (b & 7)) << 4));
+#pragma unroll
+                  for (int it = 2 * sb; it < 2 * sb + 2; ++it)
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+#pragma unroll
+                      for (int j = 0; j < 4; ++j)
+                        dr[it][j] = dp4a_us(u4_get(wv[hf][it], v) & (0x03030303u << (2 * j)), u4_get(xc[v], j), dr[it][j]);
+                }
+              }
+              continue;
+            }
             const int k0 = i * kGvStageK + hf * (kGvStageK / 2) + 64 * ch;
             if (k0 < L.K) {  // inputs past K have zero weights (K is a multiple of 64)
               uint4 xc[4];
@@ -904,6 +990,10 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       if constexpr (kAlu) {
 #pragma unroll
         for (int r = 0; r < 4; ++r) pc[0][r] = dr[r][0] + (dr[r][1] >> 2) + (dr[r][2] >> 4) + (dr[r][3] >> 6);
+        if constexpr (kNarrow) {  // rows rs and rs + 4: the two input ranges summed
+          pc[0][0] += pc[0][2];
+          pc[0][1] += pc[0][3];
+        }
       } else if constexpr (kSplit) {  // (the mma epilogue below combines them itself otherwise)
 #pragma unroll
         for (int tg = 0; tg < TG; ++tg)
@@ -943,9 +1033,24 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       // and up sums of the same output row (each output rounded to the
       // activation type first, as a stored output is), stores h and folds
       // |h| into the per-token maxima.
-      const int n_base = (kGlu ? unit : unit - L.unit0) * (kGlu ? kGvRows / 2 : kGvRows);
+      const int n_base = (kGlu ? unit : unit - L.unit0) * ((kGlu || kNarrow) ? kGvRows / 2 : kGvRows);
       TY* y = static_cast<TY*>(L.y);
-      if constexpr (kAlu) {
+      if constexpr (kNarrow) {
+        // Rows rs (lanes with ch < 4 after the first step) and rs + 4 of the
+        // warp's 8, summed over the 8 lanes of the row group.
+        const bool upper = (lane & 4) != 0;
+        int v = (upper ? pc[0][1] : pc[0][0]) + __shfl_xor_sync(0xffffffffu, upper ? pc[0][0] : pc[0][1], 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        const int n = n_base + warp * 8 + (lane >> 3) + 4 * ((lane >> 2) & 1);
+        if ((lane & 3) == 0 && n < L.N) {
+          const int a = v - rsum1;
+          const float val = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, s1tok));
+          if constexpr (sizeof(TY) == 4) y[n] = val; else y[n] = __float2bfloat16_rn(val);
+          if (L.acc_out) L.acc_out[n] = a;
+        }
+        continue;
+      } else if constexpr (kAlu) {
         // A butterfly over the 8 lanes of a row group leaves the lane's row
         // number (lane >> 3) + 4*((lane >> 1) & 3) of the warp's 16 summed in
         // lanes 2r and 2r + 1.
@@ -1042,6 +1147,11 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           }
         }
     }
+    if constexpr (kGlu) {
+      // Every consumer warp, after its last unit or after giving up.
+      glu_block_done<TG, kAlu>(P, hmax, reinterpret_cast<float*>(smem), ctl);
+      glu_quant_slices<TY>(P, P.layer[P.glu.gate].N, ctl);
+    }
   }
 
   // No CTA of a K-split cluster leaves while a peer may still read its shared
@@ -1076,11 +1186,17 @@ int gemv_smem_bytes(int M, int K_max, int nring, bool stream, int ksplit = 1) {
   return nring * slot + staged + part + 256 + 16 * nring + 16 + 1024;
 }
 
-bool gemv_fuses_quant(int M, int K, int x_bf16) {
+bool gemv_fuses_quant(int M, int K, int x_bf16, bool single) {
   // Every block quantises the activations it uses, so only tiny ones are worth it;
   // each consumer thread then holds at most kGvFuseChunks chunks of 16 inputs.
+  // One bf16 token of a single layer: up to kGvFuseChunks1 chunks, as long as
+  // the whole input fits beside a ring of four stages (K up to 9856): every
+  // block reads the input (L2-resident after the first) instead of waiting
+  // for a quantisation launch.
   const int G = kGvConsumers / token_slots(M);
   const int chunks_per_thread = (K / 16 + G - 1) / G;
+  if (single && M == 1 && x_bf16)
+    return chunks_per_thread <= kGvFuseChunks1 && gemv_smem_bytes(1, K, 4, false) <= kGvSmemPerBlock;
   const int max_chunks = x_bf16 ? kGvFuseChunks : (kGvFuseChunks + 1) / 2;
   return M >= 1 && M <= 16 && static_cast<long long>(M) * K <= kGvFuseElems && chunks_per_thread <= max_chunks &&
          gemv_smem_bytes(M, K, 4, false) <= kGvSmemPerBlock;
@@ -1090,10 +1206,13 @@ template <int TT, typename TY, typename TX>
 static cudaError_t launch_group_t(const GvParams& P, int grid, int smem, cudaStream_t stream, bool pdl) {
   // Separate instances for the plain launch, the K-split and the fused
   // gate/up launch, so that each runs none of the others' code.
-  static bool attr_set[3] = {false, false, false};  // per template instance
-  const int mode = P.glu.on ? 2 : P.ksplit > 1 ? 1 : 0;
+  static bool attr_set[4] = {false, false, false, false};  // per template instance
+  constexpr bool kHasNarrow = TT == 1 && sizeof(TX) == 1;
+  const int mode = P.glu.on ? 2 : P.ksplit > 1 ? 1 : P.narrow ? 3 : 0;
+  if (mode == 3 && !kHasNarrow) return cudaErrorInvalidValue;
   auto kernel = mode == 2   ? gemv_group_kernel<TT, TY, TX, 2>
                 : mode == 1 ? gemv_group_kernel<TT, TY, TX, 1>
+                : mode == 3 ? gemv_group_kernel<TT, TY, TX, kHasNarrow ? 3 : 0>
                             : gemv_group_kernel<TT, TY, TX, 0>;
   if (!attr_set[mode]) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemPerBlock);
@@ -1143,8 +1262,6 @@ thread_local int g_force_ksplit = 0;  // 0: automatic
 
 void gemv_force_ksplit(int ks) { g_force_ksplit = ks > 0 ? ks : 0; }
 
-constexpr int kGluQuantElems = 2048;  // elements of h per quantisation unit
-
 // Zeroed scratch of a fused gate/up launch: amax and rsum (one 128-byte line
 // per token, 16 tokens each), then done[2].
 size_t gemv_glu_scratch_bytes(int N) {
@@ -1177,41 +1294,7 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   int units = 0, k_max = 64, nst_min = 1 << 30;
   for (int i = 0; i < n_layers; ++i) {
     const GemvLayerArgs& a = layers[order[i]];
-    GvLayer& L = P.layer[i];
-    {
-      // The fused gate/up launch loads 32 rows of each layer per half-stage.
-      const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K / 4), static_cast<cuuint64_t>(a.N)};
-      const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K / 4)};
-      const cuuint32_t box[2] = {128, glu ? kGvRows / 2 : kGvRows};
-      const cuuint32_t estr[2] = {1, 1};
-      if (enc(&L.tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.packed), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
-        return cudaErrorInvalidValue;
-      }
-    }
-    if (stream_x) {
-      // Codes [M][ldx] viewed as [M][ldx/128][128]; blocks past K are zero in the buffer.
-      if (a.ldx % 128 != 0 || a.ldx < a.K) return cudaErrorInvalidValue;
-      const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(a.ldx / 128), static_cast<cuuint64_t>(M)};
-      const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(a.ldx)};
-      const cuuint32_t box[3] = {128, 4, static_cast<cuuint32_t>(tt)};
-      const cuuint32_t estr[3] = {1, 1, 1};
-      if (enc(&L.xmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(a.x), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
-        return cudaErrorInvalidValue;
-      }
-    }
-    L.x = a.x;
-    L.scale = a.scale;
-    L.rowsum = a.rowsum;
-    L.gamma = a.gamma;
-    L.y = a.y;
-    L.acc_out = a.acc_out;
-    L.N = a.N;
-    L.K = a.K;
-    L.unit0 = units;
+    if (stream_x && (a.ldx % 128 != 0 || a.ldx < a.K)) return cudaErrorInvalidValue;
     units += (a.N + kGvRows - 1) / kGvRows;
     if (a.K > k_max) k_max = a.K;
     const int nst = (a.K + kGvStageK - 1) / kGvStageK;
@@ -1219,7 +1302,6 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   }
   P.n_layers = n_layers;
   P.M = M;
-  P.total_units = units;
   P.x_pitch = gemv_x_pitch(k_max);
   P.status = status;
   P.tickets = tickets;
@@ -1238,22 +1320,65 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   if (ks > nst_min) ks = nst_min;
   if (ks < 1 || glu) ks = 1;  // the fused gate/up launch hands its quantisation units out by ticket
   P.ksplit = ks;
+  // One token on streamed codes without a split: units of 32 rows, so that
+  // the last units handed out are half as long.
+  const bool narrow = tt == 1 && stream_x && ks == 1 && !glu;
+  P.narrow = narrow ? 1 : 0;
+  const int unit_rows = (narrow || glu) ? kGvRows / 2 : kGvRows;
+  units = 0;
+  for (int i = 0; i < n_layers; ++i) {
+    const GemvLayerArgs& a = layers[order[i]];
+    GvLayer& L = P.layer[i];
+    {
+      // Boxes of 32 rows for the fused gate/up launch and narrow units.
+      const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K / 4), static_cast<cuuint64_t>(a.N)};
+      const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K / 4)};
+      const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(unit_rows)};
+      const cuuint32_t estr[2] = {1, 1};
+      if (enc(&L.tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.packed), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+        return cudaErrorInvalidValue;
+      }
+    }
+    if (stream_x) {
+      // Codes [M][ldx] viewed as [M][ldx/128][128]; blocks past K are zero in
+      // the buffer, blocks past ldx are filled with zeros by the copy.  A
+      // narrow stage takes its 16 blocks in one box.
+      const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(a.ldx / 128), static_cast<cuuint64_t>(M)};
+      const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(a.ldx)};
+      const cuuint32_t box[3] = {128, narrow ? 16u : 4u, static_cast<cuuint32_t>(tt)};
+      const cuuint32_t estr[3] = {1, 1, 1};
+      if (enc(&L.xmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(a.x), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+        return cudaErrorInvalidValue;
+      }
+    }
+    L.x = a.x;
+    L.scale = a.scale;
+    L.rowsum = a.rowsum;
+    L.gamma = a.gamma;
+    L.y = a.y;
+    L.acc_out = a.acc_out;
+    L.N = a.N;
+    L.K = a.K;
+    L.unit0 = units;
+    units += (a.N + unit_rows - 1) / unit_rows;
+  }
+  // A unit of the fused gate/up launch covers the same 32 rows of both layers.
+  if (glu) units = (layers[0].N + unit_rows - 1) / unit_rows;
+  P.total_units = units;
   if (glu) {
-    // Tickets: one per unit of 64 rows of both layers, then the quantisation units.
+    // Units of 32 rows of both layers; the quantisation slices go to the grid's
+    // warps once the grid size is known (below).
     GvGlu& G = P.glu;
-    const int N = layers[0].N;
-    const int row_units = (N + kGvRows / 2 - 1) / (kGvRows / 2);  // 32 output rows each
-    const long long elems = static_cast<long long>(M) * N;
-    const int q_units = static_cast<int>((elems + kGluQuantElems - 1) / kGluQuantElems);
     G.on = 1;
     G.act = glu->act;
     for (int i = 0; i < n_layers; ++i) {
       if (order[i] == 0) G.gate = i;
       if (order[i] == 1) G.up = i;
     }
-    G.q_unit0 = row_units;
-    G.q_elems = kGluQuantElems;
-    G.q_warps = q_units * kGvWarps;
     G.h = glu->h;
     G.xq = glu->xq;
     G.scale = glu->scale;
@@ -1262,8 +1387,6 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
     G.amax = z;
     G.rsum = reinterpret_cast<int32_t*>(z + 16 * kGluTokStride);
     G.done = z + 2 * 16 * kGluTokStride;
-    units = row_units + q_units;
-    P.total_units = units;
   }
   // kGvBlocksPerSM blocks per SM, each with the deepest weight ring that fits beside its other data.
   const int slot = kGvStageBytes + (stream_x ? 2 * x_half_bytes(tt) : 0);
@@ -1276,6 +1399,12 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   const int slots = kGvBlocksPerSM * sms;
   const int grid = ks > 1 ? units * ks : (units < slots ? units : slots);
   P.one_unit = ks > 1 || units <= slots ? 1 : 0;
+  if (glu) {
+    const long long slices = (static_cast<long long>(M) * layers[0].N + kGluSlice - 1) / kGluSlice;
+    const long long warps = static_cast<long long>(grid) * kGvWarps;
+    P.glu.q_warps = static_cast<int>(slices < warps ? slices : warps);
+    P.glu.q_blocks = (P.glu.q_warps + kGvWarps - 1) / kGvWarps;
+  }
   return y_type == kOutBF16 ? launch_group_y<__nv_bfloat16>(x_type, P, grid, smem, stream, pdl)
                             : launch_group_y<float>(x_type, P, grid, smem, stream, pdl);
 }

@@ -104,7 +104,7 @@ struct GemvLayerArgs {
   int32_t* acc_out;
 };
 constexpr int kGvMaxLayers = 8;
-bool gemv_fuses_quant(int M, int K, int x_bf16);
+bool gemv_fuses_quant(int M, int K, int x_bf16, bool single = false);
 // CTAs per unit of the decode kernel's K-split (a cluster): 0 lets the kernel
 // choose (by the unit count), else forced (1 .. 8, capped by the stages).  Per thread.
 void gemv_force_ksplit(int ks);

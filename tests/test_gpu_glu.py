@@ -52,13 +52,14 @@ def _ffn(M, N, K, dtype, seed):
     return x, dev_w, _values(yg), _values(yu)
 
 
-# Decode sizes (one launch; N past one 64-row unit, ragged unit counts),
+# Decode sizes (one launch; N past one 32-row unit, ragged unit counts, and
+# 16 x 58368, whose 512-element quantisation slices outnumber the grid's warps),
 # tokens 1..16; and many tokens (the tensor-core GEMM whose
 # tiles pair gate and up rows: one CTA up to 128 tokens, CTA pairs beyond,
 # ragged M, N (not a multiple of the 128-column tile) and K).
 RELU2 = [(1, 1024, 1024, "bf16"), (1, 2816, 2560, "bf16"), (3, 704, 4096, "f32"), (8, 2816, 1024, "bf16"),
          (16, 1088, 2048, "bf16"), (1, 6912, 2560, "bf16"), (40, 704, 512, "bf16"), (2048, 1024, 512, "bf16"),
-         (300, 1088, 576, "f32"), (513, 704, 320, "bf16")]
+         (300, 1088, 576, "f32"), (513, 704, 320, "bf16"), (16, 58368, 128, "bf16")]
 
 
 @pytest.mark.parametrize("M,N,K,dtype", RELU2)
@@ -129,8 +130,9 @@ def test_fused_equals_chain_then_glu_quant(M, act):
 
 
 def test_gate_up_glu_ignores_a_forced_split():
-    """The fused call hands its quantisation units out by ticket and never splits
-    along K; a forced split on the calling thread leaves its result unchanged."""
+    """The fused call spreads its quantisation over the warps of its grid and
+    never splits along K; a forced split on the calling thread leaves its
+    result unchanged."""
     M, N, K = 4, 1088, 5120
     x, (pg, gg, pu, gu), yg, yu = _ffn(M, N, K, "bf16", seed=55)
     want = tb.gate_up_glu(pg, gg, pu, gu, x, tb.GLU_RELU2)

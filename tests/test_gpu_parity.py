@@ -156,9 +156,11 @@ def test_forward_small_gemv(M, N, K, ydtype):
 
 # One token takes the dp4a path of the decode kernel: K from one 64-input chunk
 # to several 1024-input stages with a ragged last stage, N from one row to
-# ragged 64-row units; fp32 inputs of K <= 2048 and bf16 inputs of K <= 4096 are
-# quantised inside the kernel, longer ones by the quantisation kernel.
-ONE_TOKEN = [(1, 64), (63, 960), (65, 1024), (200, 1088), (130, 2048), (129, 4160), (64, 5120), (7, 8192)]
+# ragged 64-row units; fp32 inputs of K <= 2048 and bf16 inputs of K <= 9856
+# (the most that fits beside a four-stage ring) are quantised inside the
+# kernel, longer ones by the quantisation kernel.
+ONE_TOKEN = [(1, 64), (63, 960), (65, 1024), (200, 1088), (130, 2048), (129, 4160), (64, 5120), (7, 8192),
+             (300, 9856), (70, 9920)]
 
 
 @pytest.mark.parametrize("N,K", ONE_TOKEN)
@@ -449,3 +451,29 @@ def test_shared_workspace_across_shapes_stays_consistent():
         y2, a2 = tb.forward(packed, gamma, x, acc_out=True, workspace=tb.new_workspace(tb.workspace_bytes(M, N, K)))
         assert torch.equal(a1, a2) and torch.equal(y1, y2)
     assert int(ws[:256].count_nonzero().item()) == 0
+
+
+# One token on caller codes with enough rows that no split is taken: units of
+# 32 rows over stages of 2048 inputs.  Ragged N (not a multiple of 32), K with
+# a partial last stage (down to a single 128-input block), and several layers
+# of different K in one launch.
+NARROW = [[(128, 6400)], [(1152, 6433)], [(8640, 7000)], [(2176, 3300), (4096, 3500), (128, 130)],
+          [(14336, 3200), (8192, 3217)]]
+
+
+@pytest.mark.parametrize("specs", NARROW, ids=lambda s: "+".join("%dx%d" % kn for kn in s))
+def test_one_token_narrow_units_match_the_oracle(specs):
+    layers, refs = [], []
+    for i, (K, N) in enumerate(specs):
+        x, xf = activations(1, K, seed=300 + i, dtype="bf16")
+        xq, sc, rs = tb.quant_act(x)
+        packed, gamma, T = oracle.pack_weights(weights(N, K, seed=310 + i))
+        y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+        acc = torch.empty((1, N), dtype=torch.int32, device="cuda")
+        layers.append(tb.Layer(dev(packed), dev(np.array([gamma], np.float32)), None, y, xq=xq, scale=sc,
+                               rowsum=rs, acc_out=acc))
+        refs.append(oracle.forward(T, gamma, xf))
+    tb.layer_chain(layers)
+    for L, (acc_ref, y_ref, *_) in zip(layers, refs):
+        assert np.array_equal(L.acc_out.cpu().numpy(), acc_ref)
+        assert_y_matches(L.y, y_ref, acc_ref)
