@@ -379,6 +379,21 @@ int bitlinear_set_path(int path);
  */
 int bitlinear_set_decode_split(int ctas);
 
+/*
+ * Chooses the form of the decode product for 2 to 16 tokens whose input is
+ * int8 codes (every decode call quantises first unless the decode kernel
+ * quantises tiny inputs itself), on the calling thread: 0 (default) and 1
+ * the CUDA-core form (mma.sync); 2 the tensor-core form (tcgen05.mma
+ * kind::i8 with the unpacked ternary codes in tensor memory, one block per
+ * SM) whenever the call is eligible (2 to 16 tokens on codes, not the fused
+ * gate/up call).  Both give bit-identical results; the tensor-core form is
+ * slower (each of its 128-row x 16-token MMAs costs about as much as a
+ * full-width one, so feeding the unpacked codes through the tensor cores,
+ * not HBM, sets its pace), so it is never chosen by default.  For tests and
+ * measurement.  Returns BL_ERR_INVALID_ARG for any other value.
+ */
+int bitlinear_set_decode_form(int form);
+
 /* Message of the most recent failure on the calling thread ("" if none). */
 const char* bitlinear_last_error(void);
 

@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
             "bitlinear_selftest_wait_timeout": (i32, [vp, sz, i32, vp]),
             "bitlinear_set_path": (i32, [i32]),
             "bitlinear_set_decode_split": (i32, [i32]),
+            "bitlinear_set_decode_form": (i32, [i32]),
             "bitlinear_forward_noalloc": (i32, [vp, vp, i32, i32, vp, i32, i32, vp, i32, vp, vp]),
             "bitlinear_noalloc_status": (i32, [vp]),
             "bitlinear_last_error": (ctypes.c_char_p, []),
@@ -141,6 +142,14 @@ def set_path(path: int) -> None:
 def set_decode_split(ctas: int) -> None:
     """Force the decode kernel's K-split to ``ctas`` CTAs per unit on this thread (0: automatic)."""
     _check(lib().bitlinear_set_decode_split(int(ctas)))
+
+
+DECODE_FORM_AUTO, DECODE_FORM_CUDA_CORES, DECODE_FORM_TENSOR_CORES = 0, 1, 2
+
+
+def set_decode_form(form: int) -> None:
+    """Force the decode product's form for 9-16 tokens on this thread (DECODE_FORM_*)."""
+    _check(lib().bitlinear_set_decode_form(int(form)))
 
 
 def version() -> int:

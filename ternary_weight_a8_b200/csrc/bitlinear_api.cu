@@ -332,6 +332,12 @@ int bitlinear_set_decode_split(int ctas) {
   return BL_OK;
 }
 
+int bitlinear_set_decode_form(int form) {
+  if (form < 0 || form > 2) return fail(BL_ERR_INVALID_ARG, "form = %d not in [0, 2]", form);
+  bl::gemv_force_form(form);
+  return BL_OK;
+}
+
 int bitlinear_forward_quantized(const uint8_t* packed, const float* gamma, int N, int K,
                                 const int8_t* xq, const float* scale, const int32_t* rowsum,
                                 int M, void* y, int y_dtype, int32_t* acc_out, void* workspace,

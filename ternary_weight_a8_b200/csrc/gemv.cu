@@ -1262,6 +1262,10 @@ thread_local int g_force_ksplit = 0;  // 0: automatic
 
 void gemv_force_ksplit(int ks) { g_force_ksplit = ks > 0 ? ks : 0; }
 
+thread_local int g_force_form = 0;  // 0: by size
+
+void gemv_force_form(int form) { g_force_form = form; }
+
 // Zeroed scratch of a fused gate/up launch: amax and rsum (one 128-byte line
 // per token, 16 tokens each), then done[2].
 size_t gemv_glu_scratch_bytes(int N) {
@@ -1276,6 +1280,10 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   if (glu && (n_layers != 2 || layers[0].N != layers[1].N || layers[0].K != layers[1].K || layers[0].N % 16 != 0 ||
               !glu->zeroed || !glu->h || !glu->xq || !glu->scale || !glu->rowsum))
     return cudaErrorInvalidValue;
+  // The tensor-core form only when forced: it measures slower at every token
+  // count (its MMAs cost as much per 128 x 32 block of codes as full-width ones).
+  if (!glu && x_type == kInInt8 && g_force_form == 2 && gemv_tc_eligible(layers, n_layers, M))
+    return launch_gemv_tc(layers, n_layers, M, y_type, status, tickets, stream, pdl);
   EncodeTiledFn enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
   if (!enc) return cudaErrorNotSupported;
   const bool stream_x = x_type == kInInt8;

@@ -108,6 +108,13 @@ bool gemv_fuses_quant(int M, int K, int x_bf16, bool single = false);
 // CTAs per unit of the decode kernel's K-split (a cluster): 0 lets the kernel
 // choose (by the unit count), else forced (1 .. 8, capped by the stages).  Per thread.
 void gemv_force_ksplit(int ks);
+// Form of the decode product for 2 to 16 tokens on int8 codes: 0 (default)
+// and 1 the CUDA-core kernel, 2 the tensor-core kernel whenever eligible.  Per thread.
+void gemv_force_form(int form);
+bool gemv_tc_eligible(const GemvLayerArgs* layers, int n_layers, int M);
+int gemv_tc_units(const GemvLayerArgs* layers, int n_layers);
+cudaError_t launch_gemv_tc(const GemvLayerArgs* layers, int n_layers, int M, int y_type, uint32_t* status,
+                           uint32_t* tickets, cudaStream_t stream, bool pdl);
 
 // The FFN's gated activation fused into the launch of its gate and up
 // BitLinears (layers[0] = gate, layers[1] = up, same N and K; their y are

@@ -124,6 +124,13 @@ def test_decode_split_setting(L):
     assert L.bitlinear_set_decode_split(0) == tb.BL_OK
 
 
+def test_decode_form_setting(L):
+    for bad in (-1, 3):
+        assert L.bitlinear_set_decode_form(bad) == tb.BL_ERR_INVALID_ARG
+    for good in (tb.DECODE_FORM_TENSOR_CORES, tb.DECODE_FORM_CUDA_CORES, tb.DECODE_FORM_AUTO):
+        assert L.bitlinear_set_decode_form(good) == tb.BL_OK
+
+
 def test_chain_layer_struct_matches_the_header():
     text = open(os.path.join(ROOT, "include", "bitlinear.h")).read()
     body = re.search(r"typedef struct \{(.*?)\} bl_layer;", text, flags=re.S).group(1)
