@@ -14,9 +14,11 @@ is timed separately under ``pack``.
 Timing: the K steps of a run are captured in CUDA graphs; those exact graphs
 are replayed once or more before timing (warm-up), then the K steps are
 timed as a block with CUDA events, repeated until the timed blocks cover a
-minimum time, with L2 flushed before every block; ``ms_per_step`` is the
-median block over K.  Weights rotate over byte-identical copies that
-together exceed the L2 size several times, so every step reads them from HBM.
+minimum time; ``ms_per_step`` is the median block over K.  Decode weights
+rotate over byte-identical copies that together exceed the L2 size several
+times, so every step reads them from HBM (inputs larger than L2: no flush,
+whose dirty lines would be written back inside the next block); the other
+sections write a buffer of twice the L2 size before every block.
 
 Also in the same line: ``decode`` (the same chain at 8 and 16 tokens, the
 2B-class decode step and the 3B-class layers at 1 to 16 tokens), ``prefill``
@@ -264,13 +266,15 @@ class _L2Flush:
         self.buf.fill_(1)
 
 
-def timed_graph_run(step_fn, steps, warmup, world, chunk=500, sampler=None, min_region_s=0.05):
+def timed_graph_run(step_fn, steps, warmup, world, chunk=500, sampler=None, min_region_s=0.05, flush=True):
     """Times `steps` consecutive calls of step_fn replayed as CUDA graphs.
 
     The graphs holding the `steps` calls are captured once and replayed (all of
     them) at least once and for at least `warmup` steps before timing.  Then
-    the whole block of `steps` calls is timed with CUDA events, L2 flushed
-    before each block, repeated until the blocks cover `min_region_s`.
+    the whole block of `steps` calls is timed with CUDA events (L2 flushed
+    before each block unless `flush` is false: inputs larger than L2; the
+    blocks are then enqueued back to back), repeated until the blocks cover
+    `min_region_s`.
     Returns (median seconds per block of `steps` calls, max over ranks; info).
     """
     import torch
@@ -285,7 +289,7 @@ def timed_graph_run(step_fn, steps, warmup, world, chunk=500, sampler=None, min_
         for g in graphs:
             g.replay()
 
-    flush = _L2Flush()
+    flush = _L2Flush() if flush else (lambda: None)
     for _ in range(max(1, math.ceil(warmup / steps))):
         block()
     torch.cuda.synchronize()
@@ -377,7 +381,8 @@ def run_chain(args, world, peaks, L2, tokens=(1, 8, 16), steps=None, warmup=None
     steps = steps or 100
     warmup = warmup if warmup is not None else 10
     out = {"workload": CHAIN_WORKLOAD, "weight_bytes_per_step": set_bytes,
-           "l2": "%d rotating byte-identical weight sets (%.0f MB > 3x L2), L2 flushed before every timed block"
+           "l2": "%d rotating byte-identical weight sets (%.0f MB > 3x L2): inputs larger than L2, every step "
+                 "reads its weights from HBM; no flush"
                  % (len(sets), len(sets) * set_bytes / 1e6)}
     for M in tokens:
         xs, ys = make_inputs(CHAIN_70B, M, seed=1000, shared=CHAIN_70B_SHARED_INPUT)
@@ -389,7 +394,7 @@ def run_chain(args, world, peaks, L2, tokens=(1, 8, 16), steps=None, warmup=None
 
         secs, clocks, info = timed_graph_run(step, steps, warmup, world, chunk=100,
                                              sampler=sampler if M == tokens[0] else None,
-                                             min_region_s=min_region_s)
+                                             min_region_s=min_region_s, flush=False)
         per_step = secs / steps
         gbs = set_bytes * world / per_step / 1e9
         res = {"GB/s": round(gbs, 1), "pct_hbm_measured": round(100 * gbs / world / peaks["hbm"], 2),
@@ -484,7 +489,7 @@ def run_decode_2b(args, world, peaks, L2):
         tb.layer_chain(layer_sets[i % len(layer_sets)], workspace=ws)
 
     steps = 500
-    secs, _, info = timed_graph_run(step, steps, 100, world, chunk=500)
+    secs, _, info = timed_graph_run(step, steps, 100, world, chunk=500, flush=False)
     per_step = secs / steps
     x_bytes = sum(K * 2 for K, N in DECODE_LAYERS)
     y_bytes = sum(N * 2 for K, N in DECODE_LAYERS)
@@ -496,6 +501,8 @@ def run_decode_2b(args, world, peaks, L2):
             "GB/s": round(gbs, 1), "pct_hbm_measured": round(100 * gbs / world / peaks["hbm"], 2),
             "us_per_step": round(per_step * 1e6, 3), "tokens_per_s": round(world / per_step, 1),
             "weight_bytes_per_step": set_bytes, "timing": info,
+            "l2": "%d rotating byte-identical weight sets (%.0f MB > 4x L2): inputs larger than L2; no flush"
+                  % (len(sets), len(sets) * set_bytes / 1e6),
             "roofline": {"bound": "hbm", "kernel": "gemv_group_kernel (the whole step: one launch)",
                          "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
                          "frac": round(achieved / peaks["hbm"], 4),
@@ -590,6 +597,21 @@ DECODE_3B = [(3200, 8640), (8640, 3200)]  # (K in, N out)
 DECODE_3B_TOKENS = (1, 2, 4, 8, 16)
 
 
+def run_chain_tensor_core_form(args, world, peaks, L2, tokens=(8, 16)):
+    """The same chain through the decode product's tensor-core form (chosen
+    only on request), for comparison with the default CUDA-core form."""
+    import ternary_weight_a8_b200 as tb
+
+    tb.set_decode_form(tb.DECODE_FORM_TENSOR_CORES)
+    try:
+        res, _, _ = run_chain(args, world, peaks, L2, tokens=tokens, steps=20, warmup=5)
+    finally:
+        tb.set_decode_form(tb.DECODE_FORM_AUTO)
+    res = {k: v for k, v in res.items() if k != "l2"}
+    res["form"] = "tcgen05.mma kind::i8, unpacked codes in tensor memory (bitlinear_set_decode_form 2)"
+    return res
+
+
 def run_decode_3b(args, world, peaks, L2, tokens=None):
     """The 3B-class decode sweep: one BitLinear per step through the public
     single-layer call (quantisation and product), 1 to 16 tokens."""
@@ -609,7 +631,7 @@ def run_decode_3b(args, world, peaks, L2, tokens=None):
                 tb.forward(packed, gamma, x, y=y, workspace=ws)
 
             steps = 500
-            secs, _, info = timed_graph_run(step, steps, 100, world, chunk=500, min_region_s=0.03)
+            secs, _, info = timed_graph_run(step, steps, 100, world, chunk=500, min_region_s=0.03, flush=False)
             per = secs / steps
             gbs = set_bytes * world / per / 1e9
             res["k%d_n%d_m%d" % (K, N, M)] = {
@@ -850,7 +872,8 @@ def run_ours(args, world, rank, local):
         "config": {"workload": CHAIN_WORKLOAD, "tokens": 1, "layers_k_n": CHAIN_70B,
                    "weight_bytes_per_step": set_bytes, "l2": chain["l2"],
                    "timing": "the %d steps replayed as CUDA graphs; the same graphs warmed first; the block of %d "
-                             "steps timed %d times with CUDA events, L2 flushed before each; median block / %d"
+                             "steps timed %d times with CUDA events, blocks back to back (weights rotate over "
+                             "more than L2: no flush); median block / %d"
                              % (args.steps, args.steps, reps, args.steps),
                    "parallelism": "replicas x%d" % world},
         "pct_hbm_measured": round(100 * value / world / peaks["hbm"], 2),
@@ -863,6 +886,7 @@ def run_ours(args, world, rank, local):
     if not args.no_extras:
         result["prefill"] = run_prefill(args, world, peaks, L2)
         result["decode"] = {"chain_70b": {k: v for k, v in chain.items() if k != "l2"},
+                            "chain_70b_tensor_core_form": run_chain_tensor_core_form(args, world, peaks, L2),
                             "decode_2b": run_decode_2b(args, world, peaks, L2),
                             "decode_3b": run_decode_3b(args, world, peaks, L2)}
         result["pack"] = run_pack(world)
