@@ -414,6 +414,38 @@ def layer_chain(layers: Sequence[Layer], workspace: torch.Tensor | None = None, 
                                        _ptr(workspace), workspace.numel(), _stream(stream)))
 
 
+class ChainPlan:
+    """A ``layer_chain`` call marshalled once, for a loop that runs the same
+    layers (same tensors) every step: ``run`` is then a single library call.
+    The plan keeps references to the layers' tensors; it is invalid once one
+    of them is replaced or freed."""
+
+    def __init__(self, layers: Sequence[Layer], workspace: torch.Tensor | None = None, stream=None):
+        if not layers:
+            raise ValueError("a chain plan needs at least one layer")
+        self.layers = list(layers)
+        self.M = self.layers[0].tokens
+        self._arr = _layer_array(self.layers)
+        if workspace is None:
+            workspace = new_workspace(lib().bitlinear_chain_workspace_bytes(self._arr, len(self.layers), self.M))
+        self.workspace = workspace
+        x_dtype = next((L.x.dtype for L in self.layers if L.x is not None), self.layers[0].y.dtype)
+        self._args = (self._arr, len(self.layers), self.M, _dtype_code(x_dtype), _dtype_code(self.layers[0].y.dtype),
+                      _ptr(workspace), workspace.numel())
+        self._stream = _stream(stream) if stream is not None else None
+        self._call = lib().bitlinear_layer_chain
+
+    def run(self, stream=None) -> None:
+        """The chain on ``stream`` (else the plan's stream, else the current stream)."""
+        s = _stream(stream) if stream is not None else (self._stream or _stream(None))
+        _check(self._call(*self._args, s))
+
+
+def prepare_chain(layers: Sequence[Layer], workspace: torch.Tensor | None = None, stream=None) -> ChainPlan:
+    """``layer_chain``'s arguments marshalled once (see ChainPlan)."""
+    return ChainPlan(layers, workspace, stream)
+
+
 def forward_noalloc(packed: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor, y: torch.Tensor,
                     acc_out: torch.Tensor | None = None, stream=None) -> None:
     """The forward without a workspace (the library's fixed scratch): writes ``y`` (and ``acc_out``)."""

@@ -440,6 +440,27 @@ def test_layer_chain_matches_separate_forwards():
         assert torch.equal(L.y, y)
 
 
+def test_prepared_chain_equals_layer_chain():
+    """A chain marshalled once (prepare_chain) and run twice gives layer_chain's outputs."""
+    K = 1024
+    x, _ = activations(4, K, seed=3, dtype="bf16")
+    specs = [(K, 700, x), (K, 900, x), (K, 300, None)]
+    layers, singles = [], []
+    for i, (k, n, xi) in enumerate(specs):
+        packed, gamma = tb.pack_weights(dev(weights(n, k, seed=90 + i)))
+        xi = xi if xi is not None else activations(4, k, seed=11, dtype="bf16")[0]
+        layers.append(tb.Layer(packed, gamma, xi, torch.empty((4, n), dtype=torch.bfloat16, device="cuda")))
+        singles.append(tb.forward(packed, gamma, xi))
+    plan = tb.prepare_chain(layers)
+    for _ in range(2):
+        for L in layers:
+            L.y.zero_()
+        plan.run()
+        for L, y in zip(layers, singles):
+            assert torch.equal(L.y, y)
+    assert tb.device_status(plan.workspace) == tb.BL_OK
+
+
 def test_shared_workspace_across_shapes_stays_consistent():
     """One workspace serves calls of different shapes in stream order."""
     shapes = [(1, 6912, 2560), (16, 300, 8640), (8, 3200, 8640), (3, 2560, 2560), (1, 6912, 2560)]
