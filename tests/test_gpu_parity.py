@@ -498,3 +498,49 @@ def test_one_token_narrow_units_match_the_oracle(specs):
     for L, (acc_ref, y_ref, *_) in zip(layers, refs):
         assert np.array_equal(L.acc_out.cpu().numpy(), acc_ref)
         assert_y_matches(L.y, y_ref, acc_ref)
+
+
+# One token quantised by the quantisation kernel and streamed as codes in
+# 32-row units: a single layer with too many inputs for the in-kernel staging
+# and enough rows that no split is taken, and chains of several layers,
+# distinct and shared inputs, K not a multiple of 2048 (and one not a multiple
+# of 128, so the codes carry zero padding), fp32 and bf16 inputs, called twice
+# on one workspace.
+ONE_TOKEN_STREAMED = [(6400, 10240, "bf16"), (6464, 16448, "f32"), (7000, 28672, "bf16"), (6400, 12352, "bf16")]
+
+
+@pytest.mark.parametrize("N,K,xdt", ONE_TOKEN_STREAMED)
+def test_one_token_streamed_codes_match_the_oracle(N, K, xdt):
+    x, xf = activations(1, K, seed=K + 3, dtype=xdt)
+    packed, gamma, T = oracle.pack_weights(weights(N, K, seed=N + 5))
+    ws = tb.new_workspace(tb.workspace_bytes(1, N, K))
+    acc_ref, y_ref, *_ = oracle.forward(T, gamma, xf)
+    for _ in range(2):
+        y, acc = tb.forward(dev(packed), dev(np.array([gamma], np.float32)), x, acc_out=True, workspace=ws)
+        assert np.array_equal(acc.cpu().numpy(), acc_ref)
+        assert_y_matches(y, y_ref, acc_ref)
+    assert tb.device_status(ws) == tb.BL_OK
+
+
+@pytest.mark.parametrize("xdt", ["bf16", "f32"])
+def test_one_token_chain_of_streamed_codes_matches_the_oracle(xdt):
+    # (K, N, input): inputs a, a (shared), b, c; K = 8256 needs padding to 8320
+    specs = [(8192, 3000, "a"), (8192, 2500, "a"), (8256, 1800, "b"), (3072, 900, "c")]
+    xs = {}
+    layers, refs = [], []
+    for i, (K, N, name) in enumerate(specs):
+        if name not in xs:
+            xs[name] = activations(1, K, seed=200 + i, dtype=xdt)
+        x, xf = xs[name]
+        packed, gamma, T = oracle.pack_weights(weights(N, K, seed=210 + i))
+        y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+        acc = torch.empty((1, N), dtype=torch.int32, device="cuda")
+        layers.append(tb.Layer(dev(packed), dev(np.array([gamma], np.float32)), x, y, acc_out=acc))
+        refs.append(oracle.forward(T, gamma, xf))
+    ws = tb.new_workspace(tb.chain_workspace_bytes(layers, 1))
+    for _ in range(2):
+        tb.layer_chain(layers, workspace=ws)
+        for L, (acc_ref, y_ref, *_) in zip(layers, refs):
+            assert np.array_equal(L.acc_out.cpu().numpy(), acc_ref)
+            assert_y_matches(L.y, y_ref, acc_ref)
+    assert tb.device_status(ws) == tb.BL_OK
