@@ -776,10 +776,14 @@ __global__ void __launch_bounds__(kClusterThreads) glu_quant_cluster_kernel(cons
 // tokens longer than one block holds at two chunks per thread (512 threads)
 // gain: below that the cluster's launch and barriers cost more than they save
 // (measured: a one-token RMSNorm at K = 8192 went from 4.3 to 6.7 us as two
-// CTAs, the gated activation at N = 28672 from 7.6 to 5.1 us as seven).
-static int cluster_size_for(int M, int k_max) {
+// CTAs, the gated activation at N = 28672 from 7.6 to 5.1 us as seven).  The
+// plain quantisation reads one input per element instead of two: one block
+// holds up to four chunks per thread in registers, and the cluster pays only
+// past that (a one-token quantisation at K = 28672: 4.1 us as one block,
+// 4.7 us as a cluster; the 70B chain step 39.1 against 39.8 us).
+static int cluster_size_for(int M, int k_max, int min_chunks = 2 * kQuantMaxThreads) {
   const int chunks = k_max / 16;
-  if (M > 16 || chunks <= 2 * kQuantMaxThreads) return 0;
+  if (M > 16 || chunks <= min_chunks) return 0;
   int c = (chunks + 2 * kClusterThreads - 1) / (2 * kClusterThreads);  // about two chunks per thread
   if (c > kClusterMax) c = kClusterMax;
   if (chunks > c * kClusterThreads * kClusterChunks) return 0;  // does not fit the registers
@@ -837,7 +841,7 @@ cudaError_t launch_act_quant_group(const QuantArgs* items, int n_items, int M, i
     if (items[i].K > k_max) k_max = items[i].K;
   }
   P.n_items = n_items;
-  const int csize = cluster_size_for(M, k_max);
+  const int csize = cluster_size_for(M, k_max, kQuantRegChunks * kQuantMaxThreads);
   if (csize > 0) {
     const dim3 grid(M * csize, n_items);
     if (x_bf16) return launch_cluster(act_quant_cluster_kernel<__nv_bfloat16>, grid, csize, stream, pdl, P);

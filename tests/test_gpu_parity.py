@@ -98,8 +98,10 @@ def test_pack_special_matrices():
                                        # many tokens, short and long rows
                                        (700, 2048, "f32"), (600, 576, "bf16"), (640, 4096, "bf16"),
                                        (600, 4160, "bf16"), (1200, 64, "f32"),
-                                       # few long tokens: one token over a cluster of 2 to 8 CTAs
-                                       (1, 20480, "f32"), (2, 65536, "bf16"), (16, 16448, "bf16")])
+                                       # long tokens: one block up to 32768 inputs (a token in
+                                       # registers), a cluster of CTAs per token beyond
+                                       (1, 20480, "f32"), (2, 65536, "bf16"), (16, 16448, "bf16"),
+                                       (1, 32768, "bf16"), (3, 40960, "bf16"), (1, 131072, "f32")])
 def test_quant_parity(M, K, dtype):
     x, xf = activations(M, K, seed=M * 7 + K, dtype=dtype)
     q_ref, s_ref, r_ref = oracle.quant_act(xf)
