@@ -746,8 +746,8 @@ def run_ffn(args, world, peaks, L2, tokens=(1, 8, 2048)):
     import ternary_weight_a8_b200 as tb
 
     out = {}
-    shapes = {1: (1, 8192, 28672), 8: (8, 8192, 28672), 16: (16, 8192, 28672), 2048: (2048, 2560, 6912)}
-    for M, K, N in (shapes[t] for t in tokens):
+    # decode sizes at the 70B FFN width, many tokens at the 2B prefill shape
+    for M, K, N in ((t, 8192, 28672) if t <= 16 else (t, 2560, 6912) for t in tokens):
         wsets, wbytes = make_layer_sets([(K, N), (K, N)], seed=1100, min_bytes=3 * L2)
         x = torch.from_numpy(synth.activations_bf16(M, K, seed=1101)[0].view("int16")).cuda().view(torch.bfloat16)
         yg = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
@@ -779,7 +779,7 @@ def run_ffn(args, world, peaks, L2, tokens=(1, 8, 2048)):
             else:
                 tops = 2 * 2.0 * M * N * K / (us * 1e-6) / 1e12
                 res[name].update({"TOPS": round(tops, 1)})
-        res["launches"] = {"fused_one_call": 2 if M <= 16 else 3, "chain_then_glu_quant": 3 if M <= 16 else 4}
+        res["launches"] = {"fused_one_call": 2 if M <= 8 else 3, "chain_then_glu_quant": 3 if M <= 16 else 4}
         res["device_status"] = tb.device_status(ws_f)
         out["ffn_gate_up_glu_%dx%dx%d" % (M, K, N)] = res
         del wsets, lsets

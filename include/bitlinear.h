@@ -181,12 +181,15 @@ size_t bitlinear_gate_up_glu_workspace_bytes(int M, int N, int K);
  *           xq / scale / rowsum).
  *   workspace / workspace_bytes: >= bitlinear_gate_up_glu_workspace_bytes(M, N, K),
  *           its first 256 bytes zero.
- * M <= 16: one quantisation launch and one decode launch that computes gate
- * and up, forms h as soon as both halves of a group of rows are in, keeps
- * the per-token maxima of |h| and, once every row is in, quantises h with
- * the final scales (no further launch).  Larger M: the quantisation of x,
- * one tensor-core GEMM whose tiles pair 128 gate rows with the same 128 up
- * rows so that its epilogue writes h, then the quantisation of h.
+ * M <= 8: one quantisation launch (or, for tiny x, none) and one decode
+ * launch that computes gate and up, forms h as soon as both halves of a
+ * group of rows are in, keeps the per-token maxima of |h| and, once every
+ * row is in, quantises h with the final scales (no further launch).
+ * 9 <= M <= 16: the gate and up products into the workspace, then the
+ * gated-activation kernel (there the fused launch's grid-wide step cost more
+ * than the launch it saves).  Larger M: the quantisation of x, one
+ * tensor-core GEMM whose tiles pair 128 gate rows with the same 128 up rows
+ * so that its epilogue writes h, then the quantisation of h.
  */
 int bitlinear_gate_up_glu(const uint8_t* packed_gate, const float* gamma_gate, const uint8_t* packed_up,
                           const float* gamma_up, int N, int K, const void* x, int x_dtype, int M, int act, void* h,

@@ -108,11 +108,14 @@ def test_workspace_layout(L):
     # a chain gives every layer its own q, s, rowsum region (a decode group's layers run together)
     per_layer = lambda K: tb.workspace_bytes(8, 0, K) - 256
     assert L.bitlinear_chain_workspace_bytes(layers, 2, 8) == 256 + per_layer(8192) + per_layer(28672)
-    # the fused gate/up call: codes of x, then h (4-byte elements at most), then (decode
-    # sizes) its counters: per token a 128-byte line of maxima and one of code sums, 256 more bytes
+    # the fused gate/up call: codes of x, then h (4-byte elements at most), then (1 to 8
+    # tokens) its counters: per token a 128-byte line of maxima and one of code sums, 256 more
+    # bytes; (9 to 16 tokens) the gate and up outputs
     r = lambda v: (v + 255) // 256 * 256
     assert tb.gate_up_glu_workspace_bytes(8, 28672, 8192) == \
         tb.workspace_bytes(8, 0, 8192) + r(8 * 28672 * 4) + 2 * 16 * 128 + 256
+    assert tb.gate_up_glu_workspace_bytes(16, 28672, 8192) == \
+        tb.workspace_bytes(16, 0, 8192) + r(16 * 28672 * 4) + r(2 * 16 * 28672 * 4)
     assert tb.gate_up_glu_workspace_bytes(2048, 6912, 2560) == tb.workspace_bytes(2048, 0, 2560) + 2048 * 6912 * 4
 
 
