@@ -685,7 +685,12 @@ static cudaError_t launch_gemm_t(const ProductArgs& a, cudaStream_t stream, bool
                                                   0, CU_TENSOR_MAP_DATA_TYPE_INT32, 4);
     if (!ok_y || !ok_acc) return cudaErrorInvalidValue;
   }
-  static int max_clusters = 0;  // per template instance; attributes are per function
+  // Per template instance and device (function attributes belong to the
+  // device's context): the shared-memory attribute and the resident clusters.
+  static std::atomic<int> max_clusters_of[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) dev = -1;
+  int max_clusters = dev >= 0 ? max_clusters_of[dev].load(std::memory_order_acquire) : 0;
   if (max_clusters == 0) {
     cudaError_t e = cudaFuncSetAttribute(gemm_kernel<TY, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
@@ -709,6 +714,7 @@ static cudaError_t launch_gemm_t(const ProductArgs& a, cudaStream_t stream, bool
       if (c > 0 && c < n) n = c;
     }
     max_clusters = n > 0 ? n : 1;
+    if (dev >= 0) max_clusters_of[dev].store(max_clusters, std::memory_order_release);
   }
   const int tile_n = glu ? kBN / 2 : kBN;
   const int tiles = ((a.M + kBM * CG - 1) / (kBM * CG)) * ((a.N + tile_n - 1) / tile_n);

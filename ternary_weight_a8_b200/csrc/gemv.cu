@@ -1206,7 +1206,7 @@ template <int TT, typename TY, typename TX>
 static cudaError_t launch_group_t(const GvParams& P, int grid, int smem, cudaStream_t stream, bool pdl) {
   // Separate instances for the plain launch, the K-split and the fused
   // gate/up launch, so that each runs none of the others' code.
-  static bool attr_set[4] = {false, false, false, false};  // per template instance
+  static std::atomic<uint64_t> attr_done[4];  // per template instance and device
   constexpr bool kHasNarrow = TT == 1 && sizeof(TX) == 1;
   const int mode = P.glu.on ? 2 : P.ksplit > 1 ? 1 : P.narrow ? 3 : 0;
   if (mode == 3 && !kHasNarrow) return cudaErrorInvalidValue;
@@ -1214,11 +1214,10 @@ static cudaError_t launch_group_t(const GvParams& P, int grid, int smem, cudaStr
                 : mode == 1 ? gemv_group_kernel<TT, TY, TX, 1>
                 : mode == 3 ? gemv_group_kernel<TT, TY, TX, kHasNarrow ? 3 : 0>
                             : gemv_group_kernel<TT, TY, TX, 0>;
-  if (!attr_set[mode]) {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemPerBlock);
-    if (e != cudaSuccess) return e;
-    attr_set[mode] = true;
-  }
+  cudaError_t e = once_per_device(attr_done[mode], [&] {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemPerBlock);
+  });
+  if (e != cudaSuccess) return e;
   const int sp = mode == 1 ? 1 : 0;
   if (!sp) return launch(kernel, dim3(grid), dim3(kGvThreads), static_cast<size_t>(smem), stream, pdl, P);
   cudaLaunchConfig_t cfg = {};

@@ -514,14 +514,13 @@ cudaError_t launch_gemv_tc(const GemvLayerArgs* layers, int n_layers, int M, int
   const int sms = num_sms();
   const int grid = units < sms ? units : sms;
   P.one_unit = units <= grid ? 1 : 0;
-  static bool attr_set[2] = {false, false};
+  static std::atomic<uint64_t> attr_done[2];  // per output type and device
   const int yi = y_type == kOutBF16 ? 1 : 0;
   auto kernel = yi ? gemv_tc_kernel<__nv_bfloat16> : gemv_tc_kernel<float>;
-  if (!attr_set[yi]) {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[yi] = true;
-  }
+  cudaError_t e = once_per_device(attr_done[yi], [&] {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
+  });
+  if (e != cudaSuccess) return e;
   return launch(kernel, dim3(grid), dim3(kTcThreads), static_cast<size_t>(kTcSmemBytes), stream, pdl, P);
 }
 

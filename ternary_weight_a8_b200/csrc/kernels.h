@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace bl {
 
 enum OutType { kOutF32 = 0, kOutBF16 = 1 };
@@ -28,6 +30,20 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
 }
 
 int num_sms();
+
+// Runs `set` (a function attribute, which belongs to the current device's
+// context) unless it already succeeded on the calling thread's current
+// device: one bit per device, up to 64 devices (beyond that, every call).
+template <typename F>
+cudaError_t once_per_device(std::atomic<uint64_t>& done, F&& set) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 64;
+  const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  const cudaError_t e = set();
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // Offline weight path.
 cudaError_t launch_gamma(const float* W, int N, int K, double* row_sums, float* gamma,

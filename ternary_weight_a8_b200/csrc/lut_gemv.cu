@@ -114,16 +114,15 @@ cudaError_t launch_lut_gemv(const uint8_t* packed, const float* gamma, int N, in
                             cudaStream_t stream, bool pdl) {
   if (K % 64 != 0 || K > kLutMaxK || N <= 0) return cudaErrorInvalidValue;
   const int smem = lut_gemv_smem_bytes(K);
-  static bool attr_set[2] = {false, false};
+  static std::atomic<uint64_t> attr_done[2];  // per output type and device
   const int ti = y_type == kOutBF16 ? 1 : 0;
   auto kb = lut_gemv_kernel<__nv_bfloat16>;
   auto kf = lut_gemv_kernel<float>;
-  if (!attr_set[ti]) {
-    cudaError_t e = ti ? cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, 48 * 1024 * 4)
-                       : cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, 48 * 1024 * 4);
-    if (e != cudaSuccess) return e;
-    attr_set[ti] = true;
-  }
+  const cudaError_t e = once_per_device(attr_done[ti], [&] {
+    return ti ? cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, 48 * 1024 * 4)
+              : cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, 48 * 1024 * 4);
+  });
+  if (e != cudaSuccess) return e;
   // Blocks: a few per SM (as many as fit beside their tables), rows split among their warps.
   int per_sm = (224 * 1024) / (smem + 1024);
   if (per_sm < 1) per_sm = 1;

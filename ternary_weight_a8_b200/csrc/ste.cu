@@ -278,15 +278,14 @@ static cudaError_t launch_gemm_bf16(const __nv_bfloat16* A, const __nv_bfloat16*
                                    cudaStream_t stream) {
   CUtensorMap ta, tb;
   if (!map_bf16_2d(&ta, A, R, P, kFBM) || !map_bf16_2d(&tb, B, R, Q, kFBN)) return cudaErrorInvalidValue;
-  static bool attr[2] = {false, false};
-  if (!attr[out_bf16]) {
-    cudaError_t e = out_bf16 ? cudaFuncSetAttribute(gemm_bf16_kernel<__nv_bfloat16>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kFSmem)
-                             : cudaFuncSetAttribute(gemm_bf16_kernel<float>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kFSmem);
-    if (e != cudaSuccess) return e;
-    attr[out_bf16] = true;
-  }
+  static std::atomic<uint64_t> attr_done[2];  // per output type and device
+  const cudaError_t e = once_per_device(attr_done[out_bf16 ? 1 : 0], [&] {
+    return out_bf16 ? cudaFuncSetAttribute(gemm_bf16_kernel<__nv_bfloat16>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kFSmem)
+                    : cudaFuncSetAttribute(gemm_bf16_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kFSmem);
+  });
+  if (e != cudaSuccess) return e;
   const int tiles = ((P + kFBM - 1) / kFBM) * ((Q + kFBN - 1) / kFBN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   if (out_bf16)
