@@ -554,7 +554,7 @@ __device__ __noinline__ void glu_quant_slices(const GvParams& P, int N, const Wa
 }
 
 // kMode: 0 plain, 1 K-split over clusters, 2 the fused gate/up launch,
-// 3 narrow units (one token, streamed codes).
+// 3 narrow units (one token).
 template <int TT, typename TY, typename TX, int kMode>
 __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(const __grid_constant__ GvParams P) {
   constexpr bool kSplit = kMode == 1;
@@ -563,12 +563,12 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
   constexpr int TG = (TT + 7) / 8;           // mma token groups of 8
   constexpr bool kStream = sizeof(TX) == 1;  // int8 codes stream with the weights
   constexpr bool kAlu = TT == 1;             // one token: dp4a dot products instead of the mma path
-  static_assert(!kNarrow || (kAlu && kStream), "narrow units are a one-token, streamed-codes form");
+  static_assert(!kNarrow || kAlu, "narrow units are a one-token form");
   // Inputs per stage: a narrow unit's stage is 32 rows of twice the inputs.
   constexpr int kStageIn = kNarrow ? 2 * kGvStageK : kGvStageK;
   constexpr int kXHalf = x_half_bytes(TT);   // one half-stage activation tile
   constexpr int kSlot = kGvStageBytes + (kStream ? 2 * kXHalf : 0);
-  static_assert(!kNarrow || 2 * kXHalf >= 16 * 128, "a narrow stage's codes: 16 blocks of 128");
+  static_assert(!kNarrow || !kStream || 2 * kXHalf >= 16 * 128, "a narrow stage's codes: 16 blocks of 128");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nring = P.nring, M = P.M;
@@ -663,7 +663,7 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           tma_load_3d(dst + kGvStageBytes + kXHalf, &L.xmap, 0, 8 * st + 4, 0, full);
         }
       };
-      constexpr uint32_t kStageTx = kGvStageBytes + (kNarrow ? 16 * 128 : kStream ? 2 * TT * 4 * 128 : 0);
+      constexpr uint32_t kStageTx = kGvStageBytes + (!kStream ? 0 : kNarrow ? 16 * 128 : 2 * TT * 4 * 128);
       // The next ticket (none when each block takes only its own unit).
       auto next_unit = [&]() {
         if (P.one_unit) return P.total_units;
@@ -871,8 +871,8 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           for (int hf = 0; hf < 2; ++hf) {
             if constexpr (kNarrow) {
               // Rows it < 2 over inputs (2i)*1024 + hf*512 + 64ch .. +63, rows
-              // it >= 2 over the same 1024 further on: code block b = sb*8 + hf*4
-              // + ch/2 of the stage's 16-block tile.
+              // it >= 2 over the same 1024 further on: streamed codes are block
+              // b = sb*8 + hf*4 + ch/2 of the stage's 16-block tile.
 #pragma unroll
               for (int sb = 0; sb < 2; ++sb) {
                 const int k0 = (2 * i + sb) * kGvStageK + hf * (kGvStageK / 2) + 64 * ch;
@@ -880,8 +880,13 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
                   const int b = sb * 8 + hf * 4 + (ch >> 1);
                   uint4 xc[4];
 #pragma unroll
-                  for (int u = 0; u < 4; ++u)
-                    xc[u] = lds128(wt + kGvStageBytes + b * 128 + (((4 * (ch & 1) + u) ^ (b & 7)) << 4));
+                  for (int u = 0; u < 4; ++u) {
+                    if constexpr (kStream) {
+                      xc[u] = lds128(wt + kGvStageBytes + b * 128 + (((4 * (ch & 1) + u) ^ (b & 7)) << 4));
+                    } else {
+                      xc[u] = lds128(xs + x_chunk_off((k0 >> 4) + u));
+                    }
+                  }
 #pragma unroll
                   for (int it = 2 * sb; it < 2 * sb + 2; ++it)
 #pragma unroll
@@ -1044,8 +1049,8 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         v += __shfl_xor_sync(0xffffffffu, v, 1);
         const int n = n_base + warp * 8 + (lane >> 3) + 4 * ((lane >> 2) & 1);
         if ((lane & 3) == 0 && n < L.N) {
-          const int a = v - rsum1;
-          const float val = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, s1tok));
+          const int a = v - (kStream ? rsum1 : rs_tok[0]);
+          const float val = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, kStream ? s1tok : s_tok[0]));
           if constexpr (sizeof(TY) == 4) y[n] = val; else y[n] = __float2bfloat16_rn(val);
           if (L.acc_out) L.acc_out[n] = a;
         }
@@ -1207,7 +1212,7 @@ static cudaError_t launch_group_t(const GvParams& P, int grid, int smem, cudaStr
   // Separate instances for the plain launch, the K-split and the fused
   // gate/up launch, so that each runs none of the others' code.
   static std::atomic<uint64_t> attr_done[4];  // per template instance and device
-  constexpr bool kHasNarrow = TT == 1 && sizeof(TX) == 1;
+  constexpr bool kHasNarrow = TT == 1;
   const int mode = P.glu.on ? 2 : P.ksplit > 1 ? 1 : P.narrow ? 3 : 0;
   if (mode == 3 && !kHasNarrow) return cudaErrorInvalidValue;
   auto kernel = mode == 2   ? gemv_group_kernel<TT, TY, TX, 2>
@@ -1327,9 +1332,12 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   if (ks > nst_min) ks = nst_min;
   if (ks < 1 || glu) ks = 1;  // the fused gate/up launch hands its quantisation units out by ticket
   P.ksplit = ks;
-  // One token on streamed codes without a split: units of 32 rows, so that
-  // the last units handed out are half as long.
-  const bool narrow = tt == 1 && stream_x && ks == 1 && !glu;
+  // One token without a split: units of 32 rows, so that the last units
+  // handed out are half as long.  With the activations quantised by every
+  // block itself, only when the 64-row units would leave SMs without one
+  // (the 3B 3200->8640 layer: 5.9 -> 4.9 us; the 2B step, 148 units for 148
+  // SMs, went from 3.8 to 4.6 us as 296 blocks each quantising the token).
+  const bool narrow = tt == 1 && ks == 1 && !glu && (stream_x || units < sms);
   P.narrow = narrow ? 1 : 0;
   const int unit_rows = (narrow || glu) ? kGvRows / 2 : kGvRows;
   units = 0;

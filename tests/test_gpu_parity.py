@@ -546,3 +546,31 @@ def test_one_token_chain_of_streamed_codes_matches_the_oracle(xdt):
             assert np.array_equal(L.acc_out.cpu().numpy(), acc_ref)
             assert_y_matches(L.y, y_ref, acc_ref)
     assert tb.device_status(ws) == tb.BL_OK
+
+
+# One token quantised inside the decode kernel (small K, or one bf16 token of a
+# single layer up to K = 9856) on 32-row units: ragged N and K, fp32 and bf16
+# inputs and outputs; and a chain of such layers on different inputs.
+NARROW_IN_KERNEL = [(6400, 2560, "bf16"), (6433, 1088, "f32"), (7000, 4096, "bf16"), (6464, 9856, "bf16"),
+                    (6400, 64, "f32")]
+
+
+@pytest.mark.parametrize("N,K,xdt", NARROW_IN_KERNEL)
+def test_one_token_in_kernel_quantisation_narrow_units(N, K, xdt):
+    _full_case(1, N, K, xdt, torch.float32 if xdt == "f32" else torch.bfloat16, tb.PATH_GEMV, seed=N + 3 * K)
+
+
+def test_one_token_chain_in_kernel_quantisation_narrow_units():
+    specs = [(2560, 3000), (2560, 2000), (1024, 1500)]
+    layers, refs = [], []
+    for i, (K, N) in enumerate(specs):
+        x, xf = activations(1, K, seed=400 + i, dtype="bf16")
+        packed, gamma, T = oracle.pack_weights(weights(N, K, seed=410 + i))
+        layers.append(tb.Layer(dev(packed), dev(np.array([gamma], np.float32)), x,
+                               torch.empty((1, N), dtype=torch.bfloat16, device="cuda"),
+                               acc_out=torch.empty((1, N), dtype=torch.int32, device="cuda")))
+        refs.append(oracle.forward(T, gamma, xf))
+    tb.layer_chain(layers)
+    for L, (acc_ref, y_ref, *_) in zip(layers, refs):
+        assert np.array_equal(L.acc_out.cpu().numpy(), acc_ref)
+        assert_y_matches(L.y, y_ref, acc_ref)
