@@ -95,3 +95,27 @@ def test_no_writes_outside_outputs(M):
     for buf in (ybuf[:pad], ybuf[-pad:], abuf[:pad], abuf[-pad:], wbuf[ws_bytes:]):
         assert (buf == canary).all()
     assert tb.device_status(ws) == tb.BL_OK
+
+
+def test_default_argument_calls_launch_only_library_kernels():
+    """A forward or chain call without a workspace uses the cached one: after the
+    first call, the calls launch the library's kernels and nothing else (no
+    allocation, no fill)."""
+    from torch.profiler import ProfilerActivity, profile
+
+    packed, gamma = tb.pack_weights(dev(weights(640, 1024, seed=5)))
+    x, _ = activations(4, 1024, seed=6, dtype="bf16")
+    y = torch.empty((4, 640), dtype=torch.bfloat16, device="cuda")
+    layers = [tb.Layer(packed, gamma, x, torch.empty((4, 640), dtype=torch.bfloat16, device="cuda"))]
+    tb.forward(packed, gamma, x, y=y)
+    tb.layer_chain(layers)
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        for _ in range(3):
+            tb.forward(packed, gamma, x, y=y)
+            tb.layer_chain(layers)
+        torch.cuda.synchronize()
+    names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+    kernels = [n for n in names if "memcpy" not in n.lower() and "memset" not in n.lower()]
+    assert kernels, "no kernel was recorded"
+    assert all(n.startswith("void bl::") or n.startswith("bl::") for n in kernels), sorted(set(kernels))
