@@ -259,7 +259,9 @@ size_t bitlinear_workspace_bytes(int M, int N, int K);
  *   workspace / workspace_bytes: >= bitlinear_workspace_bytes(M, N, K), its
  *           first 256 bytes zero.
  * M <= 16 runs the decode GEMV kernel (which quantises small activations
- * itself); larger M the quantisation kernel and the tcgen05 tensor-core GEMM.
+ * itself: M * K up to 4096, or one bf16 token of up to 9856 inputs; else the
+ * quantisation kernel runs first); larger M the quantisation kernel and the
+ * tcgen05 tensor-core GEMM.
  */
 int bitlinear_forward(const uint8_t* packed, const float* gamma, int N, int K, const void* x,
                       int x_dtype, int M, void* y, int y_dtype, int32_t* acc_out, void* workspace,
@@ -345,7 +347,8 @@ int bitlinear_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int
  * declares once; every GPU that loads the library holds it until the
  * process exits.  What a call needs of it depends on the kernel that runs:
  * 256 bytes when the decode kernel quantises the activations itself (M * K
- * up to 4096), else 256 bytes plus about M * K bytes for the codes (exactly
+ * up to 4096, or one bf16 token of up to 9856 inputs), else 256 bytes plus
+ * about M * K bytes for the codes (exactly
  * bitlinear_workspace_bytes(M, N, K)).  Larger calls are refused with
  * BL_ERR_WORKSPACE_TOO_SMALL.  All calls share the array and each call first
  * clears its 256-byte control block, so calls in one stream are safe but
