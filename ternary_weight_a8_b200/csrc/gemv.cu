@@ -13,7 +13,8 @@
 //
 // Decode streams every weight byte once, so the kernel is built around one
 // uninterrupted weight stream per SM:
-//  * Work unit: 64 output rows of one layer over all of its K (three blocks per SM).  Units are
+//  * Work unit: 64 output rows of one layer over all of its K (32 rows for one
+//    token; three blocks per SM).  Units are
 //    ordered largest-K layer first; each block takes its first unit by index
 //    and the rest from a ticket counter in the workspace, so the blocks end
 //    within a fraction of a unit of one another.  The block that finishes
@@ -52,7 +53,12 @@
 //    rs, rs+4, rs+8, rs+12 of its warp's 16 and the matching 64 codes: the
 //    same AND per four weights, then one dp4a (unsigned codes x signed codes)
 //    per four weights into the four accumulator sets; the eight lanes of a
-//    row group finish with a three-step butterfly.
+//    row group finish with a three-step butterfly.  Without a split the unit
+//    is 32 rows over stages of 2048 inputs (narrow units: each half-stage
+//    holds the 32 rows over two 512-input ranges 1024 apart, so a lane's four
+//    rows are two rows over two ranges): twice the units, each half as long,
+//    so the blocks end closer together (with in-kernel quantisation only when
+//    the 64-row units would leave SMs idle).
 //  * Short, wide layers (few 64-row units for the SMs) are split along K: a
 //    cluster of ks CTAs shares each unit, rank r taking the contiguous stage
 //    range [r*nst/ks, (r+1)*nst/ks).  Every CTA folds its accumulator sets per
