@@ -15,11 +15,13 @@
 namespace bl {
 
 // Row sums sum_k |W[n][k]| in double, each in the fixed order k = 0, 1, ...
-// A warp takes 32 rows: it reads them 32 columns at a time, lane l loading
-// column l of each row (one 128-byte line per load, all 32 in flight), and
-// after a transpose through shared memory lane r adds row r's 32 values in
-// column order.
+// A warp takes 32 rows: it reads them kGroup x 32 columns at a time, lane l
+// loading column l of each row of each 32-column chunk (one 128-byte line
+// per load, 32 * kGroup of them in flight, which is what keeps the few warps
+// of a matrix fed), and after a transpose of each chunk through shared
+// memory lane r adds row r's values in column order.
 constexpr int kRowWarps = 4;
+constexpr int kGroup = 4;  // 32-column chunks loaded at once
 
 __global__ void __launch_bounds__(32 * kRowWarps) gamma_row_sums_kernel(const float* __restrict__ W, int N,
                                                                        int K, double* __restrict__ row_sums) {
@@ -29,19 +31,25 @@ __global__ void __launch_bounds__(32 * kRowWarps) gamma_row_sums_kernel(const fl
   if (row0 >= N) return;  // warp-uniform
   float (*t)[33] = tile[warp];
   double acc = 0.0;
-  for (int k0 = 0; k0 < K; k0 += 32) {  // K % 64 == 0: whole 32-column blocks
-    float v[32];
+  for (int k0 = 0; k0 < K; k0 += 32 * kGroup) {  // K % 64 == 0: whole 32-column chunks
+    float v[kGroup][32];
 #pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      const int n = row0 + r;
-      v[r] = n < N ? __ldg(W + static_cast<size_t>(n) * K + k0 + lane) : 0.0f;
+    for (int c = 0; c < kGroup; ++c)
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        const int n = row0 + r, k = k0 + 32 * c + lane;
+        v[c][r] = (n < N && k < K) ? __ldg(W + static_cast<size_t>(n) * K + k) : 0.0f;
+      }
+#pragma unroll
+    for (int c = 0; c < kGroup; ++c) {
+      if (k0 + 32 * c >= K) break;  // uniform
+#pragma unroll
+      for (int r = 0; r < 32; ++r) t[r][lane] = v[c][r];
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) acc = __dadd_rn(acc, fabs(static_cast<double>(t[lane][i])));
+      __syncwarp();
     }
-#pragma unroll
-    for (int r = 0; r < 32; ++r) t[r][lane] = v[r];
-    __syncwarp();
-#pragma unroll
-    for (int c = 0; c < 32; ++c) acc = __dadd_rn(acc, fabs(static_cast<double>(t[lane][c])));
-    __syncwarp();
   }
   if (row0 + lane < N) row_sums[row0 + lane] = acc;
 }
