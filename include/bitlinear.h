@@ -184,7 +184,11 @@ size_t bitlinear_gate_up_glu_workspace_bytes(int M, int N, int K);
  * M <= 8: one quantisation launch (or, for tiny x, none) and one decode
  * launch that computes gate and up, forms h as soon as both halves of a
  * group of rows are in, keeps the per-token maxima of |h| and, once every
- * row is in, quantises h with the final scales (no further launch).
+ * row is in, quantises h with the final scales (no further launch).  That
+ * launch waits grid-wide for its blocks, which it sizes for three per SM of
+ * the whole device: on a device partitioned so that fewer can be resident
+ * (an MPS limit on SMs, say) the wait runs out after 2 s and the call
+ * reports BL_ERR_DEVICE_TIMEOUT through the workspace status word.
  * 9 <= M <= 16: the gate and up products into the workspace, then the
  * gated-activation kernel (there the fused launch's grid-wide step cost more
  * than the launch it saves).  Larger M: the quantisation of x, one
