@@ -480,6 +480,41 @@ def test_shared_workspace_across_shapes_stays_consistent():
 # 32 rows over stages of 2048 inputs.  Ragged N (not a multiple of 32), K with
 # a partial last stage (down to a single 128-input block), and several layers
 # of different K in one launch.
+# Five to sixteen tokens on streamed codes (the mma path): groups with more
+# units than resident blocks (units by ticket), units of one or two stages
+# (shorter than the ring), ragged rows, K not a multiple of 1024 (a half-stage
+# past K), absent tokens of a slot (9 and 13 of 16); codes given ("q") or
+# quantised by the call ("x"); twice on one workspace.
+MMA_GROUPS = [(8, [(512, 40000, "q")]), (16, [(1024, 30000, "q")]), (9, [(1536, 20000, "q"), (576, 7001, "x")]),
+          (13, [(8192, 3000, "x"), (640, 9000, "q"), (2112, 1000, "x")]), (5, [(3200, 8640, "x")])]
+
+
+@pytest.mark.parametrize("M,specs", MMA_GROUPS,
+                         ids=["m%d-" % M + "+".join("%dx%d%s" % s for s in specs) for M, specs in MMA_GROUPS])
+def test_mma_path_groups_match_the_oracle(M, specs):
+    layers, refs = [], []
+    for i, (K, N, given) in enumerate(specs):
+        x, xf = activations(M, K, seed=400 + 7 * i + M, dtype="bf16")
+        packed, gamma, T = oracle.pack_weights(weights(N, K, seed=410 + i))
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+        if given == "q":
+            xq, sc, rs = tb.quant_act(x)
+            layers.append(tb.Layer(dev(packed), dev(np.array([gamma], np.float32)), None, y, xq=xq, scale=sc,
+                                   rowsum=rs, acc_out=acc))
+        else:
+            layers.append(tb.Layer(dev(packed), dev(np.array([gamma], np.float32)), x, y, acc_out=acc))
+        refs.append(oracle.forward(T, gamma, xf))
+    ws = tb.new_workspace(tb.chain_workspace_bytes(layers, M))
+    for _ in range(2):
+        tb.layer_chain(layers, workspace=ws)
+        for L, (acc_ref, y_ref, *_) in zip(layers, refs):
+            got = L.acc_out.cpu().numpy()
+            assert np.array_equal(got, acc_ref), "acc differs at %s" % np.argwhere(got != acc_ref)[:5].tolist()
+            assert_y_matches(L.y, y_ref, acc_ref)
+    assert tb.device_status(ws) == tb.BL_OK
+
+
 NARROW = [[(128, 6400)], [(1152, 6433)], [(8640, 7000)], [(2176, 3300), (4096, 3500), (128, 130)],
           [(14336, 3200), (8192, 3217)]]
 
