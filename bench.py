@@ -606,14 +606,13 @@ def run_decode_2b(args, world, peaks, L2):
             "device_status": tb.device_status(ws)}
 
 
-def measure_int8_peak(world, n=8192, reps=30):
-    """Dense int8 tensor-core throughput measured on this GPU: cuBLASLt's int8
-    GEMM (torch._int_mm, int32 accumulation) on n x n x n, timed with CUDA
-    events after warm-up.  The denominator of the prefill GEMM's roofline."""
+def measure_int8_gemm(world, m, n, k, reps=30):
+    """cuBLASLt's int8 GEMM (torch._int_mm, int32 accumulation) on [m][k] x [k][n],
+    timed with CUDA events after warm-up."""
     import torch
 
-    a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device="cuda")
-    b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device="cuda").t()  # column-major operand
+    a = torch.randint(-127, 128, (m, k), dtype=torch.int8, device="cuda")
+    b = torch.randint(-127, 128, (n, k), dtype=torch.int8, device="cuda").t()  # column-major operand
     for _ in range(5):
         torch._int_mm(a, b)
     torch.cuda.synchronize()
@@ -625,8 +624,16 @@ def measure_int8_peak(world, n=8192, reps=30):
     torch.cuda.synchronize()
     secs = max_over_ranks(e0.elapsed_time(e1) / 1e3 / reps, world)
     del a, b
-    return {"TOPS": round(2.0 * n ** 3 / secs / 1e12, 1), "shape": "%d^3 int8 x int8 -> int32" % n,
+    return {"TOPS": round(2.0 * m * n * k / secs / 1e12, 1), "shape": "%dx%dx%d int8 x int8 -> int32" % (m, n, k),
             "library": "cuBLASLt via torch._int_mm", "us_per_call": round(secs * 1e6, 2), "calls": reps}
+
+
+def measure_int8_peak(world, n=8192, reps=30):
+    """Dense int8 tensor-core throughput measured on this GPU: cuBLASLt's int8
+    GEMM on n x n x n.  The denominator of the prefill GEMM's roofline."""
+    r = measure_int8_gemm(world, n, n, n, reps)
+    r["shape"] = "%d^3 int8 x int8 -> int32" % n
+    return r
 
 
 def run_prefill(args, world, peaks, L2):
@@ -667,6 +674,10 @@ def run_prefill(args, world, peaks, L2):
         int8_peak = {"unavailable": "%s: %s" % (type(e).__name__, e)}
         peak_int8 = peaks["bf16"] * INT8_PER_BF16
         peak_src = "%s bf16 burst x %.0f (nominal int8/bf16 ratio)" % (peaks["source"], INT8_PER_BF16)
+    try:  # context: a library int8 GEMM of the same shape on int8 weights (no unpack, 4x the weight bytes)
+        same_shape = measure_int8_gemm(world, M, N, K)
+    except Exception as e:
+        same_shape = {"unavailable": "%s: %s" % (type(e).__name__, e)}
     k_tops = ops / mean_s / 1e12
     status = tb.device_status(ws)
     return {"metric": "prefill int8 TOPS", "value": round(tops, 1), "unit": "TOPS",
@@ -674,7 +685,7 @@ def run_prefill(args, world, peaks, L2):
                         "tcgen05 GEMM), bf16 in/out",
             "us_per_step": round(secs / steps * 1e6, 3), "tokens_per_s": round(M * world / (secs / steps), 0),
             "pct_int8_nominal_4500": round(100 * tops / world / 4500.0, 2), "timing": info,
-            "int8_peak": int8_peak,
+            "int8_peak": int8_peak, "library_int8_same_shape": same_shape,
             "roofline": {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 kind::i8), alone",
                          "achieved": round(k_tops, 1), "peak": peak_int8, "unit": "TOPS",
                          "frac": round(k_tops / peak_int8, 4),

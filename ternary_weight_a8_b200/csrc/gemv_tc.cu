@@ -448,12 +448,6 @@ bool gemv_tc_eligible(const GemvLayerArgs* layers, int n_layers, int M) {
   return true;
 }
 
-int gemv_tc_units(const GemvLayerArgs* layers, int n_layers) {
-  int units = 0;
-  for (int i = 0; i < n_layers; ++i) units += (layers[i].N + kTcRows - 1) / kTcRows;
-  return units;
-}
-
 cudaError_t launch_gemv_tc(const GemvLayerArgs* layers, int n_layers, int M, int y_type, uint32_t* status,
                            uint32_t* tickets, cudaStream_t stream, bool pdl) {
   if (!gemv_tc_eligible(layers, n_layers, M)) return cudaErrorInvalidValue;

@@ -128,7 +128,6 @@ void gemv_force_ksplit(int ks);
 // and 1 the CUDA-core kernel, 2 the tensor-core kernel whenever eligible.  Per thread.
 void gemv_force_form(int form);
 bool gemv_tc_eligible(const GemvLayerArgs* layers, int n_layers, int M);
-int gemv_tc_units(const GemvLayerArgs* layers, int n_layers);
 cudaError_t launch_gemv_tc(const GemvLayerArgs* layers, int n_layers, int M, int y_type, uint32_t* status,
                            uint32_t* tickets, cudaStream_t stream, bool pdl);
 
