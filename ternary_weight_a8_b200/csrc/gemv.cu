@@ -116,10 +116,13 @@ __host__ __device__ constexpr int x_half_bytes(int tt) { return ((tt * 4 * 128 +
 
 // The FFN's gate and up BitLinears in one launch, with the gated activation
 // and the quantisation of its result (the down BitLinear's input) done by the
-// same launch.  A unit is 32 output rows: each half-stage of its weights
-// holds those 32 gate rows, then the same 32 up rows, so that a lane's mma
-// fragment (rows g and g + 8 of its warp's 16), or a dp4a lane and its
-// partner lane ^ 4, holds the gate and up sums of one output row.  The lane
+// same launch.  With two or more tokens a unit is 32 output rows: each
+// half-stage of its weights holds those 32 gate rows, then the same 32 up
+// rows, so that a lane's mma fragment (rows g and g + 8 of its warp's 16)
+// holds the gate and up sums of one output row.  With one token a unit is 16
+// output rows over stages of 2048 inputs: each half-stage holds the 16 gate
+// rows over two 512-input ranges 1024 apart, then the same up rows over the
+// same ranges, so that a dp4a lane holds both sums of one row.  The lane
 // rounds both outputs to the activation type, as stored outputs are, forms
 // h = act(gate) * up, stores h and keeps the warp's running maximum of |h|
 // per token in registers.  When the units run out, the block folds its
@@ -570,11 +573,16 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
   constexpr bool kStream = sizeof(TX) == 1;  // int8 codes stream with the weights
   constexpr bool kAlu = TT == 1;             // one token: dp4a dot products instead of the mma path
   static_assert(!kNarrow || kAlu, "narrow units are a one-token form");
+  // The fused gate/up launch at one token: units of 16 gate and the same 16
+  // up rows over stages of 2048 inputs (each half-stage: the gate rows over two
+  // 512-input ranges 1024 apart, then the up rows over the same ranges).
+  constexpr bool kGluNarrow = kGlu && kAlu;
+  constexpr bool kWide = kNarrow || kGluNarrow;  // stages of 2048 inputs
   // Inputs per stage: a narrow unit's stage is 32 rows of twice the inputs.
-  constexpr int kStageIn = kNarrow ? 2 * kGvStageK : kGvStageK;
+  constexpr int kStageIn = kWide ? 2 * kGvStageK : kGvStageK;
   constexpr int kXHalf = x_half_bytes(TT);   // one half-stage activation tile
   constexpr int kSlot = kGvStageBytes + (kStream ? 2 * kXHalf : 0);
-  static_assert(!kNarrow || !kStream || 2 * kXHalf >= 16 * 128, "a narrow stage's codes: 16 blocks of 128");
+  static_assert(!kWide || !kStream || 2 * kXHalf >= 16 * 128, "a 2048-input stage's codes: 16 blocks of 128");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nring = P.nring, M = P.M;
@@ -620,16 +628,16 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       bool ok = true;
       int unit = unit_first;
       // The layer, row block and stage range of a unit.  A unit of the fused
-      // gate/up launch is 32 output rows: each half-stage holds those 32 gate
-      // rows, then the same 32 up rows.  A narrow unit is 32 rows too: each
-      // half-stage holds them over one 512-input range, then over the range
-      // 1024 inputs further on.
+      // gate/up launch is 32 output rows (16 at one token, over 2048-input
+      // stages; see GvGlu).  A narrow unit is 32 rows too: each half-stage
+      // holds them over one 512-input range, then over the range 1024 inputs
+      // further on.
       auto locate = [&](int u, const GvLayer*& Lp, int& rb, int& s0, int& s1) {
         if constexpr (kGlu) {
           Lp = &P.layer[P.glu.gate];
           rb = u;
           s0 = 0;
-          s1 = (Lp->K + kGvStageK - 1) / kGvStageK;
+          s1 = (Lp->K + kStageIn - 1) / kStageIn;
         } else {
           int l = 0;
           while (l + 1 < P.n_layers && u >= P.layer[l + 1].unit0) ++l;
@@ -639,7 +647,15 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         }
       };
       auto load_weights = [&](const GvLayer& L, int rb, int st, uint32_t full, uint32_t dst) {
-        if constexpr (kGlu) {
+        if constexpr (kGluNarrow) {
+          const GvLayer& LU = P.layer[P.glu.up];
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int b = 0; b < 4; ++b)  // gate range 0, gate range 1, up range 0, up range 1
+              tma_load_2d(dst + hf * (kGvStageBytes / 2) + b * (kGvRows / 4) * 128, b < 2 ? &L.tmap : &LU.tmap,
+                          (2 * st + (b & 1)) * 256 + hf * 128, rb * (kGvRows / 4), full);
+        } else if constexpr (kGlu) {
           const GvLayer& LU = P.layer[P.glu.up];
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
@@ -662,14 +678,14 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       // The stage's activation tiles (streamed codes), in the same slot after
       // the weights; a narrow stage's 2048 codes are one 16-block tile.
       auto load_act = [&](const GvLayer& L, int st, uint32_t full, uint32_t dst) {
-        if constexpr (kNarrow) {
+        if constexpr (kWide) {
           tma_load_3d(dst + kGvStageBytes, &L.xmap, 0, 16 * st, 0, full);
         } else {
           tma_load_3d(dst + kGvStageBytes, &L.xmap, 0, 8 * st, 0, full);
           tma_load_3d(dst + kGvStageBytes + kXHalf, &L.xmap, 0, 8 * st + 4, 0, full);
         }
       };
-      constexpr uint32_t kStageTx = kGvStageBytes + (!kStream ? 0 : kNarrow ? 16 * 128 : 2 * TT * 4 * 128);
+      constexpr uint32_t kStageTx = kGvStageBytes + (!kStream ? 0 : kWide ? 16 * 128 : 2 * TT * 4 * 128);
       // The next ticket (none when each block takes only its own unit).
       auto next_unit = [&]() {
         if (P.one_unit) return P.total_units;
@@ -855,18 +871,20 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           // rows of its warp in each half (inputs 64ch .. 64ch+63 of the half)
           // and the matching 64 codes: one AND and one dp4a per four weights,
           // no idle mma columns.  Each 8-lane phase reads one 128-byte swizzled
-          // row.  Rows: warp*16 + rs + 4*it; in the fused gate/up launch the
-          // first two are gate rows warp*8 + rs + 4*it, the last two the same
-          // up rows; in a narrow unit the last two are the first two over the
-          // inputs 1024 further on.
+          // row.  Rows: warp*16 + rs + 4*it; in a narrow unit the first two are
+          // rows warp*8 + rs + 4*it, the last two the same rows over the inputs
+          // 1024 further on; in the fused gate/up launch row warp*4 + rs of each
+          // of the four boxes (gate, gate 1024 further on, up, up further on).
           const int ch = lane & 7, rs = lane >> 3;
           uint4 wv[2][4];
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
             for (int it = 0; it < 4; ++it) {
-              const int row = (kGlu || kNarrow) ? (it < 2 ? warp * 8 + rs + 4 * it : 32 + warp * 8 + rs + 4 * (it - 2))
-                                                : warp * 16 + rs + 4 * it;
+              // (one-token gate/up units: row rs of the warp's 4 in box it)
+              const int row = kGluNarrow ? it * 16 + warp * 4 + rs
+                              : kNarrow ? (it < 2 ? warp * 8 + rs + 4 * it : 32 + warp * 8 + rs + 4 * (it - 2))
+                                        : warp * 16 + rs + 4 * it;
               wv[hf][it] = lds128(wt + hf * (kGvStageBytes / 2) + row * 128 + ((ch ^ (row & 7)) << 4));
             }
           if constexpr (!kStream) {
@@ -875,10 +893,12 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
           }
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
-            if constexpr (kNarrow) {
+            if constexpr (kWide) {
               // Rows it < 2 over inputs (2i)*1024 + hf*512 + 64ch .. +63, rows
-              // it >= 2 over the same 1024 further on: streamed codes are block
-              // b = sb*8 + hf*4 + ch/2 of the stage's 16-block tile.
+              // it >= 2 over the same 1024 further on (one-token gate/up
+              // units: boxes it = 0, 2 over the first range, 1, 3 over the
+              // second): streamed codes are block b = sb*8 + hf*4 + ch/2 of
+              // the stage's 16-block tile.
 #pragma unroll
               for (int sb = 0; sb < 2; ++sb) {
                 const int k0 = (2 * i + sb) * kGvStageK + hf * (kGvStageK / 2) + 64 * ch;
@@ -894,12 +914,14 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
                     }
                   }
 #pragma unroll
-                  for (int it = 2 * sb; it < 2 * sb + 2; ++it)
+                  for (int q = 0; q < 2; ++q) {
+                    const int it = kGluNarrow ? sb + 2 * q : 2 * sb + q;
 #pragma unroll
                     for (int v = 0; v < 4; ++v)
 #pragma unroll
                       for (int j = 0; j < 4; ++j)
                         dr[it][j] = dp4a_us(u4_get(wv[hf][it], v) & (0x03030303u << (2 * j)), u4_get(xc[v], j), dr[it][j]);
+                  }
                 }
               }
               continue;
@@ -1004,6 +1026,9 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         if constexpr (kNarrow) {  // rows rs and rs + 4: the two input ranges summed
           pc[0][0] += pc[0][2];
           pc[0][1] += pc[0][3];
+        } else if constexpr (kGluNarrow) {  // the gate row's and the up row's sums over both ranges
+          pc[0][0] += pc[0][1];
+          pc[0][1] = pc[0][2] + pc[0][3];
         }
       } else if constexpr (kSplit) {  // (the mma epilogue below combines them itself otherwise)
 #pragma unroll
@@ -1044,8 +1069,34 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
       // and up sums of the same output row (each output rounded to the
       // activation type first, as a stored output is), stores h and folds
       // |h| into the per-token maxima.
-      const int n_base = (kGlu ? unit : unit - L.unit0) * ((kGlu || kNarrow) ? kGvRows / 2 : kGvRows);
+      const int n_base =
+          (kGlu ? unit : unit - L.unit0) * (kGluNarrow ? kGvRows / 4 : (kGlu || kNarrow) ? kGvRows / 2 : kGvRows);
       TY* y = static_cast<TY*>(L.y);
+      if constexpr (kGluNarrow) {
+        // Gate and up sums of row rs of the warp's 4, over the 8 lanes of the row group.
+        int gs = pc[0][0], us = pc[0][1];
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) {
+          gs += __shfl_xor_sync(0xffffffffu, gs, o);
+          us += __shfl_xor_sync(0xffffffffu, us, o);
+        }
+        const int n = n_base + warp * 4 + (lane >> 3);
+        const int rsum = kStream ? rsum1 : rs_tok[0];
+        const float sm = kStream ? s1tok : s_tok[0];
+        float habs = 0.0f;
+        if ((lane & 7) == 0 && n < L.N) {
+          const float g_v = round_to<TY>(__fmul_rn(static_cast<float>(gs - rsum), __fdiv_rn(gamma, sm)));
+          const float u_v = round_to<TY>(__fmul_rn(static_cast<float>(us - rsum), __fdiv_rn(gamma_up, sm)));
+          const float h = glu_value<TY>(g_v, u_v, P.glu.act);
+          TY* hp = static_cast<TY*>(P.glu.h);
+          if constexpr (sizeof(TY) == 4) hp[n] = h; else hp[n] = __float2bfloat16_rn(h);
+          habs = fabsf(h);
+        }
+        habs = fmaxf(habs, __shfl_xor_sync(0xffffffffu, habs, 8));
+        habs = fmaxf(habs, __shfl_xor_sync(0xffffffffu, habs, 16));
+        hmax[0][0] = fmaxf(hmax[0][0], habs);
+        continue;
+      }
       if constexpr (kNarrow) {
         // Rows rs (lanes with ch < 4 after the first step) and rs + 4 of the
         // warp's 8, summed over the 8 lanes of the row group.
@@ -1082,31 +1133,12 @@ __global__ void __launch_bounds__(kGvThreads, kGvBlocksPerSM) gemv_group_kernel(
         v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
         const int rsum = kStream ? rsum1 : rs_tok[0];
         const float sm = kStream ? s1tok : s_tok[0];
-        if constexpr (kGlu) {
-          // Row numbers 0..7 of the warp's 16 are gate rows, 8..15 the same up
-          // rows: a gate lane finds its up sum in lane ^ 4.
-          const int vu = __shfl_xor_sync(0xffffffffu, v[0], 4);
-          const int n = n_base + warp * 8 + (lane >> 3) + 4 * ((lane >> 1) & 1);
-          float habs = 0.0f;
-          if ((lane & 5) == 0 && n < L.N) {
-            const float g_v = round_to<TY>(__fmul_rn(static_cast<float>(v[0] - rsum), __fdiv_rn(gamma, sm)));
-            const float u_v = round_to<TY>(__fmul_rn(static_cast<float>(vu - rsum), __fdiv_rn(gamma_up, sm)));
-            const float h = glu_value<TY>(g_v, u_v, P.glu.act);
-            TY* hp = static_cast<TY*>(P.glu.h);
-            if constexpr (sizeof(TY) == 4) hp[n] = h; else hp[n] = __float2bfloat16_rn(h);
-            habs = fabsf(h);
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) habs = fmaxf(habs, __shfl_xor_sync(0xffffffffu, habs, o));
-          hmax[0][0] = fmaxf(hmax[0][0], habs);
-        } else {
-          const int n = n_base + warp * 16 + (lane >> 3) + 4 * ((lane >> 1) & 3);
-          if ((lane & 1) == 0 && n < L.N) {
-            const int a = v[0] - rsum;
-            const float val = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, sm));
-            if constexpr (sizeof(TY) == 4) y[n] = val; else y[n] = __float2bfloat16_rn(val);
-            if (L.acc_out) L.acc_out[n] = a;
-          }
+        const int n = n_base + warp * 16 + (lane >> 3) + 4 * ((lane >> 1) & 3);
+        if ((lane & 1) == 0 && n < L.N) {
+          const int a = v[0] - rsum;
+          const float val = __fmul_rn(static_cast<float>(a), __fdiv_rn(gamma, sm));
+          if constexpr (sizeof(TY) == 4) y[n] = val; else y[n] = __float2bfloat16_rn(val);
+          if (L.acc_out) L.acc_out[n] = a;
         }
         continue;
       }
@@ -1345,13 +1377,16 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   // SMs, went from 3.8 to 4.6 us as 296 blocks each quantising the token).
   const bool narrow = tt == 1 && ks == 1 && !glu && (stream_x || units < sms);
   P.narrow = narrow ? 1 : 0;
-  const int unit_rows = (narrow || glu) ? kGvRows / 2 : kGvRows;
+  // Rows per unit: 16 (+ 16 up rows) in the fused gate/up launch at one token,
+  // 32 (+ 32) with more tokens, 32 for narrow units, 64 otherwise.
+  const bool glu_narrow = glu && tt == 1;
+  const int unit_rows = glu_narrow ? kGvRows / 4 : (narrow || glu) ? kGvRows / 2 : kGvRows;
   units = 0;
   for (int i = 0; i < n_layers; ++i) {
     const GemvLayerArgs& a = layers[order[i]];
     GvLayer& L = P.layer[i];
     {
-      // Boxes of 32 rows for the fused gate/up launch and narrow units.
+      // Boxes of one unit's rows (16 or 32 for the fused gate/up launch, 32 for narrow units).
       const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K / 4), static_cast<cuuint64_t>(a.N)};
       const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K / 4)};
       const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(unit_rows)};
@@ -1368,7 +1403,7 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
       // narrow stage takes its 16 blocks in one box.
       const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(a.ldx / 128), static_cast<cuuint64_t>(M)};
       const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(a.ldx)};
-      const cuuint32_t box[3] = {128, narrow ? 16u : 4u, static_cast<cuuint32_t>(tt)};
+      const cuuint32_t box[3] = {128, (narrow || glu_narrow) ? 16u : 4u, static_cast<cuuint32_t>(tt)};
       const cuuint32_t estr[3] = {1, 1, 1};
       if (enc(&L.xmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(a.x), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
@@ -1387,7 +1422,7 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
     L.unit0 = units;
     units += (a.N + unit_rows - 1) / unit_rows;
   }
-  // A unit of the fused gate/up launch covers the same 32 rows of both layers.
+  // A unit of the fused gate/up launch covers the same rows of both layers.
   if (glu) units = (layers[0].N + unit_rows - 1) / unit_rows;
   P.total_units = units;
   if (glu) {

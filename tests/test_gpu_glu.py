@@ -52,16 +52,19 @@ def _ffn(M, N, K, dtype, seed):
     return x, dev_w, _values(yg), _values(yu)
 
 
-# Decode sizes: 1 to 8 tokens in one launch (N past one 32-row unit, ragged
-# unit counts, and 8 x 114688, whose 512-element quantisation slices outnumber
-# the grid's warps), 9 to 16 tokens as the products then the gated-activation
-# kernel; and many tokens (the tensor-core GEMM whose
+# Decode sizes: 1 to 8 tokens in one launch (N past one unit, ragged unit
+# counts, and 8 x 114688, whose 512-element quantisation slices outnumber
+# the grid's warps; at one token 16-row units over 2048-input stages: four
+# units, K not a multiple of 2048, and more units than resident blocks), 9 to 16
+# tokens as the products then the gated-activation kernel; and many tokens
+# (the tensor-core GEMM whose
 # tiles pair gate and up rows: one CTA up to 128 tokens, CTA pairs beyond,
 # ragged M, N (not a multiple of the 128-column tile) and K).
 RELU2 = [(1, 1024, 1024, "bf16"), (1, 2816, 2560, "bf16"), (3, 704, 4096, "f32"), (8, 2816, 1024, "bf16"),
          (16, 1088, 2048, "bf16"), (1, 6912, 2560, "bf16"), (40, 704, 512, "bf16"), (2048, 1024, 512, "bf16"),
          (300, 1088, 576, "f32"), (513, 704, 320, "bf16"), (8, 114688, 128, "bf16"), (9, 1088, 1024, "f32"),
-         (12, 2816, 2560, "bf16")]
+         (12, 2816, 2560, "bf16"), (1, 1088, 3072, "bf16"), (1, 64, 8192, "bf16"), (1, 4160, 640, "f32"),
+         (1, 28736, 1024, "bf16")]
 
 
 @pytest.mark.parametrize("M,N,K,dtype", RELU2)
