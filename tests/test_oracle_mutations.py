@@ -28,6 +28,11 @@ MUTANTS = {
     "act_scale_128": ("float scale = 127.0f / fmaxf(amax, ORACLE_EPS);", "float scale = 128.0f / fmaxf(amax, ORACLE_EPS);"),
     "act_round_half_away": ("float v = rintf(x[m * K + k] * scale);", "float v = roundf(x[m * K + k] * scale);"),
     "act_signed_max": ("float a = fabsf(x[m * K + k]);", "float a = x[m * K + k];"),
+    "act_rowsum_of_abs": ("sum += (int8_t)v;", "sum += abs((int8_t)v);"),
+    "act_scale_without_eps": ("float scale = 127.0f / fmaxf(amax, ORACLE_EPS);", "float scale = 127.0f / amax;"),
+    "unpack_wrong_field": ("uint32_t code = (word >> (8 * b + 2 * j)) & 3u;", "uint32_t code = (word >> (8 * j + 2 * b)) & 3u;"),
+    "bf16_truncates": ("double r = rint(ldexp(a, -qexp));", "double r = floor(ldexp(a, -qexp));"),
+    "bf16_no_subnormal_spacing": ("if (qexp < -133) qexp = -133;", ";"),
     "acc_transposed_weight": ("(int64_t)T[n * K + k];", "(int64_t)T[k * N + n];"),
     "dequant_multiplies_scale": ("(double)gamma / (double)s[m];", "(double)gamma * (double)s[m];"),
     "dequant_gamma_plus_eps": ("(double)gamma / (double)s[m];", "((double)gamma + 1e-5) / (double)s[m];"),
