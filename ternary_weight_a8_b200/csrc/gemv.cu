@@ -1357,13 +1357,19 @@ cudaError_t launch_gemv_group(const GemvLayerArgs* layers, int n_layers, int M, 
   P.tickets = tickets;
   // Few units for the SMs (a short, wide layer): a cluster of ks CTAs shares
   // each unit, every CTA over its own contiguous range of the unit's stages.
-  // One token: about one CTA per SM.  More tokens, where one warp per SM
-  // sub-partition issuing mma.sync is the limit: about two.  ks is that target
+  // One token: about one CTA per SM to decide whether to split, about 1.35 once
+  // split.  More tokens, where one warp per SM sub-partition issuing mma.sync
+  // is the limit: about two.  ks is that target
   // over the unit count, rounded; at most 8, at most the fewest stages of any
   // layer, and no more CTAs than are resident at once.
   const int sms = num_sms();
   const int target = tt == 1 ? sms : 2 * sms;
   int ks = units < target ? (target + units / 2) / units : 1;
+  // One token split at all: about 1.35 CTAs per SM measured better than one
+  // (the 3B 8640->3200 layer 7.8 -> 7.3 us, 11008->4096 10.0 -> 8.7 us, none
+  // slower); groups that would not split are left whole, since splitting them
+  // gives up the narrow units (4096->8192: 5.1 -> 6.0 us).
+  if (tt == 1 && ks >= 2) ks = (sms * 27 / 20 + units / 2) / units;
   if (g_force_ksplit > 0) ks = g_force_ksplit;
   while (ks > 1 && units * ks > kGvBlocksPerSM * sms) --ks;
   if (ks > kGvMaxSplit) ks = kGvMaxSplit;
