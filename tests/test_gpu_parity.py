@@ -174,7 +174,9 @@ def test_forward_one_token(N, K, xdtype):
 # Layers with fewer 64-row units than SMs are split along K over the CTAs of a
 # cluster (2 to 8, each a contiguous range of 1024-input stages) whose partial
 # sums meet in one CTA's shared memory: one to 16 tokens, ragged N and K.
-KSPLIT = [(130, 3072), (64, 8192), (300, 2112), (17, 4160)]
+# Short, wide layers the decode kernel splits along K by itself; the last two
+# take 5 and 3 CTAs per unit at one token (about 1.35 CTAs per SM).
+KSPLIT = [(130, 3072), (64, 8192), (300, 2112), (17, 4160), (2560, 6912), (4096, 11008)]
 
 
 @pytest.mark.parametrize("N,K", KSPLIT)
